@@ -1,0 +1,155 @@
+"""Expert FFN: grouped w1/w3 GEMM, SwiGLU with +-10 clamp, w2 GEMM, combine.
+
+Passages:
+  * "DeepSeek-V4-Flash-SI" model card, 架构特性 (Mixture of Experts paragraph):
+    routed + shared experts, SwiGLU activation clamped to +-10.0, routing
+    scale 1.5; 低精度计算: FP4 E2M1 expert weights with an E8M0 scale per 32
+    elements, activations FP8 E4M3 with a power-of-two scale per 128.
+  * "DeepSeek-V4-Flash-0731-W4AFP8-mt" model card, 量化方式 / 权重约定: expert
+    projections are named w1, w2, w3; weights are [N, K] with K the input
+    dimension; the W4AFP8 form holds INT4 weights with a float32
+    weight_scale_inv of shape [N, K/128] and dynamic E4M3 activations.
+
+Readings: w1 = gate, w3 = up, w2 = down; both gate and up are clamped to
+[-limit, limit] before silu(gate) * up (which tensors the clamp applies to is
+not stated: parity unpinned beyond the closed forms); the router weight is
+applied in the combine, after w2; the shared expert has weight 1.0 (no route
+scale).  The GEMMs are the plain definition: dequantise both operands exactly
+to float64 and multiply (numpy matmul as the library step).  h is rounded to
+float32 before requantisation because the quantisation decision is taken in
+float32 (the kernels' precision) -- see oracle.quant.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import decode_e2m1_packed, decode_e8m0
+from .permute import gather_rows, permute
+from .quant import dequantize_fp8_pow2, quantize_act_fp8, quantize_fp8_pow2
+from .route import route_topk
+
+
+def dequant_mxfp4(packed: np.ndarray, e8m0: np.ndarray) -> np.ndarray:
+    """MXFP4 [N, K/2] + E8M0 [N, K/32] -> float64 [N, K]."""
+    v = decode_e2m1_packed(packed)
+    N, K = v.shape[-2], v.shape[-1]
+    s = decode_e8m0(e8m0)
+    return (v.reshape(*v.shape[:-1], K // 32, 32) * s[..., None]).reshape(v.shape)
+
+
+def dequant_int4g128(q_packed: np.ndarray, scale_inv: np.ndarray) -> np.ndarray:
+    """Symmetric INT4 [N, K/2] (two's complement, element 2i in the low nibble)
+    + float32 scale_inv [N, K/128] -> float64 [N, K]."""
+    q_packed = np.asarray(q_packed).view(np.uint8)
+    lo = (q_packed & 0xF).astype(np.int64)
+    hi = (q_packed >> 4).astype(np.int64)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    q = np.empty(q_packed.shape[:-1] + (q_packed.shape[-1] * 2,), np.float64)
+    q[..., 0::2] = lo
+    q[..., 1::2] = hi
+    N, K = q.shape[-2], q.shape[-1]
+    s = np.asarray(scale_inv, dtype=np.float32).astype(np.float64)
+    return (q.reshape(*q.shape[:-1], K // 128, 128) * s[..., None]).reshape(q.shape)
+
+
+def grouped_gemm(a_q, a_s, offsets, w_deq_fn, n_groups):
+    """Rows offsets[g]:offsets[g+1] of the FP8 operand times group g's weights^T.
+
+    a_q: E4M3 [R, K]; a_s: E8M0 [R, K/128]; w_deq_fn(g) -> float64 [N, K].
+    Returns float64 [R, N]."""
+    a = dequantize_fp8_pow2(a_q, a_s)
+    out = None
+    for g in range(n_groups):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        if r1 == r0:
+            continue
+        w = w_deq_fn(g)
+        if out is None:
+            out = np.zeros((a.shape[0], w.shape[0]), np.float64)
+        out[r0:r1] = a[r0:r1] @ w.T
+    if out is None:
+        out = np.zeros((a.shape[0], 0), np.float64)
+    return out
+
+
+def grouped_gemm_mxfp4(a_q, a_s, offsets, w_fp4, w_e8m0):
+    """Steps a4 / a6: FP8 rows x MXFP4 weights [G, N, K/2] -> float64 [R, N]."""
+    N = w_fp4.shape[1]
+    out = grouped_gemm(a_q, a_s, offsets, lambda g: dequant_mxfp4(w_fp4[g], w_e8m0[g]),
+                       w_fp4.shape[0])
+    return out if out.shape[1] else np.zeros((a_q.shape[0], N))
+
+
+def grouped_gemm_w4afp8(a_q, a_s, offsets, w_int4, w_scale_inv):
+    """Step a10: FP8 rows x INT4-g128 weights [G, N, K/2] -> float64 [R, N]."""
+    N = w_int4.shape[1]
+    out = grouped_gemm(a_q, a_s, offsets,
+                       lambda g: dequant_int4g128(w_int4[g], w_scale_inv[g]), w_int4.shape[0])
+    return out if out.shape[1] else np.zeros((a_q.shape[0], N))
+
+
+def silu(g: np.ndarray) -> np.ndarray:
+    return g / (1.0 + np.exp(-g))
+
+
+def swiglu_clamp(gu: np.ndarray, I: int, limit: float = 10.0) -> np.ndarray:
+    """Step a5 (activation): gu float [R, 2I] (gate | up) -> h float64 [R, I]."""
+    gu = np.asarray(gu, dtype=np.float64)
+    g = np.clip(gu[:, :I], -limit, limit)
+    u = np.clip(gu[:, I:2 * I], -limit, limit)
+    return silu(g) * u
+
+
+def swiglu_quant(gu: np.ndarray, I: int, limit: float = 10.0):
+    """Step a5: SwiGLU then the per-128 power-of-two FP8 requantisation."""
+    h = swiglu_clamp(gu, I, limit)
+    return quantize_fp8_pow2(h.astype(np.float32))
+
+
+def combine(o: np.ndarray, inv: np.ndarray, w: np.ndarray, offsets: np.ndarray,
+            has_shared: int = 1) -> np.ndarray:
+    """Step a7: y[t] = sum_j w[t, j] * o[inv[t, j]] + o[shared row of t] (float64)."""
+    T, k = w.shape
+    y = np.zeros((T, o.shape[1]), np.float64)
+    invr = np.asarray(inv).reshape(T, k)
+    for j in range(k):
+        y += np.asarray(w[:, j], np.float64)[:, None] * o[invr[:, j]]
+    if has_shared:
+        E = len(offsets) - 2
+        y += o[int(offsets[E]) + np.arange(T)]
+    return y
+
+
+def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
+              swiglu_limit=10.0, has_shared=1, route_norm=1, weights="mxfp4",
+              w13_int4=None, w13_sinv=None, w2_int4=None, w2_sinv=None, tokens=None):
+    """The whole expert path (a1 -> a7) for the tokens listed in ``tokens``
+    (all tokens when None).  Token outputs are independent given the routing,
+    so a subset gives exactly those rows of the full result.
+
+    Returns a dict of the intermediates (indices refer to the subset)."""
+    x_bf16 = np.asarray(x_bf16)
+    logits = np.asarray(logits, dtype=np.float32)
+    if tokens is not None:
+        x_bf16 = x_bf16[tokens]
+        logits = logits[tokens]
+    T, H = x_bf16.shape
+    E = logits.shape[1]
+    I = w2.shape[2] * 2 if weights == "mxfp4" else w2_int4.shape[2] * 2
+    xq, sx = quantize_act_fp8(x_bf16)
+    idx, w = route_topk(logits, topk, route_scale, route_norm)
+    counts, offsets, perm, inv, src = permute(idx, E, has_shared)
+    xq_p, sx_p = gather_rows(xq, sx, src)
+    if weights == "mxfp4":
+        gu = grouped_gemm_mxfp4(xq_p, sx_p, offsets, w13, w13_e8m0)
+    else:
+        gu = grouped_gemm_w4afp8(xq_p, sx_p, offsets, w13_int4, w13_sinv)
+    hq, sh = swiglu_quant(gu, I, swiglu_limit)
+    if weights == "mxfp4":
+        o = grouped_gemm_mxfp4(hq, sh, offsets, w2, w2_e8m0)
+    else:
+        o = grouped_gemm_w4afp8(hq, sh, offsets, w2_int4, w2_sinv)
+    y = combine(o, inv, w, offsets, has_shared)
+    return dict(xq=xq, sx=sx, idx=idx, w=w, counts=counts, offsets=offsets, perm=perm,
+                inv=inv, xq_perm=xq_p, sx_perm=sx_p, gu=gu, hq=hq, sh=sh, o=o, y=y)

@@ -1,0 +1,223 @@
+"""Seeded synthetic inputs for the routed-expert MoE layer.
+
+This module is the only code shared between the CPU oracle (``oracle/``) and
+the CUDA path: it produces *inputs* (activations, router logits, MXFP4 expert
+weights, random FP8 operands) and holds none of the arithmetic of the layer
+itself.  Everything is generated on the host with numpy from a counter-based
+generator, so both sides see identical bytes.
+
+Generator: splitmix64 (S. Vigna's published mixing function) used in counter
+mode -- output ``i`` of stream ``s`` under ``seed`` is
+``mix(key(seed, s) + (i + 1) * 0x9E3779B97F4A7C15)``; each tensor draws from
+its own stream so tensors do not depend on generation order.  Normals use the
+Box-Muller transform.
+
+The workload recipes follow the shapes of a DeepSeek-V4-Flash-class MoE layer
+(hidden 4096, expert intermediate 2048, 256 routed + 1 shared experts, top-6),
+as given on the "DeepSeek-V4-Flash-SI" model card (section 模型概述 and the
+MoE paragraph of 架构特性).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    z = (z ^ (z >> np.uint64(30))) * _M1
+    z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def splitmix64(seed: int, stream: int, n: int) -> np.ndarray:
+    """n uint64 outputs of the counter-mode splitmix64 stream (seed, stream)."""
+    with np.errstate(over="ignore"):
+        key = _mix(np.array([(seed * 0x632BE59BD9B4E019 + stream) & 0xFFFFFFFFFFFFFFFF],
+                            dtype=np.uint64))[0] if (seed or stream) else np.uint64(0)
+        ctr = np.arange(1, n + 1, dtype=np.uint64) * _GAMMA
+        return _mix(ctr + key)
+
+
+def uniform(seed: int, stream: int, n: int) -> np.ndarray:
+    """n doubles in [0, 1) with 53 random bits each."""
+    return (splitmix64(seed, stream, n) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+
+
+def normal(seed: int, stream: int, n: int) -> np.ndarray:
+    """n standard normals (Box-Muller, cosine branch)."""
+    u = uniform(seed, stream, 2 * n)
+    r = np.sqrt(-2.0 * np.log1p(-u[0::2]))   # 1-u in (0, 1]
+    return r * np.cos(2.0 * np.pi * u[1::2])
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float64 -> float32 -> bfloat16 (round to nearest even), as uint16 bits."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + np.uint64(0x7FFF) + ((b >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return b.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 weight synthesis (an input format, not a step of the layer).
+# Each block of 32 values gets the exponent e = ceil(log2(amax / 6)) so the
+# block maximum lands in (3, 6]; values are rounded to the nearest E2M1 grid
+# point with ties to the even code, saturating at 6.  All-zero blocks get e=0.
+# ---------------------------------------------------------------------------
+_E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _round_to_e2m1_code(m: np.ndarray) -> np.ndarray:
+    """Magnitudes (already divided by the block scale) -> 3-bit codes 0..7."""
+    m = np.minimum(m, 6.0)
+    # distance to every grid point; ties are resolved toward the even code
+    d = np.abs(m[..., None] - _E2M1_GRID)
+    best = d.min(axis=-1, keepdims=True)
+    cand = d == best
+    even = cand & (np.arange(8) % 2 == 0)
+    pick = np.where(even.any(axis=-1, keepdims=True), even, cand)
+    return np.argmax(pick, axis=-1).astype(np.uint8)
+
+
+def quantize_mxfp4(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """float [..., K] -> (packed nibbles uint8 [..., K/2], E8M0 uint8 [..., K/32]).
+
+    Element 2i sits in the low nibble, 2i+1 in the high nibble.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    K = w.shape[-1]
+    assert K % 32 == 0
+    blocks = w.reshape(*w.shape[:-1], K // 32, 32)
+    amax = np.abs(blocks).max(axis=-1)
+    with np.errstate(divide="ignore"):
+        ratio = amax / 6.0
+        e = np.where(amax > 0, np.ceil(np.log2(np.where(amax > 0, ratio, 1.0))), 0.0)
+    # guard against log2 rounding: make sure amax / 2^e <= 6 and > 3
+    e = np.where((amax > 0) & (amax / np.exp2(e) > 6.0), e + 1, e)
+    e = np.where((amax > 0) & (amax / np.exp2(e) <= 3.0), e - 1, e)
+    e = np.clip(e, -127, 127)
+    scaled = blocks / np.exp2(e)[..., None]
+    code = _round_to_e2m1_code(np.abs(scaled))
+    sign = ((scaled < 0) & (code > 0)).astype(np.uint8)
+    nib = (code | (sign << 3)).reshape(*w.shape[:-1], K)
+    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+    return packed, (e + 127).astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# Layer workloads
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass
+class MoeWorkload:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    topk: int
+    x_bf16: np.ndarray          # uint16 [T, H]
+    logits: np.ndarray          # float32 [T, E]
+    w13: np.ndarray             # uint8 [E+1, 2I, H/2]  (w1 = gate rows, then w3 = up rows)
+    w13_e8m0: np.ndarray        # uint8 [E+1, 2I, H/32]
+    w2: np.ndarray              # uint8 [E+1, H, I/2]
+    w2_e8m0: np.ndarray         # uint8 [E+1, H, I/32]
+    route_scale: float = 1.5
+    swiglu_limit: float = 10.0
+
+
+def expert_weights(seed: int, E1: int, H: int, I: int, std: float = 0.02,
+                   experts: np.ndarray | None = None):
+    """MXFP4 w13 [E1, 2I, H] and w2 [E1, H, I] from N(0, std).
+
+    Each expert draws from its own streams, so a subset (``experts``) can be
+    generated without the others; rows of untouched experts are left zero.
+    """
+    w13 = np.zeros((E1, 2 * I, H // 2), np.uint8)
+    s13 = np.full((E1, 2 * I, H // 32), 127, np.uint8)
+    w2 = np.zeros((E1, H, I // 2), np.uint8)
+    s2 = np.full((E1, H, I // 32), 127, np.uint8)
+    for e in (range(E1) if experts is None else experts):
+        a = normal(seed, 1000 + 2 * e, 2 * I * H).reshape(2 * I, H) * std
+        w13[e], s13[e] = quantize_mxfp4(a)
+        b = normal(seed, 1001 + 2 * e, H * I).reshape(H, I) * std
+        w2[e], s2[e] = quantize_mxfp4(b)
+    return w13, s13, w2, s2
+
+
+def tiny_layer(seed: int = 0) -> MoeWorkload:
+    """Hidden 256, intermediate 128, 8 routed + 1 shared, top-2, 16 tokens.
+
+    Router logits = x . Wg^T with Wg ~ N(0, 0.02), computed on the host (the
+    gate projection is not part of the expert path)."""
+    T, H, I, E, k = 16, 256, 128, 8, 2
+    x = to_bf16_bits(normal(seed, 1, T * H).reshape(T, H))
+    wg = normal(seed, 2, E * H).reshape(E, H) * 0.02
+    logits = (bf16_bits_to_f32(x).astype(np.float64) @ wg.T).astype(np.float32)
+    w13, s13, w2, s2 = expert_weights(seed, E + 1, H, I)
+    return MoeWorkload("tiny", T, H, I, E, k, x, logits, w13, s13, w2, s2)
+
+
+def decode_activations(seed: int, T: int, H: int) -> np.ndarray:
+    """N(0,1) with each element scaled x20 with probability 0.001 (outliers)."""
+    x = normal(seed, 1, T * H)
+    out = uniform(seed, 3, T * H) < 0.001
+    x = np.where(out, 20.0 * x, x)
+    return to_bf16_bits(x.reshape(T, H))
+
+
+def uniform_logits(seed: int, T: int, E: int) -> np.ndarray:
+    return (uniform(seed, 4, T * E) * 2.0 - 1.0).astype(np.float32).reshape(T, E)
+
+
+def zipf_logits(seed: int, T: int, E: int, s: float = 1.1) -> np.ndarray:
+    """log p_e + Gumbel(0,1) noise with p_e proportional to rank^-s.
+
+    Top-k of Gumbel-perturbed log-probabilities draws experts without
+    replacement with probabilities p, so expert loads follow the Zipf law
+    (flattened at the head because each token picks k distinct experts).
+    Expert e has rank e+1."""
+    logp = -s * np.log(np.arange(1, E + 1, dtype=np.float64))
+    logp -= np.log(np.exp(logp).sum())
+    u = uniform(seed, 5, T * E).reshape(T, E)
+    g = -np.log(-np.log(np.clip(u, 1e-300, None)))
+    return (logp[None, :] + g).astype(np.float32)
+
+
+def random_e4m3(seed: int, stream: int, shape, max_code: int = 0x7E) -> np.ndarray:
+    """Random finite E4M3 bytes (codes 0x7F / 0xFF are NaN and never drawn)."""
+    n = int(np.prod(shape))
+    r = splitmix64(seed, stream, n)
+    mag = (r % np.uint64(max_code + 1)).astype(np.uint8)
+    sign = ((r >> np.uint64(32)) & np.uint64(1)).astype(np.uint8) << 7
+    return (mag | sign).reshape(shape)
+
+
+def random_bytes(seed: int, stream: int, shape, lo: int = 0, hi: int = 255) -> np.ndarray:
+    n = int(np.prod(shape))
+    r = splitmix64(seed, stream, n)
+    return (lo + (r % np.uint64(hi - lo + 1))).astype(np.uint8).reshape(shape)
+
+
+def small_int_e4m3(seed: int, stream: int, shape) -> np.ndarray:
+    """E4M3 codes of the integers -4..4 (exact products with E2M1 integers)."""
+    table = np.array([0xC8, 0xC4, 0xC0, 0xB8, 0x00, 0x38, 0x40, 0x44, 0x48], np.uint8)
+    n = int(np.prod(shape))
+    return table[(splitmix64(seed, stream, n) % np.uint64(9)).astype(np.int64)].reshape(shape)
+
+
+def small_int_fp4(seed: int, stream: int, shape_packed) -> np.ndarray:
+    """Packed E2M1 bytes whose nibbles are the integer codes 0,+-1,+-2,+-3,+-4,+-6."""
+    codes = np.array([0x0, 0x2, 0x4, 0x5, 0x6, 0x7, 0xA, 0xC, 0xD, 0xE, 0xF], np.uint8)
+    n = int(np.prod(shape_packed))
+    r = splitmix64(seed, stream, n)
+    lo = codes[(r % np.uint64(11)).astype(np.int64)]
+    hi = codes[((r >> np.uint64(8)) % np.uint64(11)).astype(np.int64)]
+    return (lo | (hi << 4)).astype(np.uint8).reshape(shape_packed)

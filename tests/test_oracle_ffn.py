@@ -1,0 +1,100 @@
+"""Pins of the expert FFN oracle (a4-a7, a10): pure-Python loops on tiny
+shapes, integer-exact special cases, the E=1/k=1 reduction and the SwiGLU
+closed forms."""
+import numpy as np
+
+import synth
+from oracle import ffn
+from oracle import formats as F
+from oracle import quant as Q
+
+
+def test_dequant_mxfp4_loop():
+    w, s = synth.quantize_mxfp4(synth.normal(0, 31, 4 * 64).reshape(4, 64) * 0.02)
+    d = ffn.dequant_mxfp4(w, s)
+    for n in range(4):
+        for kk in range(64):
+            byte = int(w[n, kk // 2])
+            nib = (byte & 0xF) if kk % 2 == 0 else (byte >> 4)
+            assert d[n, kk] == F.E2M1_TABLE[nib] * 2.0 ** (int(s[n, kk // 32]) - 127)
+
+
+def test_grouped_gemm_matches_python_loop():
+    R, K, N, G = 9, 256, 3, 3
+    aq = synth.random_e4m3(1, 1, (R, K), max_code=0x60)
+    as_ = synth.random_bytes(1, 2, (R, K // 128), 120, 134)
+    wq = synth.random_bytes(1, 3, (G, N, K // 2))
+    ws = synth.random_bytes(1, 4, (G, N, K // 32), 118, 130)
+    offsets = np.array([0, 4, 4, 9])
+    out = ffn.grouped_gemm_mxfp4(aq, as_, offsets, wq, ws)
+    for g in range(G):
+        for r in range(offsets[g], offsets[g + 1]):
+            for n in range(N):
+                acc = 0.0
+                for kk in range(K):
+                    a = F.E4M3_TABLE[aq[r, kk]] * 2.0 ** (int(as_[r, kk // 128]) - 127)
+                    byte = int(wq[g, n, kk // 2])
+                    nib = (byte & 0xF) if kk % 2 == 0 else (byte >> 4)
+                    acc += a * F.E2M1_TABLE[nib] * 2.0 ** (int(ws[g, n, kk // 32]) - 127)
+                assert abs(out[r, n] - acc) <= 1e-12 * max(1.0, abs(acc))
+
+
+def test_integer_exact_case():
+    R, K, N = 5, 512, 4
+    aq = synth.small_int_e4m3(2, 1, (R, K))
+    wq = synth.small_int_fp4(2, 2, (1, N, K // 2))
+    out = ffn.grouped_gemm_mxfp4(aq, np.full((R, K // 128), 127, np.uint8), [0, R], wq,
+                                 np.full((1, N, K // 32), 127, np.uint8))
+    a = F.decode_e4m3(aq)
+    w = F.decode_e2m1_packed(wq[0])
+    assert (a == np.round(a)).all() and (w == np.round(w)).all()
+    assert (out == (a.astype(np.int64) @ w.astype(np.int64).T)).all()
+
+
+def test_swiglu_closed_forms():
+    I = 128
+    gu = np.zeros((4, 2 * I))
+    gu[1, :I], gu[1, I:] = 50.0, 50.0                     # both clamp to 10
+    gu[2, :I], gu[2, I:] = -50.0, 3.0                     # gate clamps to -10
+    gu[3, :I], gu[3, I:] = 2.0, -1.0
+    h = ffn.swiglu_clamp(gu, I)
+    assert (h[0] == 0).all()
+    np.testing.assert_allclose(h[1], 10.0 / (1 + np.exp(-10.0)) * 10.0, rtol=1e-15)
+    np.testing.assert_allclose(h[2], -10.0 / (1 + np.exp(10.0)) * 3.0, rtol=1e-15)
+    np.testing.assert_allclose(h[3], -2.0 / (1 + np.exp(-2.0)), rtol=1e-15)
+
+
+def test_single_expert_reduction():
+    """E = 1, k = 1, normalised: the router weight is exactly 1.5, so
+    y = 1.5 * FFN_0(x) + FFN_shared(x) with FFN the plain dense expert."""
+    T, H, I = 6, 256, 128
+    x = synth.to_bf16_bits(synth.normal(3, 1, T * H).reshape(T, H))
+    logits = synth.uniform_logits(3, T, 1)
+    w13, s13, w2, s2 = synth.expert_weights(3, 2, H, I)
+    r = ffn.moe_layer(x, logits, w13, s13, w2, s2, topk=1)
+    assert np.allclose(r["w"], 1.5)
+
+    def dense(e):
+        xq, sx = Q.quantize_act_fp8(x)
+        a = Q.dequantize_fp8_pow2(xq, sx)
+        gu = a @ ffn.dequant_mxfp4(w13[e], s13[e]).T
+        g, u = np.clip(gu[:, :I], -10, 10), np.clip(gu[:, I:], -10, 10)
+        hq, sh = Q.quantize_fp8_pow2((g / (1 + np.exp(-g)) * u).astype(np.float32))
+        return Q.dequantize_fp8_pow2(hq, sh) @ ffn.dequant_mxfp4(w2[e], s2[e]).T
+
+    np.testing.assert_allclose(r["y"], 1.5 * dense(0) + dense(1), rtol=1e-12, atol=1e-15)
+
+
+def test_token_subset_equals_full_rows():
+    wl = synth.tiny_layer(0)
+    full = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    sub = [3, 7, 11]
+    part = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk,
+                         tokens=sub)
+    np.testing.assert_array_equal(part["y"], full["y"][sub])
+
+
+def test_w4afp8_dequant_loop():
+    q = np.array([[0x7F, 0x98] + [0] * 62], np.uint8).view(np.int8)   # nibbles 15,7,8,9
+    d = ffn.dequant_int4g128(q, np.array([[0.5]], np.float32))
+    assert d[0, :4].tolist() == [-0.5, 3.5, -4.0, -3.5]

@@ -1,0 +1,38 @@
+"""The shared input generators: determinism, the published splitmix64 value,
+and the MXFP4 synthesis invariant (re-quantising a dequantised block gives
+back the same bytes)."""
+import numpy as np
+
+import synth
+from oracle import ffn
+
+
+def test_splitmix64_reference_value():
+    # first output of splitmix64 from state 0 (Vigna's reference generator)
+    assert int(synth.splitmix64(0, 0, 1)[0]) == 0xE220A8397B1DCDAF
+
+
+def test_streams_independent_and_deterministic():
+    a = synth.normal(0, 1, 1000)
+    assert (a == synth.normal(0, 1, 1000)).all()
+    assert not (a == synth.normal(0, 2, 1000)).all()
+    assert abs(a.mean()) < 0.1 and abs(a.std() - 1) < 0.1
+
+
+def test_mxfp4_synthesis_roundtrip():
+    w = synth.normal(0, 5, 64 * 256).reshape(64, 256) * 0.02
+    p, s = synth.quantize_mxfp4(w)
+    d = ffn.dequant_mxfp4(p, s)
+    p2, s2 = synth.quantize_mxfp4(d)
+    # the values come back exactly (a block whose maximum rounded down to
+    # 3 * 2^e may be re-expressed with the next lower exponent)
+    assert (ffn.dequant_mxfp4(p2, s2) == d).all()
+    blk = np.abs(d.reshape(64, 8, 32)).max(-1) / 2.0 ** (s.astype(int) - 127)
+    assert ((blk >= 3) & (blk <= 6)).all()
+
+
+def test_zipf_loads_are_skewed():
+    z = synth.zipf_logits(0, 4096, 256)
+    top = np.argsort(-z, axis=1, kind="stable")[:, :6]
+    load = np.bincount(top.reshape(-1), minlength=256)
+    assert load[0] > 3000 and load[-1] < 40 and load.sum() == 4096 * 6
