@@ -1,0 +1,407 @@
+"""Benchmark of the routed-expert MoE layer (MXFP4 experts, FP8 activations).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill|long_prefill]
+
+A step is one pass of the whole expert path (quantise, route, group, w1/w3
+GEMM + SwiGLU + requantise, w2 GEMM, combine) over one batch of synthetic
+tokens.  The default workload is the decode layer of a DeepSeek-V4-Flash-
+class model: hidden 4096, expert intermediate 2048, 256 routed + 1 shared
+experts, top-6, 64 tokens of N(0,1) activations with 0.1% outliers x20,
+uniform router logits, MXFP4 experts from N(0, 0.02).  Each rank runs its own
+replica on its own tokens (data parallel, no collective on the data path);
+`value` is the tokens of all ranks divided by the slowest rank's device time.
+
+One JSON line is printed by rank 0.  `--impl reference` times the CPU oracle
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s or HBM GB/s vs B200 roofline"
+KERNELS_PER_STEP = 13     # quant 1, route 1, permute 4, gemm 3 + 3, combine 1
+
+WORKLOADS = {
+    "decode": dict(T=64, H=4096, I=2048, E=256, k=6, logits="uniform"),
+    "prefill": dict(T=4096, H=4096, I=2048, E=256, k=6, logits="zipf"),
+    "long_prefill": dict(T=16384, H=4096, I=2048, E=384, k=6, logits="zipf"),
+}
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_block_scaled_pow2_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, or None when the kernels changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(workload)
+    if not d or d.get("source_digest") != source_digest():
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+def make_inputs(wl: dict, seed: int, rank: int):
+    import synth
+    T, H, I, E = wl["T"], wl["H"], wl["I"], wl["E"]
+    w13, s13, w2, s2 = synth.expert_weights(seed, E + 1, H, I, n_proto=4)
+    x = synth.decode_activations(seed + 1000 * rank, T, H)
+    logits = (synth.uniform_logits if wl["logits"] == "uniform" else synth.zipf_logits)(seed + 1000 * rank, T, E)
+    return x, logits, (w13, s13, w2, s2)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                p = [c.strip() for c in ln.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx.append(float(p[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local, pg
+
+
+def max_over_ranks(value: float, pg) -> float:
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def algorithmic_bytes(layer, buf, wl) -> dict:
+    """Bytes each GEMM must move at least once: weights of every expert that
+    received rows (nibbles + E8M0 scales), FP8 inputs with their scales, outputs."""
+    counts = buf.counts.cpu().numpy()
+    active = int((counts > 0).sum())
+    R = int(counts.sum())
+    H, I = wl["H"], wl["I"]
+    w13 = 2 * I * H // 2 + 2 * I * H // 32
+    w2 = H * I // 2 + H * I // 32
+    return dict(active_experts=active, rows=R,
+                w13=active * w13 + R * (H + H // 128) + R * (I + I // 128),
+                w2=active * w2 + R * (I + I // 128) + R * H * 4,
+                flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
+
+
+def run_ours(args, wl):
+    import torch
+
+    from fp8_block_scaled_pow2_b200 import moe
+    from fp8_block_scaled_pow2_b200.layer import MoeLayer
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    x, logits, (w13, s13, w2, s2) = make_inputs(wl, args.seed, rank)
+    layer = MoeLayer(w13, s13, w2, s2, wl["k"])
+    T = wl["T"]
+    buf = layer.alloc(T)
+    xd = torch.from_numpy(x.view(np.int16)).cuda()
+    ld = torch.from_numpy(logits).cuda()
+    stream = torch.cuda.current_stream()
+
+    # per-GEMM events: the step is the same sequence of ABI calls as
+    # MoeLayer.forward, with events around the two grouped GEMMs
+    def step(ev=None):
+        b = buf
+        moe.moe_quantize_act_fp8(xd, b.xq, b.sx)
+        moe.moe_route_topk(ld, layer.topk, b.idx, b.w, layer.route_scale, layer.route_norm)
+        moe.moe_permute(b.idx, layer.E, layer.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
+                        b.xq_perm, b.sx_perm, b.ws_permute)
+        if ev: ev[0].record(stream)
+        moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, b.offsets, layer.w13, layer.w13_sf,
+                                   moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, layer.swiglu_limit, b.block_n)
+        if ev: ev[1].record(stream)
+        moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, b.offsets, layer.w2, layer.w2_sf, moe.MOE_EPI_STORE_F32, b.o,
+                                   None, b.ws_gemm, layer.swiglu_limit, b.block_n)
+        if ev: ev[2].record(stream)
+        moe.moe_combine(b.o, b.inv, b.w, layer.has_shared, b.offsets, layer.E, b.y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error() == 0
+    ab = algorithmic_bytes(layer, buf, wl)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(pg)
+    ms = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms, pg)
+    g13 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    g2 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    # end to end through the public API with host buffers: pinned x / logits
+    # in, y out, copies inside the timed region
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    lh = torch.from_numpy(logits).pin_memory()
+    yh = torch.empty((T, wl["H"]), dtype=torch.bfloat16).pin_memory()
+    xd2, ld2 = torch.empty_like(xd), torch.empty_like(ld)
+
+    def e2e_step():
+        xd2.copy_(xh, non_blocking=True)
+        ld2.copy_(lh, non_blocking=True)
+        y = layer.forward(xd2, ld2, buf)
+        yh.copy_(y, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(pg)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg)
+    assert moe.moe_get_device_error() == 0
+
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    peaks = read_peaks()
+    tokens = T * world * args.steps
+    value = tokens / (ms_max / 1e3)
+    clocks = clk.summary()
+    dominant = "w13" if args.workload == "decode" else "w13"
+    if args.workload == "decode":
+        achieved = ab["w13"] / (g13 / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": recorded_traffic(args.workload),
+                "kernel": "moe_grouped_gemm_mxfp4 (w1/w3, SwiGLU epilogue)",
+                "peak_source": f"{peaks['src']} HBM copy"}
+    else:
+        fp8_peak = 2.0 * peaks["bf16_sustained"]
+        achieved = ab["flops13"] / (g13 / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak, 4), "traffic": recorded_traffic(args.workload),
+                "kernel": "moe_grouped_gemm_mxfp4 (w1/w3, SwiGLU epilogue)",
+                "peak_source": f"{peaks['src']} bf16 sustained x 2 (FP8 rate)"}
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe2m1->f32",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload} layer: hidden {wl['H']}, intermediate {wl['I']}, "
+                               f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {T} tokens per GPU",
+                   "tokens_per_gpu": T, "parallelism": f"replicas x{world} (data parallel, no collective)",
+                   "l2": f"inputs larger than L2: {ab['active_experts']} active experts stream "
+                         f"{(ab['w13'] + ab['w2']) / 1e9:.2f} GB of weights per step"},
+        "roofline": roof,
+        "gemm": {"w13_ms": round(g13, 4), "w2_ms": round(g2, 4),
+                 "w13_GBps": round(ab["w13"] / (g13 / 1e3) / 1e9, 1),
+                 "w2_GBps": round(ab["w2"] / (g2 / 1e3) / 1e9, 1),
+                 "w13_TFLOPs": round(ab["flops13"] / (g13 / 1e3) / 1e12, 2),
+                 "w2_TFLOPs": round(ab["flops2"] / (g2 / 1e3) / 1e12, 2),
+                 "active_experts": ab["active_experts"], "rows": ab["rows"]},
+        "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(xh.numel() * 2 + lh.numel() * 4),
+                "d2h_bytes_per_step": int(yh.numel() * 2)},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.seed, budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(wl, seed, budget_s=15.0, tokens_per_step=None):
+    """Time the oracle on a bounded sample of tokens (rank 0 only)."""
+    import synth
+    from oracle import ffn
+    x, logits, (w13, s13, w2, s2) = make_inputs(wl, seed, 0)
+    n, done, t_used = 0, 0, 0.0
+    order = (synth.splitmix64(seed, 99, wl["T"]) % np.uint64(wl["T"])).astype(np.int64)
+    t_start = time.perf_counter()
+    while t_used < budget_s and done < wl["T"]:
+        tok = np.unique(order[done:done + (tokens_per_step or 1)])
+        t = time.perf_counter()
+        ffn.moe_layer(x, logits, w13, s13, w2, s2, wl["k"], tokens=tok)
+        t_used += time.perf_counter() - t
+        n += len(tok)
+        done += tokens_per_step or 1
+    return {"value": round(n / t_used, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} tokens of the {wl['T']}-token batch, one oracle call per token "
+                      f"({t_used:.1f} s of CPU work, numpy float64, BLAS threads for the matmuls)",
+            "wall_s": round(time.perf_counter() - t_start, 1)}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synth
+    from oracle import ffn
+    x, logits, (w13, s13, w2, s2) = make_inputs(wl, args.seed, 0)
+    order = (synth.splitmix64(args.seed, 99, wl["T"]) % np.uint64(wl["T"])).astype(np.int64)
+    times = []
+    for i in range(args.warmup + args.steps):
+        tok = order[i % wl["T"]:i % wl["T"] + 1]
+        t = time.perf_counter()
+        ffn.moe_layer(x, logits, w13, s13, w2, s2, wl["k"], tokens=tok)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    total = sum(times)
+    value = len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / len(times), 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload} layer: hidden {wl['H']}, intermediate {wl['I']}, "
+                               f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {wl['T']} tokens per GPU",
+                   "tokens_per_gpu": wl["T"], "parallelism": "CPU oracle, rank 0 only"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one token of the batch per step, {len(times)} steps"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

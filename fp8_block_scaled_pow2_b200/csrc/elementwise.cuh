@@ -1,0 +1,284 @@
+// Bandwidth-bound kernels of the expert path: activation quantisation (a1),
+// standalone SwiGLU + requantisation (a5), routing (a2), grouping (a3) and
+// the weighted combine (a7).  All are one pass over their data with 8-16
+// byte accesses per thread.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// ------------------------------- a1 ---------------------------------------
+// One warp per (row, 128-column group): each lane owns 4 consecutive columns
+// (8 bytes of bf16 in, 4 bytes of E4M3 out).  "DeepSeek-V4-Flash-SI",
+// 低精度计算: FP8 E4M3 per 128 elements with a power-of-two scale.
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict__ x, int64_t n_groups,
+                                                        int gpr, uint32_t* __restrict__ xq,
+                                                        uint8_t* __restrict__ sx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t grp = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (grp >= n_groups) return;
+  const int64_t v = grp * 32 + lane;               // index in units of 4 elements
+  const uint2 w = __ldg(x + v);
+  const float a = bf16_lo(w.x), b = bf16_hi(w.x), c = bf16_lo(w.y), d = bf16_hi(w.y);
+  const float m = warp_max_nonneg(fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d))));
+  const int k = pow2_scale_exponent(m);
+  const float s = exp2_int(-k);
+  xq[v] = e4m3x4(__fmul_rn(a, s), __fmul_rn(b, s), __fmul_rn(c, s), __fmul_rn(d, s));
+  if (lane == 0) sx[grp] = (uint8_t)(k + 127);
+  (void)gpr;
+}
+
+// ------------------------------- a5 ---------------------------------------
+// One warp per (row, 128 columns of h); gate at column c, up at column I + c.
+__global__ void __launch_bounds__(256) swiglu_quant_kernel(const float4* __restrict__ gu, int rows, int I,
+                                                           float limit, uint32_t* __restrict__ hq,
+                                                           uint8_t* __restrict__ sh) {
+  const int lane = threadIdx.x & 31;
+  const int gpr = I / 128;
+  const int64_t grp = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (grp >= (int64_t)rows * gpr) return;
+  const int64_t row = grp / gpr;
+  const int gi = (int)(grp % gpr);
+  const int64_t q4 = (row * 2 * I + gi * 128) / 4 + lane;     // float4 index of the gate
+  const float4 g = __ldg(gu + q4);
+  const float4 u = __ldg(gu + q4 + I / 4);
+  const float h0 = swiglu_clamped(g.x, u.x, limit), h1 = swiglu_clamped(g.y, u.y, limit);
+  const float h2 = swiglu_clamped(g.z, u.z, limit), h3 = swiglu_clamped(g.w, u.w, limit);
+  const float m = warp_max_nonneg(fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+  const int k = pow2_scale_exponent(m);
+  const float s = exp2_int(-k);
+  hq[(row * I + gi * 128) / 4 + lane] =
+      e4m3x4(__fmul_rn(h0, s), __fmul_rn(h1, s), __fmul_rn(h2, s), __fmul_rn(h3, s));
+  if (lane == 0) sh[row * gpr + gi] = (uint8_t)(k + 127);
+}
+
+// ------------------------------- a2 ---------------------------------------
+// One warp per token.  Lane l holds logits of experts l, l+32, ...; k rounds
+// of a warp arg-max on (value desc, index asc).  "DeepSeek-V4-Flash-SI",
+// 架构特性: sqrtsoftplus scores, top-k, routing scale 1.5.
+__device__ __forceinline__ float softplus_f(float z) { return z > 20.0f ? z : log1pf(expf(z)); }
+
+template <int V>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                         int k, float route_scale, int route_norm,
+                                                         int32_t* __restrict__ idx, float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + (int64_t)t * E;
+  float v[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __ldg(row + e) : 0.0f;
+  }
+  uint32_t taken = 0;
+  int sel_e[16];
+  float sel_v[16];
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j == r) { sel_e[j] = be; sel_v[j] = bv; }
+  }
+  // every lane computes all k scores in slot order (identical on all lanes)
+  float s_sel = 0.0f, sum = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < k) {
+      const float s = sqrtf(softplus_f(sel_v[j]));
+      sum += s;
+      if (j == lane) s_sel = s;
+    }
+  }
+  if (lane < k) {
+    int e_sel = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j == lane) e_sel = sel_e[j];
+    idx[(int64_t)t * k + lane] = e_sel;
+    w[(int64_t)t * k + lane] = route_norm ? route_scale * __fdiv_rn(s_sel, sum) : route_scale * s_sel;
+  }
+}
+
+// ------------------------------- a3 ---------------------------------------
+// Grouping in four deterministic passes:
+//   count:   per chunk of kChunk pairs, a histogram over experts
+//   scan:    per expert the running sum over chunks, then offsets
+//   scatter: per chunk, one warp walks its pairs in order; __match_any_sync
+//            gives each pair its rank among equal experts -> stable rows
+//   gather:  one warp per output row copies the FP8 row and its scales
+constexpr int kChunk = 2048;
+
+__global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __restrict__ idx, int P, int E,
+                                                            int32_t* __restrict__ chunk_hist) {
+  __shared__ int hist[1024];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int p0 = blockIdx.x * kChunk;
+  for (int p = p0 + threadIdx.x; p < min(P, p0 + kChunk); p += blockDim.x) {
+    const int e = __ldg(idx + p);
+    if (e < 0 || e >= E) record_error(MOE_ERR_INVALID);
+    else atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ chunk_hist, int n_chunks,
+                                                            int E, int T, int has_shared,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int warp_sums[32];
+  const int e = threadIdx.x;          // E + 1 <= 1024 groups
+  int c = 0;
+  if (e < E) {
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const int h = chunk_hist[(int64_t)ch * E + e];
+      chunk_hist[(int64_t)ch * E + e] = c;
+      c += h;
+    }
+  } else if (e == E) {
+    c = has_shared ? T : 0;
+  }
+  // exclusive scan of c over threads
+  const int lane = e & 31, wid = e >> 5;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int s = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+      if (lane >= o) s += y;
+    }
+    warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int excl = (wid ? warp_sums[wid - 1] : 0) + x - c;
+  if (e <= E) {
+    counts[e] = c;
+    offsets[e] = excl;
+    if (e == E) offsets[E + 1] = excl + c;
+  }
+}
+
+__global__ void __launch_bounds__(32) permute_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
+                                                             const int32_t* __restrict__ chunk_hist,
+                                                             const int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm,
+                                                             int32_t* __restrict__ inv) {
+  __shared__ int ctr[1024];
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) ctr[e] = offsets[e] + chunk_hist[(int64_t)blockIdx.x * E + e];
+  __syncwarp();
+  const int p0 = blockIdx.x * kChunk;
+  const int p1 = min(P, p0 + kChunk);
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    int e = (p < p1) ? __ldg(idx + p) : -1;
+    if (e >= E) e = -1;                             // invalid ids were flagged by the count pass
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = 0;
+    if (e >= 0) pos = ctr[e] + rank;
+    __syncwarp();
+    if (e >= 0 && (__ffs(peers) - 1) == lane) ctr[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      perm[pos] = p;
+      inv[p] = pos;
+    }
+  }
+}
+
+// One warp per row.  H % 128 == 0, rows 16-byte aligned.
+__global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __restrict__ xq,
+                                                             const uint8_t* __restrict__ sx, int H, int T,
+                                                             int k, const int32_t* __restrict__ offsets,
+                                                             int E, int32_t* __restrict__ perm,
+                                                             uint4* __restrict__ xq_perm,
+                                                             uint8_t* __restrict__ sx_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int R = offsets[E + 1];
+  if (r >= R) return;
+  const int shared0 = offsets[E];
+  const int P = T * k;
+  int t;
+  if (r >= shared0) {
+    t = (int)(r - shared0);
+    if (lane == 0) perm[r] = P + t;
+  } else {
+    t = perm[r] / k;
+  }
+  const int n16 = H / 16;
+  const uint4* src = xq + (int64_t)t * n16;
+  uint4* dst = xq_perm + r * n16;
+  for (int i = lane; i < n16; i += 32) dst[i] = __ldg(src + i);
+  const int ns = H / 128;
+  for (int i = lane; i < ns; i += 32) sx_perm[r * ns + i] = __ldg(sx + (int64_t)t * ns + i);
+}
+
+// ------------------------------- a7 ---------------------------------------
+// One thread per (token, 4 columns): slot-order float32 sum, one bf16 rounding.
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ w, int T, int k, int H,
+                                                      int has_shared, const int32_t* __restrict__ offsets,
+                                                      int E, uint2* __restrict__ y) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int h4 = H / 4;
+  if (i >= (int64_t)T * h4) return;
+  const int t = (int)(i / h4);
+  const int c = (int)(i % h4);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const int r = __ldg(inv + (int64_t)t * k + j);
+    const float wj = __ldg(w + (int64_t)t * k + j);
+    const float4 v = __ldg(o + (int64_t)r * h4 + c);
+    acc.x = fmaf(wj, v.x, acc.x);
+    acc.y = fmaf(wj, v.y, acc.y);
+    acc.z = fmaf(wj, v.z, acc.z);
+    acc.w = fmaf(wj, v.w, acc.w);
+  }
+  if (has_shared) {
+    const int r = __ldg(offsets + E) + t;
+    const float4 v = __ldg(o + (int64_t)r * h4 + c);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  y[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+}  // namespace moe

@@ -1,0 +1,317 @@
+// C-ABI entry points of libmoe: argument validation, tensor-map creation and
+// kernel launches.  All kernels are compiled in this one translation unit so
+// they share the device error word.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm_mxfp4.cuh"
+#include "repack.cuh"
+
+using namespace moe;
+
+namespace {
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_LAUNCH;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D tiled map, inner dimension first.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pick_block_n(int a_rows, int G) {
+  const double avg = (double)a_rows / (G > 0 ? G : 1);
+  if (avg <= 12) return 16;
+  if (avg <= 28) return 32;
+  if (avg <= 56) return 64;
+  return 128;
+}
+
+template <int BN, bool DUAL, int EPI>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a, cudaStream_t st) {
+  using C = gemm::Cfg<BN, DUAL>;
+  auto k = gemm::gemm_mxfp4_kernel<BN, DUAL, EPI>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  k<<<sm_count(), gemm::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  return launch_status();
+}
+
+template <bool DUAL, int EPI>
+int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a,
+                   cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_gemm<16, DUAL, EPI>(ta, tb, a, st);
+    case 32: return launch_gemm<32, DUAL, EPI>(ta, tb, a, st);
+    case 64: return launch_gemm<64, DUAL, EPI>(ta, tb, a, st);
+    case 128: return launch_gemm<128, DUAL, EPI>(ta, tb, a, st);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_NAN_SCALE: return "E8M0 NaN scale (byte 255)";
+    case MOE_ERR_RANGE: return "value not representable in the target format";
+    case MOE_ERR_LAUNCH: return "CUDA launch or copy failed";
+    case MOE_ERR_TIMEOUT: return "bounded device wait expired";
+    default: return "unknown status";
+  }
+}
+
+int moe_version(void) { return 100; }
+
+int moe_get_device_error(int* code, void* stream) {
+  if (!code) return MOE_ERR_INVALID;
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, S(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MOE_ERR_LAUNCH;
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, S(stream)) !=
+      cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MOE_ERR_LAUNCH;
+  *code = v;
+  return MOE_OK;
+}
+
+int moe_quantize_act_fp8(const void* x, int rows, int cols, uint8_t* xq, uint8_t* sx, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 128) return MOE_ERR_INVALID;
+  if (rows == 0) return MOE_OK;
+  if (!x || !xq || !sx || !aligned(x, 8) || !aligned(xq, 4)) return MOE_ERR_INVALID;
+  const int64_t n_groups = (int64_t)rows * (cols / 128);
+  quant_act_kernel<<<(unsigned)((n_groups + 7) / 8), 256, 0, S(stream)>>>(
+      reinterpret_cast<const uint2*>(x), n_groups, cols / 128, reinterpret_cast<uint32_t*>(xq), sx);
+  return launch_status();
+}
+
+int moe_route_topk(const float* logits, int T, int E, int k, float route_scale, int route_norm, int32_t* idx,
+                   float* w, void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 16 || k > E) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!logits || !idx || !w) return MOE_ERR_INVALID;
+  const int V = (E + 31) / 32;
+  const dim3 grid((T + 7) / 8);
+  cudaStream_t st = S(stream);
+  if (V <= 1) route_topk_kernel<1><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 2) route_topk_kernel<2><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 4) route_topk_kernel<4><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 8) route_topk_kernel<8><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 16) route_topk_kernel<16><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  else route_topk_kernel<32><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  return launch_status();
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k) {
+  if (T <= 0 || E <= 0 || k <= 0) return 256;
+  const int64_t P = (int64_t)T * k;
+  const int64_t chunks = (P + kChunk - 1) / kChunk;
+  return (size_t)((chunks * E * 4 + 255) / 256 * 256);
+}
+
+int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared, const uint8_t* xq, const uint8_t* sx,
+                int H, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, uint8_t* xq_perm,
+                uint8_t* sx_perm, void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || E < 1 || E > 1023 || k < 1 || H <= 0 || H % 128) return MOE_ERR_INVALID;
+  if (!counts || !offsets) return MOE_ERR_INVALID;
+  if ((int64_t)T * k > (int64_t)1 << 30) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t st = S(stream);
+  const int P = T * k;
+  const int n_chunks = (P + kChunk - 1) / kChunk;
+  if (T > 0) {
+    if (!idx || !xq || !sx || !perm || !inv || !xq_perm || !sx_perm || !workspace) return MOE_ERR_INVALID;
+    if (!aligned(xq, 16) || !aligned(xq_perm, 16) || !aligned(workspace, 16)) return MOE_ERR_INVALID;
+    if (workspace_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_INVALID;
+  }
+  int32_t* hist = reinterpret_cast<int32_t*>(workspace);
+  if (n_chunks > 0) permute_count_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist);
+  permute_scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
+  if (n_chunks > 0) permute_scatter_kernel<<<n_chunks, 32, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
+  const int64_t R = (int64_t)P + (has_shared ? T : 0);
+  if (R > 0)
+    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
+        sx_perm);
+  return launch_status();
+}
+
+int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, uint8_t* tiled, void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return MOE_ERR_INVALID;
+  if (n_mats == 0) return MOE_OK;
+  if (!e8m0 || !tiled || !aligned(e8m0, 4) || !aligned(tiled, 4)) return MOE_ERR_INVALID;
+  const int64_t n_blocks = n_mats * (N / 128);
+  const int64_t total = n_blocks * (K / 128) * 128;
+  const int64_t grid = std::min<int64_t>((total + 255) / 256, 65535LL * 8);
+  gemm::prepare_weight_scales_kernel<<<(unsigned)grid, 256, 0, S(stream)>>>(e8m0, n_blocks, K, tiled);
+  return launch_status();
+}
+
+size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n) {
+  if (a_rows < 0 || n_groups <= 0 || K <= 0) return 0;
+  if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
+  return gemm::ws_layout(a_rows, n_groups, K, block_n).total;
+}
+
+int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets,
+                           int n_groups, const uint8_t* w_fp4, const uint8_t* w_scale_tiled, int N, int K,
+                           int epilogue, float swiglu_limit, int block_n, void* out, uint8_t* out_scale,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
+    return MOE_ERR_INVALID;
+  if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
+  if (epilogue == MOE_EPI_SWIGLU_QUANT && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
+  if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
+  if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128) return MOE_ERR_UNSUPPORTED;
+  if (a_rows == 0) return MOE_OK;
+  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_fp4 || !w_scale_tiled || !out || !workspace)
+    return MOE_ERR_INVALID;
+  if (!aligned(a_e4m3, 16) || !aligned(w_fp4, 32) || !aligned(w_scale_tiled, 16) || !aligned(workspace, 256))
+    return MOE_ERR_INVALID;
+  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
+  if (workspace_bytes < L.total) return MOE_ERR_INVALID;
+
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_fp4, (uint64_t)K, (uint64_t)n_groups * N,
+                (uint64_t)K / 2, 128, 128))
+    return MOE_ERR_LAUNCH;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
+                (uint32_t)block_n))
+    return MOE_ERR_LAUNCH;
+
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  gemm::GemmArgs args;
+  args.w_sf = w_scale_tiled;
+  args.a_sf = ws + L.a_sf;
+  args.header = reinterpret_cast<const int*>(ws + L.header);
+  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
+  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
+  args.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  args.G = n_groups;
+  args.N = N;
+  args.K = K;
+  args.out = out;
+  args.out_scale = out_scale;
+  args.limit = swiglu_limit;
+
+  cudaStream_t st = S(stream);
+  const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
+  const int n_ft = dual ? N / 256 : N / 128;
+  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
+                                        reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+                                        reinterpret_cast<int2*>(ws + L.tiles));
+  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, K / 128), 128, 0, st>>>(
+      a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
+      reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  switch (epilogue) {
+    case MOE_EPI_STORE_F32: return launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
+    case MOE_EPI_STORE_BF16: return launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
+    default: return launch_gemm_bn<true, MOE_EPI_SWIGLU_QUANT>(block_n, ta, tb, args, st);
+  }
+}
+
+int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq, uint8_t* sh, void* stream) {
+  if (rows < 0 || I <= 0 || I % 128) return MOE_ERR_INVALID;
+  if (rows == 0) return MOE_OK;
+  if (!gu || !hq || !sh || !aligned(gu, 16) || !aligned(hq, 4)) return MOE_ERR_INVALID;
+  const int64_t groups = (int64_t)rows * (I / 128);
+  swiglu_quant_kernel<<<(unsigned)((groups + 7) / 8), 256, 0, S(stream)>>>(
+      reinterpret_cast<const float4*>(gu), rows, I, limit, reinterpret_cast<uint32_t*>(hq), sh);
+  return launch_status();
+}
+
+int moe_combine(const float* o, const int32_t* inv, const float* w, int T, int k, int H, int has_shared,
+                const int32_t* offsets, int E, void* y, void* stream) {
+  if (T < 0 || k < 0 || H <= 0 || H % 4 || E < 0) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!o || !y || (k > 0 && (!inv || !w)) || (has_shared && !offsets)) return MOE_ERR_INVALID;
+  if (!aligned(o, 16) || !aligned(y, 8)) return MOE_ERR_INVALID;
+  const int64_t n = (int64_t)T * (H / 4);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
+      reinterpret_cast<const float4*>(o), inv, w, T, k, H, has_shared ? 1 : 0, offsets, E,
+      reinterpret_cast<uint2*>(y));
+  return launch_status();
+}
+
+int repack_mxfp4_to_nvfp4(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K, uint8_t* out_fp4,
+                          uint8_t* out_e4m3, float* out_global, void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID;
+  if (n_mats == 0) return MOE_OK;
+  if (!fp4 || !e8m0 || !out_fp4 || !out_e4m3 || !out_global) return MOE_ERR_INVALID;
+  if (!aligned(fp4, 16) || !aligned(out_fp4, 16) || !aligned(out_e4m3, 2)) return MOE_ERR_INVALID;
+  const int64_t per_mat = (int64_t)N * (K / 32);
+  const int64_t n_scale = n_mats * per_mat;
+  const int64_t fp4_bytes = n_mats * (int64_t)N * (K / 2);
+  if (fp4_bytes % 16) return MOE_ERR_INVALID;
+  cudaStream_t st = S(stream);
+  nvfp4_global_kernel<<<(unsigned)n_mats, 256, 0, st>>>(e8m0, per_mat, out_global);
+  const bool alias = out_fp4 == fp4;
+  const int64_t work = std::max<int64_t>(n_scale, alias ? 0 : fp4_bytes / 16);
+  const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
+  nvfp4_convert_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
+      e8m0, n_scale, per_mat, out_global, out_e4m3, reinterpret_cast<const uint4*>(fp4),
+      alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
+  return launch_status();
+}
+
+int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                             int8_t* out_int4, float* out_scale_inv, void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || K % 128) return MOE_ERR_INVALID;
+  if (n_mats == 0) return MOE_OK;
+  if (!fp4 || !e8m0 || !out_int4 || !out_scale_inv) return MOE_ERR_INVALID;
+  if (!aligned(fp4, 16) || !aligned(out_int4, 16) || !aligned(e8m0, 4) || !aligned(out_scale_inv, 4))
+    return MOE_ERR_INVALID;
+  const int64_t groups = n_mats * (int64_t)N * (K / 128);
+  int4g128_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, S(stream)>>>(
+      reinterpret_cast<const uint4*>(fp4), reinterpret_cast<const uint32_t*>(e8m0), groups,
+      reinterpret_cast<uint4*>(out_int4), out_scale_inv);
+  return launch_status();
+}
+
+}  // extern "C"

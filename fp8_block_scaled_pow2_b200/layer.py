@@ -1,0 +1,114 @@
+"""A routed-expert MoE FFN layer on top of the C ABI.
+
+MoeLayer owns the device copies of the expert weights (MXFP4, w13 = w1 (gate)
+rows followed by w3 (up) rows, then w2) with their scales prepared once for
+the tensor cores, and runs one forward pass as a fixed sequence of library
+calls on one stream, with no host synchronisation:
+
+    moe_quantize_act_fp8 -> moe_route_topk -> moe_permute
+    -> moe_grouped_gemm_mxfp4(w13, SwiGLU + FP8 requant)
+    -> moe_grouped_gemm_mxfp4(w2, float32) -> moe_combine
+
+The shared expert is group E, fed every token with weight 1 ("DeepSeek-V4-
+Flash-SI" model card, 架构特性: one shared expert per layer, always active).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+from . import moe
+
+
+def _dev(a, device) -> torch.Tensor:
+    if isinstance(a, torch.Tensor):
+        return a.to(device).contiguous()
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+@dataclasses.dataclass
+class Buffers:
+    T: int
+    xq: torch.Tensor
+    sx: torch.Tensor
+    idx: torch.Tensor
+    w: torch.Tensor
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    perm: torch.Tensor
+    inv: torch.Tensor
+    xq_perm: torch.Tensor
+    sx_perm: torch.Tensor
+    hq: torch.Tensor
+    sh: torch.Tensor
+    o: torch.Tensor
+    y: torch.Tensor
+    ws_permute: torch.Tensor
+    ws_gemm: torch.Tensor
+    block_n: int
+
+
+class MoeLayer:
+    def __init__(self, w13, w13_e8m0, w2, w2_e8m0, topk: int, route_scale: float = 1.5,
+                 swiglu_limit: float = 10.0, has_shared: int = 1, route_norm: int = 1, device="cuda"):
+        self.device = torch.device(device)
+        self.G = w13.shape[0]                      # routed experts + shared expert
+        self.E = self.G - (1 if has_shared else 0)
+        self.I = w13.shape[1] // 2
+        self.H = w13.shape[2] * 2
+        assert w2.shape[1] == self.H and w2.shape[2] * 2 == self.I
+        self.topk, self.route_scale, self.swiglu_limit = topk, route_scale, swiglu_limit
+        self.has_shared, self.route_norm = has_shared, route_norm
+        self.w13 = _dev(w13, self.device)
+        self.w2 = _dev(w2, self.device)
+        self.w13_sf = torch.empty((self.G, 2 * self.I // 128, self.H // 128, 512), dtype=torch.uint8,
+                                  device=self.device)
+        self.w2_sf = torch.empty((self.G, self.H // 128, self.I // 128, 512), dtype=torch.uint8,
+                                 device=self.device)
+        moe.moe_prepare_weight_scales(_dev(w13_e8m0, self.device), self.w13_sf)
+        moe.moe_prepare_weight_scales(_dev(w2_e8m0, self.device), self.w2_sf)
+
+    def weight_bytes_per_expert(self) -> int:
+        """MXFP4 bytes of one expert (nibbles + E8M0 scales of w1, w3, w2)."""
+        return 3 * self.I * self.H // 2 + 3 * self.I * self.H // 32
+
+    def alloc(self, T: int, block_n: int = 0) -> Buffers:
+        d, H, I, k = self.device, self.H, self.I, self.topk
+        R = T * k + (T if self.has_shared else 0)
+        u8, i32, f32 = torch.uint8, torch.int32, torch.float32
+        ws_g = max(moe.moe_gemm_workspace_size(R, self.G, H, block_n),
+                   moe.moe_gemm_workspace_size(R, self.G, I, block_n), 256)
+        return Buffers(
+            T=T,
+            xq=torch.empty((T, H), dtype=u8, device=d), sx=torch.empty((T, H // 128), dtype=u8, device=d),
+            idx=torch.empty((T, k), dtype=i32, device=d), w=torch.empty((T, k), dtype=f32, device=d),
+            counts=torch.empty(self.E + 1, dtype=i32, device=d),
+            offsets=torch.empty(self.E + 2, dtype=i32, device=d),
+            perm=torch.empty(max(R, 1), dtype=i32, device=d), inv=torch.empty(max(T * k, 1), dtype=i32, device=d),
+            xq_perm=torch.empty((R, H), dtype=u8, device=d), sx_perm=torch.empty((R, H // 128), dtype=u8, device=d),
+            hq=torch.empty((R, I), dtype=u8, device=d), sh=torch.empty((R, I // 128), dtype=u8, device=d),
+            o=torch.empty((R, H), dtype=f32, device=d), y=torch.empty((T, H), dtype=torch.bfloat16, device=d),
+            ws_permute=torch.empty(moe.moe_permute_workspace_size(T, self.E, k), dtype=u8, device=d),
+            ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n)
+
+    def forward(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers | None = None,
+                stream=None) -> torch.Tensor:
+        """x bfloat16 [T, H] (or its uint16 bits), logits float32 [T, E] -> y bfloat16 [T, H]."""
+        T = x.shape[0]
+        if buf is None or buf.T != T:
+            buf = self.alloc(T)
+        b = buf
+        moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
+        moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
+        moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
+                        b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
+        g_off = b.offsets if self.has_shared else b.offsets[: self.G + 1]
+        moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13, self.w13_sf,
+                                   moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
+                                   b.block_n, stream=stream)
+        moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2, self.w2_sf, moe.MOE_EPI_STORE_F32, b.o, None,
+                                   b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)
+        return b.y

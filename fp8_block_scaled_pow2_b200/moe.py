@@ -1,0 +1,130 @@
+"""Python binding of libmoe (the C ABI declared in include/moe_fp8_pow2.h).
+
+Each function has the name of its C entry point, takes torch tensors that
+already live on the GPU, and only marshals arguments: pointers, sizes and the
+current CUDA stream.  Every step runs in the library's kernels; there is no
+fallback.  A non-zero status raises MoeError.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import load
+
+MOE_EPI_STORE_F32 = 0
+MOE_EPI_STORE_BF16 = 1
+MOE_EPI_SWIGLU_QUANT = 2
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = _lib().moe_status_string(status).decode()
+        super().__init__(f"{fn}: {msg} ({status})")
+        self.status = status
+
+
+def _lib():
+    return load()
+
+
+def _ptr(t: torch.Tensor | None) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise MoeError(fn, status)
+
+
+def moe_get_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    _check("moe_get_device_error", _lib().moe_get_device_error(ctypes.byref(code), _stream(stream)))
+    return code.value
+
+
+def moe_quantize_act_fp8(x, xq, sx, stream=None):
+    rows, cols = x.shape
+    _check("moe_quantize_act_fp8",
+           _lib().moe_quantize_act_fp8(_ptr(x), rows, cols, _ptr(xq), _ptr(sx), _stream(stream)))
+
+
+def moe_route_topk(logits, k, idx, w, route_scale=1.5, route_norm=1, stream=None):
+    T, E = logits.shape
+    _check("moe_route_topk", _lib().moe_route_topk(_ptr(logits), T, E, k, ctypes.c_float(route_scale),
+                                                   int(route_norm), _ptr(idx), _ptr(w), _stream(stream)))
+
+
+def moe_permute_workspace_size(T: int, E: int, k: int) -> int:
+    return int(_lib().moe_permute_workspace_size(T, E, k))
+
+
+def moe_permute(idx, E, has_shared, xq, sx, counts, offsets, perm, inv, xq_perm, sx_perm, workspace,
+                stream=None):
+    T, k = idx.shape
+    H = xq.shape[1]
+    _check("moe_permute", _lib().moe_permute(
+        _ptr(idx), T, E, k, int(has_shared), _ptr(xq), _ptr(sx), H, _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(inv), _ptr(xq_perm), _ptr(sx_perm), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_prepare_weight_scales(e8m0, tiled, stream=None):
+    """e8m0 uint8 [n_mats, N, K/32] -> tiled uint8 [n_mats, N/128, K/128, 512]."""
+    n_mats, N, k32 = e8m0.shape
+    _check("moe_prepare_weight_scales", _lib().moe_prepare_weight_scales(
+        _ptr(e8m0), n_mats, N, k32 * 32, _ptr(tiled), _stream(stream)))
+
+
+def moe_gemm_workspace_size(a_rows: int, n_groups: int, K: int, block_n: int = 0) -> int:
+    return int(_lib().moe_gemm_workspace_size(a_rows, n_groups, K, block_n))
+
+
+def moe_grouped_gemm_mxfp4(a, a_scale, offsets, w_fp4, w_scale_tiled, epilogue, out, out_scale=None,
+                           workspace=None, swiglu_limit=10.0, block_n=0, stream=None):
+    a_rows, K = a.shape
+    G, N = w_fp4.shape[0], w_fp4.shape[1]
+    _check("moe_grouped_gemm_mxfp4", _lib().moe_grouped_gemm_mxfp4(
+        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_fp4), _ptr(w_scale_tiled), N, K,
+        int(epilogue), ctypes.c_float(swiglu_limit), int(block_n), _ptr(out), _ptr(out_scale),
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def moe_swiglu_clamp(gu, hq, sh, limit=10.0, stream=None):
+    rows, two_i = gu.shape
+    _check("moe_swiglu_clamp", _lib().moe_swiglu_clamp(_ptr(gu), rows, two_i // 2, ctypes.c_float(limit),
+                                                       _ptr(hq), _ptr(sh), _stream(stream)))
+
+
+def moe_combine(o, inv, w, has_shared, offsets, E, y, stream=None):
+    T, k = w.shape
+    H = o.shape[1]
+    _check("moe_combine", _lib().moe_combine(_ptr(o), _ptr(inv), _ptr(w), T, k, H, int(has_shared),
+                                             _ptr(offsets), E, _ptr(y), _stream(stream)))
+
+
+def repack_mxfp4_to_nvfp4(fp4, e8m0, out_fp4, out_e4m3, out_global, stream=None):
+    n_mats, N, k2 = fp4.shape
+    _check("repack_mxfp4_to_nvfp4", _lib().repack_mxfp4_to_nvfp4(
+        _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_fp4), _ptr(out_e4m3), _ptr(out_global),
+        _stream(stream)))
+
+
+def repack_mxfp4_to_int4g128(fp4, e8m0, out_int4, out_scale_inv, stream=None):
+    n_mats, N, k2 = fp4.shape
+    _check("repack_mxfp4_to_int4g128", _lib().repack_mxfp4_to_int4g128(
+        _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_int4), _ptr(out_scale_inv), _stream(stream)))

@@ -1,0 +1,225 @@
+/*
+ * moe_fp8_pow2.h -- C ABI of the B200 (sm_100a) routed-expert MoE FFN with
+ * MXFP4 expert weights and FP8 E4M3 activations scaled by powers of two.
+ *
+ * Conventions (all entry points)
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     the argument description says "host".  The library never frees caller
+ *     memory and allocates nothing on these calls; scratch memory, where a
+ *     call needs it, is passed in as `workspace` and sized by the matching
+ *     *_workspace_size() query.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream) and returns an int status:
+ *        MOE_OK (0)            launched
+ *        MOE_ERR_INVALID (-1)  null pointer, bad shape, misaligned pointer
+ *        MOE_ERR_UNSUPPORTED   configuration outside the compiled kernels
+ *        MOE_ERR_NAN_SCALE     (device word only) an E8M0 byte 255 was met
+ *        MOE_ERR_RANGE         (device word only) a value is not representable
+ *        MOE_ERR_LAUNCH (-5)   the CUDA launch failed (cudaGetLastError)
+ *        MOE_ERR_TIMEOUT (-6)  (device word only) a bounded device wait expired
+ *     Problems that depend on tensor CONTENTS (NaN scales, range) cannot be
+ *     seen at launch; kernels record them in a device error word that
+ *     moe_get_device_error() returns (first error wins).  Outputs of a call
+ *     that recorded a device error are unspecified.
+ *   - Row-major layouts throughout; weights are [N, K] with K (the input
+ *     dimension) contiguous, the orientation of torch.nn.functional.linear.
+ *   - Packed FP4 / INT4: element 2i is the LOW nibble of byte i, 2i+1 the high.
+ *   - No exceptions cross this boundary; calls on different streams may run
+ *     concurrently when their buffers are disjoint.
+ *
+ * Sources (web pages describing the method; cited by title and section)
+ *   [SI]    "DeepSeek-V4-Flash-SI" model card: 架构特性 (Mixture of Experts
+ *           paragraph: 256 routed + 1 shared expert, top-6, sqrtsoftplus
+ *           scoring, routing scale 1.5, SwiGLU clamp +-10) and 低精度计算
+ *           (FP4 E2M1 experts with an F8_E8M0 scale per 32 elements; online
+ *           FP8 E4M3 activations, one power-of-2 scale per 128 elements);
+ *           模型训练 table (dynamic FP8 E4M3 activations, ue8m0 scale).
+ *   [NVFP4] "DeepSeek-V4-Pro-0813-nvfp4-DSpark" walkthrough: 阶段三 and its
+ *           MXFP4 vs NVFP4 storage table (same E2M1 nibbles, E4M3 scale per
+ *           16, weight bits not recomputed, scale bytes doubled).
+ *   [W4A]   "DeepSeek-V4-Flash-0731-W4AFP8-mt" model card: 量化方式 and
+ *           权重约定 (FP4 -> signed INT4, group 128, two INT4 per int8,
+ *           float32 weight_scale_inv [N, K/128], dynamic E4M3 activations).
+ */
+#ifndef MOE_FP8_POW2_H
+#define MOE_FP8_POW2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID (-1)
+#define MOE_ERR_UNSUPPORTED (-2)
+#define MOE_ERR_NAN_SCALE (-3)
+#define MOE_ERR_RANGE (-4)
+#define MOE_ERR_LAUNCH (-5)
+#define MOE_ERR_TIMEOUT (-6)
+
+/* Grouped-GEMM epilogues. */
+#define MOE_EPI_STORE_F32 0    /* out: float32 [rows, N]                                   */
+#define MOE_EPI_STORE_BF16 1   /* out: bfloat16 [rows, N]                                  */
+#define MOE_EPI_SWIGLU_QUANT 2 /* out: E4M3 h [rows, N/2]; out_scale: E8M0 [rows, N/256] */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int moe_version(void);
+
+/*
+ * Device error word: waits for `stream`, copies the word to *code (host) and
+ * clears it.  Returns MOE_OK, or MOE_ERR_LAUNCH if the copy itself failed.
+ */
+int moe_get_device_error(int* code, void* stream);
+
+/*
+ * a1 -- activation quantisation [SI 低精度计算, 模型训练].
+ * For each row and each group of 128 columns: amax = max |x|;
+ * k = ceil(log2(amax / 448)) with amax / 448 a float32 round-to-nearest-even
+ * divide and the ceiling taken exactly; k clamped to [-127, 127]; k = 0 for
+ * an all-zero group.  xq = E4M3(x * 2^-k) rounded to nearest even and
+ * saturated to +-448; sx = k + 127 (E8M0).
+ *   x   bfloat16 [rows, cols], 8-byte aligned; cols % 128 == 0
+ *   xq  uint8 E4M3 [rows, cols], 4-byte aligned
+ *   sx  uint8 E8M0 [rows, cols / 128]
+ * rows == 0 is a no-op.  NaN/Inf inputs are a precondition violation.
+ */
+int moe_quantize_act_fp8(const void* x, int rows, int cols, uint8_t* xq, uint8_t* sx,
+                         void* stream);
+
+/*
+ * a2 -- router [SI 架构特性]: idx[t, :] = the k largest logits of row t in
+ * descending order, ties to the lower expert index; s_j = sqrt(softplus(z_j));
+ * w[t, j] = route_scale * s_j / sum_j s_j   (route_norm != 0)
+ *         = route_scale * s_j               (route_norm == 0).
+ *   logits float32 [T, E]; 1 <= k <= min(E, 16); E <= 1024
+ *   idx    int32 [T, k];  w float32 [T, k]
+ * Indices are exact; weights use the device expf/log1pf/sqrtf (within a few
+ * float32 ulps of the exact value).
+ */
+int moe_route_topk(const float* logits, int T, int E, int k, float route_scale,
+                   int route_norm, int32_t* idx, float* w, void* stream);
+
+/*
+ * a3 -- grouping by expert.  Groups g = 0..E-1 are the routed experts,
+ * group E the shared expert (one row per token when has_shared != 0, none
+ * otherwise).  Within a routed group rows are in ascending pair id p = t*k+j;
+ * shared rows follow in token order.
+ *   idx      int32 [T, k] expert ids in [0, E)   (out-of-range ids: device
+ *            error MOE_ERR_INVALID, outputs unspecified)
+ *   xq, sx   outputs of moe_quantize_act_fp8 for H columns (H % 128 == 0)
+ *   counts   int32 [E+1];  offsets int32 [E+2] (exclusive prefix of counts)
+ *   perm     int32 [R], R = T*k + (has_shared ? T : 0): source id of row r,
+ *            the pair id p for routed rows, T*k + t for the shared row of t
+ *   inv      int32 [T*k]: row of pair p
+ *   xq_perm  uint8 [R, H] (16-byte aligned), sx_perm uint8 [R, H/128]:
+ *            the rows of xq / sx of each row's source token
+ *   workspace  device scratch of moe_permute_workspace_size(T, E, k) bytes,
+ *            256-byte aligned; its contents on entry do not matter
+ */
+size_t moe_permute_workspace_size(int T, int E, int k);
+int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared,
+                const uint8_t* xq, const uint8_t* sx, int H,
+                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                uint8_t* xq_perm, uint8_t* sx_perm,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Weight-scale preparation (once per weight tensor, at load time).  The
+ * block-scaled tensor-core MMA reads its scale factors from tensor memory in
+ * a fixed interleave; this call rewrites MXFP4 E8M0 scales [n_mats, N, K/32]
+ * into that order, [n_mats, N/128, K/128, 512] bytes, where byte
+ * (m % 32) * 16 + (m / 32) * 4 + b of a 512-byte block holds the scale of row
+ * m (0..127 within the block) for 32-element block b (0..3 within 128).
+ * N % 128 == 0, K % 128 == 0.  The values are unchanged.
+ */
+int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                              uint8_t* tiled, void* stream);
+
+/*
+ * a4 / a5 / a6 -- grouped expert GEMM with MXFP4 weights [SI 低精度计算],
+ * tcgen05 block-scaled MMA (kind::mxf8f6f4, E2M1 x E4M3, E8M0 scales) with
+ * float32 accumulation.  For every group g and row r in
+ * [offsets[g], offsets[g+1]):  acc[r, n] = sum_k a[r, k] * 2^(sa[r, k/128]-127)
+ *                                          * w[g, n, k] * 2^(sw[g, n, k/32]-127)
+ *   a_e4m3       uint8 [a_rows, K] (16-byte aligned), a_rows >= offsets[G]
+ *   a_e8m0_128   uint8 [a_rows, K/128]
+ *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0
+ *   w_fp4        uint8 [G, N, K/2] packed E2M1 (32-byte aligned)
+ *   w_scale_tiled  output of moe_prepare_weight_scales for [G, N, K/32]
+ *   N % 128 == 0 (N % 256 == 0 for SWIGLU_QUANT), K % 128 == 0
+ *   epilogue  MOE_EPI_STORE_F32 / MOE_EPI_STORE_BF16: out = acc [a_rows, N]
+ *             (rows past offsets[G] untouched);
+ *             MOE_EPI_SWIGLU_QUANT [SI 架构特性]: columns [0, N/2) are the
+ *             gate (w1) and [N/2, N) the up (w3) projection; with I = N/2,
+ *             h = silu(clamp(g, +-limit)) * clamp(u, +-limit) in float32,
+ *             then the a1 rule per 128 columns of h: out = E4M3 [a_rows, I],
+ *             out_scale = E8M0 [a_rows, I/128]
+ *   block_n   token rows per tile: 16, 32, 64 or 128 (0 = choose from
+ *             a_rows and G)
+ *   workspace scratch of moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
+ */
+size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n);
+int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
+                           const int32_t* offsets, int n_groups,
+                           const uint8_t* w_fp4, const uint8_t* w_scale_tiled, int N, int K,
+                           int epilogue, float swiglu_limit, int block_n,
+                           void* out, uint8_t* out_scale,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * a5 standalone -- SwiGLU with clamp and per-128 power-of-two requantisation
+ * [SI 架构特性 / 低精度计算], same arithmetic as MOE_EPI_SWIGLU_QUANT.
+ *   gu  float32 [rows, 2I] (gate | up), 16-byte aligned; I % 128 == 0
+ *   hq  uint8 E4M3 [rows, I];  sh uint8 E8M0 [rows, I/128]
+ */
+int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq, uint8_t* sh,
+                     void* stream);
+
+/*
+ * a7 -- combine [SI 架构特性]:
+ *   y[t] = sum_{j<k} w[t, j] * o[inv[t*k+j]] + (has_shared ? o[offsets[E] + t] : 0)
+ * accumulated in float32 in slot order, rounded once to bfloat16 (nearest even).
+ *   o  float32 [R, H] (16-byte aligned), H % 4 == 0;  inv int32 [T*k];
+ *   w  float32 [T, k];  offsets int32 [E+2] (device);  y bfloat16 [T, H]
+ */
+int moe_combine(const float* o, const int32_t* inv, const float* w, int T, int k, int H,
+                int has_shared, const int32_t* offsets, int E, void* y, void* stream);
+
+/*
+ * a8 -- MXFP4 -> NVFP4 [NVFP4 阶段三].  For each of n_mats matrices [N, K]:
+ * nibbles are copied unchanged (out_fp4 may equal fp4: then nothing is
+ * written there); every E8M0 scale 2^e (per 32) becomes two E4M3 scales
+ * 2^(e - G) (per 16), with G = 0 when all exponents of the matrix lie in
+ * [-9, 8], else G = max_e - 8 when max_e - min_e <= 17; out_global[m] = 2^G.
+ * Device errors: MOE_ERR_NAN_SCALE (byte 255), MOE_ERR_RANGE (span > 17).
+ *   fp4, out_fp4  uint8 [n_mats, N, K/2] (16-byte aligned);
+ *   e8m0 [n_mats, N, K/32];  out_e4m3 [n_mats, N, K/16];  out_global float32 [n_mats]
+ *   K % 32 == 0
+ */
+int repack_mxfp4_to_nvfp4(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                          uint8_t* out_fp4, uint8_t* out_e4m3, float* out_global, void* stream);
+
+/*
+ * a9 -- MXFP4 -> symmetric INT4, group 128 [W4A 量化方式 / 权重约定].  Per row
+ * and group of 128: x = exact float32 dequantisation; amax; scale_inv =
+ * amax / 7 (float32 IEEE divide; 1.0 when amax == 0);
+ * q = clamp(rint(x / scale_inv), -7, 7) (IEEE divide, ties to even);
+ * two's complement nibbles, element 2i low.
+ * Device errors: MOE_ERR_NAN_SCALE, MOE_ERR_RANGE (x overflows float32).
+ *   fp4 uint8 [n_mats, N, K/2] (16-byte aligned); e8m0 [n_mats, N, K/32];
+ *   out_int4 int8 [n_mats, N, K/2]; out_scale_inv float32 [n_mats, N, K/128];
+ *   K % 128 == 0
+ */
+int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N,
+                             int K, int8_t* out_int4, float* out_scale_inv, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FP8_POW2_H */

@@ -29,18 +29,63 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
-    z = (z ^ (z >> np.uint64(30))) * _M1
-    z = (z ^ (z >> np.uint64(27))) * _M2
-    return z ^ (z >> np.uint64(31))
+    """splitmix64 finaliser, in place on a uint64 array (returns it)."""
+    t = np.empty_like(z)
+    np.right_shift(z, np.uint64(30), out=t)
+    np.bitwise_xor(z, t, out=z)
+    np.multiply(z, _M1, out=z)
+    np.right_shift(z, np.uint64(27), out=t)
+    np.bitwise_xor(z, t, out=z)
+    np.multiply(z, _M2, out=z)
+    np.right_shift(z, np.uint64(31), out=t)
+    np.bitwise_xor(z, t, out=z)
+    return z
+
+
+def _key(seed: int, stream: int) -> np.uint64:
+    if not (seed or stream):
+        return np.uint64(0)
+    with np.errstate(over="ignore"):
+        return _mix(np.array([(seed * 0x632BE59BD9B4E019 + stream) & 0xFFFFFFFFFFFFFFFF],
+                             dtype=np.uint64))[0]
+
+
+_STEP = 1 << 20
+
+
+def _parallel(n: int, fn) -> None:
+    """Run fn(i0, i1) over chunks of [0, n); numpy ufuncs release the GIL, so
+    chunks run on several host cores.  Results do not depend on the split."""
+    chunks = [(i0, min(n, i0 + _STEP)) for i0 in range(0, n, _STEP)]
+    if len(chunks) <= 2:
+        for c in chunks:
+            fn(*c)
+        return
+    import concurrent.futures as cf
+    import os
+    with cf.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(lambda c: fn(*c), chunks))
+
+
+def _stream_values(key: np.uint64, c0: int, c1: int) -> np.ndarray:
+    """Outputs c0 .. c1-1 (0-based) of the stream with the given key."""
+    with np.errstate(over="ignore"):
+        z = np.arange(c0 + 1, c1 + 1, dtype=np.uint64)
+        np.multiply(z, _GAMMA, out=z)
+        np.add(z, key, out=z)
+        return _mix(z)
 
 
 def splitmix64(seed: int, stream: int, n: int) -> np.ndarray:
     """n uint64 outputs of the counter-mode splitmix64 stream (seed, stream)."""
-    with np.errstate(over="ignore"):
-        key = _mix(np.array([(seed * 0x632BE59BD9B4E019 + stream) & 0xFFFFFFFFFFFFFFFF],
-                            dtype=np.uint64))[0] if (seed or stream) else np.uint64(0)
-        ctr = np.arange(1, n + 1, dtype=np.uint64) * _GAMMA
-        return _mix(ctr + key)
+    key = _key(seed, stream)
+    out = np.empty(n, np.uint64)
+
+    def work(i0, i1):
+        out[i0:i1] = _stream_values(key, i0, i1)
+
+    _parallel(n, work)
+    return out
 
 
 def uniform(seed: int, stream: int, n: int) -> np.ndarray:
@@ -49,10 +94,17 @@ def uniform(seed: int, stream: int, n: int) -> np.ndarray:
 
 
 def normal(seed: int, stream: int, n: int) -> np.ndarray:
-    """n standard normals (Box-Muller, cosine branch)."""
-    u = uniform(seed, stream, 2 * n)
-    r = np.sqrt(-2.0 * np.log1p(-u[0::2]))   # 1-u in (0, 1]
-    return r * np.cos(2.0 * np.pi * u[1::2])
+    """n standard normals (Box-Muller, cosine branch): normal i uses stream
+    outputs 2i (radius) and 2i+1 (angle)."""
+    key = _key(seed, stream)
+    out = np.empty(n, np.float64)
+
+    def work(i0, i1):
+        u = (_stream_values(key, 2 * i0, 2 * i1) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+        out[i0:i1] = np.sqrt(-2.0 * np.log1p(-u[0::2])) * np.cos(2.0 * np.pi * u[1::2])
+
+    _parallel(n, work)
+    return out
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -76,18 +128,39 @@ _E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
 def _round_to_e2m1_code(m: np.ndarray) -> np.ndarray:
-    """Magnitudes (already divided by the block scale) -> 3-bit codes 0..7."""
-    m = np.minimum(m, 6.0)
-    # distance to every grid point; ties are resolved toward the even code
-    d = np.abs(m[..., None] - _E2M1_GRID)
-    best = d.min(axis=-1, keepdims=True)
-    cand = d == best
-    even = cand & (np.arange(8) % 2 == 0)
-    pick = np.where(even.any(axis=-1, keepdims=True), even, cand)
-    return np.argmax(pick, axis=-1).astype(np.uint8)
+    """Magnitudes (already divided by the block scale) -> 3-bit codes 0..7,
+    nearest grid point, ties to the even code, saturating at 6."""
+    mid = (_E2M1_GRID[1:] + _E2M1_GRID[:-1]) / 2          # 0.25, 0.75, ..., 5
+    c = np.searchsorted(mid, m, side="left")              # number of midpoints below m
+    tie = (c < 7) & (m == mid[np.minimum(c, 6)]) & (c % 2 == 1)
+    return (c + tie).astype(np.uint8)
 
 
 def quantize_mxfp4(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Row-parallel wrapper of _quantize_mxfp4 (same result for any split)."""
+    w = np.asarray(w, dtype=np.float64)
+    if w.ndim != 2 or w.shape[0] < 64:
+        return _quantize_mxfp4(w)
+    rows = w.shape[0]
+    packed = np.empty((rows, w.shape[1] // 2), np.uint8)
+    scales = np.empty((rows, w.shape[1] // 32), np.uint8)
+    step = max(1, (1 << 18) // w.shape[1])
+
+    def work(r0, r1):
+        for a in range(r0, r1, step):
+            b = min(r1, a + step)
+            packed[a:b], scales[a:b] = _quantize_mxfp4(w[a:b])
+
+    import concurrent.futures as cf
+    import os
+    n = min(16, os.cpu_count() or 1)
+    bounds = [(rows * i // n, rows * (i + 1) // n) for i in range(n)]
+    with cf.ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(lambda c: work(*c), bounds))
+    return packed, scales
+
+
+def _quantize_mxfp4(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """float [..., K] -> (packed nibbles uint8 [..., K/2], E8M0 uint8 [..., K/32]).
 
     Element 2i sits in the low nibble, 2i+1 in the high nibble.
@@ -100,6 +173,7 @@ def quantize_mxfp4(w: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     with np.errstate(divide="ignore"):
         ratio = amax / 6.0
         e = np.where(amax > 0, np.ceil(np.log2(np.where(amax > 0, ratio, 1.0))), 0.0)
+    # (the code below keeps every step vectorised; memory stays O(size))
     # guard against log2 rounding: make sure amax / 2^e <= 6 and > 3
     e = np.where((amax > 0) & (amax / np.exp2(e) > 6.0), e + 1, e)
     e = np.where((amax > 0) & (amax / np.exp2(e) <= 3.0), e - 1, e)
@@ -133,22 +207,26 @@ class MoeWorkload:
     swiglu_limit: float = 10.0
 
 
-def expert_weights(seed: int, E1: int, H: int, I: int, std: float = 0.02,
-                   experts: np.ndarray | None = None):
-    """MXFP4 w13 [E1, 2I, H] and w2 [E1, H, I] from N(0, std).
+def expert_weights(seed: int, E1: int, H: int, I: int, std: float = 0.02, n_proto: int | None = None):
+    """MXFP4 w13 [E1, 2I, H] (w1 rows then w3 rows) and w2 [E1, H, I] from N(0, std).
 
-    Each expert draws from its own streams, so a subset (``experts``) can be
-    generated without the others; rows of untouched experts are left zero.
-    """
-    w13 = np.zeros((E1, 2 * I, H // 2), np.uint8)
-    s13 = np.full((E1, 2 * I, H // 32), 127, np.uint8)
-    w2 = np.zeros((E1, H, I // 2), np.uint8)
-    s2 = np.full((E1, H, I // 32), 127, np.uint8)
-    for e in (range(E1) if experts is None else experts):
+    Expert e draws from its own streams.  With ``n_proto`` set, only the first
+    n_proto experts are drawn and expert e repeats expert e % n_proto (distinct
+    memory, same values): full-size layers then take seconds to synthesise
+    while every expert still streams its own bytes."""
+    n_draw = E1 if n_proto is None else min(E1, n_proto)
+    w13 = np.empty((E1, 2 * I, H // 2), np.uint8)
+    s13 = np.empty((E1, 2 * I, H // 32), np.uint8)
+    w2 = np.empty((E1, H, I // 2), np.uint8)
+    s2 = np.empty((E1, H, I // 32), np.uint8)
+    for e in range(n_draw):
         a = normal(seed, 1000 + 2 * e, 2 * I * H).reshape(2 * I, H) * std
         w13[e], s13[e] = quantize_mxfp4(a)
         b = normal(seed, 1001 + 2 * e, H * I).reshape(H, I) * std
         w2[e], s2[e] = quantize_mxfp4(b)
+    for e in range(n_draw, E1):
+        p = e % n_draw
+        w13[e], s13[e], w2[e], s2[e] = w13[p], s13[p], w2[p], s2[p]
     return w13, s13, w2, s2
 
 

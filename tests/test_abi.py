@@ -1,0 +1,57 @@
+"""The C ABI library loads on a machine without a GPU and exports every entry
+point include/moe_fp8_pow2.h declares (no compute calls here)."""
+import ctypes
+import os
+import re
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moe_fp8_pow2.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ["moe_quantize_act_fp8", "moe_route_topk", "moe_permute", "moe_grouped_gemm_mxfp4",
+              "moe_swiglu_clamp", "moe_combine", "repack_mxfp4_to_nvfp4", "repack_mxfp4_to_int4g128"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from fp8_block_scaled_pow2_b200 import build
+    build.build()
+    lib = ctypes.CDLL(build.LIB)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_signatures_cover_header():
+    from fp8_block_scaled_pow2_b200 import _lib
+    assert set(declared_functions()) <= set(_lib.SIGNATURES)
+
+
+def test_status_strings_without_gpu():
+    from fp8_block_scaled_pow2_b200 import _lib
+    lib = _lib.load()
+    assert lib.moe_status_string(0) == b"ok"
+    assert lib.moe_status_string(-6).startswith(b"bounded")
+    assert lib.moe_version() >= 100
+
+
+def test_argument_validation_without_gpu():
+    """Invalid shapes are rejected on the host before any CUDA call."""
+    from fp8_block_scaled_pow2_b200 import _lib
+    lib = _lib.load()
+    assert lib.moe_quantize_act_fp8(None, 4, 100, None, None, None) == -1      # cols % 128
+    assert lib.moe_quantize_act_fp8(None, 0, 128, None, None, None) == 0       # empty: no-op
+    assert lib.moe_route_topk(None, 4, 8, 9, ctypes.c_float(1.5), 1, None, None, None) == -1
+    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, None, 256, 100, 0,
+                                      ctypes.c_float(10), 0, None, None, None, 0, None) == -1
+    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, None, 256, 128, 0,
+                                      ctypes.c_float(10), 48, None, None, None, 0, None) == -2
+    assert lib.repack_mxfp4_to_int4g128(None, None, 1, 8, 96, None, None, None) == -1

@@ -1,0 +1,303 @@
+"""GPU parity of each step against the oracle, through the C ABI.
+
+Bit-exact: quantisation codes and scales, routing indices, grouping outputs,
+repacks, and the integer-exact GEMM case.  Tolerances: routing weights
+(1e-6 relative, libm differences), GEMM float32 accumulation, combine bf16.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import ffn
+from oracle import formats as F
+from oracle import permute as Pm
+from oracle import quant as Q
+from oracle import repack as Rp
+from oracle import route as R
+
+pytestmark = pytest.mark.gpu
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def no_device_error(lib):
+    assert lib.moe_get_device_error() == 0
+
+
+# ------------------------------- a1 ---------------------------------------
+@pytest.mark.parametrize("T,H", [(1, 128), (37, 512), (300, 4096)])
+def test_quantize_act_bit_exact(lib, T, H):
+    x = synth.decode_activations(7 + T, T, H)
+    xq = torch.empty((T, H), dtype=torch.uint8, device="cuda")
+    sx = torch.empty((T, H // 128), dtype=torch.uint8, device="cuda")
+    lib.moe_quantize_act_fp8(dev(x.view(np.int16)), xq, sx)
+    q_ref, s_ref = Q.quantize_act_fp8(x)
+    np.testing.assert_array_equal(host(sx), s_ref)
+    np.testing.assert_array_equal(host(xq), q_ref)
+    no_device_error(lib)
+
+
+def test_quantize_act_exhaustive_bf16(lib):
+    """Every finite bf16 value alone in a group, and in a group with 448 * 2^j."""
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    b = b[np.isfinite(F.decode_bf16_bits(b))]
+    x = np.zeros((len(b), 256), np.uint16)
+    x[:, 3] = b
+    x[:, 128 + 77] = b
+    x[:, 128 + 5] = synth.to_bf16_bits(np.full(len(b), 448.0) * np.exp2((np.arange(len(b)) % 61) - 30))
+    xq = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    sx = torch.empty((len(b), 2), dtype=torch.uint8, device="cuda")
+    lib.moe_quantize_act_fp8(dev(x.view(np.int16)), xq, sx)
+    q_ref, s_ref = Q.quantize_act_fp8(x)
+    np.testing.assert_array_equal(host(sx), s_ref)
+    np.testing.assert_array_equal(host(xq), q_ref)
+
+
+# ------------------------------- a2 ---------------------------------------
+@pytest.mark.parametrize("T,E,k", [(16, 8, 2), (64, 256, 6), (1000, 257, 6), (33, 385, 6), (5, 1024, 16),
+                                   (7, 3, 3)])
+def test_route_topk(lib, T, E, k):
+    z = (synth.uniform(T + E, 4, T * E) * 8 - 4).astype(np.float32).reshape(T, E)
+    z[:, ::3] = np.round(z[:, ::3] * 2) / 2                # ties
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    for norm in (1, 0):
+        lib.moe_route_topk(dev(z), k, idx, w, 1.5, norm)
+        i_ref, w_ref = R.route_topk(z, k, 1.5, norm)
+        np.testing.assert_array_equal(host(idx), i_ref)
+        np.testing.assert_allclose(host(w), w_ref, rtol=1e-6, atol=0)
+
+
+# ------------------------------- a3 ---------------------------------------
+@pytest.mark.parametrize("T,E,k,has_shared", [(0, 8, 2, 1), (1, 8, 2, 1), (16, 8, 2, 0), (700, 257, 6, 1),
+                                              (2049, 3, 1, 1), (4096, 256, 6, 1)])
+def test_permute_bit_exact(lib, T, E, k, has_shared):
+    H = 256
+    if T:
+        z = synth.zipf_logits(T, T, E)
+        idx_np, _ = R.route_topk(z, k)
+    else:
+        idx_np = np.zeros((0, k), np.int32)
+    xq_np = synth.random_bytes(1, 1, (T, H))
+    sx_np = synth.random_bytes(1, 2, (T, H // 128))
+    Rn = T * k + (T if has_shared else 0)
+    counts = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 2, dtype=torch.int32, device="cuda")
+    perm = torch.empty(max(Rn, 1), dtype=torch.int32, device="cuda")
+    inv = torch.empty(max(T * k, 1), dtype=torch.int32, device="cuda")
+    xqp = torch.empty((Rn, H), dtype=torch.uint8, device="cuda")
+    sxp = torch.empty((Rn, H // 128), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(lib.moe_permute_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
+    idx_t = dev(idx_np.astype(np.int32)) if T else torch.empty((0, k), dtype=torch.int32, device="cuda")
+    lib.moe_permute(idx_t, E, has_shared, dev(xq_np) if T else torch.empty((0, H), dtype=torch.uint8, device="cuda"),
+                    dev(sx_np) if T else torch.empty((0, H // 128), dtype=torch.uint8, device="cuda"),
+                    counts, offsets, perm, inv, xqp, sxp, ws)
+    c_ref, o_ref, p_ref, i_ref, src = Pm.permute(idx_np, E, has_shared)
+    np.testing.assert_array_equal(host(counts), c_ref)
+    np.testing.assert_array_equal(host(offsets), o_ref)
+    np.testing.assert_array_equal(host(perm)[:Rn], p_ref)
+    np.testing.assert_array_equal(host(inv)[:T * k], i_ref)
+    if Rn:
+        xr, sr = Pm.gather_rows(xq_np, sx_np, src)
+        np.testing.assert_array_equal(host(xqp), xr)
+        np.testing.assert_array_equal(host(sxp), sr)
+    no_device_error(lib)
+
+
+# ------------------------------- a4/a6 ------------------------------------
+def _gemm_inputs(seed, sizes, N, K, integer):
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Rn, G = int(offsets[-1]), len(sizes)
+    if integer:
+        a = synth.small_int_e4m3(seed, 1, (Rn, K))
+        asc = np.full((Rn, K // 128), 127, np.uint8)
+        w = synth.small_int_fp4(seed, 2, (G, N, K // 2))
+        wsc = np.full((G, N, K // 32), 127, np.uint8)
+    else:
+        a = synth.random_e4m3(seed, 1, (Rn, K))
+        asc = synth.random_bytes(seed, 2, (Rn, K // 128), 118, 130)
+        w = synth.random_bytes(seed, 3, (G, N, K // 2))
+        wsc = synth.random_bytes(seed, 4, (G, N, K // 32), 116, 132)
+    return a, asc, offsets, w, wsc
+
+
+def _run_gemm(lib, a, asc, offsets, w, wsc, epi, block_n):
+    G, N, K = w.shape[0], w.shape[1], w.shape[2] * 2
+    Rn = a.shape[0]
+    w_t = dev(w)
+    sf = torch.empty((G, N // 128, K // 128, 512), dtype=torch.uint8, device="cuda")
+    lib.moe_prepare_weight_scales(dev(wsc), sf)
+    ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
+    if epi == lib.MOE_EPI_SWIGLU_QUANT:
+        out = torch.empty((Rn, N // 2), dtype=torch.uint8, device="cuda")
+        osc = torch.empty((Rn, N // 256), dtype=torch.uint8, device="cuda")
+    elif epi == lib.MOE_EPI_STORE_F32:
+        out, osc = torch.empty((Rn, N), dtype=torch.float32, device="cuda"), None
+    else:
+        out, osc = torch.empty((Rn, N), dtype=torch.bfloat16, device="cuda"), None
+    lib.moe_grouped_gemm_mxfp4(dev(a), dev(asc), dev(offsets), w_t, sf, epi, out, osc, ws, 10.0, block_n)
+    torch.cuda.synchronize()
+    return out, osc
+
+
+GROUPS = [0, 1, 15, 16, 17, 0, 127, 128, 129, 300, 2]
+
+
+@pytest.mark.parametrize("block_n", [16, 32, 64, 128])
+def test_gemm_integer_exact(lib, block_n):
+    """All scales 2^0 and small-integer operands: every partial sum is an
+    integer below 2^24, so the float32 result is exact in any order."""
+    a, asc, offsets, w, wsc = _gemm_inputs(3, GROUPS, 256, 512, True)
+    out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("block_n", [16, 128])
+def test_gemm_random_scaled(lib, block_n):
+    a, asc, offsets, w, wsc = _gemm_inputs(5, [3, 0, 40, 130, 1], 384, 1024, False)
+    out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
+    # float32 accumulation of K terms: error <= K * 2^-24 * sum |a w|
+    av = Q.dequantize_fp8_pow2(a, asc)
+    bound = np.zeros_like(ref)
+    for g in range(len(offsets) - 1):
+        r0, r1 = offsets[g], offsets[g + 1]
+        if r1 > r0:
+            bound[r0:r1] = np.abs(av[r0:r1]) @ np.abs(ffn.dequant_mxfp4(w[g], wsc[g])).T
+    got = out.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= 1024 * 2.0 ** -24 * bound + 1e-30).all()
+    out16, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_BF16, block_n)
+    np.testing.assert_array_equal(out16.view(torch.int16).cpu().numpy(),
+                                  torch.from_numpy(got.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy())
+
+
+def _swiglu_ok(hq, sh, gu_ref, I, limit=10.0):
+    """Codes equal the oracle's, except where the oracle's h lies within a few
+    float32 ulps of a rounding boundary (h itself comes from libm expf)."""
+    q_ref, s_ref = ffn.swiglu_quant(gu_ref, I, limit)
+    h = ffn.swiglu_clamp(gu_ref, I, limit)
+    k = np.repeat(s_ref.astype(np.int64) - 127, 128, axis=1)
+    bad = (hq != q_ref)
+    if bad.any():
+        y = np.abs(h[bad]) / np.ldexp(1.0, k[bad])
+        lo = np.abs(F.decode_e4m3(q_ref[bad]))
+        hi = np.abs(F.decode_e4m3(hq[bad]))
+        mid = (lo + hi) / 2
+        assert (np.abs(y - mid) <= 8 * np.spacing(np.float32(y)).astype(np.float64) * 2).all(), (y, lo, hi)
+        assert bad.mean() < 1e-3
+    sbad = sh != s_ref
+    assert sbad.mean() < 1e-3
+
+
+def test_gemm_swiglu_epilogue_matches_standalone(lib):
+    I = 256
+    a, asc, offsets, w, wsc = _gemm_inputs(9, [5, 0, 33, 140], 2 * I, 512, False)
+    wsc[:] = np.clip(wsc, 0, 124)                          # keep gu mostly inside the clamp
+    gu, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, 32)
+    hq, sh = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_SWIGLU_QUANT, 32)
+    hq2 = torch.empty_like(hq)
+    sh2 = torch.empty_like(sh)
+    lib.moe_swiglu_clamp(gu, hq2, sh2, 10.0)
+    np.testing.assert_array_equal(host(hq), host(hq2))
+    np.testing.assert_array_equal(host(sh), host(sh2))
+    _swiglu_ok(host(hq), host(sh), ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc), I)
+
+
+def test_swiglu_standalone(lib):
+    I, rows = 384, 200
+    gu = (synth.normal(2, 8, rows * 2 * I) * 6).astype(np.float32).reshape(rows, 2 * I)
+    gu[3, :] = 0
+    gu[4, :I] = 50
+    gu[4, I:] = -50
+    hq = torch.empty((rows, I), dtype=torch.uint8, device="cuda")
+    sh = torch.empty((rows, I // 128), dtype=torch.uint8, device="cuda")
+    lib.moe_swiglu_clamp(dev(gu), hq, sh, 10.0)
+    _swiglu_ok(host(hq), host(sh), gu.astype(np.float64), I)
+
+
+# ------------------------------- a7 ---------------------------------------
+def test_combine(lib):
+    T, k, E, H = 50, 6, 16, 512
+    idx, w = R.route_topk(synth.uniform_logits(3, T, E), k)
+    counts, offsets, perm, inv, src = Pm.permute(idx, E, 1)
+    o = synth.normal(3, 9, len(perm) * H).astype(np.float32).reshape(len(perm), H)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    lib.moe_combine(dev(o), dev(inv), dev(w.astype(np.float32)), 1, dev(offsets), E, y)
+    ref = ffn.combine(o.astype(np.float64), inv, w.astype(np.float32).astype(np.float64), offsets, 1)
+    got = host(y.float())
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-6 * (np.abs(o).max() * (k + 1))
+    assert (np.abs(got - ref) <= tol).all()
+
+
+# ------------------------------- a8/a9 ------------------------------------
+def test_repack_nvfp4_bit_exact(lib):
+    M, N, K = 3, 256, 512
+    fp4 = synth.random_bytes(4, 1, (M, N, K // 2))
+    e8 = synth.random_bytes(4, 2, (M, N, K // 32), 118, 135)
+    e8[1] = synth.random_bytes(4, 3, (N, K // 32), 90, 107)   # needs a global scale
+    o_fp4 = torch.empty((M, N, K // 2), dtype=torch.uint8, device="cuda")
+    o_s = torch.empty((M, N, K // 16), dtype=torch.uint8, device="cuda")
+    o_g = torch.empty(M, dtype=torch.float32, device="cuda")
+    lib.repack_mxfp4_to_nvfp4(dev(fp4), dev(e8), o_fp4, o_s, o_g)
+    r_fp4, r_s, r_g = Rp.repack_mxfp4_to_nvfp4(fp4, e8)
+    np.testing.assert_array_equal(host(o_fp4), r_fp4)
+    np.testing.assert_array_equal(host(o_s), r_s)
+    np.testing.assert_array_equal(host(o_g), r_g)
+    no_device_error(lib)
+    # in place: nibbles aliased
+    t = dev(fp4)
+    lib.repack_mxfp4_to_nvfp4(t, dev(e8), t, o_s, o_g)
+    np.testing.assert_array_equal(host(t), fp4)
+
+
+def test_repack_nvfp4_errors(lib):
+    e8 = np.full((1, 128, 4), 127, np.uint8)
+    e8[0, 5, 1] = 255
+    o_s = torch.empty((1, 128, 8), dtype=torch.uint8, device="cuda")
+    o_g = torch.empty(1, dtype=torch.float32, device="cuda")
+    t = torch.zeros((1, 128, 64), dtype=torch.uint8, device="cuda")
+    lib.repack_mxfp4_to_nvfp4(t, dev(e8), t, o_s, o_g)
+    assert lib.moe_get_device_error() == -3
+    e8[0, 5, 1] = 127 + 9
+    e8[0, 6, 0] = 127 - 9
+    lib.repack_mxfp4_to_nvfp4(t, dev(e8), t, o_s, o_g)
+    assert lib.moe_get_device_error() == -4
+    assert lib.moe_get_device_error() == 0
+
+
+def test_repack_int4_bit_exact(lib):
+    M, N, K = 2, 256, 1024
+    fp4 = synth.random_bytes(6, 1, (M, N, K // 2))
+    e8 = synth.random_bytes(6, 2, (M, N, K // 32), 1, 250)
+    e8[0, :7] = 127                                         # ordinary blocks too
+    fp4[0, 3] = 0                                           # an all-zero row
+    q = torch.empty((M, N, K // 2), dtype=torch.int8, device="cuda")
+    s = torch.empty((M, N, K // 128), dtype=torch.float32, device="cuda")
+    lib.repack_mxfp4_to_int4g128(dev(fp4), dev(e8), q, s)
+    q_ref, s_ref = Rp.repack_mxfp4_to_int4g128(fp4, e8)
+    np.testing.assert_array_equal(host(s).view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(host(q), q_ref)
+    no_device_error(lib)
+
+
+def test_repack_int4_errors(lib):
+    q = torch.empty((1, 128, 64), dtype=torch.int8, device="cuda")
+    s = torch.empty((1, 128, 1), dtype=torch.float32, device="cuda")
+    fp4 = torch.full((1, 128, 64), 0x77, dtype=torch.uint8, device="cuda")
+    e8 = np.full((1, 128, 4), 127, np.uint8)
+    e8[0, 9, 2] = 255
+    lib.repack_mxfp4_to_int4g128(fp4, dev(e8), q, s)
+    assert lib.moe_get_device_error() == -3
+    e8[0, 9, 2] = 254
+    lib.repack_mxfp4_to_int4g128(fp4, dev(e8), q, s)
+    assert lib.moe_get_device_error() == -4
