@@ -52,10 +52,15 @@ def read_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
+GEMM_SOURCES = ("common.cuh", "gemm_mxfp4.cuh", "sm100.cuh")
+
+
 def source_digest() -> str:
+    """Digest of the grouped-GEMM kernel sources: recorded DRAM traffic is only
+    reported while these are unchanged since the ncu capture."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_block_scaled_pow2_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMM_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -84,30 +89,48 @@ def make_inputs(wl: dict, seed: int, rank: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms from before
+    the warm-up to after the timed region; summary() keeps the samples whose
+    nvidia-smi timestamp falls inside the timed window (widened to the two
+    nearest samples when the window is shorter than the sampling period)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        self.gpu = str(gpu_index)
+        try:                                    # address the GPU by UUID: robust to device remapping
+            import torch
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+        except Exception:
+            pass
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.window = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
 
-    def __enter__(self):
+    def start(self):
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100", "-i", str(self.gpu)], stdout=self.fh,
+                                          "-lms", "20", "-i", self.gpu], stdout=self.fh,
                                          stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
+        except OSError:
             self.proc = None
+            return self
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+            time.sleep(0.02)
         return self
 
-    def __exit__(self, *a):
+    def mark(self, t_begin: float, t_end: float):
+        self.window = (t_begin, t_end)
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.06)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -116,27 +139,29 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if self.proc is None or self.window is None or not os.path.exists(self.path):
             return None
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        import datetime
+        rows = []
         with open(self.path) as f:
             for ln in f:
                 p = [c.strip() for c in ln.split(",")]
-                if len(p) < 9:
+                if len(p) < 10:
                     continue
                 try:
-                    sm.append(float(p[1]))
-                    mx.append(float(p[2]))
+                    ts = datetime.datetime.strptime(p[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(p[2]), float(p[3]), p[6:10]))
                 except ValueError:
                     continue
-                for n, v in zip(names, p[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        b, e = self.window
+        inside = [r for r in rows if b <= r[0] <= e]
+        if len(inside) < 2:
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - b), abs(r[0] - e)))[:2]
+        reasons = sorted({n for r in inside for n, v in zip(self.REASONS, r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window_ms": round(1e3 * (e - b), 1)}
 
 
 def dist_setup(n_gpus: int):
@@ -221,6 +246,7 @@ def run_ours(args, wl):
         if ev: ev[2].record(stream)
         moe.moe_combine(b.o, b.inv, b.w, layer.has_shared, b.offsets, layer.E, b.y)
 
+    clk = ClockSampler(local).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -231,12 +257,14 @@ def run_ours(args, wl):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
+    w_begin = time.time()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk.mark(w_begin, time.time())
+    clk.stop()
     barrier(pg)
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, pg)
