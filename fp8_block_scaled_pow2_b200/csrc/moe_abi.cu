@@ -314,4 +314,74 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Grouping without caller scratch.  The per-chunk expert histograms live in a
+// fixed device array owned by this library instead of a caller workspace.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr int64_t kNoAllocScratchInts = 65536;   // 256 KiB: n_chunks * E int32 counters
+static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
+
+// Device address of g_permute_scratch, looked up once per device with that
+// device current (the host-side symbol is not a device address).
+int32_t* permute_scratch_ptr(int* status) {
+  static std::mutex mu;
+  static int32_t* ptrs[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    *status = MOE_ERR_LAUNCH;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) {
+      *status = MOE_ERR_LAUNCH;
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<int32_t*>(p);
+  }
+  *status = MOE_OK;
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_permute_noalloc_max_counters(void) { return kNoAllocScratchInts; }
+
+int moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int has_shared, const uint8_t* xq,
+                        const uint8_t* sx, int H, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                        uint8_t* xq_perm, uint8_t* sx_perm, void* stream) {
+  if (T < 0 || E < 1 || E > 1023 || k < 1 || H <= 0 || H % 128) return MOE_ERR_INVALID;
+  if (!counts || !offsets) return MOE_ERR_INVALID;
+  if ((int64_t)T * k > (int64_t)1 << 30) return MOE_ERR_UNSUPPORTED;
+  const int P = T * k;
+  const int64_t n_chunks = (P + kChunk - 1) / kChunk;
+  if (n_chunks * E > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;   // beyond the fixed scratch
+  if (T > 0) {
+    if (!idx || !xq || !sx || !perm || !inv || !xq_perm || !sx_perm) return MOE_ERR_INVALID;
+    if (!aligned(xq, 16) || !aligned(xq_perm, 16)) return MOE_ERR_INVALID;
+  }
+  int st_code = MOE_OK;
+  int32_t* hist = permute_scratch_ptr(&st_code);
+  if (!hist) return st_code;
+  cudaStream_t st = S(stream);
+  // every counter the scan reads is written by the count pass of this call,
+  // so the scratch needs no clearing between calls
+  if (n_chunks > 0) permute_count_kernel<<<(unsigned)n_chunks, 256, 0, st>>>(idx, P, E, hist);
+  permute_scan_kernel<<<1, 1024, 0, st>>>(hist, (int)n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
+  if (n_chunks > 0) permute_scatter_kernel<<<(unsigned)n_chunks, 32, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
+  const int64_t R = (int64_t)P + (has_shared ? T : 0);
+  if (R > 0)
+    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
+        sx_perm);
+  return launch_status();
+}
+
 }  // extern "C"

@@ -82,6 +82,21 @@ def moe_permute(idx, E, has_shared, xq, sx, counts, offsets, perm, inv, xq_perm,
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_permute_noalloc(idx, E, has_shared, xq, sx, counts, offsets, perm, inv, xq_perm, sx_perm, stream=None):
+    """moe_permute for callers that cannot allocate device scratch: the library
+    keeps the counters in its own fixed device array (see the C header for the
+    size limit and the rule that overlapping calls race)."""
+    T, k = idx.shape
+    H = xq.shape[1]
+    _check("moe_permute_noalloc", _lib().moe_permute_noalloc(
+        _ptr(idx), T, E, k, int(has_shared), _ptr(xq), _ptr(sx), H, _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(inv), _ptr(xq_perm), _ptr(sx_perm), _stream(stream)))
+
+
+def moe_permute_noalloc_max_counters() -> int:
+    return int(_lib().moe_permute_noalloc_max_counters())
+
+
 def moe_prepare_weight_scales(e8m0, tiled, stream=None):
     """e8m0 uint8 [n_mats, N, K/32] -> tiled uint8 [n_mats, N/128, K/128, 512]."""
     n_mats, N, k32 = e8m0.shape

@@ -129,6 +129,32 @@ int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared,
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Grouping without caller scratch.  The source pages have no counterpart to
+ * this call; it exists for callers that cannot allocate device memory: a host
+ * runtime working from a fixed memory plan that hands the layer only its
+ * input and output buffers, or a caller that is not allowed to call
+ * cudaMalloc at this point.  Same arguments, outputs and results as
+ * moe_permute, minus the workspace: the per-chunk expert counters live in a
+ * file-scope device array of moe_permute_noalloc_max_counters() int32
+ * (256 KiB), which every GPU that loads this library holds until the process
+ * exits.  Requires ceil(T*k / 2048) * E <= that maximum, else it returns
+ * MOE_ERR_UNSUPPORTED without launching anything.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture on the device.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero (each call writes every counter it
+ *     reads).  Calls whose executions overlap on the GPU (different streams,
+ *     no ordering between them) race on the array and give wrong results.
+ */
+int64_t moe_permute_noalloc_max_counters(void);
+int moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int has_shared,
+                        const uint8_t* xq, const uint8_t* sx, int H,
+                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                        uint8_t* xq_perm, uint8_t* sx_perm, void* stream);
+
+/*
  * Weight-scale preparation (once per weight tensor, at load time).  The
  * block-scaled tensor-core MMA reads its scale factors from tensor memory in
  * a fixed interleave; this call rewrites MXFP4 E8M0 scales [n_mats, N, K/32]
