@@ -52,21 +52,22 @@ def read_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
-GEMM_SOURCES = ("common.cuh", "gemm_mxfp4.cuh", "sm100.cuh")
+GEMM_SOURCES = {"mxfp4": ("common.cuh", "gemm_mxfp4.cuh", "sm100.cuh"),
+                "w4afp8": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh")}
 
 
-def source_digest() -> str:
+def source_digest(weights: str = "mxfp4") -> str:
     """Digest of the grouped-GEMM kernel sources: recorded DRAM traffic is only
     reported while these are unchanged since the ncu capture."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_block_scaled_pow2_b200", "csrc")
-    for f in GEMM_SOURCES:
+    for f in GEMM_SOURCES[weights]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, weights: str = "mxfp4"):
     """DRAM bytes per launch of the dominant kernel from a committed ncu
     summary, or None when the kernels changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -74,7 +75,7 @@ def recorded_traffic(workload: str):
         return None
     with open(p) as f:
         d = json.load(f).get(workload)
-    if not d or d.get("source_digest") != source_digest():
+    if not d or d.get("source_digest") != source_digest(weights) or d.get("weights", "mxfp4") != weights:
         return None
     return d.get("traffic_bytes_per_launch")
 
@@ -222,29 +223,15 @@ def run_ours(args, wl):
 
     rank, world, local, pg = dist_setup(args.gpus)
     x, logits, (w13, s13, w2, s2) = make_inputs(wl, args.seed, rank)
-    layer = MoeLayer(w13, s13, w2, s2, wl["k"])
+    layer = MoeLayer(w13, s13, w2, s2, wl["k"], weights=args.weights)
     T = wl["T"]
     buf = layer.alloc(T)
     xd = torch.from_numpy(x.view(np.int16)).cuda()
     ld = torch.from_numpy(logits).cuda()
     stream = torch.cuda.current_stream()
 
-    # per-GEMM events: the step is the same sequence of ABI calls as
-    # MoeLayer.forward, with events around the two grouped GEMMs
     def step(ev=None):
-        b = buf
-        moe.moe_quantize_act_fp8(xd, b.xq, b.sx)
-        moe.moe_route_topk(ld, layer.topk, b.idx, b.w, layer.route_scale, layer.route_norm)
-        moe.moe_permute(b.idx, layer.E, layer.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
-                        b.xq_perm, b.sx_perm, b.ws_permute)
-        if ev: ev[0].record(stream)
-        moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, b.offsets, layer.w13, layer.w13_sf,
-                                   moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, layer.swiglu_limit, b.block_n)
-        if ev: ev[1].record(stream)
-        moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, b.offsets, layer.w2, layer.w2_sf, moe.MOE_EPI_STORE_F32, b.o,
-                                   None, b.ws_gemm, layer.swiglu_limit, b.block_n)
-        if ev: ev[2].record(stream)
-        moe.moe_combine(b.o, b.inv, b.w, layer.has_shared, b.offsets, layer.E, b.y)
+        layer.forward(xd, ld, buf, marks=ev)
 
     clk = ClockSampler(local).start()
     for _ in range(args.warmup):
@@ -305,27 +292,27 @@ def run_ours(args, wl):
     tokens = T * world * args.steps
     value = tokens / (ms_max / 1e3)
     clocks = clk.summary()
-    dominant = "w13" if args.workload == "decode" else "w13"
     if args.workload == "decode":
         achieved = ab["w13"] / (g13 / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm"], 4), "traffic": recorded_traffic(args.workload),
-                "kernel": "moe_grouped_gemm_mxfp4 (w1/w3, SwiGLU epilogue)",
+                "frac": round(achieved / peaks["hbm"], 4), "traffic": recorded_traffic(args.workload, args.weights),
+                "kernel": f"moe_grouped_gemm_{args.weights} (w1/w3, SwiGLU epilogue)",
                 "peak_source": f"{peaks['src']} HBM copy"}
     else:
         fp8_peak = 2.0 * peaks["bf16_sustained"]
         achieved = ab["flops13"] / (g13 / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": round(achieved / fp8_peak, 4), "traffic": recorded_traffic(args.workload),
-                "kernel": "moe_grouped_gemm_mxfp4 (w1/w3, SwiGLU epilogue)",
+                "frac": round(achieved / fp8_peak, 4), "traffic": recorded_traffic(args.workload, args.weights),
+                "kernel": f"moe_grouped_gemm_{args.weights} (w1/w3, SwiGLU epilogue)",
                 "peak_source": f"{peaks['src']} bf16 sustained x 2 (FP8 rate)"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe2m1->f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe2m1->f32" if args.weights == "mxfp4" else "e4m3xint4->f32",
         "data": "synthetic",
         "config": {"workload": f"{args.workload} layer: hidden {wl['H']}, intermediate {wl['I']}, "
                                f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {T} tokens per GPU",
+                   "weights": args.weights,
                    "tokens_per_gpu": T, "parallelism": f"replicas x{world} (data parallel, no collective)",
                    "l2": f"inputs larger than L2: {ab['active_experts']} active experts stream "
                          f"{(ab['w13'] + ab['w2']) / 1e9:.2f} GB of weights per step"},
@@ -419,6 +406,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--weights", choices=["mxfp4", "w4afp8"], default="mxfp4")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

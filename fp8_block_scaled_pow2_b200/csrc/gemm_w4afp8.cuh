@@ -1,0 +1,348 @@
+// Grouped expert GEMM with W4AFP8 weights: symmetric INT4, group 128, float32
+// weight_scale_inv [N, K/128] ("DeepSeek-V4-Flash-0731-W4AFP8-mt" model card,
+// 量化方式 / 权重约定), times FP8 E4M3 activations with per-128 power-of-two
+// scales (dynamic, e4m3).
+//
+// The weight scale is an arbitrary float32 per (row, 128-column group), so it
+// cannot ride in the MMA's E8M0 scale slots.  Each 128-wide K step is one
+// weight group:
+//   * converter warps transcode the INT4 tile to E4M3 in shared memory (every
+//     integer -8..7 is an exact E4M3 value) in the 128-byte-swizzled K-major
+//     layout the tensor core reads;
+//   * the MMA (kind::mxf8f6f4, E4M3 x E4M3, unit weight scales, per-128
+//     activation scales) writes the group's partial sum into one of two
+//     tensor-memory buffers;
+//   * promotion warps multiply each partial by the row's scale_inv and add it
+//     into float32 registers, then run the same epilogues as the MXFP4 GEMM.
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 converters,
+// 6..9 promotion + epilogue.
+#pragma once
+
+#include "gemm_mxfp4.cuh"
+
+namespace moe {
+namespace w4a {
+
+using namespace sm100;
+using gemm::Item;
+using gemm::decode_item;
+
+constexpr int kThreads = 320;
+
+template <int BN, bool DUAL>
+struct Cfg {
+  static constexpr int NA = (BN + 127) / 128;
+  static constexpr int NUM_A = DUAL ? 2 : 1;
+  static constexpr int RAW_BYTES = 128 * 64;          // INT4 tile as loaded (64 B per row)
+  static constexpr int A_BYTES = 128 * 128;           // E4M3 tile for the MMA
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int A_OFF = 0;                      // NUM_A E4M3 tiles (1024-aligned)
+  static constexpr int B_OFF = NUM_A * A_BYTES;
+  static constexpr int RAW_OFF = B_OFF + B_BYTES;      // NUM_A raw tiles
+  static constexpr int SFB_OFF = RAW_OFF + NUM_A * RAW_BYTES;
+  static constexpr int STAGE_RAW = SFB_OFF + NA * 512;
+  static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int STAGES_FIT = (196 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int TX = NUM_A * RAW_BYTES + B_BYTES + NA * 512;
+  // TMEM: two partial buffers of NUM_A * BN columns, then scale factors
+  static constexpr int P_COLS = NUM_A * BN;
+  static constexpr int SFA_COL = 2 * P_COLS;
+  static constexpr int SFB_COL = SFA_COL + 4;
+  static constexpr int TMEM_USED = SFB_COL + 4 * NA;
+  static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+  static constexpr int SFA_SMEM_OFF = STAGES * STAGE;  // 512 bytes of unit scales
+  static constexpr int BAR_OFF = SFA_SMEM_OFF + 512;
+  static constexpr int RED_OFF = BAR_OFF + 512;
+  static constexpr int SMEM_USED = RED_OFF + 4 * BN * 4;
+  static constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+  static_assert(TMEM_USED <= 512, "tensor memory overflow");
+  static_assert(STAGES >= 2, "too few stages");
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
+  static_assert(!DUAL || BN <= 64, "register accumulators: BN <= 64 with gate and up");
+  static_assert(BN <= 128, "register accumulators: BN <= 128");
+};
+
+// Eight INT4 (two's complement nibbles, element 0 in the low nibble) ->
+// eight E4M3 bytes, by byte-permute table lookups.
+__device__ __forceinline__ uint32_t int4x4_to_e4m3x4(uint32_t h) {
+  // codes of 0..7 and of -8..-1
+  const uint32_t P0 = 0x44403800u, P1 = 0x4E4C4A48u;
+  const uint32_t N0 = 0xCACCCED0u, N1 = 0xB8C0C4C8u;
+  const uint32_t pos = __byte_perm(P0, P1, h);
+  const uint32_t neg = __byte_perm(N0, N1, h);
+  const uint32_t mask = __byte_perm(0x0000FF00u, 0u, (h >> 3) & 0x1111u);
+  return (pos & ~mask) | (neg & mask);
+}
+
+struct W4Args {
+  const float* w_sinv;     // [G, N, K/128]
+  const uint8_t* a_sf;     // per-tile activation scales (as in the MXFP4 GEMM)
+  const int* header;
+  const int* prefix;
+  const int* tstart;
+  const int2* tiles;
+  int G, N, K;
+  void* out;
+  uint8_t* out_scale;
+  float limit;
+};
+
+template <int BN, bool DUAL, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4afp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const W4Args args) {
+  using C = Cfg<BN, DUAL>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* conv = full + C::STAGES;
+  uint64_t* empty = conv + C::STAGES;
+  uint64_t* pfull = empty + C::STAGES;      // [2]
+  uint64_t* pempty = pfull + 2;             // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = args.G, N = args.N, K = args.K;
+  const int KT = K / 128;
+  const int n_ft = DUAL ? N / 256 : N / 128;
+  const int n_items = args.header[0];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pfull[b], 1);
+      mbar_init(&pempty[b], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  // unit weight scales (E8M0 127 = 2^0) for every row and sub-block
+  if (threadIdx.x < 128) reinterpret_cast<uint32_t*>(smem + C::SFA_SMEM_OFF)[threadIdx.x] = 0x7F7F7F7Fu;
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+        const int rb_per_g = N / 128;
+        const int rb0 = it.g * rb_per_g + it.ft;
+        const int rb1 = rb0 + rb_per_g / 2;
+        const uint8_t* sfb = args.a_sf + (size_t)it.t * KT * C::NA * 512;
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + stage * C::STAGE;
+          mbar_arrive_expect_tx(&full[stage], C::TX);
+          tma_load_2d(st + C::RAW_OFF, &tmA, kt * 64, rb0 * 128, &full[stage]);
+          if (DUAL) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, &tmA, kt * 64, rb1 * 128, &full[stage]);
+          tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
+          bulk_load(st + C::SFB_OFF, sfb + (size_t)kt * C::NA * 512, C::NA * 512, &full[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------
+    if (lane == 0) {
+      const uint32_t sfa_smem = smem_u32(smem + C::SFA_SMEM_OFF);
+      tmem_cp_32x128b_warpx4(tmem + C::SFA_COL, sdesc_sf(sfa_smem));
+      uint32_t stage = 0, phase = 0;
+      uint32_t pb = 0, pbits = 0;            // bit b: phase of partial buffer b
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+        const int n_mma = max(16, (it.rows + 15) & ~15);
+        const uint32_t idesc = idesc_mxf8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
+        bool ok = true;
+        for (int kt = 0; kt < KT && ok; ++kt) {
+          if (!mbar_wait(&pempty[pb], ((pbits >> pb) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + stage * C::STAGE);
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a)
+            tmem_cp_32x128b_warpx4(tmem + C::SFB_COL + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+          const uint32_t dcol = tmem + pb * C::P_COLS;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint32_t id = idesc_with_sf_ids(idesc, kb, kb);
+            const uint64_t bdesc = sdesc_kmajor_sw128(st + C::B_OFF + kb * 32);
+            const uint32_t sfa = (tmem + C::SFA_COL) | ((uint32_t)kb << 30);
+            const uint32_t sfb = (tmem + C::SFB_COL) | ((uint32_t)kb << 30);
+            mma_mxf8f6f4(dcol, sdesc_kmajor_sw128(st + C::A_OFF + kb * 32), bdesc, id, sfa, sfb, kb != 0);
+            if (DUAL)
+              mma_mxf8f6f4(dcol + BN, sdesc_kmajor_sw128(st + C::A_OFF + C::A_BYTES + kb * 32), bdesc, id, sfa,
+                           sfb, kb != 0);
+          }
+          tc_commit(&empty[stage]);
+          tc_commit(&pfull[pb]);
+          pbits ^= 1u << pb;
+          pb ^= 1u;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------ converters ----------------------------
+    // thread layout: warp w (0..3), lane l -> 16-byte input chunk (l & 3) of
+    // rows w*8 + (l >> 2) + 32 j; conflict-free reads of the raw tile and
+    // conflict-free writes into the 128-byte swizzle.
+    const int w = warp - 2;
+    const int chunk = lane & 3;
+    uint32_t stage = 0, phase = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        uint8_t* st = smem + stage * C::STAGE;
+#pragma unroll
+        for (int a = 0; a < C::NUM_A; ++a) {
+          const uint8_t* raw = st + C::RAW_OFF + a * C::RAW_BYTES;
+          uint8_t* dst = st + C::A_OFF + a * C::A_BYTES;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = w * 8 + (lane >> 2) + 32 * j;
+            const uint4 in = *reinterpret_cast<const uint4*>(raw + r * 64 + chunk * 16);
+            uint4 o0, o1;
+            o0.x = int4x4_to_e4m3x4(in.x & 0xFFFFu);
+            o0.y = int4x4_to_e4m3x4(in.x >> 16);
+            o0.z = int4x4_to_e4m3x4(in.y & 0xFFFFu);
+            o0.w = int4x4_to_e4m3x4(in.y >> 16);
+            o1.x = int4x4_to_e4m3x4(in.z & 0xFFFFu);
+            o1.y = int4x4_to_e4m3x4(in.z >> 16);
+            o1.z = int4x4_to_e4m3x4(in.w & 0xFFFFu);
+            o1.w = int4x4_to_e4m3x4(in.w >> 16);
+            const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
+            *reinterpret_cast<uint4*>(dst + r * 128 + ((c0 ^ (r & 7)) << 4)) = o0;
+            *reinterpret_cast<uint4*>(dst + r * 128 + ((c1 ^ (r & 7)) << 4)) = o1;
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&conv[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  } else {
+    // --------------------------- promotion + epilogue ---------------------
+    const int q = warp & 3;
+    const int f = q * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+    uint32_t pb = 0, pbits = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+      const int rb_per_g = N / 128;
+      const float* s0 = args.w_sinv + ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT;
+      const float* s1 = args.w_sinv + ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT;
+      float acc0[BN], acc1[DUAL ? BN : 1];
+#pragma unroll
+      for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+#pragma unroll
+      for (int c = 0; c < (DUAL ? BN : 1); ++c) acc1[c] = 0.0f;
+      const int nchunks = (it.rows + 15) >> 4;
+      bool ok = true;
+      float sc0 = __ldg(s0), sc1 = DUAL ? __ldg(s1) : 0.0f;
+      for (int kt = 0; kt < KT; ++kt) {
+        const float nx0 = (kt + 1 < KT) ? __ldg(s0 + kt + 1) : 0.0f;
+        const float nx1 = (DUAL && kt + 1 < KT) ? __ldg(s1 + kt + 1) : 0.0f;
+        if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t base = lane_addr + pb * C::P_COLS;
+#pragma unroll
+        for (int ch = 0; ch < BN / 16; ++ch) {
+          if (ch < nchunks) {
+            uint32_t r0[16];
+            tmem_ld16(base + ch * 16, r0);
+            if constexpr (DUAL) {
+              uint32_t r1[16];
+              tmem_ld16(base + BN + ch * 16, r1);
+              tmem_wait_ld(r0, r1);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]), acc0[ch * 16 + j]);
+                acc1[ch * 16 + j] = fmaf(sc1, __uint_as_float(r1[j]), acc1[ch * 16 + j]);
+              }
+            } else {
+              tmem_wait_ld(r0);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]), acc0[ch * 16 + j]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&pempty[pb]);
+        pbits ^= 1u << pb;
+        pb ^= 1u;
+        sc0 = nx0;
+        sc1 = nx1;
+      }
+      if (!ok) break;
+      // ---- epilogue from registers ----
+      if constexpr (EPI == MOE_EPI_SWIGLU_QUANT) {
+        const int I = N / 2;
+        uint8_t* hq = reinterpret_cast<uint8_t*>(args.out);
+        float* h = acc0;                    // h replaces the gate accumulators
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          h[c] = swiglu_clamped(acc0[c], acc1[DUAL ? c : 0], args.limit);
+          const float m = warp_max_nonneg(fabsf(h[c]));
+          if (lane == 0) red[q * BN + c] = m;
+        }
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          if (c < it.rows) {
+            const float amax = fmaxf(fmaxf(red[c], red[BN + c]), fmaxf(red[2 * BN + c], red[3 * BN + c]));
+            const int k = pow2_scale_exponent(amax);
+            const size_t row = (size_t)(it.row0 + c);
+            hq[row * I + it.ft * 128 + f] = (uint8_t)(e4m3x2(__fmul_rn(h[c], exp2_int(-k)), 0.0f) & 0xFFu);
+            if (f == 0) args.out_scale[row * (I / 128) + it.ft] = (uint8_t)(k + 127);
+          }
+        }
+        named_bar_sync(1, 128);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          if (c < it.rows) {
+            const size_t o = (size_t)(it.row0 + c) * N + it.ft * 128 + f;
+            if constexpr (EPI == MOE_EPI_STORE_F32)
+              reinterpret_cast<float*>(args.out)[o] = acc0[c];
+            else
+              reinterpret_cast<__nv_bfloat16*>(args.out)[o] = __float2bfloat16_rn(acc0[c]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace w4a
+}  // namespace moe

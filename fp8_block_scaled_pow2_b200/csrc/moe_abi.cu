@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "elementwise.cuh"
 #include "gemm_mxfp4.cuh"
+#include "gemm_w4afp8.cuh"
 #include "repack.cuh"
 
 using namespace moe;
@@ -44,7 +45,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D tiled map, inner dimension first.
 bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -52,7 +54,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -84,6 +86,16 @@ int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const g
     case 128: return launch_gemm<128, DUAL, EPI>(ta, tb, a, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
+}
+
+template <int BN, bool DUAL, int EPI>
+int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& a, cudaStream_t st) {
+  using C = w4a::Cfg<BN, DUAL>;
+  auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  k<<<sm_count(), w4a::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  return launch_status();
 }
 
 }  // namespace
@@ -253,6 +265,76 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
     case MOE_EPI_STORE_F32: return launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
     case MOE_EPI_STORE_BF16: return launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
     default: return launch_gemm_bn<true, MOE_EPI_SWIGLU_QUANT>(block_n, ta, tb, args, st);
+  }
+}
+
+int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets,
+                            int n_groups, const int8_t* w_int4, const float* w_scale_inv, int N, int K,
+                            int epilogue, float swiglu_limit, int block_n, void* out, uint8_t* out_scale,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
+    return MOE_ERR_INVALID;
+  if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
+  const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
+  if (dual && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
+  if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
+  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual)) return MOE_ERR_UNSUPPORTED;
+  if (a_rows == 0) return MOE_OK;
+  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_int4 || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
+  if (!aligned(a_e4m3, 16) || !aligned(w_int4, 16) || !aligned(w_scale_inv, 4) || !aligned(workspace, 256))
+    return MOE_ERR_INVALID;
+  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
+  if (workspace_bytes < L.total) return MOE_ERR_INVALID;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_int4, (uint64_t)K / 2, (uint64_t)n_groups * N,
+                (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MOE_ERR_LAUNCH;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
+                (uint32_t)block_n))
+    return MOE_ERR_LAUNCH;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  w4a::W4Args args;
+  args.w_sinv = w_scale_inv;
+  args.a_sf = ws + L.a_sf;
+  args.header = reinterpret_cast<const int*>(ws + L.header);
+  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
+  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
+  args.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  args.G = n_groups;
+  args.N = N;
+  args.K = K;
+  args.out = out;
+  args.out_scale = out_scale;
+  args.limit = swiglu_limit;
+  cudaStream_t st = S(stream);
+  const int n_ft = dual ? N / 256 : N / 128;
+  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
+                                        reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+                                        reinterpret_cast<int2*>(ws + L.tiles));
+  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, K / 128), 128, 0, st>>>(
+      a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
+      reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  if (dual) {
+    switch (block_n) {
+      case 16: return launch_w4a<16, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
+      case 32: return launch_w4a<32, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
+      default: return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
+    }
+  }
+  if (epilogue == MOE_EPI_STORE_F32) {
+    switch (block_n) {
+      case 16: return launch_w4a<16, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
+      case 32: return launch_w4a<32, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
+      case 64: return launch_w4a<64, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
+      default: return launch_w4a<128, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
+    }
+  }
+  switch (block_n) {
+    case 16: return launch_w4a<16, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
+    case 32: return launch_w4a<32, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
+    case 64: return launch_w4a<64, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
+    default: return launch_w4a<128, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
   }
 }
 

@@ -52,7 +52,11 @@ class Buffers:
 
 class MoeLayer:
     def __init__(self, w13, w13_e8m0, w2, w2_e8m0, topk: int, route_scale: float = 1.5,
-                 swiglu_limit: float = 10.0, has_shared: int = 1, route_norm: int = 1, device="cuda"):
+                 swiglu_limit: float = 10.0, has_shared: int = 1, route_norm: int = 1, device="cuda",
+                 weights: str = "mxfp4"):
+        """weights="mxfp4" runs the block-scaled MXFP4 GEMMs; weights="w4afp8"
+        repacks the experts once on the GPU to symmetric INT4 group-128
+        (repack_mxfp4_to_int4g128) and runs the W4AFP8 GEMMs."""
         self.device = torch.device(device)
         self.G = w13.shape[0]                      # routed experts + shared expert
         self.E = self.G - (1 if has_shared else 0)
@@ -69,6 +73,19 @@ class MoeLayer:
                                  device=self.device)
         moe.moe_prepare_weight_scales(_dev(w13_e8m0, self.device), self.w13_sf)
         moe.moe_prepare_weight_scales(_dev(w2_e8m0, self.device), self.w2_sf)
+        self.weights = weights
+        if weights == "w4afp8":
+            d = self.device
+            self.w13_q = torch.empty(self.w13.shape, dtype=torch.int8, device=d)
+            self.w13_sinv = torch.empty((self.G, 2 * self.I, self.H // 128), dtype=torch.float32, device=d)
+            self.w2_q = torch.empty(self.w2.shape, dtype=torch.int8, device=d)
+            self.w2_sinv = torch.empty((self.G, self.H, self.I // 128), dtype=torch.float32, device=d)
+            moe.repack_mxfp4_to_int4g128(self.w13, _dev(w13_e8m0, d), self.w13_q, self.w13_sinv)
+            moe.repack_mxfp4_to_int4g128(self.w2, _dev(w2_e8m0, d), self.w2_q, self.w2_sinv)
+            if moe.moe_get_device_error() != 0:
+                raise moe.MoeError("repack_mxfp4_to_int4g128", -4)
+        elif weights != "mxfp4":
+            raise ValueError(weights)
 
     def weight_bytes_per_expert(self) -> int:
         """MXFP4 bytes of one expert (nibbles + E8M0 scales of w1, w3, w2)."""
@@ -78,8 +95,9 @@ class MoeLayer:
         d, H, I, k = self.device, self.H, self.I, self.topk
         R = T * k + (T if self.has_shared else 0)
         u8, i32, f32 = torch.uint8, torch.int32, torch.float32
-        ws_g = max(moe.moe_gemm_workspace_size(R, self.G, H, block_n),
-                   moe.moe_gemm_workspace_size(R, self.G, I, block_n), 256)
+        # the W4AFP8 w1/w3 GEMM may use narrower token tiles than block_n
+        bns = (block_n, 16) if self.weights == "w4afp8" else (block_n,)
+        ws_g = max([moe.moe_gemm_workspace_size(R, self.G, K, bn) for bn in bns for K in (H, I)] + [256])
         return Buffers(
             T=T,
             xq=torch.empty((T, H), dtype=u8, device=d), sx=torch.empty((T, H // 128), dtype=u8, device=d),
@@ -94,8 +112,11 @@ class MoeLayer:
             ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n)
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers | None = None,
-                stream=None) -> torch.Tensor:
-        """x bfloat16 [T, H] (or its uint16 bits), logits float32 [T, E] -> y bfloat16 [T, H]."""
+                stream=None, marks=None) -> torch.Tensor:
+        """x bfloat16 [T, H] (or its uint16 bits), logits float32 [T, E] -> y bfloat16 [T, H].
+
+        marks: optional three torch.cuda.Event recorded on the stream before the
+        w1/w3 GEMM, between the GEMMs and after the w2 GEMM (for timing)."""
         T = x.shape[0]
         if buf is None or buf.T != T:
             buf = self.alloc(T)
@@ -105,10 +126,27 @@ class MoeLayer:
         moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
                         b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
         g_off = b.offsets if self.has_shared else b.offsets[: self.G + 1]
-        moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13, self.w13_sf,
-                                   moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
-                                   b.block_n, stream=stream)
-        moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2, self.w2_sf, moe.MOE_EPI_STORE_F32, b.o, None,
-                                   b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        ev_stream = stream if stream is not None else torch.cuda.current_stream()
+        if marks:
+            marks[0].record(ev_stream)
+        if self.weights == "mxfp4":
+            moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13, self.w13_sf,
+                                       moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
+                                       b.block_n, stream=stream)
+            if marks:
+                marks[1].record(ev_stream)
+            moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2, self.w2_sf, moe.MOE_EPI_STORE_F32, b.o,
+                                       None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        else:
+            bn = min(b.block_n, 64) if b.block_n else 0
+            moe.moe_grouped_gemm_w4afp8(b.xq_perm, b.sx_perm, g_off, self.w13_q, self.w13_sinv,
+                                        moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
+                                        bn, stream=stream)
+            if marks:
+                marks[1].record(ev_stream)
+            moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
+                                        b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        if marks:
+            marks[2].record(ev_stream)
         moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)
         return b.y

@@ -119,6 +119,17 @@ def moe_grouped_gemm_mxfp4(a, a_scale, offsets, w_fp4, w_scale_tiled, epilogue, 
         _stream(stream)))
 
 
+def moe_grouped_gemm_w4afp8(a, a_scale, offsets, w_int4, w_scale_inv, epilogue, out, out_scale=None,
+                            workspace=None, swiglu_limit=10.0, block_n=0, stream=None):
+    a_rows, K = a.shape
+    G, N = w_int4.shape[0], w_int4.shape[1]
+    _check("moe_grouped_gemm_w4afp8", _lib().moe_grouped_gemm_w4afp8(
+        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_int4), _ptr(w_scale_inv), N, K,
+        int(epilogue), ctypes.c_float(swiglu_limit), int(block_n), _ptr(out), _ptr(out_scale),
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 def moe_swiglu_clamp(gu, hq, sh, limit=10.0, stream=None):
     rows, two_i = gu.shape
     _check("moe_swiglu_clamp", _lib().moe_swiglu_clamp(_ptr(gu), rows, two_i // 2, ctypes.c_float(limit),

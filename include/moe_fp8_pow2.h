@@ -198,6 +198,28 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * a10 -- grouped expert GEMM with W4AFP8 weights [W4A 量化方式 / 权重约定]:
+ * symmetric INT4 weights (two's complement nibbles, element 2i low) with a
+ * float32 dequantisation multiplier per (row, 128 columns), times the same
+ * FP8 activations as moe_grouped_gemm_mxfp4:
+ *   acc[r, n] = sum_g scale_inv[g', n, g] * sum_{k in group g}
+ *               a[r, k] * 2^(sa[r, g]-127) * q[g', n, k]        (g' = r's group)
+ * Each 128-wide group is one block-scaled MMA (INT4 transcoded exactly to
+ * E4M3 in shared memory) whose float32 partial is scaled and summed in
+ * registers, groups in ascending order.
+ *   w_int4       int8 [G, N, K/2] (16-byte aligned); w_scale_inv float32 [G, N, K/128]
+ *   other arguments, layouts and epilogues as moe_grouped_gemm_mxfp4;
+ *   block_n: 16, 32, 64 (SWIGLU_QUANT) or up to 128 (STORE_F32 / STORE_BF16);
+ *   workspace: moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
+ */
+int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
+                            const int32_t* offsets, int n_groups,
+                            const int8_t* w_int4, const float* w_scale_inv, int N, int K,
+                            int epilogue, float swiglu_limit, int block_n,
+                            void* out, uint8_t* out_scale,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * a5 standalone -- SwiGLU with clamp and per-128 power-of-two requantisation
  * [SI 架构特性 / 低精度计算], same arithmetic as MOE_EPI_SWIGLU_QUANT.
  *   gu  float32 [rows, 2I] (gate | up), 16-byte aligned; I % 128 == 0

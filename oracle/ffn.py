@@ -136,7 +136,7 @@ def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
         logits = logits[tokens]
     T, H = x_bf16.shape
     E = logits.shape[1]
-    I = w2.shape[2] * 2 if weights == "mxfp4" else w2_int4.shape[2] * 2
+    I = (w2 if weights == "mxfp4" else w2_int4).shape[2] * 2
     xq, sx = quantize_act_fp8(x_bf16)
     idx, w = route_topk(logits, topk, route_scale, route_norm)
     counts, offsets, perm, inv, src = permute(idx, E, has_shared)

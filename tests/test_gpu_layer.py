@@ -74,3 +74,56 @@ def test_decode_layer_full_size(lib):
 def test_prefill_layer_full_size(lib):
     """Same shapes, 4096 tokens with Zipf(1.1) expert loads."""
     _full_size(4096, synth.zipf_logits, sample=8)
+
+
+def _w4a_ref(x, logits, w13, s13, w2, s2, k, tokens=None, n_proto=None):
+    """Oracle W4AFP8 layer: the oracle's INT4 repack of the experts, then its FFN.
+    With n_proto set (expert e holds the values of expert e % n_proto) only
+    the prototypes the sampled tokens reach are repacked."""
+    from oracle import repack as Rp
+    from oracle import route as R
+    G = w13.shape[0]
+    q13 = np.zeros(w13.shape, np.int8)
+    i13 = np.ones(w13.shape[:2] + (w13.shape[2] * 2 // 128,), np.float32)
+    q2 = np.zeros(w2.shape, np.int8)
+    i2 = np.ones(w2.shape[:2] + (w2.shape[2] * 2 // 128,), np.float32)
+    lg = logits if tokens is None else logits[tokens]
+    used = sorted(set(R.route_topk(lg, k)[0].reshape(-1).tolist()) | {G - 1})
+    done = {}
+    for e in used:
+        p = e if n_proto is None else e % n_proto
+        if p not in done:
+            done[p] = (Rp.repack_mxfp4_to_int4g128(w13[p:p + 1], s13[p:p + 1]),
+                       Rp.repack_mxfp4_to_int4g128(w2[p:p + 1], s2[p:p + 1]))
+        (a, b), (c, d) = done[p]
+        q13[e], i13[e], q2[e], i2[e] = a[0], b[0], c[0], d[0]
+    return ffn.moe_layer(x, logits, None, None, None, None, k, weights="w4afp8", w13_int4=q13, w13_sinv=i13,
+                         w2_int4=q2, w2_sinv=i2, tokens=tokens)
+
+
+@pytest.mark.parametrize("block_n", [0, 16])
+def test_tiny_layer_w4afp8(lib, block_n):
+    """The W4AFP8 path: experts repacked to INT4 group-128 on the GPU, then the
+    INT4 x FP8 GEMMs; compared with the oracle's repack and FFN."""
+    wl = synth.tiny_layer(0)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk, weights="w4afp8")
+    buf = layer.alloc(wl.T, block_n)
+    y = layer.forward(torch.from_numpy(wl.x_bf16.view(np.int16)).cuda(), torch.from_numpy(wl.logits).cuda(), buf)
+    ref = _w4a_ref(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    check_y(y.float().cpu().numpy(), ref["y"])
+    assert lib.moe_get_device_error() == 0
+
+
+def test_long_prefill_w4afp8_sampled(lib):
+    """Hidden 4096, intermediate 2048, 384 routed + 1 shared, top-6, 16384 tokens
+    with Zipf loads, W4AFP8 path; sampled tokens against the oracle."""
+    T, H, I, E, k = 16384, 4096, 2048, 384, 6
+    w13, s13, w2, s2 = synth.expert_weights(0, E + 1, H, I, n_proto=2)
+    x = synth.decode_activations(0, T, H)
+    logits = synth.zipf_logits(0, T, E)
+    layer = MoeLayer(w13, s13, w2, s2, k, weights="w4afp8")
+    buf = layer.alloc(T)
+    y = layer.forward(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(logits).cuda(), buf)
+    toks = np.sort((synth.splitmix64(0, 78, 4) % np.uint64(T)).astype(np.int64))
+    ref = _w4a_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
+    check_y(y.float().cpu().numpy()[toks], ref["y"])
