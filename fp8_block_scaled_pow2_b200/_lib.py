@@ -7,7 +7,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe.so")
+# MOE_LIBRARY may point at another build of the same C ABI (e.g. a debug build)
+LIB_PATH = os.environ.get("MOE_LIBRARY") or os.path.join(_HERE, "libmoe.so")
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -26,7 +27,7 @@ SIGNATURES = {
     "moe_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_noalloc_max_counters": (_I64, []),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_prepare_weight_scales": (_I, [_P, _I64, _I, _I, _P, _P]),
+    "moe_prepare_weight_scales": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
     "moe_gemm_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "moe_grouped_gemm_mxfp4": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_grouped_gemm_w4afp8": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),

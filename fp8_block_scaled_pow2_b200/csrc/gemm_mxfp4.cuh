@@ -36,42 +36,70 @@ namespace gemm {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                   // 10 warps: producer, MMA, 8 workers
+constexpr int kPrefetchStages = 0;              // default L2 prefetch run-ahead (K steps)
 
+// Two shared-memory pipelines:
+//  * direct (BN >= 64): TMA writes the weight tile straight into the unpacked
+//    one-nibble-per-byte layout the MMA reads (16U4_ALIGN16B); 8 epilogue warps.
+//  * staged (BN <= 32, weight streaming): TMA brings the packed nibbles (half
+//    the bytes) into a deep ring; 4 converter warps spread them into a 2-slot
+//    ring of MMA-ready tiles just in time, so twice as many weight bytes are
+//    in flight per SM; 4 epilogue warps.
 template <int BN, bool DUAL>
 struct Cfg {
+  static constexpr bool STAGED = BN <= 32;
   static constexpr int NA = (BN + 127) / 128;            // 128-row scale blocks of the token tile
   static constexpr int NUM_A = DUAL ? 2 : 1;
-  static constexpr int A_BYTES = 128 * 128;              // one FP4 weight tile in shared memory
-  static constexpr int A_TX = 128 * 128 / 2;             // bytes the tensor copy moves for it
+  static constexpr int A_BYTES = 128 * 128;              // one MMA-ready FP4 weight tile
+  static constexpr int A_PACKED = 128 * 64;              // the same tile packed (global layout)
   static constexpr int B_BYTES = BN * 128;
   static constexpr int SF_BYTES = 512;
+  // ring slot: [weight tiles][token tile][weight scales][token scales]
+  static constexpr int A_SLOT = STAGED ? A_PACKED : A_BYTES;
   static constexpr int A0_OFF = 0;
-  static constexpr int A1_OFF = A_BYTES;
-  static constexpr int B_OFF = NUM_A * A_BYTES;
+  static constexpr int B_OFF = (NUM_A * A_SLOT + 1023) / 1024 * 1024;
   static constexpr int SFA_OFF = B_OFF + B_BYTES;
   static constexpr int SFB_OFF = SFA_OFF + NUM_A * SF_BYTES;
   static constexpr int STAGE_RAW = SFB_OFF + NA * SF_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int STAGES_FIT = (200 * 1024) / STAGE;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int TX = NUM_A * A_TX + B_BYTES + NUM_A * SF_BYTES + NA * SF_BYTES;
-  // tensor-memory columns
-  static constexpr int D0_COL = 0;
-  static constexpr int D1_COL = BN;
-  static constexpr int SFA_COL = NUM_A * BN;             // 4 columns per weight tile
-  static constexpr int SFB_COL = SFA_COL + 4 * NUM_A;    // 4 columns per 128 tokens
-  static constexpr int TMEM_USED = SFB_COL + 4 * NA;
-  static constexpr int TMEM_COLS = 512;
-  // shared memory after the stages
-  static constexpr int BAR_OFF = STAGES * STAGE;
-  static constexpr int RED_OFF = BAR_OFF + 256;
-  static constexpr int SMEM_USED = RED_OFF + 4 * 16 * 4;
+  static constexpr int PAD_SLOTS = STAGED ? 2 : 0;       // MMA-ready tiles (staged mode)
+  static constexpr int PAD_STAGE = NUM_A * A_BYTES;
+  static constexpr int RING_BUDGET = 200 * 1024 - PAD_SLOTS * PAD_STAGE;
+  static constexpr int STAGES_FIT = RING_BUDGET / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
+  static constexpr int TX = NUM_A * A_SLOT / (STAGED ? 1 : 2) + B_BYTES + NUM_A * SF_BYTES;  // + NA*512 every 4th step
+  static constexpr int PAD_OFF = STAGES * STAGE;
+  // tensor-memory columns: ACC_BUFS accumulators of NUM_A * BN columns, then scales
+  static constexpr int ACC_COLS = NUM_A * BN;
+  // scale factors are double-buffered so a copy never overwrites columns the
+  // previous K step's MMAs may still read
+  static constexpr int SF_SET = 4 * NUM_A + 4 * NA;       // one set: weight + token scales
+  static constexpr int SF_COLS = 2 * SF_SET;
+  static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
+  static constexpr int SFA_COL = ACC_BUFS * ACC_COLS;     // 4 columns per weight tile (+ SF_SET odd steps)
+  static constexpr int SFB_COL = SFA_COL + 4 * NUM_A;     // 4 columns per 128 tokens (+ SF_SET odd groups)
+  static constexpr int TMEM_USED = SFA_COL + SF_COLS;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
+  // epilogue warps: each owns 32 weight rows (its TMEM sub-partition) and
+  // BN / (EPI_WARPS / 4) token columns
+  static constexpr int EPI_WARPS = STAGED ? 4 : 8;
+  static constexpr int EPI_FIRST = STAGED ? 6 : 2;        // warps 2..5 convert in staged mode
+  static constexpr int CW = BN / (EPI_WARPS / 4);
+  // shared memory after the rings
+  static constexpr int BAR_OFF = PAD_OFF + PAD_SLOTS * PAD_STAGE;
+  static constexpr int RED_OFF = BAR_OFF + 512;
+  static constexpr int PREFIX_OFF = RED_OFF + 2 * 4 * CW * 4;     // group item prefix, int32[G+1]
+  static constexpr int TSTART_OFF = PREFIX_OFF + 4 * 1028;        // first token tile per group, int32[G]
+  static constexpr int SMEM_USED = TSTART_OFF + 4 * 1028;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;     // slack for 1024-byte alignment
-  static_assert(TMEM_USED <= TMEM_COLS, "tensor memory overflow");
+  static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few pipeline stages");
+  static_assert(2 * STAGES + 2 * PAD_SLOTS + 4 <= 64, "barrier area overflow");
+  static_assert(!STAGED || STAGES > PAD_SLOTS, "converters reuse the ring's empty barriers");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "bad token tile");
+  static_assert(SMEM_ALLOC > 116 * 1024, "one CTA per SM keeps tensor-memory allocation uncontended");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "bad token tile");
 };
 
 // ----------------------- plan (work decomposition) -------------------------
@@ -80,7 +108,8 @@ struct Cfg {
 //   prefix   int32[G+1]: first work item of each group
 //   tstart   int32[G]:   first token tile of each group
 //   tiles    int2[max_tiles]: (first row, rows) of each token tile
-//   a_sf     uint8[max_tiles * KT * NA * 512]: per-tile interleaved activation scales
+//   a_sf     uint8[max_tiles * KG * NA * 512]: per-tile activation scales, interleaved
+//            for tensor memory, four 128-wide K steps per 512-byte block (KG = ceil(KT/4))
 struct WsLayout {
   size_t header, prefix, tstart, tiles, a_sf, total;
   int max_tiles;
@@ -97,7 +126,7 @@ inline WsLayout ws_layout(int a_rows, int G, int K, int BN) {
   L.tstart = L.prefix + align256(4 * (size_t)(G + 1));
   L.tiles = L.tstart + align256(4 * (size_t)G);
   L.a_sf = L.tiles + align256(8 * (size_t)L.max_tiles);
-  L.total = L.a_sf + align256((size_t)L.max_tiles * KT * NA * 512);
+  L.total = L.a_sf + align256((size_t)L.max_tiles * ((KT + 3) / 4) * NA * 512);
   return L;
 }
 
@@ -163,22 +192,30 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 }
 
 // Interleave the per-128 activation scales of each token tile into the
-// tensor-memory scale order: for token n of a 128-row block, the 32-bit word
-// at byte (n % 32) * 16 + (n / 32) * 4 holds its scale four times (one per
-// 32-element sub-block of the 128-wide K step).  Rows past the tile are 0.
+// tensor-memory scale order.  For token n of a 128-row block, the 32-bit word
+// at byte (n % 32) * 16 + (n / 32) * 4 of block (tile, g) holds its scales
+// of the four K steps 4g .. 4g+3, one per byte; the MMA of K step kt selects
+// byte kt % 4.  Rows past the tile and K steps past K are 0.
 __global__ void __launch_bounds__(128) tile_act_scales_kernel(const uint8_t* __restrict__ sx, int KT,
                                                               const int* __restrict__ header,
                                                               const int2* __restrict__ tiles, int NA,
                                                               uint8_t* __restrict__ a_sf) {
-  const int t = blockIdx.x, kt = blockIdx.y;
+  const int t = blockIdx.x, g = blockIdx.y;
   if (t >= header[1]) return;
+  const int KG = (KT + 3) / 4;
   const int2 tr = tiles[t];
   const int n = threadIdx.x;
   for (int a = 0; a < NA; ++a) {
     const int r = a * 128 + n;
-    uint32_t b = (r < tr.y) ? (uint32_t)sx[(size_t)(tr.x + r) * KT + kt] : 0u;
-    uint8_t* blk = a_sf + ((size_t)(t * KT + kt) * NA + a) * 512;
-    *reinterpret_cast<uint32_t*>(blk + (n & 31) * 16 + (n >> 5) * 4) = b * 0x01010101u;
+    uint32_t w = 0;
+    if (r < tr.y) {
+      const uint8_t* src = sx + (size_t)(tr.x + r) * KT;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (4 * g + j < KT) w |= (uint32_t)src[4 * g + j] << (8 * j);
+    }
+    uint8_t* blk = a_sf + ((size_t)(t * KG + g) * NA + a) * 512;
+    *reinterpret_cast<uint32_t*>(blk + (n & 31) * 16 + (n >> 5) * 4) = w;
   }
 }
 
@@ -186,21 +223,21 @@ struct Item {
   int g, ft, t, row0, rows;
 };
 
-__device__ __forceinline__ Item decode_item(int item, const int* __restrict__ prefix,
-                                            const int* __restrict__ tstart,
+// prefix: the group item prefix, copied to shared memory by the kernel.
+__device__ __forceinline__ Item decode_item(int item, const int* prefix, const int* tstart,
                                             const int2* __restrict__ tiles, int G, int n_ft) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(prefix + mid) <= item) lo = mid; else hi = mid - 1;
+    if (prefix[mid] <= item) lo = mid; else hi = mid - 1;
   }
   Item it;
   it.g = lo;
-  const int base = __ldg(prefix + lo);
-  const int nt = (__ldg(prefix + lo + 1) - base) / n_ft;
+  const int base = prefix[lo];
+  const int nt = (prefix[lo + 1] - base) / n_ft;
   const int local = item - base;
   it.ft = local / nt;
-  it.t = __ldg(tstart + lo) + local % nt;
+  it.t = tstart[lo] + local % nt;
   const int2 tr = __ldg(tiles + it.t);
   it.row0 = tr.x;
   it.rows = tr.y;
@@ -218,7 +255,74 @@ struct GemmArgs {
   void* out;
   uint8_t* out_scale;
   float limit;
+  int prefetch;           // L2 prefetch run-ahead in K steps
 };
+
+// Epilogue of one work item for one epilogue warp: copy the warp's slice of
+// the accumulator (32 weight rows x CW token columns) to registers, release
+// the TMEM buffer (the next item's MMAs may start), then finish from registers:
+// float32 / bf16 stores, or SwiGLU + per-128 power-of-two FP8 requantisation
+// with the group maximum reduced across the four warps of a column slice.
+template <int BN, bool DUAL, int EPI, int CW>
+__device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int f, int q, int half, int lane,
+                                              int N, const GemmArgs& args, float* red, uint64_t* acc_empty_bar) {
+  const int c_base = half * CW;
+  const int my_cols = max(0, min(CW, it.rows - c_base));     // valid columns of this warp
+  uint32_t v0[CW];
+  uint32_t v1[DUAL ? CW : 1];
+#pragma unroll
+  for (int c = 0; c < CW; c += (CW >= 16 ? 16 : 8)) {
+    if (c < my_cols) {
+      if constexpr (CW >= 16) {
+        tmem_ld16(src + c, *reinterpret_cast<uint32_t(*)[16]>(v0 + c));
+        if constexpr (DUAL) tmem_ld16(src + BN + c, *reinterpret_cast<uint32_t(*)[16]>(v1 + c));
+      } else {
+        tmem_ld8(src + c, v0 + c);
+        if constexpr (DUAL) tmem_ld8(src + BN + c, v1 + c);
+      }
+    }
+  }
+  tmem_wait_ld_n<CW>(v0);
+  if constexpr (DUAL) tmem_wait_ld_n<CW>(v1);
+  tc_fence_before();
+  mbar_arrive(acc_empty_bar);
+
+  if constexpr (EPI == MOE_EPI_SWIGLU_QUANT) {
+    const int I = N / 2;
+    float* rr = red + half * 4 * CW;
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      const float h = swiglu_clamped(__uint_as_float(v0[c]), __uint_as_float(v1[c]), args.limit);
+      v0[c] = __float_as_uint(h);
+      const float m = warp_max_nonneg(fabsf(h));
+      if (lane == 0) rr[q * CW + c] = m;
+    }
+    named_bar_sync(1 + half, 128);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(args.out);
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      if (c < my_cols) {
+        const float amax = fmaxf(fmaxf(rr[c], rr[CW + c]), fmaxf(rr[2 * CW + c], rr[3 * CW + c]));
+        const int k = pow2_scale_exponent(amax);
+        const size_t row = (size_t)(it.row0 + c_base + c);
+        hq[row * I + it.ft * 128 + f] = (uint8_t)(e4m3x2(__fmul_rn(__uint_as_float(v0[c]), exp2_int(-k)), 0.0f) & 0xFFu);
+        if (f == 0) args.out_scale[row * (I / 128) + it.ft] = (uint8_t)(k + 127);
+      }
+    }
+    named_bar_sync(1 + half, 128);
+  } else {
+#pragma unroll
+    for (int c = 0; c < CW; ++c) {
+      if (c < my_cols) {
+        const size_t o = (size_t)(it.row0 + c_base + c) * N + it.ft * 128 + f;
+        if constexpr (EPI == MOE_EPI_STORE_F32)
+          reinterpret_cast<float*>(args.out)[o] = __uint_as_float(v0[c]);
+        else
+          reinterpret_cast<__nv_bfloat16*>(args.out)[o] = __float2bfloat16_rn(__uint_as_float(v0[c]));
+      }
+    }
+  }
+}
 
 template <int BN, bool DUAL, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -230,25 +334,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* acc_full = empty + C::STAGES;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* pad_full = empty + C::STAGES;       // [PAD_SLOTS] (staged mode)
+  uint64_t* acc_full = pad_full + 2;            // [ACC_BUFS]
+  uint64_t* acc_empty = acc_full + 2;           // [ACC_BUFS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
+  int* s_tstart = reinterpret_cast<int*>(smem + C::TSTART_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.G, N = args.N, K = args.K;
   const int KT = K / 128;
   const int n_ft = DUAL ? N / 256 : N / 128;
+  const int rb_per_g = N / 128;
   const int n_items = args.header[0];
+  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+    s_prefix[g] = args.prefix[g];
+    if (g < G) s_tstart[g] = args.tstart[g];
+  }
+  if constexpr (C::STAGED) {      // padding halves of the MMA-ready tiles stay zero
+    for (int i = threadIdx.x; i < C::PAD_SLOTS * C::PAD_STAGE / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + C::PAD_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pad_full[b], 128);
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 32 * C::EPI_WARPS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
@@ -266,26 +386,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
+      // optional L2 prefetch stream running args.prefetch K steps ahead of the loads
+      int pf_item = blockIdx.x, pf_kt = 0;
+      Item pf_it{};
+      if (pf_item < n_items && args.prefetch > 0)
+        pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      auto prefetch_next = [&]() {
+        if (args.prefetch <= 0 || pf_item >= n_items) return;
+        const int rb0 = pf_it.g * rb_per_g + pf_it.ft;
+        tma_prefetch_2d(&tmA, C::STAGED ? pf_kt * 64 : pf_kt * 128, rb0 * 128);
+        if (DUAL) tma_prefetch_2d(&tmA, C::STAGED ? pf_kt * 64 : pf_kt * 128, (rb0 + rb_per_g / 2) * 128);
+        if (++pf_kt == KT) {
+          pf_kt = 0;
+          pf_item += gridDim.x;
+          if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
+        }
+      };
+      for (int i = 0; i < args.prefetch; ++i) prefetch_next();
+
       uint32_t stage = 0, phase = 0;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
-        const int rb_per_g = N / 128;
+        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
         const int rb0 = it.g * rb_per_g + it.ft;
         const int rb1 = rb0 + rb_per_g / 2;
-        const uint8_t* sfa0 = args.w_sf + (size_t)rb0 * KT * 512;
-        const uint8_t* sfa1 = args.w_sf + (size_t)rb1 * KT * 512;
-        const uint8_t* sfb = args.a_sf + (size_t)it.t * KT * C::NA * 512;
+        // weight scales: paired [gate | up] blocks for the SwiGLU projection
+        const uint8_t* sfa = DUAL ? args.w_sf + ((size_t)(it.g * n_ft + it.ft) * KT) * 1024
+                                  : args.w_sf + (size_t)rb0 * KT * 512;
+        const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE;
-          mbar_arrive_expect_tx(&full[stage], C::TX);
-          tma_load_2d(st + C::A0_OFF, &tmA, kt * 128, rb0 * 128, &full[stage]);
-          if (DUAL) tma_load_2d(st + C::A1_OFF, &tmA, kt * 128, rb1 * 128, &full[stage]);
+          const bool new_group = (kt & 3) == 0;
+          mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
+          const int ax = C::STAGED ? kt * 64 : kt * 128;
+          tma_load_2d(st + C::A0_OFF, &tmA, ax, rb0 * 128, &full[stage]);
+          if (DUAL) tma_load_2d(st + C::A0_OFF + C::A_SLOT, &tmA, ax, rb1 * 128, &full[stage]);
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
-          bulk_load(st + C::SFA_OFF, sfa0 + (size_t)kt * 512, 512, &full[stage]);
-          if (DUAL) bulk_load(st + C::SFA_OFF + 512, sfa1 + (size_t)kt * 512, 512, &full[stage]);
-          bulk_load(st + C::SFB_OFF, sfb + (size_t)kt * C::NA * 512, C::NA * 512, &full[stage]);
+          bulk_load(st + C::SFA_OFF, sfa + (size_t)kt * C::NUM_A * 512, C::NUM_A * 512, &full[stage]);
+          if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
+          prefetch_next();
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -293,101 +433,131 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------
+    // One thread issues everything in order; every value that does not change
+    // within an item is computed before its K loop, and per-K-block operands
+    // are constant offsets of per-stage bases (a descriptor's start-address
+    // field is the byte address / 16, so +32 bytes is +2).
     if (lane == 0) {
-      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0, ps = 0, pbits = 0;   // pbits: pad_full phases
+      const uint32_t ring0 = smem_u32(smem);
+      const uint32_t pad0 = smem_u32(smem + C::PAD_OFF);
+      const uint32_t sfa_t = tmem + C::SFA_COL, sfb_t = tmem + C::SFB_COL;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
         const int n_mma = max(16, (it.rows + 15) & ~15);
         const uint32_t idesc = idesc_mxf8f6f4(5u /*E2M1*/, 0u /*E4M3*/, 128, n_mma);
-        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) break;
-        acc_phase ^= 1u;
+        uint32_t id_kb[4];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) id_kb[kb] = idesc_with_sf_ids(idesc, kb, 0);
+        if (!mbar_wait(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
+        const uint32_t d0 = tmem + ab * C::ACC_COLS;
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + stage * C::STAGE);
-          tmem_cp_32x128b_warpx4(tmem + C::SFA_COL, sdesc_sf(st + C::SFA_OFF));
-          if (DUAL) tmem_cp_32x128b_warpx4(tmem + C::SFA_COL + 4, sdesc_sf(st + C::SFA_OFF + 512));
+          uint32_t a_base;
+          if constexpr (C::STAGED) {
+            // the converters waited for this stage's loads before filling pad slot ps
+            if (!mbar_wait(&pad_full[ps], (pbits >> ps) & 1u, abort_flag)) { ok = false; break; }
+            a_base = pad0 + ps * C::PAD_STAGE;
+          } else {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            a_base = ring0 + stage * C::STAGE;
+          }
+          // shared-memory operands arrive through the mbarrier (async proxy);
+          // no tensor-memory hand-off here, so no tcgen05 fence per step
+          const uint32_t st = ring0 + stage * C::STAGE;
+          const uint32_t sfa_k = sfa_t + (kt & 1) * C::SF_SET;          // alternate sets by step
+          const uint32_t sfb_k = sfb_t + ((kt >> 2) & 1) * C::SF_SET;   // and by 4-step group
+          tmem_cp_32x128b_warpx4(sfa_k, sdesc_sf(st + C::SFA_OFF));
+          if (DUAL) tmem_cp_32x128b_warpx4(sfa_k + 4, sdesc_sf(st + C::SFA_OFF + 512));
+          if ((kt & 3) == 0) {
 #pragma unroll
-          for (int a = 0; a < C::NA; ++a)
-            tmem_cp_32x128b_warpx4(tmem + C::SFB_COL + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+            for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_k + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+          }
+          const uint32_t bsel = (uint32_t)(kt & 3);
+          const uint32_t sfb = sfb_k | (bsel << 30);
+          const uint64_t da = sdesc_kmajor_sw128(a_base);
+          const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
+          const uint32_t first = kt != 0;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t id = idesc_with_sf_ids(idesc, kb, kb);
-            const uint64_t bdesc = sdesc_kmajor_sw128(st + C::B_OFF + kb * 32);
-            const uint32_t acc = (kt | kb) != 0;
-            mma_mxf8f6f4(tmem + C::D0_COL, sdesc_kmajor_sw128(st + C::A0_OFF + kb * 32), bdesc, id,
-                         (tmem + C::SFA_COL) | ((uint32_t)kb << 30),
-                         (tmem + C::SFB_COL) | ((uint32_t)kb << 30), acc);
+            const uint32_t id = id_kb[kb] | (bsel << 4);
+            const uint32_t acc = kb ? 1u : first;
+            mma_mxf8f6f4(d0, da + 2 * kb, db + 2 * kb, id, sfa_k | ((uint32_t)kb << 30), sfb, acc);
             if (DUAL)
-              mma_mxf8f6f4(tmem + C::D1_COL, sdesc_kmajor_sw128(st + C::A1_OFF + kb * 32), bdesc, id,
-                           (tmem + C::SFA_COL + 4) | ((uint32_t)kb << 30),
-                           (tmem + C::SFB_COL) | ((uint32_t)kb << 30), acc);
+              mma_mxf8f6f4(d0 + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id,
+                           (sfa_k + 4) | ((uint32_t)kb << 30), sfb, acc);
           }
           tc_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if constexpr (C::STAGED) {
+            pbits ^= 1u << ps;
+            ps ^= 1u;
+          }
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(&acc_full[ab]);
+        acc_bits ^= 1u << ab;
+        if (C::ACC_BUFS == 2) ab ^= 1u;
       }
+    }
+  } else if (C::STAGED && warp < C::EPI_FIRST) {
+    // ------------------------------ converters ----------------------------
+    // Spread packed nibbles (64 B per weight row) into the MMA's layout:
+    // every 8 packed bytes start a 16-byte chunk, chunks 128-byte swizzled.
+    // warp w (0..3), lane l: 16-byte input chunk (l & 3) of rows
+    // w*8 + (l >> 2) + 32 j: conflict-free reads and writes.
+    const int w = warp - 2;
+    const int chunk = lane & 3;
+    uint32_t stage = 0, phase = 0, ps = 0;
+    uint32_t n = 0;                           // running K-step count of this CTA
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt, ++n) {
+        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        if (n >= (uint32_t)C::PAD_SLOTS) {
+          // pad slot ps was last read by the MMAs of step n - PAD_SLOTS; the
+          // ring's empty barrier of that step completes when they are done
+          const uint32_t m = n - C::PAD_SLOTS;
+          if (!mbar_wait(&empty[m % C::STAGES], (m / C::STAGES) & 1u, abort_flag)) { ok = false; break; }
+        }
+        const uint8_t* raw = smem + stage * C::STAGE + C::A0_OFF;
+        uint8_t* dst = smem + C::PAD_OFF + ps * C::PAD_STAGE;
+#pragma unroll
+        for (int a = 0; a < C::NUM_A; ++a) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = w * 8 + (lane >> 2) + 32 * j;
+            const uint4 in = *reinterpret_cast<const uint4*>(raw + a * C::A_PACKED + r * 64 + chunk * 16);
+            const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
+            uint8_t* row = dst + a * C::A_BYTES + r * 128;
+            *reinterpret_cast<uint2*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint2(in.x, in.y);
+            *reinterpret_cast<uint2*>(row + ((c1 ^ (r & 7)) << 4)) = make_uint2(in.z, in.w);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(&pad_full[ps]);
+        ps ^= 1u;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
     }
   } else {
     // ------------------------------ epilogue ------------------------------
+    const int e = warp - C::EPI_FIRST;
     const int q = warp & 3;                 // TMEM sub-partition of this warp
+    const int half = e >> 2;                // which token-column slice (8 epilogue warps)
     const int f = q * 32 + lane;            // weight row (output feature) within the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
-    uint32_t acc_phase = 0;
+    uint32_t ab = 0, acc_bits = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
-      if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
-      acc_phase ^= 1u;
+      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      if (!mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag)) break;
       tc_fence_after();
-      for (int c0 = 0; c0 < it.rows; c0 += 16) {
-        uint32_t r0[16];
-        tmem_ld16(lane_addr + C::D0_COL + c0, r0);
-        if constexpr (EPI == MOE_EPI_SWIGLU_QUANT) {
-          uint32_t r1[16];
-          tmem_ld16(lane_addr + C::D1_COL + c0, r1);
-          tmem_wait_ld(r0, r1);
-          const int I = N / 2;
-          float h[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            h[j] = swiglu_clamped(__uint_as_float(r0[j]), __uint_as_float(r1[j]), args.limit);
-            const float m = warp_max_nonneg(fabsf(h[j]));
-            if (lane == 0) red[q * 16 + j] = m;
-          }
-          named_bar_sync(1, 128);
-          uint8_t* hq = reinterpret_cast<uint8_t*>(args.out);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float amax = fmaxf(fmaxf(red[j], red[16 + j]), fmaxf(red[32 + j], red[48 + j]));
-            const int k = pow2_scale_exponent(amax);
-            const float s = exp2_int(-k);
-            if (c0 + j < it.rows) {
-              const size_t row = (size_t)(it.row0 + c0 + j);
-              hq[row * I + it.ft * 128 + f] = (uint8_t)(e4m3x2(__fmul_rn(h[j], s), 0.0f) & 0xFFu);
-              if (f == 0) args.out_scale[row * (I / 128) + it.ft] = (uint8_t)(k + 127);
-            }
-          }
-          named_bar_sync(1, 128);
-        } else {
-          tmem_wait_ld(r0);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c0 + j < it.rows) {
-              const size_t o = (size_t)(it.row0 + c0 + j) * N + it.ft * 128 + f;
-              if constexpr (EPI == MOE_EPI_STORE_F32)
-                reinterpret_cast<float*>(args.out)[o] = __uint_as_float(r0[j]);
-              else
-                reinterpret_cast<__nv_bfloat16*>(args.out)[o] = __float2bfloat16_rn(__uint_as_float(r0[j]));
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(acc_empty);
+      epilogue_item<BN, DUAL, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,
+                                          args, red, &acc_empty[ab]);
+      acc_bits ^= 1u << ab;
+      if (C::ACC_BUFS == 2) ab ^= 1u;
     }
   }
 
@@ -399,21 +569,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Weight-scale interleave (load-time): [M, N, K/32] -> [M, N/128, K/128, 512].
-__global__ void prepare_weight_scales_kernel(const uint8_t* __restrict__ src, int64_t n_blocks, int K,
-                                             uint8_t* __restrict__ dst) {
-  // one thread per (128-row block, 128-column step, row): 4 bytes
-  const int KT = K / 128;
-  const int64_t total = n_blocks * KT * 128;
+// Weight-scale interleave (load-time): [M, N, K/32] -> 512-byte blocks per
+// (128-row block, 128-wide K step).  Plain order: [M, N/128, K/128].  Paired
+// order (gate | up halves of a w1/w3 matrix): [M, N/256, K/128, 2], so the two
+// blocks one SwiGLU work item needs are adjacent.
+__global__ void prepare_weight_scales_kernel(const uint8_t* __restrict__ src, int64_t n_mats, int N, int K,
+                                             int paired, uint8_t* __restrict__ dst) {
+  // one thread per (128-row block, 128-wide K step, row): 4 bytes
+  const int KT = K / 128, RB = N / 128;
+  const int64_t total = n_mats * RB * KT * 128;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int m = (int)(i & 127);
-    const int64_t bk = i >> 7;               // (block, kt)
+    const int64_t bk = i >> 7;               // (matrix, row block, kt)
     const int kt = (int)(bk % KT);
-    const int64_t blk = bk / KT;
+    const int64_t blk = bk / KT;             // matrix * RB + rb
+    const int64_t mat = blk / RB;
+    const int rb = (int)(blk % RB);
     const int64_t row = blk * 128 + m;
     const uint32_t v = *reinterpret_cast<const uint32_t*>(src + row * (K / 32) + kt * 4);
-    *reinterpret_cast<uint32_t*>(dst + bk * 512 + (m & 31) * 16 + (m >> 5) * 4) = v;
+    int64_t o;
+    if (paired) {
+      const int half_rb = RB / 2, h = rb / half_rb, ft = rb % half_rb;
+      o = ((mat * half_rb + ft) * KT + kt) * 2 + h;
+    } else {
+      o = bk;
+    }
+    *reinterpret_cast<uint32_t*>(dst + o * 512 + (m & 31) * 16 + (m >> 5) * 4) = v;
   }
 }
 

@@ -44,7 +44,7 @@ struct Cfg {
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int STAGES_FIT = (196 * 1024) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int TX = NUM_A * RAW_BYTES + B_BYTES + NA * 512;
+  static constexpr int TX = NUM_A * RAW_BYTES + B_BYTES;   // + NA * 512 every 4th K step
   // TMEM: two partial buffers of NUM_A * BN columns, then scale factors
   static constexpr int P_COLS = NUM_A * BN;
   static constexpr int SFA_COL = 2 * P_COLS;
@@ -54,7 +54,9 @@ struct Cfg {
   static constexpr int SFA_SMEM_OFF = STAGES * STAGE;  // 512 bytes of unit scales
   static constexpr int BAR_OFF = SFA_SMEM_OFF + 512;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int SMEM_USED = RED_OFF + 4 * BN * 4;
+  static constexpr int PREFIX_OFF = RED_OFF + 4 * BN * 4;    // group item prefix, int32[G+1]
+  static constexpr int TSTART_OFF = PREFIX_OFF + 4 * 1028;   // first token tile per group, int32[G]
+  static constexpr int SMEM_USED = TSTART_OFF + 4 * 1028;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few stages");
@@ -86,6 +88,7 @@ struct W4Args {
   void* out;
   uint8_t* out_scale;
   float limit;
+  int prefetch;           // L2 prefetch run-ahead in K steps
 };
 
 template <int BN, bool DUAL, int EPI>
@@ -104,12 +107,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.G, N = args.N, K = args.K;
   const int KT = K / 128;
   const int n_ft = DUAL ? N / 256 : N / 128;
   const int n_items = args.header[0];
+  int* s_tstart = reinterpret_cast<int*>(smem + C::TSTART_OFF);
+  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+    s_prefix[g] = args.prefix[g];
+    if (g < G) s_tstart[g] = args.tstart[g];
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -141,22 +150,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
+      const int rb_per_g = N / 128;
+      // L2 prefetch stream running kPrefetchStages stages ahead of the loads
+      int pf_item = blockIdx.x, pf_kt = 0;
+      Item pf_it{};
+      if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      auto prefetch_next = [&]() {
+        if (pf_item >= n_items) return;
+        const int rb0 = pf_it.g * rb_per_g + pf_it.ft;
+        if (pf_kt == 0) {                 // the item's float32 scales: 128 rows x KT, contiguous
+          bulk_prefetch(args.w_sinv + (size_t)rb0 * 128 * KT, 128 * KT * 4);
+          if (DUAL) bulk_prefetch(args.w_sinv + (size_t)(rb0 + rb_per_g / 2) * 128 * KT, 128 * KT * 4);
+        }
+        tma_prefetch_2d(&tmA, pf_kt * 64, rb0 * 128);
+        if (DUAL) tma_prefetch_2d(&tmA, pf_kt * 64, (rb0 + rb_per_g / 2) * 128);
+        tma_prefetch_2d(&tmB, pf_kt * 128, pf_it.row0);
+        if (++pf_kt == KT) {
+          pf_kt = 0;
+          pf_item += gridDim.x;
+          if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
+        }
+      };
+      for (int i = 0; i < args.prefetch; ++i) prefetch_next();
       uint32_t stage = 0, phase = 0;
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
-        const int rb_per_g = N / 128;
+        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
         const int rb0 = it.g * rb_per_g + it.ft;
         const int rb1 = rb0 + rb_per_g / 2;
-        const uint8_t* sfb = args.a_sf + (size_t)it.t * KT * C::NA * 512;
+        const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE;
-          mbar_arrive_expect_tx(&full[stage], C::TX);
+          const bool new_group = (kt & 3) == 0;
+          mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
           tma_load_2d(st + C::RAW_OFF, &tmA, kt * 64, rb0 * 128, &full[stage]);
           if (DUAL) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, &tmA, kt * 64, rb1 * 128, &full[stage]);
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
-          bulk_load(st + C::SFB_OFF, sfb + (size_t)kt * C::NA * 512, C::NA * 512, &full[stage]);
+          if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
+          prefetch_next();
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -170,25 +202,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t pb = 0, pbits = 0;            // bit b: phase of partial buffer b
       for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
         const int n_mma = max(16, (it.rows + 15) & ~15);
         const uint32_t idesc = idesc_mxf8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
         bool ok = true;
         for (int kt = 0; kt < KT && ok; ++kt) {
           if (!mbar_wait(&pempty[pb], ((pbits >> pb) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+          tc_fence_after();     // orders the MMA after the promotion warps' release of the partial buffer
           const uint32_t st = smem_u32(smem + stage * C::STAGE);
+          if ((kt & 3) == 0) {
 #pragma unroll
-          for (int a = 0; a < C::NA; ++a)
-            tmem_cp_32x128b_warpx4(tmem + C::SFB_COL + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+            for (int a = 0; a < C::NA; ++a)
+              tmem_cp_32x128b_warpx4(tmem + C::SFB_COL + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+          }
           const uint32_t dcol = tmem + pb * C::P_COLS;
+          const uint32_t kb_b = (uint32_t)(kt & 3);
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t id = idesc_with_sf_ids(idesc, kb, kb);
+            const uint32_t id = idesc_with_sf_ids(idesc, kb, kb_b);
             const uint64_t bdesc = sdesc_kmajor_sw128(st + C::B_OFF + kb * 32);
             const uint32_t sfa = (tmem + C::SFA_COL) | ((uint32_t)kb << 30);
-            const uint32_t sfb = (tmem + C::SFB_COL) | ((uint32_t)kb << 30);
+            const uint32_t sfb = (tmem + C::SFB_COL) | (kb_b << 30);
             mma_mxf8f6f4(dcol, sdesc_kmajor_sw128(st + C::A_OFF + kb * 32), bdesc, id, sfa, sfb, kb != 0);
             if (DUAL)
               mma_mxf8f6f4(dcol + BN, sdesc_kmajor_sw128(st + C::A_OFF + C::A_BYTES + kb * 32), bdesc, id, sfa,
@@ -251,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t pb = 0, pbits = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, args.prefix, args.tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
       const int rb_per_g = N / 128;
       const float* s0 = args.w_sinv + ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT;
       const float* s1 = args.w_sinv + ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT;

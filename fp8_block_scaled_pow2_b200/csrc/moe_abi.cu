@@ -3,6 +3,7 @@
 // they share the device error word.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -56,6 +57,19 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// L2 prefetch run-ahead of the grouped GEMMs in 128-wide K steps; the
+// environment variable MOE_GEMM_PREFETCH overrides the default (tuning).
+int prefetch_steps() {
+  static int v = [] {
+    const char* e = getenv("MOE_GEMM_PREFETCH");
+    const int d = gemm::kPrefetchStages;
+    if (!e) return d;
+    const int x = atoi(e);
+    return (x >= 0 && x <= 256) ? x : d;
+  }();
+  return v;
 }
 
 int pick_block_n(int a_rows, int G) {
@@ -193,14 +207,15 @@ int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared, const u
   return launch_status();
 }
 
-int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, uint8_t* tiled, void* stream) {
-  if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return MOE_ERR_INVALID;
+int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired, uint8_t* tiled,
+                              void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128 || (paired && N % 256)) return MOE_ERR_INVALID;
   if (n_mats == 0) return MOE_OK;
   if (!e8m0 || !tiled || !aligned(e8m0, 4) || !aligned(tiled, 4)) return MOE_ERR_INVALID;
-  const int64_t n_blocks = n_mats * (N / 128);
-  const int64_t total = n_blocks * (K / 128) * 128;
+  const int64_t total = n_mats * (N / 128) * (K / 128) * 128;
   const int64_t grid = std::min<int64_t>((total + 255) / 256, 65535LL * 8);
-  gemm::prepare_weight_scales_kernel<<<(unsigned)grid, 256, 0, S(stream)>>>(e8m0, n_blocks, K, tiled);
+  gemm::prepare_weight_scales_kernel<<<(unsigned)grid, 256, 0, S(stream)>>>(e8m0, n_mats, N, K, paired ? 1 : 0,
+                                                                           tiled);
   return launch_status();
 }
 
@@ -229,9 +244,14 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
 
   CUtensorMap ta, tb;
-  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_fp4, (uint64_t)K, (uint64_t)n_groups * N,
-                (uint64_t)K / 2, 128, 128))
+  if (block_n <= 32) {            // staged pipeline: packed nibbles, spread in shared memory
+    if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_fp4, (uint64_t)K / 2, (uint64_t)n_groups * N,
+                  (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_LAUNCH;
+  } else if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_fp4, (uint64_t)K, (uint64_t)n_groups * N,
+                       (uint64_t)K / 2, 128, 128)) {
     return MOE_ERR_LAUNCH;
+  }
   if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
                 (uint32_t)block_n))
     return MOE_ERR_LAUNCH;
@@ -250,6 +270,7 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   args.out = out;
   args.out_scale = out_scale;
   args.limit = swiglu_limit;
+  args.prefetch = prefetch_steps();
 
   cudaStream_t st = S(stream);
   const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
@@ -257,7 +278,7 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
                                         reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
                                         reinterpret_cast<int2*>(ws + L.tiles));
-  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, K / 128), 128, 0, st>>>(
+  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
       a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
       reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
@@ -306,12 +327,13 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
   args.out = out;
   args.out_scale = out_scale;
   args.limit = swiglu_limit;
+  args.prefetch = prefetch_steps();
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
   gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
                                         reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
                                         reinterpret_cast<int2*>(ws + L.tiles));
-  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, K / 128), 128, 0, st>>>(
+  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
       a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
       reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;

@@ -71,7 +71,7 @@ class MoeLayer:
                                   device=self.device)
         self.w2_sf = torch.empty((self.G, self.H // 128, self.I // 128, 512), dtype=torch.uint8,
                                  device=self.device)
-        moe.moe_prepare_weight_scales(_dev(w13_e8m0, self.device), self.w13_sf)
+        moe.moe_prepare_weight_scales(_dev(w13_e8m0, self.device), self.w13_sf, paired=True)
         moe.moe_prepare_weight_scales(_dev(w2_e8m0, self.device), self.w2_sf)
         self.weights = weights
         if weights == "w4afp8":

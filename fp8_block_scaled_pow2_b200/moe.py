@@ -97,11 +97,13 @@ def moe_permute_noalloc_max_counters() -> int:
     return int(_lib().moe_permute_noalloc_max_counters())
 
 
-def moe_prepare_weight_scales(e8m0, tiled, stream=None):
-    """e8m0 uint8 [n_mats, N, K/32] -> tiled uint8 [n_mats, N/128, K/128, 512]."""
+def moe_prepare_weight_scales(e8m0, tiled, paired=False, stream=None):
+    """e8m0 uint8 [n_mats, N, K/32] -> tiled uint8 (n_mats * N * K/32 bytes) in
+    the tensor-memory scale order; paired=True for w1/w3 used with
+    MOE_EPI_SWIGLU_QUANT (gate and up blocks side by side)."""
     n_mats, N, k32 = e8m0.shape
     _check("moe_prepare_weight_scales", _lib().moe_prepare_weight_scales(
-        _ptr(e8m0), n_mats, N, k32 * 32, _ptr(tiled), _stream(stream)))
+        _ptr(e8m0), n_mats, N, k32 * 32, int(bool(paired)), _ptr(tiled), _stream(stream)))
 
 
 def moe_gemm_workspace_size(a_rows: int, n_groups: int, K: int, block_n: int = 0) -> int:

@@ -158,12 +158,18 @@ int moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int has_shared,
  * Weight-scale preparation (once per weight tensor, at load time).  The
  * block-scaled tensor-core MMA reads its scale factors from tensor memory in
  * a fixed interleave; this call rewrites MXFP4 E8M0 scales [n_mats, N, K/32]
- * into that order, [n_mats, N/128, K/128, 512] bytes, where byte
- * (m % 32) * 16 + (m / 32) * 4 + b of a 512-byte block holds the scale of row
- * m (0..127 within the block) for 32-element block b (0..3 within 128).
- * N % 128 == 0, K % 128 == 0.  The values are unchanged.
+ * into 512-byte blocks, one per (128-row block, 128-wide K step), where byte
+ * (m % 32) * 16 + (m / 32) * 4 + b of a block holds the scale of row m
+ * (0..127 within the block) for 32-element sub-block b (0..3).  Block order:
+ *   paired == 0: [n_mats, N/128, K/128]                  (MOE_EPI_STORE_F32 / BF16)
+ *   paired != 0: [n_mats, N/256, K/128, 2] with the row block of the first
+ *                half (gate, w1) and the matching block of the second half
+ *                (up, w3) side by side; required by MOE_EPI_SWIGLU_QUANT;
+ *                N % 256 == 0
+ * N % 128 == 0, K % 128 == 0.  The scale values are unchanged; `tiled` holds
+ * n_mats * N * K / 32 bytes.
  */
-int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K,
+int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired,
                               uint8_t* tiled, void* stream);
 
 /*
@@ -176,7 +182,8 @@ int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K,
  *   a_e8m0_128   uint8 [a_rows, K/128]
  *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0
  *   w_fp4        uint8 [G, N, K/2] packed E2M1 (32-byte aligned)
- *   w_scale_tiled  output of moe_prepare_weight_scales for [G, N, K/32]
+ *   w_scale_tiled  output of moe_prepare_weight_scales for [G, N, K/32] (paired
+ *                layout for MOE_EPI_SWIGLU_QUANT, plain otherwise)
  *   N % 128 == 0 (N % 256 == 0 for SWIGLU_QUANT), K % 128 == 0
  *   epilogue  MOE_EPI_STORE_F32 / MOE_EPI_STORE_BF16: out = acc [a_rows, N]
  *             (rows past offsets[G] untouched);

@@ -134,7 +134,7 @@ def _run_gemm(lib, a, asc, offsets, w, wsc, epi, block_n):
     Rn = a.shape[0]
     w_t = dev(w)
     sf = torch.empty((G, N // 128, K // 128, 512), dtype=torch.uint8, device="cuda")
-    lib.moe_prepare_weight_scales(dev(wsc), sf)
+    lib.moe_prepare_weight_scales(dev(wsc), sf, paired=(epi == lib.MOE_EPI_SWIGLU_QUANT))
     ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
     if epi == lib.MOE_EPI_SWIGLU_QUANT:
         out = torch.empty((Rn, N // 2), dtype=torch.uint8, device="cuda")
