@@ -27,9 +27,10 @@ SIGNATURES = {
     "moe_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_noalloc_max_counters": (_I64, []),
     "moe_permute_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_prepare_weight_scales": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
+    "moe_prepared_weights_size": (_SZ, [_I64, _I, _I]),
+    "moe_prepare_weights": (_I, [_P, _P, _I64, _I, _I, _I, _P, _P]),
     "moe_gemm_workspace_size": (_SZ, [_I, _I, _I, _I]),
-    "moe_grouped_gemm_mxfp4": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
+    "moe_grouped_gemm_mxfp4": (_I, [_P, _P, _I, _P, _I, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_grouped_gemm_w4afp8": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_swiglu_clamp": (_I, [_P, _I, _I, _F, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P]),

@@ -36,16 +36,23 @@ namespace gemm {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;                   // 10 warps: producer, MMA, 8 workers
+constexpr int kThreads = 352;                   // 11 warps: producer, 2 MMA issuers, 8 workers
 constexpr int kPrefetchStages = 0;              // default L2 prefetch run-ahead (K steps)
 
+// Prepared weights (moe_prepare_weights): one 8704-byte block per (128-row
+// block, 128-wide K step): 128 rows x 64 bytes of packed E2M1 nibbles, then
+// the 512-byte scale block in tensor-memory order.  For the SwiGLU projection
+// the gate block and the matching up block of each K step are adjacent.
+constexpr int kWBlock = 8192 + 512;
+
 // Two shared-memory pipelines:
-//  * direct (BN >= 64): TMA writes the weight tile straight into the unpacked
-//    one-nibble-per-byte layout the MMA reads (16U4_ALIGN16B); 8 epilogue warps.
-//  * staged (BN <= 32, weight streaming): TMA brings the packed nibbles (half
-//    the bytes) into a deep ring; 4 converter warps spread them into a 2-slot
-//    ring of MMA-ready tiles just in time, so twice as many weight bytes are
-//    in flight per SM; 4 epilogue warps.
+//  * direct (BN >= 64): a 3-D TMA copy writes the weight tile straight into
+//    the unpacked one-nibble-per-byte layout the MMA reads (16U4_ALIGN16B);
+//    8 epilogue warps.
+//  * staged (BN <= 32, weight streaming): one bulk copy brings the packed
+//    blocks (nibbles + scales, half the bytes of the unpacked tile) into a
+//    deep ring; 4 converter warps spread the nibbles into a 2-slot ring of
+//    MMA-ready tiles just in time; 4 epilogue warps.
 template <int BN, bool DUAL>
 struct Cfg {
   static constexpr bool STAGED = BN <= 32;
@@ -55,12 +62,14 @@ struct Cfg {
   static constexpr int A_PACKED = 128 * 64;              // the same tile packed (global layout)
   static constexpr int B_BYTES = BN * 128;
   static constexpr int SF_BYTES = 512;
-  // ring slot: [weight tiles][token tile][weight scales][token scales]
-  static constexpr int A_SLOT = STAGED ? A_PACKED : A_BYTES;
+  // ring slot, direct: [unpacked weight tiles][token tile][weight scales][token scales]
+  //            staged: [prepared weight blocks (nibbles + scales)][token tile][token scales]
+  static constexpr int A_SLOT = STAGED ? kWBlock : A_BYTES;
   static constexpr int A0_OFF = 0;
   static constexpr int B_OFF = (NUM_A * A_SLOT + 1023) / 1024 * 1024;
-  static constexpr int SFA_OFF = B_OFF + B_BYTES;
-  static constexpr int SFB_OFF = SFA_OFF + NUM_A * SF_BYTES;
+  static constexpr int SFA_OFF = STAGED ? 8192 : B_OFF + B_BYTES;       // weight scales of tile a:
+  static constexpr int SFA_STRIDE = STAGED ? kWBlock : SF_BYTES;       //   SFA_OFF + a * SFA_STRIDE
+  static constexpr int SFB_OFF = STAGED ? B_OFF + B_BYTES : SFA_OFF + NUM_A * SF_BYTES;
   static constexpr int STAGE_RAW = SFB_OFF + NA * SF_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int PAD_SLOTS = STAGED ? 2 : 0;       // MMA-ready tiles (staged mode)
@@ -68,18 +77,26 @@ struct Cfg {
   static constexpr int RING_BUDGET = 200 * 1024 - PAD_SLOTS * PAD_STAGE;
   static constexpr int STAGES_FIT = RING_BUDGET / STAGE;
   static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
-  static constexpr int TX = NUM_A * A_SLOT / (STAGED ? 1 : 2) + B_BYTES + NUM_A * SF_BYTES;  // + NA*512 every 4th step
+  static constexpr int TX = STAGED ? NUM_A * kWBlock + B_BYTES
+                                   : NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;   // + token scales, see below
   static constexpr int PAD_OFF = STAGES * STAGE;
-  // tensor-memory columns: ACC_BUFS accumulators of NUM_A * BN columns, then scales
-  static constexpr int ACC_COLS = NUM_A * BN;
-  // scale factors are double-buffered so a copy never overwrites columns the
-  // previous K step's MMAs may still read
-  static constexpr int SF_SET = 4 * NUM_A + 4 * NA;       // one set: weight + token scales
+  // MMA issue: a single thread issuing small-N MMAs is bound by its own issue
+  // latency, so narrow tiles use two issuing threads.  With gate and up (DUAL)
+  // issuer 0 computes the gate tile and issuer 1 the up tile; otherwise they
+  // take alternate K steps into two partial accumulators the epilogue adds.
+  // Wide gate/up tiles keep one issuer (its gate and up MMAs share the token
+  // operand back to back).
+  // tensor-memory columns: ACC_BUFS accumulators of 2 * BN columns, then one
+  // scale set (weight + token scales) per issuer
+  static constexpr int ISSUERS = (DUAL && BN >= 64) ? 1 : 2;
+  static constexpr int TILES_PER_ISSUER = (DUAL && ISSUERS == 1) ? 2 : 1;
+  static constexpr int ACC_COLS = 2 * BN;
+  static constexpr int SF_SET = 4 * TILES_PER_ISSUER + 4 * NA;
   static constexpr int SF_COLS = 2 * SF_SET;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
-  static constexpr int SFA_COL = ACC_BUFS * ACC_COLS;     // 4 columns per weight tile (+ SF_SET odd steps)
-  static constexpr int SFB_COL = SFA_COL + 4 * NUM_A;     // 4 columns per 128 tokens (+ SF_SET odd groups)
-  static constexpr int TMEM_USED = SFA_COL + SF_COLS;
+  static constexpr int SF_COL = ACC_BUFS * ACC_COLS;      // issuer i: SF_COL + i * SF_SET
+  static constexpr int TMEM_USED = SF_COL + SF_COLS;
+  static constexpr int CONSUMERS = DUAL ? ISSUERS : 1;    // issuers reading each ring stage
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   // epilogue warps: each owns 32 weight rows (its TMEM sub-partition) and
   // BN / (EPI_WARPS / 4) token columns
@@ -245,7 +262,7 @@ __device__ __forceinline__ Item decode_item(int item, const int* prefix, const i
 }
 
 struct GemmArgs {
-  const uint8_t* w_sf;     // prepared weight scales [G, N/128, KT, 512]
+  const uint8_t* w;        // prepared weights (nibbles + scales), see kWBlock
   const uint8_t* a_sf;     // per-tile activation scales
   const int* header;
   const int* prefix;
@@ -265,27 +282,37 @@ struct GemmArgs {
 // with the group maximum reduced across the four warps of a column slice.
 template <int BN, bool DUAL, int EPI, int CW>
 __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int f, int q, int half, int lane,
-                                              int N, const GemmArgs& args, float* red, uint64_t* acc_empty_bar) {
+                                              int N, int KT, const GemmArgs& args, float* red,
+                                              uint64_t* acc_empty_bar) {
   const int c_base = half * CW;
   const int my_cols = max(0, min(CW, it.rows - c_base));     // valid columns of this warp
+  // DUAL: v0 = gate, v1 = up.  Otherwise v0 / v1 are the even / odd K-step
+  // partial sums (v1 holds nothing when there is a single K step).
+  const bool use_v1 = DUAL || KT > 1;
   uint32_t v0[CW];
-  uint32_t v1[DUAL ? CW : 1];
+  uint32_t v1[CW];
 #pragma unroll
   for (int c = 0; c < CW; c += (CW >= 16 ? 16 : 8)) {
     if (c < my_cols) {
       if constexpr (CW >= 16) {
         tmem_ld16(src + c, *reinterpret_cast<uint32_t(*)[16]>(v0 + c));
-        if constexpr (DUAL) tmem_ld16(src + BN + c, *reinterpret_cast<uint32_t(*)[16]>(v1 + c));
+        if (use_v1) tmem_ld16(src + BN + c, *reinterpret_cast<uint32_t(*)[16]>(v1 + c));
       } else {
         tmem_ld8(src + c, v0 + c);
-        if constexpr (DUAL) tmem_ld8(src + BN + c, v1 + c);
+        if (use_v1) tmem_ld8(src + BN + c, v1 + c);
       }
     }
   }
   tmem_wait_ld_n<CW>(v0);
-  if constexpr (DUAL) tmem_wait_ld_n<CW>(v1);
+  tmem_wait_ld_n<CW>(v1);
   tc_fence_before();
   mbar_arrive(acc_empty_bar);
+  if constexpr (!DUAL) {
+    if (use_v1) {
+#pragma unroll
+      for (int c = 0; c < CW; ++c) v0[c] = __float_as_uint(__uint_as_float(v0[c]) + __uint_as_float(v1[c]));
+    }
+  }
 
   if constexpr (EPI == MOE_EPI_SWIGLU_QUANT) {
     const int I = N / 2;
@@ -321,6 +348,76 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
           reinterpret_cast<__nv_bfloat16*>(args.out)[o] = __float2bfloat16_rn(__uint_as_float(v0[c]));
       }
     }
+  }
+}
+
+// One MMA-issuing thread.  Every value that does not change within an item
+// is computed before its K loop; per-K-block operands are constant offsets of
+// per-stage bases (a descriptor's start-address field is the byte address /
+// 16, so +32 bytes is +2).
+template <int BN, bool DUAL>
+__device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const uint32_t tmem, uint64_t* full,
+                                           uint64_t* pad_full, uint64_t* empty, uint64_t* acc_full,
+                                           uint64_t* acc_empty, volatile int* abort_flag, const int* s_prefix,
+                                           const int* s_tstart, const GemmArgs& args, const int n_items,
+                                           const int KT, const int n_ft) {
+  using C = Cfg<BN, DUAL>;
+  const uint32_t ring0 = smem_u32(smem);
+  const uint32_t pad0 = smem_u32(smem + C::PAD_OFF);
+  const uint32_t sfa_t = tmem + C::SF_COL + iss * C::SF_SET;     // 4 columns per weight tile
+  const uint32_t sfb_t = sfa_t + 4 * C::TILES_PER_ISSUER;
+  uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0, n = 0;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, args.G, n_ft);
+    const int n_mma = max(16, (it.rows + 15) & ~15);
+    const uint32_t idesc = idesc_mxf8f6f4(5u /*E2M1*/, 0u /*E4M3*/, 128, n_mma);
+    uint32_t id_kb[4];
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) id_kb[kb] = idesc_with_sf_ids(idesc, kb, 0);
+    if (!mbar_wait(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) return;
+    tc_fence_after();
+    const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
+    for (int kt = 0; kt < KT; ++kt, ++n) {
+      const bool mine = DUAL || C::ISSUERS == 1 || (kt & 1) == iss;
+      if (mine) {
+        uint32_t a_base;
+        if constexpr (C::STAGED) {
+          // the converters waited for this step's loads before filling pad slot n % 2
+          if (!mbar_wait(&pad_full[n & 1u], (n >> 1) & 1u, abort_flag)) return;
+          a_base = pad0 + (n & 1u) * C::PAD_STAGE;
+        } else {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) return;
+          a_base = ring0 + stage * C::STAGE;
+        }
+        if (DUAL) a_base += iss * C::A_BYTES;
+        const uint32_t st = ring0 + stage * C::STAGE;
+        tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SFA_STRIDE : 0)));
+        if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SFA_STRIDE));
+        if ((kt & 3) == (DUAL || C::ISSUERS == 1 ? 0 : iss)) {
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+        }
+        const uint32_t bsel = (uint32_t)(kt & 3);
+        const uint32_t sfb = sfb_t | (bsel << 30);
+        const uint64_t da = sdesc_kmajor_sw128(a_base);
+        const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
+        // this issuer's first step of the item starts a fresh accumulator
+        const uint32_t first = (DUAL || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          mma_mxf8f6f4(d, da + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4), sfa_t | ((uint32_t)kb << 30), sfb,
+                       kb ? 1u : first);
+          if (C::TILES_PER_ISSUER == 2)
+            mma_mxf8f6f4(d + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4),
+                         (sfa_t + 4) | ((uint32_t)kb << 30), sfb, kb ? 1u : first);
+        }
+        tc_commit(&empty[stage]);
+      }
+      if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+    }
+    tc_commit(&acc_full[ab]);
+    acc_bits ^= 1u << ab;
+    if (C::ACC_BUFS == 2) ab ^= 1u;
   }
 }
 
@@ -362,11 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], C::CONSUMERS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&pad_full[b], 128);
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], C::ISSUERS);
       mbar_init(&acc_empty[b], 32 * C::EPI_WARPS);
     }
     *abort_flag = 0;
@@ -393,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
       auto prefetch_next = [&]() {
         if (args.prefetch <= 0 || pf_item >= n_items) return;
-        const int rb0 = pf_it.g * rb_per_g + pf_it.ft;
-        tma_prefetch_2d(&tmA, C::STAGED ? pf_kt * 64 : pf_kt * 128, rb0 * 128);
-        if (DUAL) tma_prefetch_2d(&tmA, C::STAGED ? pf_kt * 64 : pf_kt * 128, (rb0 + rb_per_g / 2) * 128);
+        const size_t pblk = (DUAL ? ((size_t)(pf_it.g * n_ft + pf_it.ft) * KT) * 2
+                                  : (size_t)(pf_it.g * rb_per_g + pf_it.ft) * KT) + (size_t)pf_kt * C::NUM_A;
+        bulk_prefetch(args.w + pblk * kWBlock, C::NUM_A * kWBlock);
         if (++pf_kt == KT) {
           pf_kt = 0;
           pf_item += gridDim.x;
@@ -409,21 +506,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
         const int rb0 = it.g * rb_per_g + it.ft;
         const int rb1 = rb0 + rb_per_g / 2;
-        // weight scales: paired [gate | up] blocks for the SwiGLU projection
-        const uint8_t* sfa = DUAL ? args.w_sf + ((size_t)(it.g * n_ft + it.ft) * KT) * 1024
-                                  : args.w_sf + (size_t)rb0 * KT * 512;
+        // first prepared block of this item's weight tile(s); per K step the
+        // blocks of gate and up (DUAL, paired order) or of the tile are adjacent
+        const size_t blk0 = DUAL ? ((size_t)(it.g * n_ft + it.ft) * KT) * 2 : (size_t)rb0 * KT;
         const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
         bool ok = true;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* st = smem + stage * C::STAGE;
-          const bool new_group = (kt & 3) == 0;
+          // token scales: one block per 4 K steps, read by each issuer at its
+          // first step of the group (issuers alternate steps without DUAL)
+          const bool new_group = (DUAL || C::ISSUERS == 1) ? (kt & 3) == 0 : (kt & 3) < 2;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
-          const int ax = C::STAGED ? kt * 64 : kt * 128;
-          tma_load_2d(st + C::A0_OFF, &tmA, ax, rb0 * 128, &full[stage]);
-          if (DUAL) tma_load_2d(st + C::A0_OFF + C::A_SLOT, &tmA, ax, rb1 * 128, &full[stage]);
+          const size_t blk = blk0 + (size_t)kt * C::NUM_A;
+          if constexpr (C::STAGED) {
+            bulk_load(st + C::A0_OFF, args.w + blk * kWBlock, C::NUM_A * kWBlock, &full[stage]);
+          } else {
+#pragma unroll
+            for (int a = 0; a < C::NUM_A; ++a) {
+              tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)(blk + a), &full[stage]);
+              bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + (blk + a) * kWBlock + 8192, 512, &full[stage]);
+            }
+          }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
-          bulk_load(st + C::SFA_OFF, sfa + (size_t)kt * C::NUM_A * 512, C::NUM_A * 512, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
           prefetch_next();
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -432,75 +537,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer ----------------------------
-    // One thread issues everything in order; every value that does not change
-    // within an item is computed before its K loop, and per-K-block operands
-    // are constant offsets of per-stage bases (a descriptor's start-address
-    // field is the byte address / 16, so +32 bytes is +2).
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0, ps = 0, pbits = 0;   // pbits: pad_full phases
-      const uint32_t ring0 = smem_u32(smem);
-      const uint32_t pad0 = smem_u32(smem + C::PAD_OFF);
-      const uint32_t sfa_t = tmem + C::SFA_COL, sfb_t = tmem + C::SFB_COL;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        const int n_mma = max(16, (it.rows + 15) & ~15);
-        const uint32_t idesc = idesc_mxf8f6f4(5u /*E2M1*/, 0u /*E4M3*/, 128, n_mma);
-        uint32_t id_kb[4];
-#pragma unroll
-        for (int kb = 0; kb < 4; ++kb) id_kb[kb] = idesc_with_sf_ids(idesc, kb, 0);
-        if (!mbar_wait(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d0 = tmem + ab * C::ACC_COLS;
-        bool ok = true;
-        for (int kt = 0; kt < KT; ++kt) {
-          uint32_t a_base;
-          if constexpr (C::STAGED) {
-            // the converters waited for this stage's loads before filling pad slot ps
-            if (!mbar_wait(&pad_full[ps], (pbits >> ps) & 1u, abort_flag)) { ok = false; break; }
-            a_base = pad0 + ps * C::PAD_STAGE;
-          } else {
-            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-            a_base = ring0 + stage * C::STAGE;
-          }
-          // shared-memory operands arrive through the mbarrier (async proxy);
-          // no tensor-memory hand-off here, so no tcgen05 fence per step
-          const uint32_t st = ring0 + stage * C::STAGE;
-          const uint32_t sfa_k = sfa_t + (kt & 1) * C::SF_SET;          // alternate sets by step
-          const uint32_t sfb_k = sfb_t + ((kt >> 2) & 1) * C::SF_SET;   // and by 4-step group
-          tmem_cp_32x128b_warpx4(sfa_k, sdesc_sf(st + C::SFA_OFF));
-          if (DUAL) tmem_cp_32x128b_warpx4(sfa_k + 4, sdesc_sf(st + C::SFA_OFF + 512));
-          if ((kt & 3) == 0) {
-#pragma unroll
-            for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_k + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
-          }
-          const uint32_t bsel = (uint32_t)(kt & 3);
-          const uint32_t sfb = sfb_k | (bsel << 30);
-          const uint64_t da = sdesc_kmajor_sw128(a_base);
-          const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
-          const uint32_t first = kt != 0;
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t id = id_kb[kb] | (bsel << 4);
-            const uint32_t acc = kb ? 1u : first;
-            mma_mxf8f6f4(d0, da + 2 * kb, db + 2 * kb, id, sfa_k | ((uint32_t)kb << 30), sfb, acc);
-            if (DUAL)
-              mma_mxf8f6f4(d0 + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id,
-                           (sfa_k + 4) | ((uint32_t)kb << 30), sfb, acc);
-          }
-          tc_commit(&empty[stage]);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-          if constexpr (C::STAGED) {
-            pbits ^= 1u << ps;
-            ps ^= 1u;
-          }
-        }
-        if (!ok) break;
-        tc_commit(&acc_full[ab]);
-        acc_bits ^= 1u << ab;
-        if (C::ACC_BUFS == 2) ab ^= 1u;
-      }
-    }
+    // ------------------------------ MMA issuer 0 ---------------------------
+    if (lane == 0) mma_issuer<BN, DUAL>(0, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag,
+                                        s_prefix, s_tstart, args, n_items, KT, n_ft);
+  } else if (warp == kThreads / 32 - 1) {
+    // ------------------------------ MMA issuer 1 ---------------------------
+    if (lane == 0 && C::ISSUERS == 2) mma_issuer<BN, DUAL>(1, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag,
+                                        s_prefix, s_tstart, args, n_items, KT, n_ft);
   } else if (C::STAGED && warp < C::EPI_FIRST) {
     // ------------------------------ converters ----------------------------
     // Spread packed nibbles (64 B per weight row) into the MMA's layout:
@@ -528,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int r = w * 8 + (lane >> 2) + 32 * j;
-            const uint4 in = *reinterpret_cast<const uint4*>(raw + a * C::A_PACKED + r * 64 + chunk * 16);
+            const uint4 in = *reinterpret_cast<const uint4*>(raw + a * kWBlock + r * 64 + chunk * 16);
             const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
             uint8_t* row = dst + a * C::A_BYTES + r * 128;
             *reinterpret_cast<uint2*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint2(in.x, in.y);
@@ -555,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag)) break;
       tc_fence_after();
       epilogue_item<BN, DUAL, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,
-                                          args, red, &acc_empty[ab]);
+                                          KT, args, red, &acc_empty[ab]);
       acc_bits ^= 1u << ab;
       if (C::ACC_BUFS == 2) ab ^= 1u;
     }
@@ -569,34 +612,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Weight-scale interleave (load-time): [M, N, K/32] -> 512-byte blocks per
-// (128-row block, 128-wide K step).  Plain order: [M, N/128, K/128].  Paired
-// order (gate | up halves of a w1/w3 matrix): [M, N/256, K/128, 2], so the two
-// blocks one SwiGLU work item needs are adjacent.
-__global__ void prepare_weight_scales_kernel(const uint8_t* __restrict__ src, int64_t n_mats, int N, int K,
-                                             int paired, uint8_t* __restrict__ dst) {
-  // one thread per (128-row block, 128-wide K step, row): 4 bytes
+// Weight preparation (load-time): MXFP4 [M, N, K/2] nibbles + [M, N, K/32]
+// E8M0 -> 8704-byte blocks (kWBlock), one per (128-row block, 128-wide K step):
+// rows of 64 packed bytes, then the scales in tensor-memory order (byte
+// (m % 32) * 16 + (m / 32) * 4 + b: row m, 32-element sub-block b).  Block order
+// plain [M, N/128, K/128]; paired (gate | up halves of a w1/w3 matrix)
+// [M, N/256, K/128, 2].  One block of 128 threads per output block; thread m
+// moves row m.
+__global__ void __launch_bounds__(128) prepare_weights_kernel(const uint8_t* __restrict__ fp4,
+                                                              const uint8_t* __restrict__ e8m0, int N, int K,
+                                                              int paired, uint8_t* __restrict__ out) {
   const int KT = K / 128, RB = N / 128;
-  const int64_t total = n_mats * RB * KT * 128;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int m = (int)(i & 127);
-    const int64_t bk = i >> 7;               // (matrix, row block, kt)
-    const int kt = (int)(bk % KT);
-    const int64_t blk = bk / KT;             // matrix * RB + rb
-    const int64_t mat = blk / RB;
-    const int rb = (int)(blk % RB);
-    const int64_t row = blk * 128 + m;
-    const uint32_t v = *reinterpret_cast<const uint32_t*>(src + row * (K / 32) + kt * 4);
-    int64_t o;
-    if (paired) {
-      const int half_rb = RB / 2, h = rb / half_rb, ft = rb % half_rb;
-      o = ((mat * half_rb + ft) * KT + kt) * 2 + h;
-    } else {
-      o = bk;
-    }
-    *reinterpret_cast<uint32_t*>(dst + o * 512 + (m & 31) * 16 + (m >> 5) * 4) = v;
+  const int64_t ob = blockIdx.x;            // output block index
+  int64_t mat, rb;
+  int kt;
+  if (paired) {
+    const int h = (int)(ob & 1);
+    const int64_t t = ob >> 1;              // (mat, ft, kt)
+    kt = (int)(t % KT);
+    const int64_t mf = t / KT;
+    mat = mf / (RB / 2);
+    rb = (mf % (RB / 2)) + h * (RB / 2);
+  } else {
+    kt = (int)(ob % KT);
+    const int64_t mr = ob / KT;
+    mat = mr / RB;
+    rb = mr % RB;
   }
+  const int m = threadIdx.x;
+  const int64_t row = (mat * RB + rb) * 128 + m;
+  const uint4* src = reinterpret_cast<const uint4*>(fp4 + row * (K / 2) + kt * 64);
+  uint4* dst = reinterpret_cast<uint4*>(out + ob * kWBlock + m * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = __ldg(src + i);
+  const uint32_t v = *reinterpret_cast<const uint32_t*>(e8m0 + row * (K / 32) + kt * 4);
+  *reinterpret_cast<uint32_t*>(out + ob * kWBlock + 8192 + (m & 31) * 16 + (m >> 5) * 4) = v;
 }
 
 }  // namespace gemm

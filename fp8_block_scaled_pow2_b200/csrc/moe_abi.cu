@@ -72,6 +72,20 @@ int prefetch_steps() {
   return v;
 }
 
+// 3-D tiled map (inner dimension first) over equally spaced 2-D blocks.
+bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int pick_block_n(int a_rows, int G) {
   const double avg = (double)a_rows / (G > 0 ? G : 1);
   if (avg <= 12) return 16;
@@ -207,15 +221,20 @@ int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared, const u
   return launch_status();
 }
 
-int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired, uint8_t* tiled,
-                              void* stream) {
+size_t moe_prepared_weights_size(int64_t n_mats, int N, int K) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return 0;
+  return (size_t)n_mats * (N / 128) * (K / 128) * gemm::kWBlock;
+}
+
+int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired,
+                        uint8_t* prepared, void* stream) {
   if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128 || (paired && N % 256)) return MOE_ERR_INVALID;
   if (n_mats == 0) return MOE_OK;
-  if (!e8m0 || !tiled || !aligned(e8m0, 4) || !aligned(tiled, 4)) return MOE_ERR_INVALID;
-  const int64_t total = n_mats * (N / 128) * (K / 128) * 128;
-  const int64_t grid = std::min<int64_t>((total + 255) / 256, 65535LL * 8);
-  gemm::prepare_weight_scales_kernel<<<(unsigned)grid, 256, 0, S(stream)>>>(e8m0, n_mats, N, K, paired ? 1 : 0,
-                                                                           tiled);
+  if (!fp4 || !e8m0 || !prepared || !aligned(fp4, 16) || !aligned(e8m0, 4) || !aligned(prepared, 16))
+    return MOE_ERR_INVALID;
+  const int64_t blocks = n_mats * (N / 128) * (K / 128);
+  if (blocks > 0x7FFFFFFFLL) return MOE_ERR_UNSUPPORTED;
+  gemm::prepare_weights_kernel<<<(unsigned)blocks, 128, 0, S(stream)>>>(fp4, e8m0, N, K, paired ? 1 : 0, prepared);
   return launch_status();
 }
 
@@ -226,9 +245,9 @@ size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n) {
 }
 
 int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets,
-                           int n_groups, const uint8_t* w_fp4, const uint8_t* w_scale_tiled, int N, int K,
-                           int epilogue, float swiglu_limit, int block_n, void* out, uint8_t* out_scale,
-                           void* workspace, size_t workspace_bytes, void* stream) {
+                           int n_groups, const uint8_t* w_prepared, int N, int K, int epilogue, float swiglu_limit,
+                           int block_n, void* out, uint8_t* out_scale, void* workspace, size_t workspace_bytes,
+                           void* stream) {
   if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
     return MOE_ERR_INVALID;
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
@@ -236,29 +255,25 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
   if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128) return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
-  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_fp4 || !w_scale_tiled || !out || !workspace)
-    return MOE_ERR_INVALID;
-  if (!aligned(a_e4m3, 16) || !aligned(w_fp4, 32) || !aligned(w_scale_tiled, 16) || !aligned(workspace, 256))
-    return MOE_ERR_INVALID;
+  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_prepared || !out || !workspace) return MOE_ERR_INVALID;
+  if (!aligned(a_e4m3, 16) || !aligned(w_prepared, 32) || !aligned(workspace, 256)) return MOE_ERR_INVALID;
   const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
 
   CUtensorMap ta, tb;
-  if (block_n <= 32) {            // staged pipeline: packed nibbles, spread in shared memory
-    if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_fp4, (uint64_t)K / 2, (uint64_t)n_groups * N,
-                  (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return MOE_ERR_LAUNCH;
-  } else if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_fp4, (uint64_t)K, (uint64_t)n_groups * N,
-                       (uint64_t)K / 2, 128, 128)) {
+  // weight tiles of the direct pipeline: 3-D view [blocks][128 rows][128 nibbles]
+  // of the prepared blocks (the staged pipeline copies whole blocks instead)
+  const uint64_t n_blocks = (uint64_t)n_groups * (N / 128) * (K / 128);
+  if (!make_map_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_prepared, 128, 128, n_blocks, 64,
+                   (uint64_t)gemm::kWBlock, 128, 128))
     return MOE_ERR_LAUNCH;
-  }
   if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
                 (uint32_t)block_n))
     return MOE_ERR_LAUNCH;
 
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   gemm::GemmArgs args;
-  args.w_sf = w_scale_tiled;
+  args.w = w_prepared;
   args.a_sf = ws + L.a_sf;
   args.header = reinterpret_cast<const int*>(ws + L.header);
   args.prefix = reinterpret_cast<const int*>(ws + L.prefix);

@@ -1,9 +1,9 @@
 """A routed-expert MoE FFN layer on top of the C ABI.
 
 MoeLayer owns the device copies of the expert weights (MXFP4, w13 = w1 (gate)
-rows followed by w3 (up) rows, then w2) with their scales prepared once for
-the tensor cores, and runs one forward pass as a fixed sequence of library
-calls on one stream, with no host synchronisation:
+rows followed by w3 (up) rows, then w2), prepared once into the blocks the
+tensor-core GEMM streams (moe_prepare_weights), and runs one forward pass as a
+fixed sequence of library calls on one stream, with no host synchronisation:
 
     moe_quantize_act_fp8 -> moe_route_topk -> moe_permute
     -> moe_grouped_gemm_mxfp4(w13, SwiGLU + FP8 requant)
@@ -65,26 +65,30 @@ class MoeLayer:
         assert w2.shape[1] == self.H and w2.shape[2] * 2 == self.I
         self.topk, self.route_scale, self.swiglu_limit = topk, route_scale, swiglu_limit
         self.has_shared, self.route_norm = has_shared, route_norm
-        self.w13 = _dev(w13, self.device)
-        self.w2 = _dev(w2, self.device)
-        self.w13_sf = torch.empty((self.G, 2 * self.I // 128, self.H // 128, 512), dtype=torch.uint8,
-                                  device=self.device)
-        self.w2_sf = torch.empty((self.G, self.H // 128, self.I // 128, 512), dtype=torch.uint8,
-                                 device=self.device)
-        moe.moe_prepare_weight_scales(_dev(w13_e8m0, self.device), self.w13_sf, paired=True)
-        moe.moe_prepare_weight_scales(_dev(w2_e8m0, self.device), self.w2_sf)
+        d = self.device
         self.weights = weights
-        if weights == "w4afp8":
-            d = self.device
-            self.w13_q = torch.empty(self.w13.shape, dtype=torch.int8, device=d)
+        if weights == "mxfp4":
+            # prepared blocks (nibbles + tensor-memory-order scales); the raw
+            # MXFP4 arrays are not kept
+            w13_d, s13_d = _dev(w13, d), _dev(w13_e8m0, d)
+            self.w13_p = torch.empty(moe.moe_prepared_weights_size(self.G, 2 * self.I, self.H), dtype=torch.uint8,
+                                     device=d)
+            moe.moe_prepare_weights(w13_d, s13_d, self.w13_p, paired=True)
+            del w13_d, s13_d
+            w2_d, s2_d = _dev(w2, d), _dev(w2_e8m0, d)
+            self.w2_p = torch.empty(moe.moe_prepared_weights_size(self.G, self.H, self.I), dtype=torch.uint8, device=d)
+            moe.moe_prepare_weights(w2_d, s2_d, self.w2_p)
+            del w2_d, s2_d
+        elif weights == "w4afp8":
+            self.w13_q = torch.empty((self.G, 2 * self.I, self.H // 2), dtype=torch.int8, device=d)
             self.w13_sinv = torch.empty((self.G, 2 * self.I, self.H // 128), dtype=torch.float32, device=d)
-            self.w2_q = torch.empty(self.w2.shape, dtype=torch.int8, device=d)
+            self.w2_q = torch.empty((self.G, self.H, self.I // 2), dtype=torch.int8, device=d)
             self.w2_sinv = torch.empty((self.G, self.H, self.I // 128), dtype=torch.float32, device=d)
-            moe.repack_mxfp4_to_int4g128(self.w13, _dev(w13_e8m0, d), self.w13_q, self.w13_sinv)
-            moe.repack_mxfp4_to_int4g128(self.w2, _dev(w2_e8m0, d), self.w2_q, self.w2_sinv)
+            moe.repack_mxfp4_to_int4g128(_dev(w13, d), _dev(w13_e8m0, d), self.w13_q, self.w13_sinv)
+            moe.repack_mxfp4_to_int4g128(_dev(w2, d), _dev(w2_e8m0, d), self.w2_q, self.w2_sinv)
             if moe.moe_get_device_error() != 0:
                 raise moe.MoeError("repack_mxfp4_to_int4g128", -4)
-        elif weights != "mxfp4":
+        else:
             raise ValueError(weights)
 
     def weight_bytes_per_expert(self) -> int:
@@ -130,12 +134,12 @@ class MoeLayer:
         if marks:
             marks[0].record(ev_stream)
         if self.weights == "mxfp4":
-            moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13, self.w13_sf,
+            moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13_p, self.G, 2 * self.I,
                                        moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
                                        b.block_n, stream=stream)
             if marks:
                 marks[1].record(ev_stream)
-            moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2, self.w2_sf, moe.MOE_EPI_STORE_F32, b.o,
+            moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.G, self.H, moe.MOE_EPI_STORE_F32, b.o,
                                        None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
         else:
             bn = min(b.block_n, 64) if b.block_n else 0

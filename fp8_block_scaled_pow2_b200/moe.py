@@ -97,25 +97,29 @@ def moe_permute_noalloc_max_counters() -> int:
     return int(_lib().moe_permute_noalloc_max_counters())
 
 
-def moe_prepare_weight_scales(e8m0, tiled, paired=False, stream=None):
-    """e8m0 uint8 [n_mats, N, K/32] -> tiled uint8 (n_mats * N * K/32 bytes) in
-    the tensor-memory scale order; paired=True for w1/w3 used with
+def moe_prepared_weights_size(n_mats: int, N: int, K: int) -> int:
+    return int(_lib().moe_prepared_weights_size(n_mats, N, K))
+
+
+def moe_prepare_weights(fp4, e8m0, prepared, paired=False, stream=None):
+    """MXFP4 nibbles [n_mats, N, K/2] + E8M0 [n_mats, N, K/32] -> prepared
+    blocks (moe_prepared_weights_size bytes); paired=True for w1/w3 used with
     MOE_EPI_SWIGLU_QUANT (gate and up blocks side by side)."""
-    n_mats, N, k32 = e8m0.shape
-    _check("moe_prepare_weight_scales", _lib().moe_prepare_weight_scales(
-        _ptr(e8m0), n_mats, N, k32 * 32, int(bool(paired)), _ptr(tiled), _stream(stream)))
+    n_mats, N, k2 = fp4.shape
+    _check("moe_prepare_weights", _lib().moe_prepare_weights(
+        _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, int(bool(paired)), _ptr(prepared), _stream(stream)))
 
 
 def moe_gemm_workspace_size(a_rows: int, n_groups: int, K: int, block_n: int = 0) -> int:
     return int(_lib().moe_gemm_workspace_size(a_rows, n_groups, K, block_n))
 
 
-def moe_grouped_gemm_mxfp4(a, a_scale, offsets, w_fp4, w_scale_tiled, epilogue, out, out_scale=None,
+def moe_grouped_gemm_mxfp4(a, a_scale, offsets, w_prepared, G, N, epilogue, out, out_scale=None,
                            workspace=None, swiglu_limit=10.0, block_n=0, stream=None):
+    """w_prepared: moe_prepare_weights output for G matrices [N, K] (K = a.shape[1])."""
     a_rows, K = a.shape
-    G, N = w_fp4.shape[0], w_fp4.shape[1]
     _check("moe_grouped_gemm_mxfp4", _lib().moe_grouped_gemm_mxfp4(
-        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_fp4), _ptr(w_scale_tiled), N, K,
+        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_prepared), N, K,
         int(epilogue), ctypes.c_float(swiglu_limit), int(block_n), _ptr(out), _ptr(out_scale),
         _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
         _stream(stream)))

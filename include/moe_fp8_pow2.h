@@ -155,22 +155,24 @@ int moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int has_shared,
                         uint8_t* xq_perm, uint8_t* sx_perm, void* stream);
 
 /*
- * Weight-scale preparation (once per weight tensor, at load time).  The
- * block-scaled tensor-core MMA reads its scale factors from tensor memory in
- * a fixed interleave; this call rewrites MXFP4 E8M0 scales [n_mats, N, K/32]
- * into 512-byte blocks, one per (128-row block, 128-wide K step), where byte
- * (m % 32) * 16 + (m / 32) * 4 + b of a block holds the scale of row m
- * (0..127 within the block) for 32-element sub-block b (0..3).  Block order:
- *   paired == 0: [n_mats, N/128, K/128]                  (MOE_EPI_STORE_F32 / BF16)
- *   paired != 0: [n_mats, N/256, K/128, 2] with the row block of the first
- *                half (gate, w1) and the matching block of the second half
- *                (up, w3) side by side; required by MOE_EPI_SWIGLU_QUANT;
- *                N % 256 == 0
- * N % 128 == 0, K % 128 == 0.  The scale values are unchanged; `tiled` holds
- * n_mats * N * K / 32 bytes.
+ * Weight preparation (once per weight tensor, at load time): MXFP4 nibbles
+ * [n_mats, N, K/2] and E8M0 scales [n_mats, N, K/32] -> blocks of 8704 bytes,
+ * one per (128-row block, 128-wide K step): the block's 128 rows x 64 bytes of
+ * packed nibbles (the source rows, unchanged), then its 512 scale bytes in the
+ * order the block-scaled tensor-core MMA reads from tensor memory (byte
+ * (m % 32) * 16 + (m / 32) * 4 + b holds row m's scale of 32-element sub-block
+ * b).  Block order:
+ *   paired == 0: [n_mats, N/128, K/128]                   (MOE_EPI_STORE_F32 / BF16)
+ *   paired != 0: [n_mats, N/256, K/128, 2]: the block of the first half (gate,
+ *                w1) and the matching block of the second half (up, w3) side by
+ *                side; required by MOE_EPI_SWIGLU_QUANT; N % 256 == 0
+ * N % 128 == 0, K % 128 == 0; fp4 16-byte aligned; `prepared` holds
+ * moe_prepared_weights_size(n_mats, N, K) bytes (N*K/2 * 17/16 per matrix),
+ * 32-byte aligned.  The values are unchanged (a relayout).
  */
-int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired,
-                              uint8_t* tiled, void* stream);
+size_t moe_prepared_weights_size(int64_t n_mats, int N, int K);
+int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K, int paired,
+                        uint8_t* prepared, void* stream);
 
 /*
  * a4 / a5 / a6 -- grouped expert GEMM with MXFP4 weights [SI 低精度计算],
@@ -181,9 +183,9 @@ int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K,
  *   a_e4m3       uint8 [a_rows, K] (16-byte aligned), a_rows >= offsets[G]
  *   a_e8m0_128   uint8 [a_rows, K/128]
  *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0
- *   w_fp4        uint8 [G, N, K/2] packed E2M1 (32-byte aligned)
- *   w_scale_tiled  output of moe_prepare_weight_scales for [G, N, K/32] (paired
- *                layout for MOE_EPI_SWIGLU_QUANT, plain otherwise)
+ *   w_prepared   output of moe_prepare_weights for the MXFP4 weights [G, N, K/2]
+ *                and scales [G, N, K/32] (paired order for
+ *                MOE_EPI_SWIGLU_QUANT, plain otherwise)
  *   N % 128 == 0 (N % 256 == 0 for SWIGLU_QUANT), K % 128 == 0
  *   epilogue  MOE_EPI_STORE_F32 / MOE_EPI_STORE_BF16: out = acc [a_rows, N]
  *             (rows past offsets[G] untouched);
@@ -199,7 +201,7 @@ int moe_prepare_weight_scales(const uint8_t* e8m0, int64_t n_mats, int N, int K,
 size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n);
 int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
                            const int32_t* offsets, int n_groups,
-                           const uint8_t* w_fp4, const uint8_t* w_scale_tiled, int N, int K,
+                           const uint8_t* w_prepared, int N, int K,
                            int epilogue, float swiglu_limit, int block_n,
                            void* out, uint8_t* out_scale,
                            void* workspace, size_t workspace_bytes, void* stream);

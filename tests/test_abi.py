@@ -50,8 +50,9 @@ def test_argument_validation_without_gpu():
     assert lib.moe_quantize_act_fp8(None, 4, 100, None, None, None) == -1      # cols % 128
     assert lib.moe_quantize_act_fp8(None, 0, 128, None, None, None) == 0       # empty: no-op
     assert lib.moe_route_topk(None, 4, 8, 9, ctypes.c_float(1.5), 1, None, None, None) == -1
-    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, None, 256, 100, 0,
+    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 256, 100, 0,
                                       ctypes.c_float(10), 0, None, None, None, 0, None) == -1
-    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, None, 256, 128, 0,
+    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 256, 128, 0,
                                       ctypes.c_float(10), 48, None, None, None, 0, None) == -2
+    assert lib.moe_prepared_weights_size(3, 256, 512) == 3 * 2 * 4 * 8704
     assert lib.repack_mxfp4_to_int4g128(None, None, 1, 8, 96, None, None, None) == -1

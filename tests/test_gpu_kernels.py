@@ -132,9 +132,8 @@ def _gemm_inputs(seed, sizes, N, K, integer):
 def _run_gemm(lib, a, asc, offsets, w, wsc, epi, block_n):
     G, N, K = w.shape[0], w.shape[1], w.shape[2] * 2
     Rn = a.shape[0]
-    w_t = dev(w)
-    sf = torch.empty((G, N // 128, K // 128, 512), dtype=torch.uint8, device="cuda")
-    lib.moe_prepare_weight_scales(dev(wsc), sf, paired=(epi == lib.MOE_EPI_SWIGLU_QUANT))
+    wp = torch.empty(lib.moe_prepared_weights_size(G, N, K), dtype=torch.uint8, device="cuda")
+    lib.moe_prepare_weights(dev(w), dev(wsc), wp, paired=(epi == lib.MOE_EPI_SWIGLU_QUANT))
     ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
     if epi == lib.MOE_EPI_SWIGLU_QUANT:
         out = torch.empty((Rn, N // 2), dtype=torch.uint8, device="cuda")
@@ -143,7 +142,7 @@ def _run_gemm(lib, a, asc, offsets, w, wsc, epi, block_n):
         out, osc = torch.empty((Rn, N), dtype=torch.float32, device="cuda"), None
     else:
         out, osc = torch.empty((Rn, N), dtype=torch.bfloat16, device="cuda"), None
-    lib.moe_grouped_gemm_mxfp4(dev(a), dev(asc), dev(offsets), w_t, sf, epi, out, osc, ws, 10.0, block_n)
+    lib.moe_grouped_gemm_mxfp4(dev(a), dev(asc), dev(offsets), wp, G, N, epi, out, osc, ws, 10.0, block_n)
     torch.cuda.synchronize()
     return out, osc
 
