@@ -36,6 +36,7 @@ METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s or HBM GB/s vs B200 rooflin
 KERNELS_PER_STEP = 13     # quant 1, route 1, permute 4, gemm 3 + 3, combine 1
 
 WORKLOADS = {
+    "repack": dict(T=0, H=4096, I=2048, E=256, k=6, logits="uniform"),
     "decode": dict(T=64, H=4096, I=2048, E=256, k=6, logits="uniform"),
     "prefill": dict(T=4096, H=4096, I=2048, E=256, k=6, logits="zipf"),
     "long_prefill": dict(T=16384, H=4096, I=2048, E=384, k=6, logits="zipf"),
@@ -187,10 +188,12 @@ def dist_setup(n_gpus: int):
 
 
 def max_over_ranks(value: float, pg) -> float:
+    """The slowest rank's time (every rank gets it); plumbing only."""
     if pg is None:
         return value
     import torch
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
 
@@ -213,6 +216,94 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
                 w13=active * w13 + R * (H + H // 128) + R * (I + I // 128),
                 w2=active * w2 + R * (I + I // 128) + R * H * 4,
                 flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
+
+
+def run_repack(args, wl):
+    """Weight repack sweep: one layer of E experts x (w1, w3 [I, H], w2 [H, I])
+    MXFP4 -> NVFP4 (E4M3 scale per 16, per-matrix global scale) and -> symmetric
+    INT4 group 128 (fp32 scale_inv [N, K/128]).  One step = both repacks of
+    the whole layer.  Metric: GB/s of algorithmic bytes (each repack reads its
+    source once and writes its outputs once)."""
+    import torch
+
+    import synth
+    from fp8_block_scaled_pow2_b200 import moe
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    E, H, I = wl["E"], wl["H"], wl["I"]
+    w13, s13, w2, s2 = synth.expert_weights(args.seed, E, H, I, n_proto=4)
+    # w1 and w3 are separate [I, H] matrices: view w13 [E, 2I, H/2] as [2E, I, H/2]
+    mats = [(torch.from_numpy(w13.reshape(2 * E, I, H // 2)).cuda(), torch.from_numpy(s13.reshape(2 * E, I, H // 32)).cuda()),
+            (torch.from_numpy(w2).cuda(), torch.from_numpy(s2).cuda())]
+    outs = []
+    nv_bytes = int4_bytes = 0
+    for fp4, e8 in mats:
+        M, N, k2 = fp4.shape
+        K = 2 * k2
+        o = dict(nv_fp4=torch.empty_like(fp4), nv_s=torch.empty((M, N, K // 16), dtype=torch.uint8, device="cuda"),
+                 nv_g=torch.empty(M, dtype=torch.float32, device="cuda"),
+                 q=torch.empty((M, N, k2), dtype=torch.int8, device="cuda"),
+                 sinv=torch.empty((M, N, K // 128), dtype=torch.float32, device="cuda"))
+        outs.append(o)
+        nv_bytes += 2 * fp4.numel() + e8.numel() + o["nv_s"].numel() + 4 * M
+        int4_bytes += fp4.numel() + e8.numel() + o["q"].numel() + 4 * o["sinv"].numel()
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        for (fp4, e8), o in zip(mats, outs):
+            moe.repack_mxfp4_to_nvfp4(fp4, e8, o["nv_fp4"], o["nv_s"], o["nv_g"])
+        if ev: ev[1].record(stream)
+        for (fp4, e8), o in zip(mats, outs):
+            moe.repack_mxfp4_to_int4g128(fp4, e8, o["q"], o["sinv"])
+        if ev: ev[2].record(stream)
+
+    clk = ClockSampler(local).start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(pg)
+    torch.cuda.synchronize()
+    w_begin = time.time()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk.mark(w_begin, time.time())
+    clk.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), pg)
+    nv_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    i4_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+    peaks = read_peaks()
+    total = (nv_bytes + int4_bytes) * world * args.steps
+    gbs = total / (ms / 1e3) / 1e9
+    nv_gbs = nv_bytes / (nv_ms / 1e3) / 1e9
+    line = {
+        "metric": "weight repack GB/s vs B200 HBM roofline", "value": round(gbs, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4 "
+                               f"and -> INT4 group 128", "l2": "inputs larger than L2 (3.4 GB per repack)"},
+        "roofline": {"bound": "hbm", "achieved": round(nv_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": round(nv_gbs / peaks["hbm"], 4), "traffic": None, "kernel": "repack_mxfp4_to_nvfp4",
+                     "peak_source": f"{peaks['src']} HBM copy"},
+        "repack": {"nvfp4_ms": round(nv_ms, 4), "nvfp4_GBps": round(nv_gbs, 1),
+                   "int4_ms": round(i4_ms, 4), "int4_GBps": round(int4_bytes / (i4_ms / 1e3) / 1e9, 1),
+                   "nvfp4_bytes": nv_bytes, "int4_bytes": int4_bytes},
+        "gpu_launches": 6 * args.steps,     # per step: 2 x (2 NVFP4 kernels + 1 INT4 kernel)
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
 
 
 def run_ours(args, wl):
@@ -366,10 +457,43 @@ def cpu_baseline(wl, seed, budget_s=15.0, tokens_per_step=None):
             "wall_s": round(time.perf_counter() - t_start, 1)}
 
 
+def run_reference_repack(args, wl):
+    """The oracle's repacks on one expert's three matrices per step."""
+    import synth
+    from oracle import repack as Rp
+    E, H, I = wl["E"], wl["H"], wl["I"]
+    w13, s13, w2, s2 = synth.expert_weights(args.seed, 1, H, I)
+    per = (2 * w13.nbytes + s13.nbytes + 2 * s13.nbytes + 4 * 2) + (2 * w2.nbytes + s2.nbytes + 2 * s2.nbytes + 4) \
+        + (2 * w13.nbytes + s13.nbytes + 4 * w13.nbytes * 2 // 128) + (2 * w2.nbytes + s2.nbytes + 4 * w2.nbytes * 2 // 128)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = time.perf_counter()
+        Rp.repack_mxfp4_to_nvfp4(w13.reshape(2, I, H // 2), s13.reshape(2, I, H // 32))
+        Rp.repack_mxfp4_to_nvfp4(w2, s2)
+        Rp.repack_mxfp4_to_int4g128(w13.reshape(2, I, H // 2), s13.reshape(2, I, H // 32))
+        Rp.repack_mxfp4_to_int4g128(w2, s2)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t)
+    value = per * len(times) / sum(times) / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": "weight repack GB/s vs B200 HBM roofline", "value": round(value, 4),
+        "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * sum(times) / len(times), 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4 "
+                               f"and -> INT4 group 128"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one expert's three matrices per step, {len(times)} steps"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+        flush=True)
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    if args.workload == "repack":
+        return run_reference_repack(args, wl)
     import synth
     from oracle import ffn
     x, logits, (w13, s13, w2, s2) = make_inputs(wl, args.seed, 0)
@@ -415,6 +539,8 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.workload == "repack":
+        run_repack(args, wl)
     else:
         run_ours(args, wl)
 

@@ -21,6 +21,7 @@ SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_version": (_I, []),
     "moe_get_device_error": (_I, [ctypes.POINTER(_I), _P]),
+    "moe_selftest_wait_timeout": (_I, [_I64, _P]),
     "moe_quantize_act_fp8": (_I, [_P, _I, _I, _P, _P, _P]),
     "moe_route_topk": (_I, [_P, _I, _I, _I, _F, _I, _P, _P, _P]),
     "moe_permute_workspace_size": (_SZ, [_I, _I, _I]),

@@ -126,9 +126,29 @@ int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& 
   return launch_status();
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that no
+// one arrives at; the wait gives up after timeout_ns and records
+// MOE_ERR_TIMEOUT in the device error word.
+__global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  sm100::mbar_init(&bar, 1);
+  abort_flag = 0;
+  sm100::fence_mbar_init();
+  __syncwarp();
+  volatile int* ab = &abort_flag;
+  if (sm100::mbar_wait(&bar, 0, ab, timeout_ns)) record_error(MOE_ERR_INVALID);   // cannot complete
+}
+
 }  // namespace
 
 extern "C" {
+
+int moe_selftest_wait_timeout(int64_t timeout_ns, void* stream) {
+  if (timeout_ns <= 0 || timeout_ns > 2000000000LL) return MOE_ERR_INVALID;
+  wait_timeout_selftest_kernel<<<1, 1, 0, S(stream)>>>((uint64_t)timeout_ns);
+  return launch_status();
+}
 
 const char* moe_status_string(int s) {
   switch (s) {

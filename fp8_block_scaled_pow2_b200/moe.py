@@ -56,6 +56,10 @@ def moe_get_device_error(stream=None) -> int:
     return code.value
 
 
+def moe_selftest_wait_timeout(timeout_ns: int, stream=None):
+    _check("moe_selftest_wait_timeout", _lib().moe_selftest_wait_timeout(int(timeout_ns), _stream(stream)))
+
+
 def moe_quantize_act_fp8(x, xq, sx, stream=None):
     rows, cols = x.shape
     _check("moe_quantize_act_fp8",

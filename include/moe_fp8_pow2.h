@@ -77,6 +77,15 @@ int moe_version(void);
 int moe_get_device_error(int* code, void* stream);
 
 /*
+ * Failure-detection self-test (no counterpart on the source pages): launches
+ * one thread that waits on a barrier nothing ever arrives at, using the same
+ * bounded wait as the GEMM pipelines with a limit of timeout_ns (0 <
+ * timeout_ns <= 2 s).  The wait gives up, the kernel records MOE_ERR_TIMEOUT
+ * in the device error word and exits; the CUDA context stays usable.
+ */
+int moe_selftest_wait_timeout(int64_t timeout_ns, void* stream);
+
+/*
  * a1 -- activation quantisation [SI 低精度计算, 模型训练].
  * For each row and each group of 128 columns: amax = max |x|;
  * k = ceil(log2(amax / 448)) with amax / 448 a float32 round-to-nearest-even
