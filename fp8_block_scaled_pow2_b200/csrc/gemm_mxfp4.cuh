@@ -37,7 +37,6 @@ namespace gemm {
 using namespace sm100;
 
 constexpr int kThreads = 352;                   // 11 warps: producer, 2 MMA issuers, 8 workers
-constexpr int kPrefetchStages = 0;              // default L2 prefetch run-ahead (K steps)
 
 // Prepared weights (moe_prepare_weights): one 8704-byte block per (128-row
 // block, 128-wide K step): 128 rows x 64 bytes of packed E2M1 nibbles, then
@@ -272,7 +271,6 @@ struct GemmArgs {
   void* out;
   uint8_t* out_scale;
   float limit;
-  int prefetch;           // L2 prefetch run-ahead in K steps
 };
 
 // Epilogue of one work item for one epilogue warp: copy the warp's slice of
@@ -351,10 +349,11 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
   }
 }
 
-// One MMA-issuing thread.  Every value that does not change within an item
-// is computed before its K loop; per-K-block operands are constant offsets of
-// per-stage bases (a descriptor's start-address field is the byte address /
-// 16, so +32 bytes is +2).
+// One MMA-issuing warp: the whole warp runs the loop and waits, one elected
+// lane issues the scale copies, MMAs and commits.  Every value that does not
+// change within an item is computed before its K loop; per-K-block operands
+// are constant offsets of per-stage bases (a descriptor's start-address field
+// is the byte address / 16, so +32 bytes is +2).
 template <int BN, bool DUAL>
 __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const uint32_t tmem, uint64_t* full,
                                            uint64_t* pad_full, uint64_t* empty, uint64_t* acc_full,
@@ -374,7 +373,7 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
     uint32_t id_kb[4];
 #pragma unroll
     for (int kb = 0; kb < 4; ++kb) id_kb[kb] = idesc_with_sf_ids(idesc, kb, 0);
-    if (!mbar_wait(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) return;
+    if (!mbar_wait_warp(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) return;
     tc_fence_after();
     const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
     for (int kt = 0; kt < KT; ++kt, ++n) {
@@ -383,39 +382,43 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
         uint32_t a_base;
         if constexpr (C::STAGED) {
           // the converters waited for this step's loads before filling pad slot n % 2
-          if (!mbar_wait(&pad_full[n & 1u], (n >> 1) & 1u, abort_flag)) return;
+          if (!mbar_wait_warp(&pad_full[n & 1u], (n >> 1) & 1u, abort_flag)) return;
           a_base = pad0 + (n & 1u) * C::PAD_STAGE;
         } else {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) return;
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) return;
           a_base = ring0 + stage * C::STAGE;
         }
         if (DUAL) a_base += iss * C::A_BYTES;
         const uint32_t st = ring0 + stage * C::STAGE;
-        tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SFA_STRIDE : 0)));
-        if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SFA_STRIDE));
-        if ((kt & 3) == (DUAL || C::ISSUERS == 1 ? 0 : iss)) {
-#pragma unroll
-          for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
-        }
         const uint32_t bsel = (uint32_t)(kt & 3);
         const uint32_t sfb = sfb_t | (bsel << 30);
         const uint64_t da = sdesc_kmajor_sw128(a_base);
         const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
         // this issuer's first step of the item starts a fresh accumulator
         const uint32_t first = (DUAL || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
+        if (elect_one()) {
+          tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SFA_STRIDE : 0)));
+          if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SFA_STRIDE));
+          if ((kt & 3) == (DUAL || C::ISSUERS == 1 ? 0 : iss)) {
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          mma_mxf8f6f4(d, da + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4), sfa_t | ((uint32_t)kb << 30), sfb,
-                       kb ? 1u : first);
-          if (C::TILES_PER_ISSUER == 2)
-            mma_mxf8f6f4(d + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4),
-                         (sfa_t + 4) | ((uint32_t)kb << 30), sfb, kb ? 1u : first);
+            for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
+          }
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            mma_mxf8f6f4(d, da + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4), sfa_t | ((uint32_t)kb << 30), sfb,
+                         kb ? 1u : first);
+            if (C::TILES_PER_ISSUER == 2)
+              mma_mxf8f6f4(d + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4),
+                           (sfa_t + 4) | ((uint32_t)kb << 30), sfb, kb ? 1u : first);
+          }
+          tc_commit(&empty[stage]);
         }
-        tc_commit(&empty[stage]);
+        __syncwarp();
       }
       if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
     }
-    tc_commit(&acc_full[ab]);
+    if (elect_one()) tc_commit(&acc_full[ab]);
+    __syncwarp();
     acc_bits ^= 1u << ab;
     if (C::ACC_BUFS == 2) ab ^= 1u;
   }
@@ -482,37 +485,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
-    if (lane == 0) {
-      // optional L2 prefetch stream running args.prefetch K steps ahead of the loads
-      int pf_item = blockIdx.x, pf_kt = 0;
-      Item pf_it{};
-      if (pf_item < n_items && args.prefetch > 0)
-        pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
-      auto prefetch_next = [&]() {
-        if (args.prefetch <= 0 || pf_item >= n_items) return;
-        const size_t pblk = (DUAL ? ((size_t)(pf_it.g * n_ft + pf_it.ft) * KT) * 2
-                                  : (size_t)(pf_it.g * rb_per_g + pf_it.ft) * KT) + (size_t)pf_kt * C::NUM_A;
-        bulk_prefetch(args.w + pblk * kWBlock, C::NUM_A * kWBlock);
-        if (++pf_kt == KT) {
-          pf_kt = 0;
-          pf_item += gridDim.x;
-          if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        }
-      };
-      for (int i = 0; i < args.prefetch; ++i) prefetch_next();
-
-      uint32_t stage = 0, phase = 0;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        const int rb0 = it.g * rb_per_g + it.ft;
-        const int rb1 = rb0 + rb_per_g / 2;
-        // first prepared block of this item's weight tile(s); per K step the
-        // blocks of gate and up (DUAL, paired order) or of the tile are adjacent
-        const size_t blk0 = DUAL ? ((size_t)(it.g * n_ft + it.ft) * KT) * 2 : (size_t)rb0 * KT;
-        const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
-        bool ok = true;
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+    // The whole warp walks the items (its coordinates stay warp-uniform); one
+    // elected lane issues each step's copies.
+    uint32_t stage = 0, phase = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const int rb0 = it.g * rb_per_g + it.ft;
+      // first prepared block of this item's weight tile(s); per K step the
+      // blocks of gate and up (DUAL, paired order) or of the tile are adjacent
+      const size_t blk0 = DUAL ? ((size_t)(it.g * n_ft + it.ft) * KT) * 2 : (size_t)rb0 * KT;
+      const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (elect_one()) {
           uint8_t* st = smem + stage * C::STAGE;
           // token scales: one block per 4 K steps, read by each issuer at its
           // first step of the group (issuers alternate steps without DUAL)
@@ -530,20 +516,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
-          prefetch_next();
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
+      if (!ok) break;
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer 0 ---------------------------
-    if (lane == 0) mma_issuer<BN, DUAL>(0, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag,
-                                        s_prefix, s_tstart, args, n_items, KT, n_ft);
+    mma_issuer<BN, DUAL>(0, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag, s_prefix, s_tstart,
+                         args, n_items, KT, n_ft);
   } else if (warp == kThreads / 32 - 1) {
     // ------------------------------ MMA issuer 1 ---------------------------
-    if (lane == 0 && C::ISSUERS == 2) mma_issuer<BN, DUAL>(1, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag,
-                                        s_prefix, s_tstart, args, n_items, KT, n_ft);
+    if (C::ISSUERS == 2)
+      mma_issuer<BN, DUAL>(1, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag, s_prefix,
+                           s_tstart, args, n_items, KT, n_ft);
   } else if (C::STAGED && warp < C::EPI_FIRST) {
     // ------------------------------ converters ----------------------------
     // Spread packed nibbles (64 B per weight row) into the MMA's layout:

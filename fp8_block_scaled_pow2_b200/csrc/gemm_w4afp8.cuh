@@ -88,7 +88,6 @@ struct W4Args {
   void* out;
   uint8_t* out_scale;
   float limit;
-  int prefetch;           // L2 prefetch run-ahead in K steps
 };
 
 template <int BN, bool DUAL, int EPI>
@@ -149,38 +148,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
-    if (lane == 0) {
-      const int rb_per_g = N / 128;
-      // L2 prefetch stream running kPrefetchStages stages ahead of the loads
-      int pf_item = blockIdx.x, pf_kt = 0;
-      Item pf_it{};
-      if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
-      auto prefetch_next = [&]() {
-        if (pf_item >= n_items) return;
-        const int rb0 = pf_it.g * rb_per_g + pf_it.ft;
-        if (pf_kt == 0) {                 // the item's float32 scales: 128 rows x KT, contiguous
-          bulk_prefetch(args.w_sinv + (size_t)rb0 * 128 * KT, 128 * KT * 4);
-          if (DUAL) bulk_prefetch(args.w_sinv + (size_t)(rb0 + rb_per_g / 2) * 128 * KT, 128 * KT * 4);
-        }
-        tma_prefetch_2d(&tmA, pf_kt * 64, rb0 * 128);
-        if (DUAL) tma_prefetch_2d(&tmA, pf_kt * 64, (rb0 + rb_per_g / 2) * 128);
-        tma_prefetch_2d(&tmB, pf_kt * 128, pf_it.row0);
-        if (++pf_kt == KT) {
-          pf_kt = 0;
-          pf_item += gridDim.x;
-          if (pf_item < n_items) pf_it = decode_item(pf_item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        }
-      };
-      for (int i = 0; i < args.prefetch; ++i) prefetch_next();
-      uint32_t stage = 0, phase = 0;
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        const int rb0 = it.g * rb_per_g + it.ft;
-        const int rb1 = rb0 + rb_per_g / 2;
-        const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
-        bool ok = true;
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+    // The whole warp walks the items; one elected lane issues the copies.
+    const int rb_per_g = N / 128;
+    uint32_t stage = 0, phase = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const int rb0 = it.g * rb_per_g + it.ft;
+      const int rb1 = rb0 + rb_per_g / 2;
+      const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
+      bool ok = true;
+      for (int kt = 0; kt < KT; ++kt) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (elect_one()) {
           uint8_t* st = smem + stage * C::STAGE;
           const bool new_group = (kt & 3) == 0;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
@@ -188,36 +167,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (DUAL) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, &tmA, kt * 64, rb1 * 128, &full[stage]);
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
-          prefetch_next();
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
+      if (!ok) break;
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------
-    if (lane == 0) {
-      const uint32_t sfa_smem = smem_u32(smem + C::SFA_SMEM_OFF);
-      tmem_cp_32x128b_warpx4(tmem + C::SFA_COL, sdesc_sf(sfa_smem));
-      uint32_t stage = 0, phase = 0;
-      uint32_t pb = 0, pbits = 0;            // bit b: phase of partial buffer b
-      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
-        const int n_mma = max(16, (it.rows + 15) & ~15);
-        const uint32_t idesc = idesc_mxf8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
-        bool ok = true;
-        for (int kt = 0; kt < KT && ok; ++kt) {
-          if (!mbar_wait(&pempty[pb], ((pbits >> pb) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();     // orders the MMA after the promotion warps' release of the partial buffer
-          const uint32_t st = smem_u32(smem + stage * C::STAGE);
+    // The whole warp runs the loop and waits; one elected lane issues.
+    const uint32_t sfa_smem = smem_u32(smem + C::SFA_SMEM_OFF);
+    if (elect_one()) tmem_cp_32x128b_warpx4(tmem + C::SFA_COL, sdesc_sf(sfa_smem));
+    __syncwarp();
+    uint32_t stage = 0, phase = 0;
+    uint32_t pb = 0, pbits = 0;            // bit b: phase of partial buffer b
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const int n_mma = max(16, (it.rows + 15) & ~15);
+      const uint32_t idesc = idesc_mxf8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
+      bool ok = true;
+      for (int kt = 0; kt < KT && ok; ++kt) {
+        if (!mbar_wait_warp(&pempty[pb], ((pbits >> pb) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&conv[stage], phase, abort_flag)) { ok = false; break; }
+        tc_fence_after();     // orders the MMA after the promotion warps' release of the partial buffer
+        const uint32_t st = smem_u32(smem + stage * C::STAGE);
+        const uint32_t dcol = tmem + pb * C::P_COLS;
+        const uint32_t kb_b = (uint32_t)(kt & 3);
+        if (elect_one()) {
           if ((kt & 3) == 0) {
 #pragma unroll
             for (int a = 0; a < C::NA; ++a)
               tmem_cp_32x128b_warpx4(tmem + C::SFB_COL + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
           }
-          const uint32_t dcol = tmem + pb * C::P_COLS;
-          const uint32_t kb_b = (uint32_t)(kt & 3);
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             const uint32_t id = idesc_with_sf_ids(idesc, kb, kb_b);
@@ -231,12 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(&empty[stage]);
           tc_commit(&pfull[pb]);
-          pbits ^= 1u << pb;
-          pb ^= 1u;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        __syncwarp();
+        pbits ^= 1u << pb;
+        pb ^= 1u;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
+      if (!ok) break;
     }
   } else if (warp < 6) {
     // ------------------------------ converters ----------------------------

@@ -59,18 +59,6 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// L2 prefetch run-ahead of the grouped GEMMs in 128-wide K steps; the
-// environment variable MOE_GEMM_PREFETCH overrides the default (tuning).
-int prefetch_steps() {
-  static int v = [] {
-    const char* e = getenv("MOE_GEMM_PREFETCH");
-    const int d = gemm::kPrefetchStages;
-    if (!e) return d;
-    const int x = atoi(e);
-    return (x >= 0 && x <= 256) ? x : d;
-  }();
-  return v;
-}
 
 // 3-D tiled map (inner dimension first) over equally spaced 2-D blocks.
 bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -305,7 +293,6 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   args.out = out;
   args.out_scale = out_scale;
   args.limit = swiglu_limit;
-  args.prefetch = prefetch_steps();
 
   cudaStream_t st = S(stream);
   const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
@@ -362,7 +349,6 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
   args.out = out;
   args.out_scale = out_scale;
   args.limit = swiglu_limit;
-  args.prefetch = prefetch_steps();
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
   gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),

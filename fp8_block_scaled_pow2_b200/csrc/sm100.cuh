@@ -61,6 +61,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait run by every lane of a converged warp; the result is the same in
+// all lanes (false if any lane gave up), so the warp stays converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t timeout_ns = kWaitTimeoutNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, timeout_ns);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+// One lane of a fully active warp (the lowest, so the same lane on every
+// call).  Issue loops run converged on the whole warp, which keeps their
+// descriptors and coordinates warp-uniform, and only the elected lane issues
+// the tensor-core and TMA instructions: a loop confined to a single lane
+// issues them far more slowly.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -181,8 +181,10 @@ def test_gemm_random_scaled(lib, block_n):
 
 
 def _swiglu_ok(hq, sh, gu_ref, I, limit=10.0):
-    """Codes equal the oracle's, except where the oracle's h lies within a few
-    float32 ulps of a rounding boundary (h itself comes from libm expf)."""
+    """Codes equal the oracle's, except where the oracle's h lies within 24
+    float32 ulps of a rounding boundary: the kernels' silu uses the hardware
+    exponential (at most 13 ulp on |g| <= 10) and the approximate divide
+    (2 ulp), about 16 ulp in all, and the pages fix no precision for it."""
     q_ref, s_ref = ffn.swiglu_quant(gu_ref, I, limit)
     h = ffn.swiglu_clamp(gu_ref, I, limit)
     k = np.repeat(s_ref.astype(np.int64) - 127, 128, axis=1)
@@ -192,7 +194,7 @@ def _swiglu_ok(hq, sh, gu_ref, I, limit=10.0):
         lo = np.abs(F.decode_e4m3(q_ref[bad]))
         hi = np.abs(F.decode_e4m3(hq[bad]))
         mid = (lo + hi) / 2
-        assert (np.abs(y - mid) <= 8 * np.spacing(np.float32(y)).astype(np.float64) * 2).all(), (y, lo, hi)
+        assert (np.abs(y - mid) <= 24 * np.spacing(np.float32(y)).astype(np.float64)).all(), (y, lo, hi)
         assert bad.mean() < 1e-3
     sbad = sh != s_ref
     assert sbad.mean() < 1e-3
