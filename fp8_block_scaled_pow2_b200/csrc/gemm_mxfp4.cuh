@@ -18,14 +18,18 @@
 // are ordered group-major, then weight tile, then token tile, so CTAs running
 // at the same time stream the same weight tile from L2.
 //
-// CTA roles (persistent kernel, one CTA per SM, 6 warps):
-//   warp 0        TMA producer: weight tiles (FP4 unpacked to bytes in shared
-//                 memory by the 16U4_ALIGN16B tensor-map type), token tile, and
-//                 the pre-interleaved scale-factor blocks (1-D bulk copies)
-//   warp 1        TMEM owner and MMA issuer (one thread): scale factors
-//                 shared -> TMEM (tcgen05.cp), 4 MMAs of K = 32 per stage
-//   warps 2..5    epilogue: TMEM -> registers -> global (float32 / bf16 /
+// CTA roles (persistent kernel, one CTA per SM, 11 warps):
+//   warp 0        TMA producer: weight tiles (FP4 unpacked to one nibble per
+//                 byte in shared memory by the 16U4_ALIGN16B tensor-map type),
+//                 token tile, and the pre-interleaved scale blocks (1-D bulk
+//                 copies)
+//   warp 1        TMEM owner and MMA issuer 0: scale factors shared -> TMEM
+//                 (tcgen05.cp), 4 MMAs of K = 32 per 128-wide K step
+//   warp 10       MMA issuer 1 (narrow token tiles, see Cfg::ISSUERS)
+//   warps 2..9    epilogue: TMEM -> registers -> global (float32 / bf16 /
 //                 SwiGLU + per-128 FP8 requantisation)
+// The producer and issuer loops run converged on their whole warp and one
+// elected lane issues the copies and tensor-core instructions.
 #pragma once
 
 #include "common.cuh"
@@ -44,43 +48,33 @@ constexpr int kThreads = 352;                   // 11 warps: producer, 2 MMA iss
 // the gate block and the matching up block of each K step are adjacent.
 constexpr int kWBlock = 8192 + 512;
 
-// Two shared-memory pipelines:
-//  * direct (BN >= 64): a 3-D TMA copy writes the weight tile straight into
-//    the unpacked one-nibble-per-byte layout the MMA reads (16U4_ALIGN16B);
-//    8 epilogue warps.
-//  * staged (BN <= 32, weight streaming): one bulk copy brings the packed
-//    blocks (nibbles + scales, half the bytes of the unpacked tile) into a
-//    deep ring; 4 converter warps spread the nibbles into a 2-slot ring of
-//    MMA-ready tiles just in time; 4 epilogue warps.
+// Pipeline: per 128-wide K step a 3-D TMA copy writes each weight tile
+// straight into the unpacked one-nibble-per-byte layout the MMA reads
+// (16U4_ALIGN16B), a 1-D bulk copy brings its 512-byte scale block, a 2-D TMA
+// copy the token tile, and every fourth step a bulk copy the token scales.
 template <int BN, bool DUAL>
 struct Cfg {
-  static constexpr bool STAGED = BN <= 32;
   static constexpr int NA = (BN + 127) / 128;            // 128-row scale blocks of the token tile
   static constexpr int NUM_A = DUAL ? 2 : 1;
   static constexpr int A_BYTES = 128 * 128;              // one MMA-ready FP4 weight tile
   static constexpr int A_PACKED = 128 * 64;              // the same tile packed (global layout)
   static constexpr int B_BYTES = BN * 128;
   static constexpr int SF_BYTES = 512;
-  // ring slot, direct: [unpacked weight tiles][token tile][weight scales][token scales]
-  //            staged: [prepared weight blocks (nibbles + scales)][token tile][token scales]
-  static constexpr int A_SLOT = STAGED ? kWBlock : A_BYTES;
+  // ring slot: [unpacked weight tiles][token tile][weight scales][token scales]
   static constexpr int A0_OFF = 0;
-  static constexpr int B_OFF = (NUM_A * A_SLOT + 1023) / 1024 * 1024;
-  static constexpr int SFA_OFF = STAGED ? 8192 : B_OFF + B_BYTES;       // weight scales of tile a:
-  static constexpr int SFA_STRIDE = STAGED ? kWBlock : SF_BYTES;       //   SFA_OFF + a * SFA_STRIDE
-  static constexpr int SFB_OFF = STAGED ? B_OFF + B_BYTES : SFA_OFF + NUM_A * SF_BYTES;
+  static constexpr int B_OFF = NUM_A * A_BYTES;
+  static constexpr int SFA_OFF = B_OFF + B_BYTES;          // weight scales of tile a: SFA_OFF + a * SF_BYTES
+  static constexpr int SFB_OFF = SFA_OFF + NUM_A * SF_BYTES;
   static constexpr int STAGE_RAW = SFB_OFF + NA * SF_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int PAD_SLOTS = STAGED ? 2 : 0;       // MMA-ready tiles (staged mode)
-  static constexpr int PAD_STAGE = NUM_A * A_BYTES;
-  static constexpr int RING_BUDGET = 200 * 1024 - PAD_SLOTS * PAD_STAGE;
+  static constexpr int RING_BUDGET = 200 * 1024;
   static constexpr int STAGES_FIT = RING_BUDGET / STAGE;
   static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
-  static constexpr int TX = STAGED ? NUM_A * kWBlock + B_BYTES
-                                   : NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;   // + token scales, see below
-  static constexpr int PAD_OFF = STAGES * STAGE;
-  // MMA issue: a single thread issuing small-N MMAs is bound by its own issue
-  // latency, so narrow tiles use two issuing threads.  With gate and up (DUAL)
+  // transaction bytes of a step (the TMA counts the packed weight bytes);
+  // steps that also load token scales add NA * 512
+  static constexpr int TX = NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;
+  // MMA issue: one warp issuing small-N MMAs is bound by its own issue
+  // latency, so narrow tiles use two issuing warps.  With gate and up (DUAL)
   // issuer 0 computes the gate tile and issuer 1 the up tile; otherwise they
   // take alternate K steps into two partial accumulators the epilogue adds.
   // Wide gate/up tiles keep one issuer (its gate and up MMAs share the token
@@ -99,11 +93,11 @@ struct Cfg {
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   // epilogue warps: each owns 32 weight rows (its TMEM sub-partition) and
   // BN / (EPI_WARPS / 4) token columns
-  static constexpr int EPI_WARPS = STAGED ? 4 : 8;
-  static constexpr int EPI_FIRST = STAGED ? 6 : 2;        // warps 2..5 convert in staged mode
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_FIRST = 2;
   static constexpr int CW = BN / (EPI_WARPS / 4);
-  // shared memory after the rings
-  static constexpr int BAR_OFF = PAD_OFF + PAD_SLOTS * PAD_STAGE;
+  // shared memory after the ring
+  static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int RED_OFF = BAR_OFF + 512;
   static constexpr int PREFIX_OFF = RED_OFF + 2 * 4 * CW * 4;     // group item prefix, int32[G+1]
   static constexpr int TSTART_OFF = PREFIX_OFF + 4 * 1028;        // first token tile per group, int32[G]
@@ -111,8 +105,7 @@ struct Cfg {
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;     // slack for 1024-byte alignment
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few pipeline stages");
-  static_assert(2 * STAGES + 2 * PAD_SLOTS + 4 <= 64, "barrier area overflow");
-  static_assert(!STAGED || STAGES > PAD_SLOTS, "converters reuse the ring's empty barriers");
+  static_assert(2 * STAGES + 4 + 1 <= 64, "barrier area overflow");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
   static_assert(SMEM_ALLOC > 116 * 1024, "one CTA per SM keeps tensor-memory allocation uncontended");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "bad token tile");
@@ -356,16 +349,15 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
 // is the byte address / 16, so +32 bytes is +2).
 template <int BN, bool DUAL>
 __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const uint32_t tmem, uint64_t* full,
-                                           uint64_t* pad_full, uint64_t* empty, uint64_t* acc_full,
+                                           uint64_t* empty, uint64_t* acc_full,
                                            uint64_t* acc_empty, volatile int* abort_flag, const int* s_prefix,
                                            const int* s_tstart, const GemmArgs& args, const int n_items,
                                            const int KT, const int n_ft) {
   using C = Cfg<BN, DUAL>;
   const uint32_t ring0 = smem_u32(smem);
-  const uint32_t pad0 = smem_u32(smem + C::PAD_OFF);
   const uint32_t sfa_t = tmem + C::SF_COL + iss * C::SF_SET;     // 4 columns per weight tile
   const uint32_t sfb_t = sfa_t + 4 * C::TILES_PER_ISSUER;
-  uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0, n = 0;
+  uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, args.G, n_ft);
     const int n_mma = max(16, (it.rows + 15) & ~15);
@@ -376,20 +368,12 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
     if (!mbar_wait_warp(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) return;
     tc_fence_after();
     const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
-    for (int kt = 0; kt < KT; ++kt, ++n) {
+    for (int kt = 0; kt < KT; ++kt) {
       const bool mine = DUAL || C::ISSUERS == 1 || (kt & 1) == iss;
       if (mine) {
-        uint32_t a_base;
-        if constexpr (C::STAGED) {
-          // the converters waited for this step's loads before filling pad slot n % 2
-          if (!mbar_wait_warp(&pad_full[n & 1u], (n >> 1) & 1u, abort_flag)) return;
-          a_base = pad0 + (n & 1u) * C::PAD_STAGE;
-        } else {
-          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) return;
-          a_base = ring0 + stage * C::STAGE;
-        }
-        if (DUAL) a_base += iss * C::A_BYTES;
+        if (!mbar_wait_warp(&full[stage], phase, abort_flag)) return;
         const uint32_t st = ring0 + stage * C::STAGE;
+        const uint32_t a_base = st + (DUAL ? iss * C::A_BYTES : 0);
         const uint32_t bsel = (uint32_t)(kt & 3);
         const uint32_t sfb = sfb_t | (bsel << 30);
         const uint64_t da = sdesc_kmajor_sw128(a_base);
@@ -397,8 +381,8 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
         // this issuer's first step of the item starts a fresh accumulator
         const uint32_t first = (DUAL || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
         if (elect_one()) {
-          tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SFA_STRIDE : 0)));
-          if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SFA_STRIDE));
+          tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SF_BYTES : 0)));
+          if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SF_BYTES));
           if ((kt & 3) == (DUAL || C::ISSUERS == 1 ? 0 : iss)) {
 #pragma unroll
             for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
@@ -434,8 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~(uintptr_t)1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* pad_full = empty + C::STAGES;       // [PAD_SLOTS] (staged mode)
-  uint64_t* acc_full = pad_full + 2;            // [ACC_BUFS]
+  uint64_t* acc_full = empty + C::STAGES;       // [ACC_BUFS]
   uint64_t* acc_empty = acc_full + 2;           // [ACC_BUFS]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -453,11 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_prefix[g] = args.prefix[g];
     if (g < G) s_tstart[g] = args.tstart[g];
   }
-  if constexpr (C::STAGED) {      // padding halves of the MMA-ready tiles stay zero
-    for (int i = threadIdx.x; i < C::PAD_SLOTS * C::PAD_STAGE / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(smem + C::PAD_OFF)[i] = make_uint4(0u, 0u, 0u, 0u);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -465,7 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], C::CONSUMERS);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&pad_full[b], 128);
       mbar_init(&acc_full[b], C::ISSUERS);
       mbar_init(&acc_empty[b], 32 * C::EPI_WARPS);
     }
@@ -505,14 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool new_group = (DUAL || C::ISSUERS == 1) ? (kt & 3) == 0 : (kt & 3) < 2;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
           const size_t blk = blk0 + (size_t)kt * C::NUM_A;
-          if constexpr (C::STAGED) {
-            bulk_load(st + C::A0_OFF, args.w + blk * kWBlock, C::NUM_A * kWBlock, &full[stage]);
-          } else {
 #pragma unroll
-            for (int a = 0; a < C::NUM_A; ++a) {
-              tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)(blk + a), &full[stage]);
-              bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + (blk + a) * kWBlock + 8192, 512, &full[stage]);
-            }
+          for (int a = 0; a < C::NUM_A; ++a) {
+            tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)(blk + a), &full[stage]);
+            bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + (blk + a) * kWBlock + 8192, 512, &full[stage]);
           }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
@@ -524,54 +497,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer 0 ---------------------------
-    mma_issuer<BN, DUAL>(0, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag, s_prefix, s_tstart,
+    mma_issuer<BN, DUAL>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, s_prefix, s_tstart,
                          args, n_items, KT, n_ft);
   } else if (warp == kThreads / 32 - 1) {
     // ------------------------------ MMA issuer 1 ---------------------------
     if (C::ISSUERS == 2)
-      mma_issuer<BN, DUAL>(1, smem, tmem, full, pad_full, empty, acc_full, acc_empty, abort_flag, s_prefix,
+      mma_issuer<BN, DUAL>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, s_prefix,
                            s_tstart, args, n_items, KT, n_ft);
-  } else if (C::STAGED && warp < C::EPI_FIRST) {
-    // ------------------------------ converters ----------------------------
-    // Spread packed nibbles (64 B per weight row) into the MMA's layout:
-    // every 8 packed bytes start a 16-byte chunk, chunks 128-byte swizzled.
-    // warp w (0..3), lane l: 16-byte input chunk (l & 3) of rows
-    // w*8 + (l >> 2) + 32 j: conflict-free reads and writes.
-    const int w = warp - 2;
-    const int chunk = lane & 3;
-    uint32_t stage = 0, phase = 0, ps = 0;
-    uint32_t n = 0;                           // running K-step count of this CTA
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      bool ok = true;
-      for (int kt = 0; kt < KT; ++kt, ++n) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-        if (n >= (uint32_t)C::PAD_SLOTS) {
-          // pad slot ps was last read by the MMAs of step n - PAD_SLOTS; the
-          // ring's empty barrier of that step completes when they are done
-          const uint32_t m = n - C::PAD_SLOTS;
-          if (!mbar_wait(&empty[m % C::STAGES], (m / C::STAGES) & 1u, abort_flag)) { ok = false; break; }
-        }
-        const uint8_t* raw = smem + stage * C::STAGE + C::A0_OFF;
-        uint8_t* dst = smem + C::PAD_OFF + ps * C::PAD_STAGE;
-#pragma unroll
-        for (int a = 0; a < C::NUM_A; ++a) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = w * 8 + (lane >> 2) + 32 * j;
-            const uint4 in = *reinterpret_cast<const uint4*>(raw + a * kWBlock + r * 64 + chunk * 16);
-            const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
-            uint8_t* row = dst + a * C::A_BYTES + r * 128;
-            *reinterpret_cast<uint2*>(row + ((c0 ^ (r & 7)) << 4)) = make_uint2(in.x, in.y);
-            *reinterpret_cast<uint2*>(row + ((c1 ^ (r & 7)) << 4)) = make_uint2(in.z, in.w);
-          }
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&pad_full[ps]);
-        ps ^= 1u;
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) break;
-    }
   } else {
     // ------------------------------ epilogue ------------------------------
     const int e = warp - C::EPI_FIRST;

@@ -269,8 +269,8 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
 
   CUtensorMap ta, tb;
-  // weight tiles of the direct pipeline: 3-D view [blocks][128 rows][128 nibbles]
-  // of the prepared blocks (the staged pipeline copies whole blocks instead)
+  // weight tiles: 3-D view [blocks][128 rows][128 nibbles] of the prepared
+  // blocks (the scale block that ends each prepared block is a bulk copy)
   const uint64_t n_blocks = (uint64_t)n_groups * (N / 128) * (K / 128);
   if (!make_map_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_prepared, 128, 128, n_blocks, 64,
                    (uint64_t)gemm::kWBlock, 128, 128))
