@@ -48,6 +48,11 @@ constexpr int kThreads = 352;                   // 11 warps: producer, 2 MMA iss
 // the gate block and the matching up block of each K step are adjacent.
 constexpr int kWBlock = 8192 + 512;
 
+// Groups per call (one plan thread per group) and the shared-memory copy of
+// the plan: prefix [G + 1], tstart [G], groups [G].
+constexpr int kMaxGroups = 1024;
+constexpr int kPlanSmemBytes = 16 * (kMaxGroups + 4);
+
 // Pipeline: per 128-wide K step a 3-D TMA copy writes each weight tile
 // straight into the unpacked one-nibble-per-byte layout the MMA reads
 // (16U4_ALIGN16B), a 1-D bulk copy brings its 512-byte scale block, a 2-D TMA
@@ -67,7 +72,10 @@ struct Cfg {
   static constexpr int SFB_OFF = SFA_OFF + NUM_A * SF_BYTES;
   static constexpr int STAGE_RAW = SFB_OFF + NA * SF_BYTES;
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int RING_BUDGET = 200 * 1024;
+  // the ring takes the shared memory the rest of the kernel leaves (227 KB
+  // per CTA; barriers, SwiGLU reduction, plan and alignment slack)
+  static constexpr int CW0 = BN / 2;                     // epilogue columns per warp, see CW
+  static constexpr int RING_BUDGET = 227 * 1024 - (512 + 2 * 4 * CW0 * 4 + kPlanSmemBytes + 1024);
   static constexpr int STAGES_FIT = RING_BUDGET / STAGE;
   static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
   // transaction bytes of a step (the TMA counts the packed weight bytes);
@@ -96,12 +104,12 @@ struct Cfg {
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_FIRST = 2;
   static constexpr int CW = BN / (EPI_WARPS / 4);
+  static_assert(CW == CW0, "ring budget assumes 8 epilogue warps");
   // shared memory after the ring
   static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int PREFIX_OFF = RED_OFF + 2 * 4 * CW * 4;     // group item prefix, int32[G+1]
-  static constexpr int TSTART_OFF = PREFIX_OFF + 4 * 1028;        // first token tile per group, int32[G]
-  static constexpr int SMEM_USED = TSTART_OFF + 4 * 1028;
+  static constexpr int PLAN_OFF = RED_OFF + 2 * 4 * CW * 4;       // SmemPlan (kPlanSmemBytes)
+  static constexpr int SMEM_USED = PLAN_OFF + kPlanSmemBytes;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;     // slack for 1024-byte alignment
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few pipeline stages");
@@ -116,11 +124,12 @@ struct Cfg {
 //   header   int32[4]: n_items, n_tiles, n_ft, BN
 //   prefix   int32[G+1]: first work item of each group
 //   tstart   int32[G]:   first token tile of each group
+//   groups   int2[G]:    (first row, rows) of each group, rows 0 for an invalid group
 //   tiles    int2[max_tiles]: (first row, rows) of each token tile
 //   a_sf     uint8[max_tiles * KG * NA * 512]: per-tile activation scales, interleaved
 //            for tensor memory, four 128-wide K steps per 512-byte block (KG = ceil(KT/4))
 struct WsLayout {
-  size_t header, prefix, tstart, tiles, a_sf, total;
+  size_t header, prefix, tstart, groups, tiles, a_sf, total;
   int max_tiles;
 };
 
@@ -133,7 +142,8 @@ inline WsLayout ws_layout(int a_rows, int G, int K, int BN) {
   L.header = 0;
   L.prefix = align256(16);
   L.tstart = L.prefix + align256(4 * (size_t)(G + 1));
-  L.tiles = L.tstart + align256(4 * (size_t)G);
+  L.groups = L.tstart + align256(4 * (size_t)G);
+  L.tiles = L.groups + align256(8 * (size_t)G);
   L.a_sf = L.tiles + align256(8 * (size_t)L.max_tiles);
   L.total = L.a_sf + align256((size_t)L.max_tiles * ((KT + 3) / 4) * NA * 512);
   return L;
@@ -167,20 +177,26 @@ __device__ inline int block_exclusive_scan_1024(int v, int* total) {
   return base + x - v;
 }
 
-// One block of 1024 threads; thread g handles group g (G <= 1024).
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ offsets, int G, int BN,
-                                                    int n_ft, int* __restrict__ header,
+// One block of 1024 threads; thread g handles group g (G <= 1024).  Unless
+// the offsets are nondecreasing from offsets[0] = 0 to offsets[G] <= a_rows,
+// the call records MOE_ERR_INVALID and plans no work at all, so no tile ever
+// addresses rows outside the operands or the workspace.
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ offsets, int G, int a_rows,
+                                                    int BN, int n_ft, int* __restrict__ header,
                                                     int* __restrict__ prefix, int* __restrict__ tstart,
-                                                    int2* __restrict__ tiles) {
+                                                    int2* __restrict__ groups, int2* __restrict__ tiles) {
   const int g = threadIdx.x;
   int rows = 0, r0 = 0;
+  bool bad = false;
   if (g < G) {
     r0 = offsets[g];
     rows = offsets[g + 1] - r0;
-    if (rows < 0 || (g == 0 && r0 != 0)) {
-      record_error(MOE_ERR_INVALID);
-      rows = 0;
-    }
+    bad = rows < 0 || (g == 0 && r0 != 0) || (g == G - 1 && offsets[G] > a_rows);
+  }
+  if (__syncthreads_or(bad)) {
+    if (g == 0) record_error(MOE_ERR_INVALID);
+    rows = 0;
+    r0 = 0;
   }
   const int nt = ceil_div(rows, BN);
   int n_tiles, n_items;
@@ -189,6 +205,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   if (g < G) {
     tstart[g] = t0;
     prefix[g] = i0;
+    groups[g] = make_int2(r0, rows);
     for (int j = 0; j < nt; ++j) tiles[t0 + j] = make_int2(r0 + j * BN, min(BN, rows - j * BN));
   }
   if (g == 0) {
@@ -232,24 +249,47 @@ struct Item {
   int g, ft, t, row0, rows;
 };
 
-// prefix: the group item prefix, copied to shared memory by the kernel.
-__device__ __forceinline__ Item decode_item(int item, const int* prefix, const int* tstart,
-                                            const int2* __restrict__ tiles, int G, int n_ft) {
+// The plan of one GEMM call, copied to shared memory at kernel start so that
+// decoding a work item reads no global memory.
+struct SmemPlan {
+  int* prefix;     // [G + 1]
+  int* tstart;     // [G]
+  int2* groups;    // [G]
+  __device__ explicit SmemPlan(uint8_t* base)
+      : prefix(reinterpret_cast<int*>(base)),
+        tstart(reinterpret_cast<int*>(base + 4 * (kMaxGroups + 4))),
+        groups(reinterpret_cast<int2*>(base + 8 * (kMaxGroups + 4))) {}
+  // all threads of the block; the caller synchronises before use
+  __device__ void load(const int* g_prefix, const int* g_tstart, const int2* g_groups, int G) {
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+      prefix[g] = g_prefix[g];
+      if (g < G) {
+        tstart[g] = g_tstart[g];
+        groups[g] = g_groups[g];
+      }
+    }
+  }
+};
+
+// Work item -> (group, weight tile, token tile).  Items are group-major, then
+// weight tile, then token tile.
+__device__ __forceinline__ Item decode_item(int item, const SmemPlan& plan, int G, int n_ft, int BN) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= item) lo = mid; else hi = mid - 1;
+    if (plan.prefix[mid] <= item) lo = mid; else hi = mid - 1;
   }
   Item it;
   it.g = lo;
-  const int base = prefix[lo];
-  const int nt = (prefix[lo + 1] - base) / n_ft;
+  const int base = plan.prefix[lo];
+  const int nt = (plan.prefix[lo + 1] - base) / n_ft;
   const int local = item - base;
   it.ft = local / nt;
-  it.t = tstart[lo] + local % nt;
-  const int2 tr = __ldg(tiles + it.t);
-  it.row0 = tr.x;
-  it.rows = tr.y;
+  const int tl = local - it.ft * nt;
+  it.t = plan.tstart[lo] + tl;
+  const int2 gr = plan.groups[lo];
+  it.row0 = gr.x + tl * BN;
+  it.rows = min(BN, gr.y - tl * BN);
   return it;
 }
 
@@ -259,7 +299,7 @@ struct GemmArgs {
   const int* header;
   const int* prefix;
   const int* tstart;
-  const int2* tiles;
+  const int2* groups;
   int G, N, K;
   void* out;
   uint8_t* out_scale;
@@ -350,8 +390,8 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
 template <int BN, bool DUAL>
 __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const uint32_t tmem, uint64_t* full,
                                            uint64_t* empty, uint64_t* acc_full,
-                                           uint64_t* acc_empty, volatile int* abort_flag, const int* s_prefix,
-                                           const int* s_tstart, const GemmArgs& args, const int n_items,
+                                           uint64_t* acc_empty, volatile int* abort_flag, const SmemPlan& plan,
+                                           const GemmArgs& args, const int n_items,
                                            const int KT, const int n_ft) {
   using C = Cfg<BN, DUAL>;
   const uint32_t ring0 = smem_u32(smem);
@@ -359,7 +399,7 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
   const uint32_t sfb_t = sfa_t + 4 * C::TILES_PER_ISSUER;
   uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, args.G, n_ft);
+    const Item it = decode_item(item, plan, args.G, n_ft, BN);
     const int n_mma = max(16, (it.rows + 15) & ~15);
     const uint32_t idesc = idesc_mxf8f6f4(5u /*E2M1*/, 0u /*E4M3*/, 128, n_mma);
     uint32_t id_kb[4];
@@ -423,8 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
-  int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
-  int* s_tstart = reinterpret_cast<int*>(smem + C::TSTART_OFF);
+  SmemPlan plan(smem + C::PLAN_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.G, N = args.N, K = args.K;
@@ -432,10 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_ft = DUAL ? N / 256 : N / 128;
   const int rb_per_g = N / 128;
   const int n_items = args.header[0];
-  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
-    s_prefix[g] = args.prefix[g];
-    if (g < G) s_tstart[g] = args.tstart[g];
-  }
+  plan.load(args.prefix, args.tstart, args.groups, G);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -466,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // elected lane issues each step's copies.
     uint32_t stage = 0, phase = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb0 = it.g * rb_per_g + it.ft;
       // first prepared block of this item's weight tile(s); per K step the
       // blocks of gate and up (DUAL, paired order) or of the tile are adjacent
@@ -497,13 +533,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer 0 ---------------------------
-    mma_issuer<BN, DUAL>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, s_prefix, s_tstart,
-                         args, n_items, KT, n_ft);
+    mma_issuer<BN, DUAL>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
+                         n_items, KT, n_ft);
   } else if (warp == kThreads / 32 - 1) {
     // ------------------------------ MMA issuer 1 ---------------------------
     if (C::ISSUERS == 2)
-      mma_issuer<BN, DUAL>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, s_prefix,
-                           s_tstart, args, n_items, KT, n_ft);
+      mma_issuer<BN, DUAL>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan,
+                           args, n_items, KT, n_ft);
   } else {
     // ------------------------------ epilogue ------------------------------
     const int e = warp - C::EPI_FIRST;
@@ -513,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t ab = 0, acc_bits = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, plan, G, n_ft, BN);
       if (!mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag)) break;
       tc_fence_after();
       epilogue_item<BN, DUAL, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,

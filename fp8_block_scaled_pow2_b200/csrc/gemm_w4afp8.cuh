@@ -54,9 +54,8 @@ struct Cfg {
   static constexpr int SFA_SMEM_OFF = STAGES * STAGE;  // 512 bytes of unit scales
   static constexpr int BAR_OFF = SFA_SMEM_OFF + 512;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int PREFIX_OFF = RED_OFF + 4 * BN * 4;    // group item prefix, int32[G+1]
-  static constexpr int TSTART_OFF = PREFIX_OFF + 4 * 1028;   // first token tile per group, int32[G]
-  static constexpr int SMEM_USED = TSTART_OFF + 4 * 1028;
+  static constexpr int PLAN_OFF = RED_OFF + 4 * BN * 4;      // gemm::SmemPlan
+  static constexpr int SMEM_USED = PLAN_OFF + gemm::kPlanSmemBytes;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few stages");
@@ -83,7 +82,7 @@ struct W4Args {
   const int* header;
   const int* prefix;
   const int* tstart;
-  const int2* tiles;
+  const int2* groups;
   int G, N, K;
   void* out;
   uint8_t* out_scale;
@@ -106,18 +105,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
-  int* s_prefix = reinterpret_cast<int*>(smem + C::PREFIX_OFF);
+  gemm::SmemPlan plan(smem + C::PLAN_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.G, N = args.N, K = args.K;
   const int KT = K / 128;
   const int n_ft = DUAL ? N / 256 : N / 128;
   const int n_items = args.header[0];
-  int* s_tstart = reinterpret_cast<int*>(smem + C::TSTART_OFF);
-  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
-    s_prefix[g] = args.prefix[g];
-    if (g < G) s_tstart[g] = args.tstart[g];
-  }
+  plan.load(args.prefix, args.tstart, args.groups, G);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -152,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rb_per_g = N / 128;
     uint32_t stage = 0, phase = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb0 = it.g * rb_per_g + it.ft;
       const int rb1 = rb0 + rb_per_g / 2;
       const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
@@ -182,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t stage = 0, phase = 0;
     uint32_t pb = 0, pbits = 0;            // bit b: phase of partial buffer b
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, plan, G, n_ft, BN);
       const int n_mma = max(16, (it.rows + 15) & ~15);
       const uint32_t idesc = idesc_mxf8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
       bool ok = true;
@@ -268,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t pb = 0, pbits = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, s_prefix, s_tstart, args.tiles, G, n_ft);
+      const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb_per_g = N / 128;
       const float* s0 = args.w_sinv + ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT;
       const float* s1 = args.w_sinv + ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT;

@@ -286,7 +286,7 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   args.header = reinterpret_cast<const int*>(ws + L.header);
   args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
   args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
-  args.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
   args.G = n_groups;
   args.N = N;
   args.K = K;
@@ -297,8 +297,9 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   cudaStream_t st = S(stream);
   const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
   const int n_ft = dual ? N / 256 : N / 128;
-  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
-                                        reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, (int)a_rows, block_n, n_ft,
+                                        reinterpret_cast<int*>(ws + L.header), reinterpret_cast<int*>(ws + L.prefix),
+                                        reinterpret_cast<int*>(ws + L.tstart), reinterpret_cast<int2*>(ws + L.groups),
                                         reinterpret_cast<int2*>(ws + L.tiles));
   gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
       a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
@@ -342,7 +343,7 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
   args.header = reinterpret_cast<const int*>(ws + L.header);
   args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
   args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
-  args.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
   args.G = n_groups;
   args.N = N;
   args.K = K;
@@ -351,8 +352,9 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
   args.limit = swiglu_limit;
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
-  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, block_n, n_ft, reinterpret_cast<int*>(ws + L.header),
-                                        reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, (int)a_rows, block_n, n_ft,
+                                        reinterpret_cast<int*>(ws + L.header), reinterpret_cast<int*>(ws + L.prefix),
+                                        reinterpret_cast<int*>(ws + L.tstart), reinterpret_cast<int2*>(ws + L.groups),
                                         reinterpret_cast<int2*>(ws + L.tiles));
   gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
       a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),

@@ -191,7 +191,10 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
  *                                          * w[g, n, k] * 2^(sw[g, n, k/32]-127)
  *   a_e4m3       uint8 [a_rows, K] (16-byte aligned), a_rows >= offsets[G]
  *   a_e8m0_128   uint8 [a_rows, K/128]
- *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0
+ *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0,
+ *                offsets[G] <= a_rows; otherwise the call does no work, leaves
+ *                out untouched and records MOE_ERR_INVALID in the device error
+ *                word (moe_get_device_error)
  *   w_prepared   output of moe_prepare_weights for the MXFP4 weights [G, N, K/2]
  *                and scales [G, N, K/32] (paired order for
  *                MOE_EPI_SWIGLU_QUANT, plain otherwise)

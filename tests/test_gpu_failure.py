@@ -46,3 +46,32 @@ def test_out_of_range_expert_id_is_flagged(lib):
     ws = torch.empty(lib.moe_permute_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
     lib.moe_permute(idx, E, 1, xq, sx, *out, ws)
     assert lib.moe_get_device_error() == -1
+
+
+@pytest.mark.parametrize("bad", ["past_rows", "decreasing", "nonzero_start"])
+def test_invalid_group_offsets_plan_no_work(lib, bad):
+    """Offsets that are not nondecreasing from 0 up to at most a_rows (device
+    data the host cannot check) are caught by the GEMM's plan: it records
+    MOE_ERR_INVALID and plans no work, so the output keeps its contents and
+    no tile reads or writes outside the operands."""
+    G, N, K, R = 3, 256, 256, 40
+    offsets = {"past_rows": [0, 10, 20, 41], "decreasing": [0, 30, 10, 40],
+               "nonzero_start": [5, 10, 20, 40]}[bad]
+    a = torch.zeros((R, K), dtype=torch.uint8, device="cuda")
+    asc = torch.full((R, K // 128), 127, dtype=torch.uint8, device="cuda")
+    w = torch.zeros((G, N, K // 2), dtype=torch.uint8, device="cuda")
+    wsc = torch.full((G, N, K // 32), 127, dtype=torch.uint8, device="cuda")
+    wp = torch.empty(lib.moe_prepared_weights_size(G, N, K), dtype=torch.uint8, device="cuda")
+    lib.moe_prepare_weights(w, wsc, wp)
+    ws = torch.empty(lib.moe_gemm_workspace_size(R, G, K, 16), dtype=torch.uint8, device="cuda")
+    out = torch.full((R, N), 7.0, dtype=torch.float32, device="cuda")
+    off = torch.tensor(offsets, dtype=torch.int32, device="cuda")
+    lib.moe_grouped_gemm_mxfp4(a, asc, off, wp, G, N, lib.MOE_EPI_STORE_F32, out, None, ws, 10.0, 16)
+    torch.cuda.synchronize()
+    assert lib.moe_get_device_error() == -1
+    assert (out == 7.0).all()
+    off_ok = torch.tensor([0, 10, 20, 40], dtype=torch.int32, device="cuda")
+    lib.moe_grouped_gemm_mxfp4(a, asc, off_ok, wp, G, N, lib.MOE_EPI_STORE_F32, out, None, ws, 10.0, 16)
+    torch.cuda.synchronize()
+    assert lib.moe_get_device_error() == 0
+    assert (out == 0.0).all()
