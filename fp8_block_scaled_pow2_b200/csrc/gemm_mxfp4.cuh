@@ -75,7 +75,8 @@ struct Cfg {
   // the ring takes the shared memory the rest of the kernel leaves (227 KB
   // per CTA; barriers, SwiGLU reduction, plan and alignment slack)
   static constexpr int CW0 = BN / 2;                     // epilogue columns per warp, see CW
-  static constexpr int RING_BUDGET = 227 * 1024 - (512 + 2 * 4 * CW0 * 4 + kPlanSmemBytes + 1024);
+  static constexpr int RED_BYTES = 2 * 4 * CW0 * 4 + 2 * CW0 * 4;   // SwiGLU maxima + column scales
+  static constexpr int RING_BUDGET = 227 * 1024 - (512 + RED_BYTES + kPlanSmemBytes + 1024);
   static constexpr int STAGES_FIT = RING_BUDGET / STAGE;
   static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
   // transaction bytes of a step (the TMA counts the packed weight bytes);
@@ -108,7 +109,7 @@ struct Cfg {
   // shared memory after the ring
   static constexpr int BAR_OFF = STAGES * STAGE;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int PLAN_OFF = RED_OFF + 2 * 4 * CW * 4;       // SmemPlan (kPlanSmemBytes)
+  static constexpr int PLAN_OFF = RED_OFF + RED_BYTES;            // SmemPlan (kPlanSmemBytes)
   static constexpr int SMEM_USED = PLAN_OFF + kPlanSmemBytes;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;     // slack for 1024-byte alignment
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
@@ -346,8 +347,13 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
   }
 
   if constexpr (EPI == MOE_EPI_SWIGLU_QUANT) {
+    // The 128 features of a token column live in the four warps of this half
+    // (one TMEM sub-partition each): per-warp maxima go through shared memory,
+    // one thread per column turns the column maximum into the scale, and every
+    // thread then quantises its 128 features x CW tokens with that scale.
     const int I = N / 2;
-    float* rr = red + half * 4 * CW;
+    float* rr = red + half * 4 * CW;             // [4 warps][CW] partial maxima
+    float* sk = red + 2 * 4 * CW + half * CW;    // [CW] 2^-k per column
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
       const float h = swiglu_clamped(__uint_as_float(v0[c]), __uint_as_float(v1[c]), args.limit);
@@ -356,16 +362,19 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
       if (lane == 0) rr[q * CW + c] = m;
     }
     named_bar_sync(1 + half, 128);
-    uint8_t* hq = reinterpret_cast<uint8_t*>(args.out);
+    if (f < my_cols) {
+      const int c = f;
+      const float amax = fmaxf(fmaxf(rr[c], rr[CW + c]), fmaxf(rr[2 * CW + c], rr[3 * CW + c]));
+      const int k = pow2_scale_exponent(amax);
+      sk[c] = exp2_int(-k);
+      args.out_scale[(size_t)(it.row0 + c_base + c) * (I / 128) + it.ft] = (uint8_t)(k + 127);
+    }
+    named_bar_sync(1 + half, 128);
+    uint8_t* hq = reinterpret_cast<uint8_t*>(args.out) + (size_t)(it.row0 + c_base) * I + it.ft * 128 + f;
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
-      if (c < my_cols) {
-        const float amax = fmaxf(fmaxf(rr[c], rr[CW + c]), fmaxf(rr[2 * CW + c], rr[3 * CW + c]));
-        const int k = pow2_scale_exponent(amax);
-        const size_t row = (size_t)(it.row0 + c_base + c);
-        hq[row * I + it.ft * 128 + f] = (uint8_t)(e4m3x2(__fmul_rn(__uint_as_float(v0[c]), exp2_int(-k)), 0.0f) & 0xFFu);
-        if (f == 0) args.out_scale[row * (I / 128) + it.ft] = (uint8_t)(k + 127);
-      }
+      if (c < my_cols)
+        hq[(size_t)c * I] = (uint8_t)(e4m3x2(__fmul_rn(__uint_as_float(v0[c]), sk[c]), 0.0f) & 0xFFu);
     }
     named_bar_sync(1 + half, 128);
   } else {
