@@ -14,8 +14,9 @@
 //     tensor-memory buffers;
 //   * promotion warps multiply each partial by the row's scale_inv and add it
 //     into float32 registers, then run the same epilogues as the MXFP4 GEMM.
-// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 converters,
-// 6..9 promotion + epilogue.
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, then CONV_WARPS
+// converters (8 for narrow token tiles, where transcoding is the critical
+// path, else 4), then 4 promotion + epilogue warps.
 #pragma once
 
 #include "gemm_mxfp4.cuh"
@@ -27,10 +28,12 @@ using namespace sm100;
 using gemm::Item;
 using gemm::decode_item;
 
-constexpr int kThreads = 320;
-
 template <int BN, bool DUAL>
 struct Cfg {
+  static constexpr int CONV_WARPS = BN <= 32 ? 8 : 4;
+  static constexpr int PROMO_FIRST = 2 + CONV_WARPS;      // first promotion warp
+  static constexpr int THREADS = (PROMO_FIRST + 4) * 32;
+  static constexpr int CONV_THREADS = CONV_WARPS * 32;
   static constexpr int NA = (BN + 127) / 128;
   static constexpr int NUM_A = DUAL ? 2 : 1;
   static constexpr int RAW_BYTES = 128 * 64;          // INT4 tile as loaded (64 B per row)
@@ -54,7 +57,7 @@ struct Cfg {
   static constexpr int SFA_SMEM_OFF = STAGES * STAGE;  // 512 bytes of unit scales
   static constexpr int BAR_OFF = SFA_SMEM_OFF + 512;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int PLAN_OFF = RED_OFF + 4 * BN * 4;      // gemm::SmemPlan
+  static constexpr int PLAN_OFF = RED_OFF + 5 * BN * 4;      // after [4][BN] maxima + [BN] scales
   static constexpr int SMEM_USED = PLAN_OFF + gemm::kPlanSmemBytes;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
@@ -90,7 +93,7 @@ struct W4Args {
 };
 
 template <int BN, bool DUAL, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
     gemm_w4afp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const W4Args args) {
   using C = Cfg<BN, DUAL>;
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], 128);
+      mbar_init(&conv[s], C::CONV_THREADS);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -215,11 +218,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-  } else if (warp < 6) {
+  } else if (warp < C::PROMO_FIRST) {
     // ------------------------------ converters ----------------------------
-    // thread layout: warp w (0..3), lane l -> 16-byte input chunk (l & 3) of
-    // rows w*8 + (l >> 2) + 32 j; conflict-free reads of the raw tile and
-    // conflict-free writes into the 128-byte swizzle.
+    // thread layout: converter warp w (0..CONV_WARPS-1), lane l -> 16-byte
+    // input chunk (l & 3) of rows w*8 + (l >> 2) + 8*CONV_WARPS*j;
+    // conflict-free reads of the raw tile and conflict-free writes into the
+    // 128-byte swizzle.
     const int w = warp - 2;
     const int chunk = lane & 3;
     uint32_t stage = 0, phase = 0;
@@ -233,8 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* raw = st + C::RAW_OFF + a * C::RAW_BYTES;
           uint8_t* dst = st + C::A_OFF + a * C::A_BYTES;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = w * 8 + (lane >> 2) + 32 * j;
+          for (int j = 0; j < 128 / (8 * C::CONV_WARPS); ++j) {
+            const int r = w * 8 + (lane >> 2) + 8 * C::CONV_WARPS * j;
             const uint4 in = *reinterpret_cast<const uint4*>(raw + r * 64 + chunk * 16);
             uint4 o0, o1;
             o0.x = int4x4_to_e4m3x4(in.x & 0xFFFFu);
@@ -322,15 +326,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) red[q * BN + c] = m;
         }
         named_bar_sync(1, 128);
+        // one thread per token column turns the column maximum into the scale
+        float* sk = red + 4 * BN;
+        if (f < it.rows && f < BN) {
+          const int c = f;
+          const float amax = fmaxf(fmaxf(red[c], red[BN + c]), fmaxf(red[2 * BN + c], red[3 * BN + c]));
+          const int k = pow2_scale_exponent(amax);
+          sk[c] = exp2_int(-k);
+          args.out_scale[(size_t)(it.row0 + c) * (I / 128) + it.ft] = (uint8_t)(k + 127);
+        }
+        named_bar_sync(1, 128);
+        uint8_t* hq_f = hq + (size_t)it.row0 * I + it.ft * 128 + f;
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
-          if (c < it.rows) {
-            const float amax = fmaxf(fmaxf(red[c], red[BN + c]), fmaxf(red[2 * BN + c], red[3 * BN + c]));
-            const int k = pow2_scale_exponent(amax);
-            const size_t row = (size_t)(it.row0 + c);
-            hq[row * I + it.ft * 128 + f] = (uint8_t)(e4m3x2(__fmul_rn(h[c], exp2_int(-k)), 0.0f) & 0xFFu);
-            if (f == 0) args.out_scale[row * (I / 128) + it.ft] = (uint8_t)(k + 127);
-          }
+          if (c < it.rows) hq_f[(size_t)c * I] = (uint8_t)(e4m3x2(__fmul_rn(h[c], sk[c]), 0.0f) & 0xFFu);
         }
         named_bar_sync(1, 128);
       } else {

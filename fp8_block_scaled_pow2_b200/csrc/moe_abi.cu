@@ -110,7 +110,7 @@ int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& 
   auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
-  k<<<sm_count(), w4a::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  k<<<sm_count(), C::THREADS, C::SMEM_ALLOC, st>>>(ta, tb, a);
   return launch_status();
 }
 
