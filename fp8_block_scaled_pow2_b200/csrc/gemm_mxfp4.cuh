@@ -12,11 +12,14 @@
 // memory as [128 weight rows (lanes)] x [BN tokens (columns)].
 //
 // Work decomposition: tokens of each expert (group) are cut into tiles of BN
-// rows; a work item is (token tile, 128-row weight tile).  For the w1/w3
-// projection (DUAL) one item holds the gate tile and the up tile of the same
-// 128 output features so the SwiGLU epilogue has both in one thread.  Items
-// are ordered group-major, then weight tile, then token tile, so CTAs running
-// at the same time stream the same weight tile from L2.
+// rows; a work item is (token tile, weight tile pair).  A pair (PAIR) is two
+// 128-row weight tiles that share the token tile: for the w1/w3 projection
+// the gate tile and the up tile of the same 128 output features (paired
+// weight order), so the SwiGLU epilogue has both in one thread; otherwise two
+// adjacent 128-row blocks of the output (plain order).  Without PAIR (N not a
+// multiple of 256) an item is one weight tile.  Items are ordered
+// group-major, then weight tile, then token tile, so CTAs running at the same
+// time stream the same weight tiles from L2.
 //
 // CTA roles (persistent kernel, one CTA per SM, 11 warps):
 //   warp 0        TMA producer: weight tiles (FP4 unpacked to one nibble per
@@ -57,10 +60,10 @@ constexpr int kPlanSmemBytes = 16 * (kMaxGroups + 4);
 // straight into the unpacked one-nibble-per-byte layout the MMA reads
 // (16U4_ALIGN16B), a 1-D bulk copy brings its 512-byte scale block, a 2-D TMA
 // copy the token tile, and every fourth step a bulk copy the token scales.
-template <int BN, bool DUAL>
+template <int BN, bool PAIR>
 struct Cfg {
   static constexpr int NA = (BN + 127) / 128;            // 128-row scale blocks of the token tile
-  static constexpr int NUM_A = DUAL ? 2 : 1;
+  static constexpr int NUM_A = PAIR ? 2 : 1;
   static constexpr int A_BYTES = 128 * 128;              // one MMA-ready FP4 weight tile
   static constexpr int A_PACKED = 128 * 64;              // the same tile packed (global layout)
   static constexpr int B_BYTES = BN * 128;
@@ -83,22 +86,22 @@ struct Cfg {
   // steps that also load token scales add NA * 512
   static constexpr int TX = NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;
   // MMA issue: one warp issuing small-N MMAs is bound by its own issue
-  // latency, so narrow tiles use two issuing warps.  With gate and up (DUAL)
-  // issuer 0 computes the gate tile and issuer 1 the up tile; otherwise they
-  // take alternate K steps into two partial accumulators the epilogue adds.
-  // Wide gate/up tiles keep one issuer (its gate and up MMAs share the token
-  // operand back to back).
+  // latency, so narrow tiles use two issuing warps.  With a tile pair issuer
+  // 0 computes tile 0 and issuer 1 tile 1; with one tile they take alternate
+  // K steps into two partial accumulators the epilogue adds.  Wide pairs keep
+  // one issuer (its two MMAs per K block share the token operand back to
+  // back).
   // tensor-memory columns: ACC_BUFS accumulators of 2 * BN columns, then one
   // scale set (weight + token scales) per issuer
-  static constexpr int ISSUERS = (DUAL && BN >= 64) ? 1 : 2;
-  static constexpr int TILES_PER_ISSUER = (DUAL && ISSUERS == 1) ? 2 : 1;
+  static constexpr int ISSUERS = (PAIR && BN >= 64) ? 1 : 2;
+  static constexpr int TILES_PER_ISSUER = (PAIR && ISSUERS == 1) ? 2 : 1;
   static constexpr int ACC_COLS = 2 * BN;
   static constexpr int SF_SET = 4 * TILES_PER_ISSUER + 4 * NA;
   static constexpr int SF_COLS = 2 * SF_SET;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
   static constexpr int SF_COL = ACC_BUFS * ACC_COLS;      // issuer i: SF_COL + i * SF_SET
   static constexpr int TMEM_USED = SF_COL + SF_COLS;
-  static constexpr int CONSUMERS = DUAL ? ISSUERS : 1;    // issuers reading each ring stage
+  static constexpr int CONSUMERS = PAIR ? ISSUERS : 1;    // issuers reading each ring stage
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   // epilogue warps: each owns 32 weight rows (its TMEM sub-partition) and
   // BN / (EPI_WARPS / 4) token columns
@@ -312,15 +315,16 @@ struct GemmArgs {
 // the TMEM buffer (the next item's MMAs may start), then finish from registers:
 // float32 / bf16 stores, or SwiGLU + per-128 power-of-two FP8 requantisation
 // with the group maximum reduced across the four warps of a column slice.
-template <int BN, bool DUAL, int EPI, int CW>
+template <int BN, bool PAIR, int EPI, int CW>
 __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int f, int q, int half, int lane,
                                               int N, int KT, const GemmArgs& args, float* red,
                                               uint64_t* acc_empty_bar) {
   const int c_base = half * CW;
   const int my_cols = max(0, min(CW, it.rows - c_base));     // valid columns of this warp
-  // DUAL: v0 = gate, v1 = up.  Otherwise v0 / v1 are the even / odd K-step
-  // partial sums (v1 holds nothing when there is a single K step).
-  const bool use_v1 = DUAL || KT > 1;
+  // PAIR: v0 / v1 = tile 0 / tile 1 (gate / up for SwiGLU).  Otherwise v0 / v1
+  // are the even / odd K-step partial sums (v1 holds nothing when there is a
+  // single K step).
+  const bool use_v1 = PAIR || KT > 1;
   uint32_t v0[CW];
   uint32_t v1[CW];
 #pragma unroll
@@ -339,7 +343,7 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
   tmem_wait_ld_n<CW>(v1);
   tc_fence_before();
   mbar_arrive(acc_empty_bar);
-  if constexpr (!DUAL) {
+  if constexpr (!PAIR) {
     if (use_v1) {
 #pragma unroll
       for (int c = 0; c < CW; ++c) v0[c] = __float_as_uint(__uint_as_float(v0[c]) + __uint_as_float(v1[c]));
@@ -378,14 +382,19 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
     }
     named_bar_sync(1 + half, 128);
   } else {
+    // output column block of tile 0 (tile 1 is the next block with PAIR)
+    const int cb = PAIR ? 2 * it.ft : it.ft;
 #pragma unroll
     for (int c = 0; c < CW; ++c) {
       if (c < my_cols) {
-        const size_t o = (size_t)(it.row0 + c_base + c) * N + it.ft * 128 + f;
-        if constexpr (EPI == MOE_EPI_STORE_F32)
+        const size_t o = (size_t)(it.row0 + c_base + c) * N + cb * 128 + f;
+        if constexpr (EPI == MOE_EPI_STORE_F32) {
           reinterpret_cast<float*>(args.out)[o] = __uint_as_float(v0[c]);
-        else
+          if (PAIR) reinterpret_cast<float*>(args.out)[o + 128] = __uint_as_float(v1[c]);
+        } else {
           reinterpret_cast<__nv_bfloat16*>(args.out)[o] = __float2bfloat16_rn(__uint_as_float(v0[c]));
+          if (PAIR) reinterpret_cast<__nv_bfloat16*>(args.out)[o + 128] = __float2bfloat16_rn(__uint_as_float(v1[c]));
+        }
       }
     }
   }
@@ -396,13 +405,13 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
 // change within an item is computed before its K loop; per-K-block operands
 // are constant offsets of per-stage bases (a descriptor's start-address field
 // is the byte address / 16, so +32 bytes is +2).
-template <int BN, bool DUAL>
+template <int BN, bool PAIR>
 __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const uint32_t tmem, uint64_t* full,
                                            uint64_t* empty, uint64_t* acc_full,
                                            uint64_t* acc_empty, volatile int* abort_flag, const SmemPlan& plan,
                                            const GemmArgs& args, const int n_items,
                                            const int KT, const int n_ft) {
-  using C = Cfg<BN, DUAL>;
+  using C = Cfg<BN, PAIR>;
   const uint32_t ring0 = smem_u32(smem);
   const uint32_t sfa_t = tmem + C::SF_COL + iss * C::SF_SET;     // 4 columns per weight tile
   const uint32_t sfb_t = sfa_t + 4 * C::TILES_PER_ISSUER;
@@ -418,21 +427,21 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
     tc_fence_after();
     const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
     for (int kt = 0; kt < KT; ++kt) {
-      const bool mine = DUAL || C::ISSUERS == 1 || (kt & 1) == iss;
+      const bool mine = PAIR || C::ISSUERS == 1 || (kt & 1) == iss;
       if (mine) {
         if (!mbar_wait_warp(&full[stage], phase, abort_flag)) return;
         const uint32_t st = ring0 + stage * C::STAGE;
-        const uint32_t a_base = st + (DUAL ? iss * C::A_BYTES : 0);
+        const uint32_t a_base = st + (PAIR ? iss * C::A_BYTES : 0);
         const uint32_t bsel = (uint32_t)(kt & 3);
         const uint32_t sfb = sfb_t | (bsel << 30);
         const uint64_t da = sdesc_kmajor_sw128(a_base);
         const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
         // this issuer's first step of the item starts a fresh accumulator
-        const uint32_t first = (DUAL || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
+        const uint32_t first = (PAIR || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
         if (elect_one()) {
-          tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (DUAL ? iss * C::SF_BYTES : 0)));
+          tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (PAIR ? iss * C::SF_BYTES : 0)));
           if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SF_BYTES));
-          if ((kt & 3) == (DUAL || C::ISSUERS == 1 ? 0 : iss)) {
+          if ((kt & 3) == (PAIR || C::ISSUERS == 1 ? 0 : iss)) {
 #pragma unroll
             for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
           }
@@ -457,11 +466,14 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
   }
 }
 
-template <int BN, bool DUAL, int EPI>
+template <int BN, bool PAIR, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_mxfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmArgs args) {
-  using C = Cfg<BN, DUAL>;
+  using C = Cfg<BN, PAIR>;
+  // SwiGLU reads gate and up from the two tiles of a pair (paired weight order)
+  constexpr bool PAIRED_ORDER = EPI == MOE_EPI_SWIGLU_QUANT;
+  static_assert(!PAIRED_ORDER || PAIR, "the SwiGLU epilogue needs gate/up tile pairs");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -477,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.G, N = args.N, K = args.K;
   const int KT = K / 128;
-  const int n_ft = DUAL ? N / 256 : N / 128;
+  const int n_ft = PAIR ? N / 256 : N / 128;
   const int rb_per_g = N / 128;
   const int n_items = args.header[0];
   plan.load(args.prefix, args.tstart, args.groups, G);
@@ -512,10 +524,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t stage = 0, phase = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
-      const int rb0 = it.g * rb_per_g + it.ft;
-      // first prepared block of this item's weight tile(s); per K step the
-      // blocks of gate and up (DUAL, paired order) or of the tile are adjacent
-      const size_t blk0 = DUAL ? ((size_t)(it.g * n_ft + it.ft) * KT) * 2 : (size_t)rb0 * KT;
+      // prepared block of weight tile a at K step kt: blk0 + kt * kt_step + a * a_step
+      //   paired order: the gate and up blocks of a K step are adjacent;
+      //   plain order: each 128-row block holds its KT steps contiguously
+      size_t blk0, kt_step, a_step;
+      if (PAIRED_ORDER) {
+        blk0 = (size_t)(it.g * n_ft + it.ft) * KT * 2;
+        kt_step = 2;
+        a_step = 1;
+      } else {
+        blk0 = (size_t)(it.g * rb_per_g + (PAIR ? 2 * it.ft : it.ft)) * KT;
+        kt_step = 1;
+        a_step = KT;
+      }
       const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
       bool ok = true;
       for (int kt = 0; kt < KT; ++kt) {
@@ -523,14 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) {
           uint8_t* st = smem + stage * C::STAGE;
           // token scales: one block per 4 K steps, read by each issuer at its
-          // first step of the group (issuers alternate steps without DUAL)
-          const bool new_group = (DUAL || C::ISSUERS == 1) ? (kt & 3) == 0 : (kt & 3) < 2;
+          // first step of the group (issuers alternate steps without PAIR)
+          const bool new_group = (PAIR || C::ISSUERS == 1) ? (kt & 3) == 0 : (kt & 3) < 2;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
-          const size_t blk = blk0 + (size_t)kt * C::NUM_A;
 #pragma unroll
           for (int a = 0; a < C::NUM_A; ++a) {
-            tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)(blk + a), &full[stage]);
-            bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + (blk + a) * kWBlock + 8192, 512, &full[stage]);
+            const size_t blk = blk0 + (size_t)kt * kt_step + (size_t)a * a_step;
+            tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)blk, &full[stage]);
+            bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + blk * kWBlock + 8192, 512, &full[stage]);
           }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
@@ -542,12 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer 0 ---------------------------
-    mma_issuer<BN, DUAL>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
+    mma_issuer<BN, PAIR>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
                          n_items, KT, n_ft);
   } else if (warp == kThreads / 32 - 1) {
     // ------------------------------ MMA issuer 1 ---------------------------
     if (C::ISSUERS == 2)
-      mma_issuer<BN, DUAL>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan,
+      mma_issuer<BN, PAIR>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan,
                            args, n_items, KT, n_ft);
   } else {
     // ------------------------------ epilogue ------------------------------
@@ -561,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode_item(item, plan, G, n_ft, BN);
       if (!mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag)) break;
       tc_fence_after();
-      epilogue_item<BN, DUAL, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,
+      epilogue_item<BN, PAIR, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,
                                           KT, args, red, &acc_empty[ab]);
       acc_bits ^= 1u << ab;
       if (C::ACC_BUFS == 2) ab ^= 1u;

@@ -82,24 +82,24 @@ int pick_block_n(int a_rows, int G) {
   return 128;
 }
 
-template <int BN, bool DUAL, int EPI>
+template <int BN, bool PAIR, int EPI>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a, cudaStream_t st) {
-  using C = gemm::Cfg<BN, DUAL>;
-  auto k = gemm::gemm_mxfp4_kernel<BN, DUAL, EPI>;
+  using C = gemm::Cfg<BN, PAIR>;
+  auto k = gemm::gemm_mxfp4_kernel<BN, PAIR, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
   k<<<sm_count(), gemm::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
   return launch_status();
 }
 
-template <bool DUAL, int EPI>
+template <bool PAIR, int EPI>
 int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a,
                    cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_gemm<16, DUAL, EPI>(ta, tb, a, st);
-    case 32: return launch_gemm<32, DUAL, EPI>(ta, tb, a, st);
-    case 64: return launch_gemm<64, DUAL, EPI>(ta, tb, a, st);
-    case 128: return launch_gemm<128, DUAL, EPI>(ta, tb, a, st);
+    case 16: return launch_gemm<16, PAIR, EPI>(ta, tb, a, st);
+    case 32: return launch_gemm<32, PAIR, EPI>(ta, tb, a, st);
+    case 64: return launch_gemm<64, PAIR, EPI>(ta, tb, a, st);
+    case 128: return launch_gemm<128, PAIR, EPI>(ta, tb, a, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
@@ -295,8 +295,10 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   args.limit = swiglu_limit;
 
   cudaStream_t st = S(stream);
-  const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
-  const int n_ft = dual ? N / 256 : N / 128;
+  // work items hold two 128-row weight tiles whenever N allows (gate + up for
+  // SwiGLU, which requires N % 256 == 0)
+  const bool pair = epilogue == MOE_EPI_SWIGLU_QUANT || N % 256 == 0;
+  const int n_ft = pair ? N / 256 : N / 128;
   gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, (int)a_rows, block_n, n_ft,
                                         reinterpret_cast<int*>(ws + L.header), reinterpret_cast<int*>(ws + L.prefix),
                                         reinterpret_cast<int*>(ws + L.tstart), reinterpret_cast<int2*>(ws + L.groups),
@@ -306,8 +308,12 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
       reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   switch (epilogue) {
-    case MOE_EPI_STORE_F32: return launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
-    case MOE_EPI_STORE_BF16: return launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
+    case MOE_EPI_STORE_F32:
+      return pair ? launch_gemm_bn<true, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st)
+                  : launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
+    case MOE_EPI_STORE_BF16:
+      return pair ? launch_gemm_bn<true, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st)
+                  : launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
     default: return launch_gemm_bn<true, MOE_EPI_SWIGLU_QUANT>(block_n, ta, tb, args, st);
   }
 }

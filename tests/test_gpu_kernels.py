@@ -150,20 +150,23 @@ def _run_gemm(lib, a, asc, offsets, w, wsc, epi, block_n):
 GROUPS = [0, 1, 15, 16, 17, 0, 127, 128, 129, 300, 2]
 
 
+@pytest.mark.parametrize("N", [256, 384, 512])
 @pytest.mark.parametrize("block_n", [16, 32, 64, 128])
-def test_gemm_integer_exact(lib, block_n):
+def test_gemm_integer_exact(lib, block_n, N):
     """All scales 2^0 and small-integer operands: every partial sum is an
-    integer below 2^24, so the float32 result is exact in any order."""
-    a, asc, offsets, w, wsc = _gemm_inputs(3, GROUPS, 256, 512, True)
+    integer below 2^24, so the float32 result is exact in any order.  N = 384
+    runs single 128-row weight tiles per work item, N = 256 / 512 pairs."""
+    a, asc, offsets, w, wsc = _gemm_inputs(3, GROUPS, N, 512, True)
     out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
     ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
     np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("N", [384, 512])
 @pytest.mark.parametrize("block_n", [16, 128])
-def test_gemm_random_scaled(lib, block_n):
-    a, asc, offsets, w, wsc = _gemm_inputs(5, [3, 0, 40, 130, 1], 384, 1024, False)
+def test_gemm_random_scaled(lib, block_n, N):
+    a, asc, offsets, w, wsc = _gemm_inputs(5, [3, 0, 40, 130, 1], N, 1024, False)
     out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
     ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
     # float32 accumulation of K terms: error <= K * 2^-24 * sum |a w|
