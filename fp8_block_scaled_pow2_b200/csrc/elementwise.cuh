@@ -123,12 +123,16 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 }
 
 // ------------------------------- a3 ---------------------------------------
-// Grouping in four deterministic passes:
+// Grouping in deterministic passes:
 //   count:   per chunk of kChunk pairs, a histogram over experts
 //   scan:    per expert the running sum over chunks, then offsets
-//   scatter: per chunk, one warp walks its pairs in order; __match_any_sync
-//            gives each pair its rank among equal experts -> stable rows
+//   scatter: per chunk, the pairs are staged in shared memory and one warp
+//            walks them in order; __match_any_sync gives each pair its rank
+//            among equal experts -> stable rows
 //   gather:  one warp per output row copies the FP8 row and its scales
+// When all pairs fit in one chunk (decode), one block does count, scan and
+// scatter (permute_small_kernel).  A pair with an expert id outside [0, E)
+// is flagged (MOE_ERR_INVALID), gets no row, and its inv entry is -1.
 constexpr int kChunk = 2048;
 
 __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __restrict__ idx, int P, int E,
@@ -190,33 +194,104 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
   }
 }
 
-__global__ void __launch_bounds__(32) permute_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
-                                                             const int32_t* __restrict__ chunk_hist,
-                                                             const int32_t* __restrict__ offsets,
-                                                             int32_t* __restrict__ perm,
-                                                             int32_t* __restrict__ inv) {
-  __shared__ int ctr[1024];
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) ctr[e] = offsets[e] + chunk_hist[(int64_t)blockIdx.x * E + e];
-  __syncwarp();
-  const int p0 = blockIdx.x * kChunk;
-  const int p1 = min(P, p0 + kChunk);
-  for (int base = p0; base < p1; base += 32) {
-    const int p = base + lane;
-    int e = (p < p1) ? __ldg(idx + p) : -1;
-    if (e >= E) e = -1;                             // invalid ids were flagged by the count pass
+// Stable placement of the pairs sidx[0, n) (ids p0 + i) by one warp: ctr[e]
+// holds the next row of expert e and advances as the warp walks the pairs.
+__device__ __forceinline__ void scatter_walk(const int* sidx, int n, int p0, int* ctr, int32_t* __restrict__ perm,
+                                             int32_t* __restrict__ inv) {
+  const int lane = threadIdx.x & 31;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int e = (i < n) ? sidx[i] : -2;
     const uint32_t peers = __match_any_sync(0xFFFFFFFFu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (e >= 0) pos = ctr[e] + rank;
+    const int pos = (e >= 0) ? ctr[e] + rank : 0;
     __syncwarp();
     if (e >= 0 && (__ffs(peers) - 1) == lane) ctr[e] += __popc(peers);
     __syncwarp();
     if (e >= 0) {
-      perm[pos] = p;
-      inv[p] = pos;
+      perm[pos] = p0 + i;
+      inv[p0 + i] = pos;
+    } else if (e == -1) {
+      inv[p0 + i] = -1;
     }
   }
+}
+
+// One block of 256 threads per chunk: stage the chunk's expert ids and the
+// chunk's first row per expert in shared memory, then one warp places them.
+__global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __restrict__ idx, int P, int E,
+                                                              const int32_t* __restrict__ chunk_hist,
+                                                              const int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ perm,
+                                                              int32_t* __restrict__ inv) {
+  __shared__ int ctr[1024];
+  __shared__ int sidx[kChunk];
+  const int p0 = blockIdx.x * kChunk;
+  const int n = min(P, p0 + kChunk) - p0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) ctr[e] = offsets[e] + chunk_hist[(int64_t)blockIdx.x * E + e];
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = __ldg(idx + p0 + i);
+    sidx[i] = (e >= 0 && e < E) ? e : -1;         // invalid ids were flagged by the count pass
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) scatter_walk(sidx, n, p0, ctr, perm, inv);
+}
+
+// All pairs in one chunk (P <= kChunk): count, scan and scatter in one block of
+// 1024 threads.  Group E (the shared expert) has has_shared ? T : 0 rows.
+__global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __restrict__ idx, int P, int E, int T,
+                                                             int has_shared, int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ perm,
+                                                             int32_t* __restrict__ inv) {
+  __shared__ int hist[1024];
+  __shared__ int sidx[kChunk];
+  __shared__ int warp_sums[32];
+  const int tid = threadIdx.x;
+  hist[tid] = 0;
+  __syncthreads();
+  for (int i = tid; i < P; i += blockDim.x) {
+    int e = __ldg(idx + i);
+    if (e < 0 || e >= E) {
+      record_error(MOE_ERR_INVALID);
+      e = -1;
+    } else {
+      atomicAdd(&hist[e], 1);
+    }
+    sidx[i] = e;
+  }
+  __syncthreads();
+  // exclusive scan of the group sizes (thread e: group e, e <= E < 1024)
+  const int c = tid < E ? hist[tid] : (tid == E && has_shared ? T : 0);
+  const int lane = tid & 31, wid = tid >> 5;
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int sum = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, sum, o);
+      if (lane >= o) sum += y;
+    }
+    warp_sums[lane] = sum;
+  }
+  __syncthreads();
+  const int excl = (wid ? warp_sums[wid - 1] : 0) + x - c;
+  if (tid <= E) {
+    counts[tid] = c;
+    offsets[tid] = excl;
+    if (tid == E) offsets[E + 1] = excl + c;
+  }
+  __syncthreads();                  // every thread has read hist[tid]
+  if (tid < E) hist[tid] = excl;    // reused as the running row of each expert
+  __syncthreads();
+  if (tid < 32) scatter_walk(sidx, P, 0, hist, perm, inv);
 }
 
 // One warp per row.  H % 128 == 0, rows 16-byte aligned.
@@ -261,6 +336,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j = 0; j < k; ++j) {
     const int r = __ldg(inv + (int64_t)t * k + j);
+    if (r < 0) continue;            // a pair the grouping rejected (invalid expert id)
     const float wj = __ldg(w + (int64_t)t * k + j);
     const float4 v = __ldg(o + (int64_t)r * h4 + c);
     acc.x = fmaf(wj, v.x, acc.x);

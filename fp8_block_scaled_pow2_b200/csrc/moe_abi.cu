@@ -196,6 +196,27 @@ int moe_route_topk(const float* logits, int T, int E, int k, float route_scale, 
   return launch_status();
 }
 
+// The a3 passes on one stream (arguments already validated).  hist: per-chunk
+// expert counters, unused when all pairs fit in one chunk.
+static void launch_permute(const int32_t* idx, int T, int E, int k, int has_shared, const uint8_t* xq,
+                           const uint8_t* sx, int H, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                           uint8_t* xq_perm, uint8_t* sx_perm, int32_t* hist, cudaStream_t st) {
+  const int P = T * k;
+  const int n_chunks = (P + kChunk - 1) / kChunk;
+  if (n_chunks <= 1) {
+    permute_small_kernel<<<1, 1024, 0, st>>>(idx, P, E, T, has_shared ? 1 : 0, counts, offsets, perm, inv);
+  } else {
+    permute_count_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist);
+    permute_scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
+    permute_scatter_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
+  }
+  const int64_t R = (int64_t)P + (has_shared ? T : 0);
+  if (R > 0)
+    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
+        sx_perm);
+}
+
 size_t moe_permute_workspace_size(int T, int E, int k) {
   if (T <= 0 || E <= 0 || k <= 0) return 256;
   const int64_t P = (int64_t)T * k;
@@ -210,22 +231,13 @@ int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared, const u
   if (!counts || !offsets) return MOE_ERR_INVALID;
   if ((int64_t)T * k > (int64_t)1 << 30) return MOE_ERR_UNSUPPORTED;
   cudaStream_t st = S(stream);
-  const int P = T * k;
-  const int n_chunks = (P + kChunk - 1) / kChunk;
   if (T > 0) {
     if (!idx || !xq || !sx || !perm || !inv || !xq_perm || !sx_perm || !workspace) return MOE_ERR_INVALID;
     if (!aligned(xq, 16) || !aligned(xq_perm, 16) || !aligned(workspace, 16)) return MOE_ERR_INVALID;
     if (workspace_bytes < moe_permute_workspace_size(T, E, k)) return MOE_ERR_INVALID;
   }
   int32_t* hist = reinterpret_cast<int32_t*>(workspace);
-  if (n_chunks > 0) permute_count_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist);
-  permute_scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
-  if (n_chunks > 0) permute_scatter_kernel<<<n_chunks, 32, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
-  const int64_t R = (int64_t)P + (has_shared ? T : 0);
-  if (R > 0)
-    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
-        sx_perm);
+  launch_permute(idx, T, E, k, has_shared, xq, sx, H, counts, offsets, perm, inv, xq_perm, sx_perm, hist, st);
   return launch_status();
 }
 
@@ -506,14 +518,7 @@ int moe_permute_noalloc(const int32_t* idx, int T, int E, int k, int has_shared,
   cudaStream_t st = S(stream);
   // every counter the scan reads is written by the count pass of this call,
   // so the scratch needs no clearing between calls
-  if (n_chunks > 0) permute_count_kernel<<<(unsigned)n_chunks, 256, 0, st>>>(idx, P, E, hist);
-  permute_scan_kernel<<<1, 1024, 0, st>>>(hist, (int)n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
-  if (n_chunks > 0) permute_scatter_kernel<<<(unsigned)n_chunks, 32, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
-  const int64_t R = (int64_t)P + (has_shared ? T : 0);
-  if (R > 0)
-    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
-        sx_perm);
+  launch_permute(idx, T, E, k, has_shared, xq, sx, H, counts, offsets, perm, inv, xq_perm, sx_perm, hist, st);
   return launch_status();
 }
 

@@ -118,13 +118,13 @@ int moe_route_topk(const float* logits, int T, int E, int k, float route_scale,
  * group E the shared expert (one row per token when has_shared != 0, none
  * otherwise).  Within a routed group rows are in ascending pair id p = t*k+j;
  * shared rows follow in token order.
- *   idx      int32 [T, k] expert ids in [0, E)   (out-of-range ids: device
- *            error MOE_ERR_INVALID, outputs unspecified)
+ *   idx      int32 [T, k] expert ids in [0, E)   (an out-of-range id: device
+ *            error MOE_ERR_INVALID; that pair gets no row and inv = -1)
  *   xq, sx   outputs of moe_quantize_act_fp8 for H columns (H % 128 == 0)
  *   counts   int32 [E+1];  offsets int32 [E+2] (exclusive prefix of counts)
  *   perm     int32 [R], R = T*k + (has_shared ? T : 0): source id of row r,
  *            the pair id p for routed rows, T*k + t for the shared row of t
- *   inv      int32 [T*k]: row of pair p
+ *   inv      int32 [T*k]: row of pair p (-1 for a pair with an invalid id)
  *   xq_perm  uint8 [R, H] (16-byte aligned), sx_perm uint8 [R, H/128]:
  *            the rows of xq / sx of each row's source token
  *   workspace  device scratch of moe_permute_workspace_size(T, E, k) bytes,
@@ -253,7 +253,8 @@ int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq,
  * a7 -- combine [SI 架构特性]:
  *   y[t] = sum_{j<k} w[t, j] * o[inv[t*k+j]] + (has_shared ? o[offsets[E] + t] : 0)
  * accumulated in float32 in slot order, rounded once to bfloat16 (nearest even).
- *   o  float32 [R, H] (16-byte aligned), H % 4 == 0;  inv int32 [T*k];
+ *   o  float32 [R, H] (16-byte aligned), H % 4 == 0;  inv int32 [T*k]
+ *      (a negative entry, a pair the grouping rejected, contributes nothing);
  *   w  float32 [T, k];  offsets int32 [E+2] (device);  y bfloat16 [T, H]
  */
 int moe_combine(const float* o, const int32_t* inv, const float* w, int T, int k, int H,

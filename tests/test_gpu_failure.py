@@ -34,18 +34,44 @@ def test_invalid_arguments_raise_before_launch(lib):
                                  torch.empty((4, 1), dtype=torch.uint8, device="cuda"))
 
 
-def test_out_of_range_expert_id_is_flagged(lib):
-    T, E, k, H = 4, 8, 2, 128
-    idx = torch.tensor([[0, 1], [2, 9], [3, 4], [5, 6]], dtype=torch.int32, device="cuda")   # 9 >= E
+@pytest.mark.parametrize("T", [4, 600])
+def test_out_of_range_expert_id_is_flagged(lib, T):
+    """An expert id outside [0, E) is flagged; that pair gets no row, its inv
+    entry is -1, and the combine leaves it out.  T = 4 runs the one-block
+    grouping, T = 600 (2400 pairs) the chunked passes."""
+    E, k, H = 8, 4, 128
+    idx_np = (np.arange(T * k, dtype=np.int32) % E).reshape(T, k)
+    bad = (1, 3) if T == 4 else (577, 2)
+    idx_np[bad] = 9                                                           # 9 >= E
+    idx = torch.from_numpy(idx_np).cuda()
     xq = torch.zeros((T, H), dtype=torch.uint8, device="cuda")
     sx = torch.zeros((T, 1), dtype=torch.uint8, device="cuda")
     R = T * k + T
-    out = [torch.empty(E + 1, dtype=torch.int32, device="cuda"), torch.empty(E + 2, dtype=torch.int32, device="cuda"),
-           torch.empty(R, dtype=torch.int32, device="cuda"), torch.empty(T * k, dtype=torch.int32, device="cuda"),
-           torch.empty((R, H), dtype=torch.uint8, device="cuda"), torch.empty((R, 1), dtype=torch.uint8, device="cuda")]
+    counts, offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda"), torch.empty(E + 2, dtype=torch.int32,
+                                                                                          device="cuda")
+    perm, inv = torch.empty(R, dtype=torch.int32, device="cuda"), torch.empty(T * k, dtype=torch.int32, device="cuda")
+    xqp, sxp = torch.empty((R, H), dtype=torch.uint8, device="cuda"), torch.empty((R, 1), dtype=torch.uint8, device="cuda")
     ws = torch.empty(lib.moe_permute_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
-    lib.moe_permute(idx, E, 1, xq, sx, *out, ws)
+    lib.moe_permute(idx, E, 1, xq, sx, counts, offsets, perm, inv, xqp, sxp, ws)
+    torch.cuda.synchronize()
     assert lib.moe_get_device_error() == -1
+    p_bad = bad[0] * k + bad[1]
+    inv_h = inv.cpu().numpy()
+    assert inv_h[p_bad] == -1
+    assert int(counts[:E].sum()) == T * k - 1
+    good = np.delete(np.arange(T * k), p_bad)
+    np.testing.assert_array_equal(np.sort(inv_h[good]), np.arange(T * k - 1))
+    # combine over rows o[r] = r: the rejected slot adds nothing
+    o = torch.arange(R, dtype=torch.float32, device="cuda")[:, None].repeat(1, H).contiguous()
+    w = torch.ones((T, k), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    lib.moe_combine(o, inv, w, 1, offsets, E, y)
+    torch.cuda.synchronize()
+    off_h = offsets.cpu().numpy()
+    t = bad[0]
+    expect = sum(float(inv_h[t * k + j]) for j in range(k) if j != bad[1]) + float(off_h[E] + t)
+    assert float(y[t, 0]) == float(torch.tensor(expect).to(torch.bfloat16))
+    assert lib.moe_get_device_error() == 0
 
 
 @pytest.mark.parametrize("bad", ["past_rows", "decreasing", "nonzero_start"])

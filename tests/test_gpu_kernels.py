@@ -77,8 +77,9 @@ def test_route_topk(lib, T, E, k):
 
 
 # ------------------------------- a3 ---------------------------------------
-@pytest.mark.parametrize("T,E,k,has_shared", [(0, 8, 2, 1), (1, 8, 2, 1), (16, 8, 2, 0), (700, 257, 6, 1),
-                                              (2049, 3, 1, 1), (4096, 256, 6, 1)])
+@pytest.mark.parametrize("T,E,k,has_shared", [(0, 8, 2, 1), (1, 8, 2, 1), (16, 8, 2, 0), (341, 256, 6, 1),
+                                              (512, 64, 4, 0), (700, 257, 6, 1), (2049, 3, 1, 1),
+                                              (4096, 256, 6, 1)])
 def test_permute_bit_exact(lib, T, E, k, has_shared):
     H = 256
     if T:
