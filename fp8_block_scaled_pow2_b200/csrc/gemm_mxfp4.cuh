@@ -128,12 +128,11 @@ struct Cfg {
 //   header   int32[4]: n_items, n_tiles, n_ft, BN
 //   prefix   int32[G+1]: first work item of each group
 //   tstart   int32[G]:   first token tile of each group
-//   groups   int2[G]:    (first row, rows) of each group, rows 0 for an invalid group
-//   tiles    int2[max_tiles]: (first row, rows) of each token tile
+//   groups   int2[G]:    (first row, rows) of each group, rows 0 for an invalid plan
 //   a_sf     uint8[max_tiles * KG * NA * 512]: per-tile activation scales, interleaved
 //            for tensor memory, four 128-wide K steps per 512-byte block (KG = ceil(KT/4))
 struct WsLayout {
-  size_t header, prefix, tstart, groups, tiles, a_sf, total;
+  size_t header, prefix, tstart, groups, a_sf, total;
   int max_tiles;
 };
 
@@ -147,105 +146,112 @@ inline WsLayout ws_layout(int a_rows, int G, int K, int BN) {
   L.prefix = align256(16);
   L.tstart = L.prefix + align256(4 * (size_t)(G + 1));
   L.groups = L.tstart + align256(4 * (size_t)G);
-  L.tiles = L.groups + align256(8 * (size_t)G);
-  L.a_sf = L.tiles + align256(8 * (size_t)L.max_tiles);
+  L.a_sf = L.groups + align256(8 * (size_t)G);
   L.total = L.a_sf + align256((size_t)L.max_tiles * ((KT + 3) / 4) * NA * 512);
   return L;
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
-__device__ inline int block_exclusive_scan_1024(int v, int* total) {
-  __shared__ int warp_sums[32];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int x = v;
+constexpr int kPrepThreads = 128;
+constexpr int kPrepPerThread = (kMaxGroups + kPrepThreads) / kPrepThreads;   // covers G + 1 entries
+
+// Plan and token scales of one GEMM call in one launch; one block per token
+// tile (grid = the tile bound ceil(a_rows / BN) + G).  Every block loads the
+// group offsets and scans the tile counts itself (G <= 1024: 9 entries per
+// thread), finds its tile, and interleaves that tile's per-128 activation
+// scales into the tensor-memory scale order: for token n of a 128-row block,
+// the 32-bit word at byte (n % 32) * 16 + (n / 32) * 4 of block (tile, g)
+// holds its scales of the K steps 4g .. 4g+3, one per byte (the MMA of K step
+// kt selects byte kt % 4); rows past the tile and K steps past K are 0.
+// Block 0 writes the plan.  Unless the offsets are nondecreasing from
+// offsets[0] = 0 to offsets[G] <= a_rows, the plan has no work and
+// MOE_ERR_INVALID is recorded, so no tile ever addresses rows outside the
+// operands or the workspace.
+__global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* __restrict__ offsets, int G,
+                                                                 int a_rows, int BN, int n_ft,
+                                                                 const uint8_t* __restrict__ sx, int KT,
+                                                                 int* __restrict__ header, int* __restrict__ prefix,
+                                                                 int* __restrict__ tstart, int2* __restrict__ groups,
+                                                                 uint8_t* __restrict__ a_sf) {
+  __shared__ int s_off[kMaxGroups + 1];
+  __shared__ int s_t0[kMaxGroups + 1];      // first tile of each group; s_t0[G] = tiles in all
+  __shared__ int s_warp[kPrepThreads / 32];
+  const int tid = threadIdx.x;
+  for (int g = tid; g <= G; g += kPrepThreads) s_off[g] = offsets[g];
+  __syncthreads();
+  bool bad = false;
+  for (int g = tid; g < G; g += kPrepThreads)
+    bad |= s_off[g + 1] < s_off[g] || (g == 0 && s_off[0] != 0) || (g == G - 1 && s_off[G] > a_rows);
+  bad = __syncthreads_or(bad);
+  // exclusive scan of the tile counts; thread tid owns groups [tid*P, tid*P + P)
+  const int g0 = tid * kPrepPerThread;
+  int nt[kPrepPerThread];
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < kPrepPerThread; ++i) {
+    const int g = g0 + i;
+    nt[i] = (!bad && g < G) ? ceil_div(s_off[g + 1] - s_off[g], BN) : 0;
+    local += nt[i];
+  }
+  const int lane = tid & 31, wid = tid >> 5;
+  int x = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) warp_sums[wid] = x;
+  if (lane == 31) s_warp[wid] = x;
   __syncthreads();
-  if (wid == 0) {
-    int s = warp_sums[lane];
+  int base = x - local;
+  for (int w = 0; w < wid; ++w) base += s_warp[w];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xFFFFFFFFu, s, o);
-      if (lane >= o) s += y;
+  for (int i = 0; i < kPrepPerThread; ++i) {
+    const int g = g0 + i;
+    if (g <= G) s_t0[g] = base;
+    base += nt[i];
+  }
+  __syncthreads();
+  const int n_tiles = s_t0[G];
+  if (blockIdx.x == 0) {
+    if (bad && tid == 0) record_error(MOE_ERR_INVALID);
+    for (int g = tid; g < G; g += kPrepThreads) {
+      tstart[g] = s_t0[g];
+      prefix[g] = s_t0[g] * n_ft;
+      groups[g] = bad ? make_int2(0, 0) : make_int2(s_off[g], s_off[g + 1] - s_off[g]);
     }
-    warp_sums[lane] = s;
+    if (tid == 0) {
+      prefix[G] = n_tiles * n_ft;
+      header[0] = n_tiles * n_ft;
+      header[1] = n_tiles;
+      header[2] = n_ft;
+      header[3] = BN;
+    }
   }
-  __syncthreads();
-  const int base = wid ? warp_sums[wid - 1] : 0;
-  *total = warp_sums[31];
-  __syncthreads();
-  return base + x - v;
-}
-
-// One block of 1024 threads; thread g handles group g (G <= 1024).  Unless
-// the offsets are nondecreasing from offsets[0] = 0 to offsets[G] <= a_rows,
-// the call records MOE_ERR_INVALID and plans no work at all, so no tile ever
-// addresses rows outside the operands or the workspace.
-__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ offsets, int G, int a_rows,
-                                                    int BN, int n_ft, int* __restrict__ header,
-                                                    int* __restrict__ prefix, int* __restrict__ tstart,
-                                                    int2* __restrict__ groups, int2* __restrict__ tiles) {
-  const int g = threadIdx.x;
-  int rows = 0, r0 = 0;
-  bool bad = false;
-  if (g < G) {
-    r0 = offsets[g];
-    rows = offsets[g + 1] - r0;
-    bad = rows < 0 || (g == 0 && r0 != 0) || (g == G - 1 && offsets[G] > a_rows);
+  const int t = blockIdx.x;
+  if (t >= n_tiles) return;
+  // the group of tile t: the last g with s_t0[g] <= t (empty groups share
+  // their successor's first tile and sort before it)
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_t0[mid] <= t) lo = mid; else hi = mid - 1;
   }
-  if (__syncthreads_or(bad)) {
-    if (g == 0) record_error(MOE_ERR_INVALID);
-    rows = 0;
-    r0 = 0;
-  }
-  const int nt = ceil_div(rows, BN);
-  int n_tiles, n_items;
-  const int t0 = block_exclusive_scan_1024(nt, &n_tiles);
-  const int i0 = block_exclusive_scan_1024(nt * n_ft, &n_items);
-  if (g < G) {
-    tstart[g] = t0;
-    prefix[g] = i0;
-    groups[g] = make_int2(r0, rows);
-    for (int j = 0; j < nt; ++j) tiles[t0 + j] = make_int2(r0 + j * BN, min(BN, rows - j * BN));
-  }
-  if (g == 0) {
-    prefix[G] = n_items;
-    header[0] = n_items;
-    header[1] = n_tiles;
-    header[2] = n_ft;
-    header[3] = BN;
-  }
-}
-
-// Interleave the per-128 activation scales of each token tile into the
-// tensor-memory scale order.  For token n of a 128-row block, the 32-bit word
-// at byte (n % 32) * 16 + (n / 32) * 4 of block (tile, g) holds its scales
-// of the four K steps 4g .. 4g+3, one per byte; the MMA of K step kt selects
-// byte kt % 4.  Rows past the tile and K steps past K are 0.
-__global__ void __launch_bounds__(128) tile_act_scales_kernel(const uint8_t* __restrict__ sx, int KT,
-                                                              const int* __restrict__ header,
-                                                              const int2* __restrict__ tiles, int NA,
-                                                              uint8_t* __restrict__ a_sf) {
-  const int t = blockIdx.x, g = blockIdx.y;
-  if (t >= header[1]) return;
-  const int KG = (KT + 3) / 4;
-  const int2 tr = tiles[t];
-  const int n = threadIdx.x;
-  for (int a = 0; a < NA; ++a) {
-    const int r = a * 128 + n;
-    uint32_t w = 0;
-    if (r < tr.y) {
-      const uint8_t* src = sx + (size_t)(tr.x + r) * KT;
+  const int row0 = s_off[lo] + (t - s_t0[lo]) * BN;
+  const int rows = min(BN, s_off[lo + 1] - row0);
+  const int KG = (KT + 3) / 4, NA = ceil_div(BN, 128);
+  for (int kg = 0; kg < KG; ++kg) {
+    for (int a = 0; a < NA; ++a) {
+      const int n = tid;
+      const int r = a * 128 + n;
+      uint32_t w = 0;
+      if (r < rows) {
+        const uint8_t* src = sx + (size_t)(row0 + r) * KT;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (4 * g + j < KT) w |= (uint32_t)src[4 * g + j] << (8 * j);
+        for (int j = 0; j < 4; ++j)
+          if (4 * kg + j < KT) w |= (uint32_t)src[4 * kg + j] << (8 * j);
+      }
+      uint8_t* blk = a_sf + ((size_t)(t * KG + kg) * NA + a) * 512;
+      *reinterpret_cast<uint32_t*>(blk + (n & 31) * 16 + (n >> 5) * 4) = w;
     }
-    uint8_t* blk = a_sf + ((size_t)(t * KG + g) * NA + a) * 512;
-    *reinterpret_cast<uint32_t*>(blk + (n & 31) * 16 + (n >> 5) * 4) = w;
   }
 }
 

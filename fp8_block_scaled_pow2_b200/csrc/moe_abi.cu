@@ -311,13 +311,10 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   // SwiGLU, which requires N % 256 == 0)
   const bool pair = epilogue == MOE_EPI_SWIGLU_QUANT || N % 256 == 0;
   const int n_ft = pair ? N / 256 : N / 128;
-  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, (int)a_rows, block_n, n_ft,
-                                        reinterpret_cast<int*>(ws + L.header), reinterpret_cast<int*>(ws + L.prefix),
-                                        reinterpret_cast<int*>(ws + L.tstart), reinterpret_cast<int2*>(ws + L.groups),
-                                        reinterpret_cast<int2*>(ws + L.tiles));
-  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
-      a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
-      reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
+  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+      offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
+      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   switch (epilogue) {
     case MOE_EPI_STORE_F32:
@@ -370,13 +367,10 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
   args.limit = swiglu_limit;
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
-  gemm::plan_kernel<<<1, 1024, 0, st>>>(offsets, n_groups, (int)a_rows, block_n, n_ft,
-                                        reinterpret_cast<int*>(ws + L.header), reinterpret_cast<int*>(ws + L.prefix),
-                                        reinterpret_cast<int*>(ws + L.tstart), reinterpret_cast<int2*>(ws + L.groups),
-                                        reinterpret_cast<int2*>(ws + L.tiles));
-  gemm::tile_act_scales_kernel<<<dim3(L.max_tiles, (K / 128 + 3) / 4), 128, 0, st>>>(
-      a_e8m0_128, K / 128, reinterpret_cast<const int*>(ws + L.header),
-      reinterpret_cast<const int2*>(ws + L.tiles), (block_n + 127) / 128, ws + L.a_sf);
+  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+      offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
+      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   if (dual) {
     switch (block_n) {

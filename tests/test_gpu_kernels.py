@@ -164,6 +164,19 @@ def test_gemm_integer_exact(lib, block_n, N):
     no_device_error(lib)
 
 
+def test_gemm_max_groups(lib):
+    """1024 groups (the limit), a third of them empty: the plan's scan over
+    all groups and the tile search at the last groups."""
+    sizes = (synth.splitmix64(11, 0, 1024) % np.uint64(6)).astype(np.int64) - 2
+    sizes = np.maximum(sizes, 0)
+    sizes[-1] = 3
+    a, asc, offsets, w, wsc = _gemm_inputs(11, sizes.tolist(), 256, 128, True)
+    out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, 16)
+    ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
+
+
 @pytest.mark.parametrize("N", [384, 512])
 @pytest.mark.parametrize("block_n", [16, 128])
 def test_gemm_random_scaled(lib, block_n, N):
