@@ -33,7 +33,12 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s or HBM GB/s vs B200 roofline"
-KERNELS_PER_STEP = 13     # quant 1, route 1, permute 4, gemm 3 + 3, combine 1
+def kernels_per_step(wl: dict) -> int:
+    """Library kernels one layer step launches: quant 1, route 1, grouping 2
+    (one block for <= 2048 routed pairs, then the gather) or 4 (chunked), two
+    GEMM calls of 2 (prep + GEMM), combine 1."""
+    grouping = 2 if wl["T"] * wl["k"] <= 2048 else 4
+    return 1 + 1 + grouping + 2 * 2 + 1
 
 WORKLOADS = {
     "repack": dict(T=0, H=4096, I=2048, E=256, k=6, logits="uniform"),
@@ -320,9 +325,31 @@ def run_ours(args, wl):
     xd = torch.from_numpy(x.view(np.int16)).cuda()
     ld = torch.from_numpy(logits).cuda()
     stream = torch.cuda.current_stream()
+    use_graph = args.graph == "on"
+    segs = layer.segments(xd, ld, buf)
+    if use_graph:
+        # each of the four segments (pre, w1/w3, w2, combine) becomes a CUDA
+        # graph, so the GEMM events still fall between replays
+        for _ in range(2):
+            for f in segs:
+                f()
+        torch.cuda.synchronize()
+        graphs = []
+        for f in segs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                f()
+            graphs.append(g)
+        torch.cuda.synchronize()
+        runners = [g.replay for g in graphs]
+    else:
+        runners = list(segs)
 
     def step(ev=None):
-        layer.forward(xd, ld, buf, marks=ev)
+        for i, run in enumerate(runners):
+            if ev and i > 0:
+                ev[i - 1].record(stream)
+            run()
 
     clk = ClockSampler(local).start()
     for _ in range(args.warmup):
@@ -354,13 +381,13 @@ def run_ours(args, wl):
     xh = torch.from_numpy(x.view(np.int16)).pin_memory()
     lh = torch.from_numpy(logits).pin_memory()
     yh = torch.empty((T, wl["H"]), dtype=torch.bfloat16).pin_memory()
-    xd2, ld2 = torch.empty_like(xd), torch.empty_like(ld)
 
     def e2e_step():
-        xd2.copy_(xh, non_blocking=True)
-        ld2.copy_(lh, non_blocking=True)
-        y = layer.forward(xd2, ld2, buf)
-        yh.copy_(y, non_blocking=True)
+        # the step's inputs land in the buffers the segments (or graphs) read
+        xd.copy_(xh, non_blocking=True)
+        ld.copy_(lh, non_blocking=True)
+        step()
+        yh.copy_(buf.y, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
@@ -405,6 +432,7 @@ def run_ours(args, wl):
                                f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {T} tokens per GPU",
                    "weights": args.weights,
                    "tokens_per_gpu": T, "parallelism": f"replicas x{world} (data parallel, no collective)",
+                   "cuda_graph": use_graph,
                    "l2": f"inputs larger than L2: {ab['active_experts']} active experts stream "
                          f"{(ab['w13'] + ab['w2']) / 1e9:.2f} GB of weights per step"},
         "roofline": roof,
@@ -417,7 +445,7 @@ def run_ours(args, wl):
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xh.numel() * 2 + lh.numel() * 4),
                 "d2h_bytes_per_step": int(yh.numel() * 2)},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
@@ -531,6 +559,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--weights", choices=["mxfp4", "w4afp8"], default="mxfp4")
+    ap.add_argument("--graph", choices=["on", "off"], default="on",
+                    help="replay the layer step as four CUDA graphs (off: eager library calls)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

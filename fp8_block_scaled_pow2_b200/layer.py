@@ -115,6 +115,46 @@ class MoeLayer:
             ws_permute=torch.empty(moe.moe_permute_workspace_size(T, self.E, k), dtype=u8, device=d),
             ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n)
 
+    def segments(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers, stream=None):
+        """The forward pass as four callables run in order on `stream`:
+        (quantise + route + group, w1/w3 GEMM with SwiGLU, w2 GEMM, combine).
+        Each only enqueues library calls, so each can be captured in a CUDA
+        graph; forward() runs them eagerly."""
+        b = buf
+        g_off = b.offsets if self.has_shared else b.offsets[: self.G + 1]
+
+        def pre():
+            moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
+            moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
+            moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
+                            b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
+
+        if self.weights == "mxfp4":
+            def gemm13():
+                moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13_p, self.G, 2 * self.I,
+                                           moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
+                                           b.block_n, stream=stream)
+
+            def gemm2():
+                moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.G, self.H, moe.MOE_EPI_STORE_F32,
+                                           b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        else:
+            bn = min(b.block_n, 64) if b.block_n else 0
+
+            def gemm13():
+                moe.moe_grouped_gemm_w4afp8(b.xq_perm, b.sx_perm, g_off, self.w13_q, self.w13_sinv,
+                                            moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
+                                            bn, stream=stream)
+
+            def gemm2():
+                moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
+                                            b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+
+        def post():
+            moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)
+
+        return pre, gemm13, gemm2, post
+
     def forward(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers | None = None,
                 stream=None, marks=None) -> torch.Tensor:
         """x bfloat16 [T, H] (or its uint16 bits), logits float32 [T, E] -> y bfloat16 [T, H].
@@ -124,33 +164,9 @@ class MoeLayer:
         T = x.shape[0]
         if buf is None or buf.T != T:
             buf = self.alloc(T)
-        b = buf
-        moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
-        moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
-        moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
-                        b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
-        g_off = b.offsets if self.has_shared else b.offsets[: self.G + 1]
         ev_stream = stream if stream is not None else torch.cuda.current_stream()
-        if marks:
-            marks[0].record(ev_stream)
-        if self.weights == "mxfp4":
-            moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13_p, self.G, 2 * self.I,
-                                       moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
-                                       b.block_n, stream=stream)
-            if marks:
-                marks[1].record(ev_stream)
-            moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.G, self.H, moe.MOE_EPI_STORE_F32, b.o,
-                                       None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
-        else:
-            bn = min(b.block_n, 64) if b.block_n else 0
-            moe.moe_grouped_gemm_w4afp8(b.xq_perm, b.sx_perm, g_off, self.w13_q, self.w13_sinv,
-                                        moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
-                                        bn, stream=stream)
-            if marks:
-                marks[1].record(ev_stream)
-            moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
-                                        b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
-        if marks:
-            marks[2].record(ev_stream)
-        moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)
-        return b.y
+        for i, seg in enumerate(self.segments(x, logits, buf, stream)):
+            if marks and i > 0:
+                marks[i - 1].record(ev_stream)
+            seg()
+        return buf.y

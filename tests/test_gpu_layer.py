@@ -127,3 +127,37 @@ def test_long_prefill_w4afp8_sampled(lib):
     toks = np.sort((synth.splitmix64(0, 78, 4) % np.uint64(T)).astype(np.int64))
     ref = _w4a_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
     check_y(y.float().cpu().numpy()[toks], ref["y"])
+
+
+def test_segment_graphs_match_eager(lib):
+    """The forward pass captured as four CUDA graphs (one per segment, as the
+    decode benchmark replays it) gives the eager result bit for bit, also
+    after new inputs are copied into the captured buffers."""
+    wl = synth.tiny_layer(2)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    buf = layer.alloc(wl.T)
+    x = torch.from_numpy(wl.x_bf16.view(np.int16)).cuda()
+    lg = torch.from_numpy(wl.logits).cuda()
+    segs = layer.segments(x, lg, buf)
+    for f in segs:
+        f()
+    torch.cuda.synchronize()
+    graphs = []
+    for f in segs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        graphs.append(g)
+    wl2 = synth.tiny_layer(3)
+    for src_x, src_l in ((wl.x_bf16, wl.logits), (wl2.x_bf16, wl2.logits)):
+        x.copy_(torch.from_numpy(src_x.view(np.int16)))
+        lg.copy_(torch.from_numpy(src_l))
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+        y_graph = buf.y.clone()
+        layer.forward(x, lg, buf)
+        torch.cuda.synchronize()
+        assert torch.equal(y_graph.view(torch.int16), buf.y.view(torch.int16))
+    assert lib.moe_get_device_error() == 0
+    del graphs
