@@ -429,13 +429,26 @@ int repack_mxfp4_to_nvfp4(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mat
   const int64_t fp4_bytes = n_mats * (int64_t)N * (K / 2);
   if (fp4_bytes % 16) return MOE_ERR_INVALID;
   cudaStream_t st = S(stream);
-  nvfp4_global_kernel<<<(unsigned)n_mats, 256, 0, st>>>(e8m0, per_mat, out_global);
   const bool alias = out_fp4 == fp4;
-  const int64_t work = std::max<int64_t>(n_scale, alias ? 0 : fp4_bytes / 16);
-  const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
-  nvfp4_convert_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
-      e8m0, n_scale, per_mat, out_global, out_e4m3, reinterpret_cast<const uint4*>(fp4),
-      alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
+  // 16 scale bytes at a time when the scale arrays allow it
+  const bool vec = per_mat % 16 == 0 && aligned(e8m0, 16) && aligned(out_e4m3, 16);
+  if (vec) {
+    nvfp4_global_vec_kernel<<<(unsigned)n_mats, 512, 0, st>>>(reinterpret_cast<const uint4*>(e8m0), per_mat / 16,
+                                                             out_global);
+    const int64_t work = std::max<int64_t>(n_scale / 16, alias ? 0 : fp4_bytes / 16);
+    const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
+    nvfp4_convert_vec_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(e8m0), n_scale / 16, per_mat / 16, out_global,
+        reinterpret_cast<uint4*>(out_e4m3), reinterpret_cast<const uint4*>(fp4),
+        alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
+  } else {
+    nvfp4_global_kernel<<<(unsigned)n_mats, 256, 0, st>>>(e8m0, per_mat, out_global);
+    const int64_t work = std::max<int64_t>(n_scale, alias ? 0 : fp4_bytes / 16);
+    const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
+    nvfp4_convert_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
+        e8m0, n_scale, per_mat, out_global, out_e4m3, reinterpret_cast<const uint4*>(fp4),
+        alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
+  }
   return launch_status();
 }
 
@@ -446,10 +459,9 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
   if (!fp4 || !e8m0 || !out_int4 || !out_scale_inv) return MOE_ERR_INVALID;
   if (!aligned(fp4, 16) || !aligned(out_int4, 16) || !aligned(e8m0, 4) || !aligned(out_scale_inv, 4))
     return MOE_ERR_INVALID;
-  const int64_t groups = n_mats * (int64_t)N * (K / 128);
-  int4g128_kernel<<<(unsigned)((groups + 255) / 256), 256, 0, S(stream)>>>(
-      reinterpret_cast<const uint4*>(fp4), reinterpret_cast<const uint32_t*>(e8m0), groups,
-      reinterpret_cast<uint4*>(out_int4), out_scale_inv);
+  const int64_t blocks = n_mats * (int64_t)N * (K / 32);     // 32-element blocks, 4 per group
+  int4g128_kernel<<<(unsigned)((blocks + 255) / 256), 256, 0, S(stream)>>>(
+      reinterpret_cast<const uint4*>(fp4), e8m0, blocks, reinterpret_cast<uint4*>(out_int4), out_scale_inv);
   return launch_status();
 }
 

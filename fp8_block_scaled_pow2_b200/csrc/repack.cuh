@@ -88,68 +88,148 @@ __global__ void __launch_bounds__(256) nvfp4_convert_kernel(const uint8_t* __res
     for (int64_t i = tid; i < n_fp4_16; i += stride) out_fp4[i] = __ldg(fp4 + i);
 }
 
-// INT4 group-128: one thread per (row, group of 128): 64 nibble bytes and 4
-// scale bytes in, 64 bytes and one float32 out.
-__global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__ fp4, const uint32_t* __restrict__ e8m0,
-                                                       int64_t n_groups, uint4* __restrict__ out,
-                                                       float* __restrict__ scale_inv) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= n_groups) return;
+// Vector forms of the two NVFP4 passes, used when the scale arrays are
+// 16-byte aligned and a matrix holds a multiple of 16 scales.
+// Pass 1: min / max of the bytes 16 at a time (255 is the largest byte, so a
+// NaN scale shows as max == 255).
+__global__ void __launch_bounds__(512) nvfp4_global_vec_kernel(const uint4* __restrict__ e8m0, int64_t per_mat16,
+                                                               float* __restrict__ out_global) {
+  const int64_t m = blockIdx.x;
+  const uint4* s = e8m0 + m * per_mat16;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int64_t i = threadIdx.x; i < per_mat16; i += blockDim.x) {
+    const uint4 v = __ldg(s + i);
+    lo = __vminu4(lo, __vminu4(__vminu4(v.x, v.y), __vminu4(v.z, v.w)));
+    hi = __vmaxu4(hi, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
+  }
+  lo = __vminu4(lo, lo >> 16);
+  lo = min(lo & 0xFFu, (lo >> 8) & 0xFFu);
+  hi = __vmaxu4(hi, hi >> 16);
+  hi = max(hi & 0xFFu, (hi >> 8) & 0xFFu);
+  int l = __reduce_min_sync(0xFFFFFFFFu, (int)lo);
+  int h = __reduce_max_sync(0xFFFFFFFFu, (int)hi);
+  __shared__ int s_lo[16], s_hi[16];
+  const int wid = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) { s_lo[wid] = l; s_hi[wid] = h; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) {
+      l = min(l, s_lo[i]);
+      h = max(h, s_hi[i]);
+    }
+    int G = 0;
+    if (h == 255) {
+      record_error(MOE_ERR_NAN_SCALE);
+    } else {
+      const int elo = l - 127, ehi = h - 127;
+      if (elo >= -9 && ehi <= 8) G = 0;
+      else if (ehi - elo <= 17) G = ehi - 8;
+      else record_error(MOE_ERR_RANGE);
+    }
+    out_global[m] = exp2_int(G);
+  }
+}
+
+// Two copies of the E4M3 code of byte b's 2^(b - 127 - G), as a 16-bit pair.
+__device__ __forceinline__ uint32_t nvfp4_scale_pair(uint32_t b, int G) {
+  int j = (int)b - 127 - G;
+  j = max(-9, min(8, j));                            // only out of range after a recorded error
+  const uint32_t c = e4m3_pow2_code(j);
+  return c | (c << 8);
+}
+
+// Pass 2: 16 scale bytes per thread -> 32 output bytes; the nibble copy
+// (when not aliased) in a second grid-stride loop, 16 bytes at a time.
+__global__ void __launch_bounds__(256) nvfp4_convert_vec_kernel(const uint4* __restrict__ e8m0, int64_t n16,
+                                                                int64_t per_mat16, const float* __restrict__ glob,
+                                                                uint4* __restrict__ out_e4m3,
+                                                                const uint4* __restrict__ fp4,
+                                                                uint4* __restrict__ out_fp4, int64_t n_fp4_16) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < n16; i += stride) {
+    const int G = exponent_of_pow2(__ldg(glob + i / per_mat16));
+    const uint4 v = __ldg(e8m0 + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = nvfp4_scale_pair(w[k] & 0xFFu, G) | (nvfp4_scale_pair((w[k] >> 8) & 0xFFu, G) << 16);
+      o[2 * k + 1] = nvfp4_scale_pair((w[k] >> 16) & 0xFFu, G) | (nvfp4_scale_pair(w[k] >> 24, G) << 16);
+    }
+    out_e4m3[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+    out_e4m3[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  if (out_fp4 != nullptr)
+    for (int64_t i = tid; i < n_fp4_16; i += stride) out_fp4[i] = __ldg(fp4 + i);
+}
+
+// INT4 group-128: one thread per 32-element block (one 16-byte chunk of
+// nibbles and its E8M0 byte), four consecutive threads per 128-group, so the
+// loads and stores of a warp are contiguous.  The group maximum is reduced over
+// the four threads by shuffles.  Every E2M1 magnitude is 1 or 3 times a power of
+// two, so the seven quotients x / scale_inv of a block come from two IEEE
+// divisions (2^e / s and 3 * 2^e / s) scaled by powers of two, which is exact
+// in the normal range; below it the quotient is far under 0.5 and rounds to 0
+// either way.  Lanes of a warp must all be present (n_blocks % 4 == 0 holds).
+__global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__ fp4,
+                                                       const uint8_t* __restrict__ e8m0, int64_t n_blocks,
+                                                       uint4* __restrict__ out, float* __restrict__ scale_inv) {
+  const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool live = blk < n_blocks;
+  const uint4 in = live ? __ldg(fp4 + blk) : make_uint4(0u, 0u, 0u, 0u);
+  const int b = live ? (int)__ldg(e8m0 + blk) : 0;
+  // largest magnitude code of the block: max over the 32 three-bit fields
+  uint32_t mw = __vmaxu4(__vmaxu4(in.x & 0x07070707u, (in.x >> 4) & 0x07070707u),
+                         __vmaxu4(in.y & 0x07070707u, (in.y >> 4) & 0x07070707u));
+  mw = __vmaxu4(mw, __vmaxu4(__vmaxu4(in.z & 0x07070707u, (in.z >> 4) & 0x07070707u),
+                             __vmaxu4(in.w & 0x07070707u, (in.w >> 4) & 0x07070707u)));
+  mw = __vmaxu4(mw, mw >> 16);
+  const uint32_t mc = max(mw & 0xFFu, (mw >> 8) & 0xFFu);
   const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
-  uint4 in[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) in[i] = __ldg(fp4 + g * 4 + i);
-  const uint32_t sb = __ldg(e8m0 + g);
-  // exact float32 block maxima
-  float amax = 0.0f;
-  bool bad = false;
-#pragma unroll
-  for (int blk = 0; blk < 4; ++blk) {
-    const int b = (sb >> (8 * blk)) & 0xFF;
-    if (b == 255) { bad = true; continue; }
-    const uint32_t* words = reinterpret_cast<const uint32_t*>(&in[blk]);
-    uint32_t mc = 0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-#pragma unroll
-      for (int n = 0; n < 8; ++n) mc = max(mc, (words[w] >> (4 * n)) & 7u);
-    const float bm = __fmul_rn(kE2M1[mc], exp2_int(b - 127));
-    if (isinf(bm)) record_error(MOE_ERR_RANGE);
-    amax = fmaxf(amax, bm);
+  const float sc = exp2_int(b - 127);
+  float bm = __fmul_rn(kE2M1[mc], sc);
+  const bool nan = b == 255;
+  if (live && !nan && isinf(bm)) record_error(MOE_ERR_RANGE);
+  if (nan) bm = 0.0f;
+  float amax = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  // a NaN scale anywhere in the group (its four lanes) skips the group
+  const bool gnan = ((__ballot_sync(0xFFFFFFFFu, nan) >> (threadIdx.x & 28)) & 0xFu) != 0u;
+  if (!live) return;
+  if (gnan) {
+    if (nan) record_error(MOE_ERR_NAN_SCALE);
+    return;
   }
-  if (bad) { record_error(MOE_ERR_NAN_SCALE); return; }
   const float sinv = amax > 0.0f ? __fdiv_rn(amax, 7.0f) : 1.0f;
-  scale_inv[g] = sinv;
-  uint4 res[4];
+  if ((threadIdx.x & 3) == 0) scale_inv[blk >> 2] = sinv;
+  // q of magnitude codes 1..7 (E2M1 0.5, 1, 1.5, 2, 3, 4, 6)
+  const float d1 = __fdiv_rn(sc, sinv);
+  const float d3 = __fdiv_rn(__fmul_rn(3.0f, sc), sinv);
+  const float qv[8] = {0.0f, 0.5f * d1, d1, 0.5f * d3, 2.0f * d1, d3, 4.0f * d1, 2.0f * d3};
+  // byte tables over the magnitude code: tp = q, tn = (16 - q) & 15 (q <= 7, so
+  // the byte-wise subtraction never borrows)
+  uint32_t tp[2] = {0u, 0u};
 #pragma unroll
-  for (int blk = 0; blk < 4; ++blk) {
-    const int b = (sb >> (8 * blk)) & 0xFF;
-    const float sc = exp2_int(b - 127);
-    // quantised magnitude of each of the 8 E2M1 magnitudes in this block
-    uint32_t qm = 0;                                   // 8 x 4-bit table
+  for (int c = 1; c < 8; ++c)
+    tp[c >> 2] |= __float2uint_rn(fminf(qv[c], 7.0f)) << (8 * (c & 3));   // round half to even
+  const uint32_t tn[2] = {(0x10101010u - tp[0]) & 0x0F0F0F0Fu, (0x10101010u - tp[1]) & 0x0F0F0F0Fu};
+  const uint32_t words[4] = {in.x, in.y, in.z, in.w};
+  uint32_t ow[4];
 #pragma unroll
-    for (int c = 1; c < 8; ++c) {
-      const float x = __fmul_rn(kE2M1[c], sc);
-      const float q = fminf(rintf(__fdiv_rn(x, sinv)), 7.0f);
-      qm |= (uint32_t)q << (4 * c);
-    }
-    const uint32_t* words = reinterpret_cast<const uint32_t*>(&in[blk]);
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&res[blk]);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint32_t o = 0;
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const uint32_t nib = (words[w] >> (4 * n)) & 0xFu;
-        const uint32_t mag = (qm >> (4 * (nib & 7u))) & 0xFu;
-        const uint32_t q = (nib & 8u) ? ((16u - mag) & 0xFu) : mag;   // two's complement
-        o |= q << (4 * n);
-      }
-      ow[w] = o;
-    }
+  for (int w = 0; w < 4; ++w) {
+    // even nibbles (0, 2, 4, 6) and odd nibbles (1, 3, 5, 7) as four 4-bit
+    // byte selectors each; the lookups land in the low nibble of each byte
+    const uint32_t lo = words[w] & 0x0F0F0F0Fu, hi = (words[w] >> 4) & 0x0F0F0F0Fu;
+    const uint32_t sel_e = __byte_perm(lo | (lo >> 4), 0u, 0x0020u);
+    const uint32_t sel_o = __byte_perm(hi | (hi >> 4), 0u, 0x0020u);
+    const uint32_t m_e = __byte_perm(0x0000FF00u, 0u, (sel_e >> 3) & 0x1111u);
+    const uint32_t m_o = __byte_perm(0x0000FF00u, 0u, (sel_o >> 3) & 0x1111u);
+    const uint32_t r_e = (__byte_perm(tp[0], tp[1], sel_e) & ~m_e) | (__byte_perm(tn[0], tn[1], sel_e) & m_e);
+    const uint32_t r_o = (__byte_perm(tp[0], tp[1], sel_o) & ~m_o) | (__byte_perm(tn[0], tn[1], sel_o) & m_o);
+    ow[w] = r_e | (r_o << 4);
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) out[g * 4 + i] = res[i];
+  out[blk] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
 }
 
 }  // namespace moe

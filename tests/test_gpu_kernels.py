@@ -278,6 +278,24 @@ def test_repack_nvfp4_bit_exact(lib):
     np.testing.assert_array_equal(host(t), fp4)
 
 
+def test_repack_nvfp4_scalar_path(lib):
+    """15 scales per matrix and a scale output 2 bytes off a 16-byte boundary:
+    the byte-at-a-time passes."""
+    M, N, K = 3, 5, 96
+    fp4 = synth.random_bytes(5, 1, (M, N, K // 2))
+    e8 = synth.random_bytes(5, 2, (M, N, K // 32), 119, 136)   # span 17 up to 2^9: global scale 2^1
+    o_fp4 = torch.empty((M, N, K // 2), dtype=torch.uint8, device="cuda")
+    o_s_buf = torch.empty(M * N * K // 16 + 2, dtype=torch.uint8, device="cuda")
+    o_s = o_s_buf[2:].view(M, N, K // 16)
+    o_g = torch.empty(M, dtype=torch.float32, device="cuda")
+    lib.repack_mxfp4_to_nvfp4(dev(fp4), dev(e8), o_fp4, o_s, o_g)
+    r_fp4, r_s, r_g = Rp.repack_mxfp4_to_nvfp4(fp4, e8)
+    np.testing.assert_array_equal(host(o_fp4), r_fp4)
+    np.testing.assert_array_equal(host(o_s), r_s)
+    np.testing.assert_array_equal(host(o_g), r_g)
+    no_device_error(lib)
+
+
 def test_repack_nvfp4_errors(lib):
     e8 = np.full((1, 128, 4), 127, np.uint8)
     e8[0, 5, 1] = 255
@@ -293,10 +311,14 @@ def test_repack_nvfp4_errors(lib):
     assert lib.moe_get_device_error() == 0
 
 
-def test_repack_int4_bit_exact(lib):
+@pytest.mark.parametrize("lo,hi", [(1, 250), (120, 127)])
+def test_repack_int4_bit_exact(lib, lo, hi):
+    """Scales over the whole range, and in a narrow band where a group's blocks
+    share or neighbour the maximum exponent (many quotients near rounding
+    ties)."""
     M, N, K = 2, 256, 1024
     fp4 = synth.random_bytes(6, 1, (M, N, K // 2))
-    e8 = synth.random_bytes(6, 2, (M, N, K // 32), 1, 250)
+    e8 = synth.random_bytes(6, 2, (M, N, K // 32), lo, hi)
     e8[0, :7] = 127                                         # ordinary blocks too
     fp4[0, 3] = 0                                           # an all-zero row
     q = torch.empty((M, N, K // 2), dtype=torch.int8, device="cuda")
