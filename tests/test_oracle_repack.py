@@ -96,3 +96,67 @@ def test_int4_zero_group_and_errors():
     with pytest.raises(Rp.RepackError) as ex:
         Rp.repack_mxfp4_to_int4g128(big, np.full((1, 1, 4), 254, np.uint8))
     assert ex.value.code == -4
+
+
+# ---------------- MXFP4 -> FP8 E4M3 with a [128, 128] block scale ----------------
+def _block(codes_row, exps, N=128, K=128):
+    """One [N, K] matrix: every row holds codes_row (K nibble codes), 32-element
+    block j of every row has E8M0 byte exps[j]."""
+    codes = np.tile(np.asarray(codes_row, np.uint8), (N, 1))
+    fp4 = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)[None]
+    e8 = np.tile(np.asarray(exps, np.uint8), (N, 1))[None]
+    return fp4, e8
+
+
+def test_fp8_block_cast_lossless_roundtrip():
+    """Exponent spread <= 8 inside every [128, 128] block: decoding the codes
+    and multiplying by scale_inv gives back the MXFP4 values exactly."""
+    M, N, K = 2, 256, 512
+    fp4 = synth.random_bytes(7, 1, (M, N, K // 2))
+    e8 = synth.random_bytes(7, 2, (M, N, K // 32), 118, 126)
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(fp4, e8)
+    assert exact and q.shape == (M, N, K) and sinv.shape == (M, N // 128, K // 128)
+    ref = ffn.dequant_mxfp4(fp4, e8)
+    back = F.decode_e4m3(q) * np.repeat(np.repeat(sinv.astype(np.float64), 128, 1), 128, 2)
+    np.testing.assert_array_equal(back, ref)
+
+
+def test_fp8_block_cast_closed_forms():
+    # block maximum 6 * 2^e -> scale 2^(e-6); 6 -> 384 (0x7C), 0.5 -> 32 (0x60)
+    row = [7] + [1] * 127                         # codes 7 (6.0) and 1 (0.5)
+    e = 5
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(*_block(row, [127 + e] * 4))
+    assert exact and sinv[0, 0, 0] == np.float32(2.0 ** (e - 6))
+    assert q[0, 0, 0] == 0x7C and q[0, 0, 1] == 0x60
+    # block maximum 1.0 * 2^e -> scale 2^(e-8); 1.0 -> 256 (0x78)
+    q, sinv, _ = Rp.repack_mxfp4_to_fp8_block128(*_block([2] * 128, [127 + e] * 4))
+    assert sinv[0, 0, 0] == np.float32(2.0 ** (e - 8)) and (q == 0x78).all()
+    # all-zero block: scale 1, codes 0; negative zero keeps its sign
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(*_block([0, 8] * 64, [200] * 4))
+    assert exact and sinv[0, 0, 0] == 1.0 and (q[..., 0::2] == 0).all() and (q[..., 1::2] == 0x80).all()
+
+
+def test_fp8_block_scale_is_the_activation_rule():
+    """The block exponent is the activation quantiser's exponent of the block
+    maximum (oracle.quant, float32 ratio) wherever that maximum is a float32."""
+    from oracle import quant as Q
+    for code in range(1, 8):
+        for e in range(-126, 125, 7):
+            q, sinv, _ = Rp.repack_mxfp4_to_fp8_block128(*_block([code] + [0] * 127, [127 + e] * 4))
+            amax = np.float32(F.e2m1_value(code) * 2.0 ** e)
+            k = int(Q.pow2_scale_exponent(np.array([amax]))[0])
+            assert sinv[0, 0, 0] == np.float32(np.ldexp(1.0, k)), (code, e)
+
+
+def test_fp8_block_cast_lossy_edge_and_errors():
+    # spread 14 with the smallest codes: still exact (0.5 * 2^-14 * 2^6 = 2^-9)
+    row = [7] * 32 + [1] * 32 + [3] * 32 + [0] * 32
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(*_block(row, [140, 126, 126, 126]))
+    assert exact
+    # spread 15: 0.5 -> 2^-10 rounds to 0 (tie to even), 1.5 -> 1.5 * 2^-9 rounds to 2^-8
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(*_block(row, [140, 125, 125, 125]))
+    assert not exact
+    assert (q[0, :, 32:64] == 0x00).all() and (q[0, :, 64:96] == 0x02).all()
+    with pytest.raises(Rp.RepackError) as ex:
+        Rp.repack_mxfp4_to_fp8_block128(*_block([1] * 128, [127, 255, 127, 127]))
+    assert ex.value.code == -3
