@@ -225,9 +225,9 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
 
 def run_repack(args, wl):
     """Weight repack sweep: one layer of E experts x (w1, w3 [I, H], w2 [H, I])
-    MXFP4 -> NVFP4 (E4M3 scale per 16, per-matrix global scale) and -> symmetric
-    INT4 group 128 (fp32 scale_inv [N, K/128]).  One step = both repacks of
-    the whole layer.  Metric: GB/s of algorithmic bytes (each repack reads its
+    MXFP4 -> NVFP4 (E4M3 scale per 16, per-matrix global scale), -> symmetric
+    INT4 group 128 (fp32 scale_inv [N, K/128]) and -> FP8 E4M3 with a
+    [128, 128] block scale.  One step = the three repacks of the whole layer.  Metric: GB/s of algorithmic bytes (each repack reads its
     source once and writes its outputs once)."""
     import torch
 
@@ -241,17 +241,20 @@ def run_repack(args, wl):
     mats = [(torch.from_numpy(w13.reshape(2 * E, I, H // 2)).cuda(), torch.from_numpy(s13.reshape(2 * E, I, H // 32)).cuda()),
             (torch.from_numpy(w2).cuda(), torch.from_numpy(s2).cuda())]
     outs = []
-    nv_bytes = int4_bytes = 0
+    nv_bytes = int4_bytes = fp8_bytes = 0
     for fp4, e8 in mats:
         M, N, k2 = fp4.shape
         K = 2 * k2
         o = dict(nv_fp4=torch.empty_like(fp4), nv_s=torch.empty((M, N, K // 16), dtype=torch.uint8, device="cuda"),
                  nv_g=torch.empty(M, dtype=torch.float32, device="cuda"),
                  q=torch.empty((M, N, k2), dtype=torch.int8, device="cuda"),
-                 sinv=torch.empty((M, N, K // 128), dtype=torch.float32, device="cuda"))
+                 sinv=torch.empty((M, N, K // 128), dtype=torch.float32, device="cuda"),
+                 f8=torch.empty((M, N, K), dtype=torch.uint8, device="cuda"),
+                 f8_s=torch.empty((M, N // 128, K // 128), dtype=torch.float32, device="cuda"))
         outs.append(o)
         nv_bytes += 2 * fp4.numel() + e8.numel() + o["nv_s"].numel() + 4 * M
         int4_bytes += fp4.numel() + e8.numel() + o["q"].numel() + 4 * o["sinv"].numel()
+        fp8_bytes += fp4.numel() + e8.numel() + o["f8"].numel() + 4 * o["f8_s"].numel()
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -262,13 +265,16 @@ def run_repack(args, wl):
         for (fp4, e8), o in zip(mats, outs):
             moe.repack_mxfp4_to_int4g128(fp4, e8, o["q"], o["sinv"])
         if ev: ev[2].record(stream)
+        for (fp4, e8), o in zip(mats, outs):
+            moe.repack_mxfp4_to_fp8_block128(fp4, e8, o["f8"], o["f8_s"])
+        if ev: ev[3].record(stream)
 
     clk = ClockSampler(local).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     assert moe.moe_get_device_error() == 0
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(pg)
     torch.cuda.synchronize()
     w_begin = time.time()
@@ -283,27 +289,29 @@ def run_repack(args, wl):
     ms = max_over_ranks(t0.elapsed_time(t1), pg)
     nv_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     i4_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    f8_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     if rank != 0:
         if pg is not None:
             pg.destroy_process_group()
         return
     peaks = read_peaks()
-    total = (nv_bytes + int4_bytes) * world * args.steps
+    total = (nv_bytes + int4_bytes + fp8_bytes) * world * args.steps
     gbs = total / (ms / 1e3) / 1e9
     nv_gbs = nv_bytes / (nv_ms / 1e3) / 1e9
     line = {
         "metric": "weight repack GB/s vs B200 HBM roofline", "value": round(gbs, 1), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4 "
-                               f"and -> INT4 group 128", "l2": "inputs larger than L2 (3.4 GB per repack)"},
+        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4, "
+                               f"-> INT4 group 128 and -> FP8 E4M3 [128, 128] blocks", "l2": "inputs larger than L2 (3.4 GB per repack)"},
         "roofline": {"bound": "hbm", "achieved": round(nv_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": round(nv_gbs / peaks["hbm"], 4), "traffic": None, "kernel": "repack_mxfp4_to_nvfp4",
                      "peak_source": f"{peaks['src']} HBM copy"},
         "repack": {"nvfp4_ms": round(nv_ms, 4), "nvfp4_GBps": round(nv_gbs, 1),
                    "int4_ms": round(i4_ms, 4), "int4_GBps": round(int4_bytes / (i4_ms / 1e3) / 1e9, 1),
-                   "nvfp4_bytes": nv_bytes, "int4_bytes": int4_bytes},
-        "gpu_launches": 6 * args.steps,     # per step: 2 x (2 NVFP4 kernels + 1 INT4 kernel)
+                   "fp8_ms": round(f8_ms, 4), "fp8_GBps": round(fp8_bytes / (f8_ms / 1e3) / 1e9, 1),
+                   "nvfp4_bytes": nv_bytes, "int4_bytes": int4_bytes, "fp8_bytes": fp8_bytes},
+        "gpu_launches": 8 * args.steps,     # per step: 2 x (2 NVFP4 kernels + 1 INT4 + 1 FP8 kernel)
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
@@ -492,7 +500,9 @@ def run_reference_repack(args, wl):
     E, H, I = wl["E"], wl["H"], wl["I"]
     w13, s13, w2, s2 = synth.expert_weights(args.seed, 1, H, I)
     per = (2 * w13.nbytes + s13.nbytes + 2 * s13.nbytes + 4 * 2) + (2 * w2.nbytes + s2.nbytes + 2 * s2.nbytes + 4) \
-        + (2 * w13.nbytes + s13.nbytes + 4 * w13.nbytes * 2 // 128) + (2 * w2.nbytes + s2.nbytes + 4 * w2.nbytes * 2 // 128)
+        + (2 * w13.nbytes + s13.nbytes + 4 * w13.nbytes * 2 // 128) + (2 * w2.nbytes + s2.nbytes + 4 * w2.nbytes * 2 // 128) \
+        + (3 * w13.nbytes + s13.nbytes + 4 * w13.nbytes * 2 // (128 * 128)) \
+        + (3 * w2.nbytes + s2.nbytes + 4 * w2.nbytes * 2 // (128 * 128))
     times = []
     for i in range(args.warmup + args.steps):
         t = time.perf_counter()
@@ -500,6 +510,8 @@ def run_reference_repack(args, wl):
         Rp.repack_mxfp4_to_nvfp4(w2, s2)
         Rp.repack_mxfp4_to_int4g128(w13.reshape(2, I, H // 2), s13.reshape(2, I, H // 32))
         Rp.repack_mxfp4_to_int4g128(w2, s2)
+        Rp.repack_mxfp4_to_fp8_block128(w13.reshape(2, I, H // 2), s13.reshape(2, I, H // 32))
+        Rp.repack_mxfp4_to_fp8_block128(w2, s2)
         if i >= args.warmup:
             times.append(time.perf_counter() - t)
     value = per * len(times) / sum(times) / 1e9
@@ -508,8 +520,8 @@ def run_reference_repack(args, wl):
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * sum(times) / len(times), 2), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4 "
-                               f"and -> INT4 group 128"},
+        "config": {"workload": f"repack sweep: {E} experts x (w1, w3 [{I}, {H}], w2 [{H}, {I}]) MXFP4 -> NVFP4, "
+                               f"-> INT4 group 128 and -> FP8 E4M3 [128, 128] blocks"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": f"one expert's three matrices per step, {len(times)} steps"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),

@@ -37,6 +37,7 @@ SIGNATURES = {
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P]),
     "repack_mxfp4_to_nvfp4": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P, _P]),
     "repack_mxfp4_to_int4g128": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P]),
+    "repack_mxfp4_to_fp8_block128": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P]),
 }
 
 _lib = None

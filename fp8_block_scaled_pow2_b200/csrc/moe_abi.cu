@@ -465,6 +465,19 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
   return launch_status();
 }
 
+int repack_mxfp4_to_fp8_block128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                                 uint8_t* out_e4m3, float* out_scale_inv, void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return MOE_ERR_INVALID;
+  if (n_mats == 0) return MOE_OK;
+  if (!fp4 || !e8m0 || !out_e4m3 || !out_scale_inv) return MOE_ERR_INVALID;
+  if (!aligned(fp4, 16) || !aligned(out_e4m3, 16) || !aligned(e8m0, 4) || !aligned(out_scale_inv, 4))
+    return MOE_ERR_INVALID;
+  const int64_t blocks = n_mats * (int64_t)(N / 128) * (K / 128);
+  if (blocks > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  fp8_block128_kernel<<<(unsigned)blocks, 128, 0, S(stream)>>>(fp4, e8m0, N, K, out_e4m3, out_scale_inv);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // Grouping without caller scratch.  The per-chunk expert histograms live in a
 // fixed device array owned by this library instead of a caller workspace.

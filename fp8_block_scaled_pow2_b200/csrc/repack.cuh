@@ -8,7 +8,14 @@
 //
 // MXFP4 -> symmetric INT4 group 128: "DeepSeek-V4-Flash-0731-W4AFP8-mt",
 // 量化方式 / 权重约定: signed INT4 two per int8, float32 scale_inv [N, K/128].
+//
+// MXFP4 -> FP8 E4M3 with a [128, 128] block scale: "DeepSeek-V4-Pro-0813-
+// nvfp4-DSpark" walkthrough (the lossless MXFP4 seed: nibbles split from the
+// int8, values looked up, scale rewritten per 128 block) and the
+// "DeepSeek-V4-Flash-SI" model card's weight block size [128, 128].
 #pragma once
+
+#include <climits>
 
 #include "common.cuh"
 
@@ -230,6 +237,109 @@ __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__
     ow[w] = r_e | (r_o << 4);
   }
   out[blk] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+}
+
+// FP8 cast: one block of 128 threads per (matrix, 128-row block, 128-column
+// block).  The block's 512 16-byte chunks of nibbles (one 32-element
+// sub-block each) are handed out so that four consecutive threads read one
+// row's 64 bytes and write its 128 E4M3 bytes (a warp covers 8 rows per pass,
+// 4 passes).  The block scale is 2^s with s = ceil(log2(amax / 448)) (the
+// activation rule) for the exact block maximum, clamped to [-127, 127]; for an
+// MXFP4 maximum {1, 1.5} * 2^E this is E - 8.  Maxima are compared as the
+// order-preserving key 2 * E + [mantissa 1.5], so values beyond float32 (6 *
+// 2^127) still order correctly.  Element codes: E4M3 round to nearest even of
+// E2M1 * 2^d, d = e - s, from an 8-entry table per sub-block (four paired
+// conversions) applied with byte permutes; the sign bit is copied.  A present
+// code c is exact iff d >= -9 - lsb(c) (its lowest set bit must stay at or
+// above E4M3's 2^-9); otherwise MOE_ERR_RANGE is recorded and the rounded
+// code is kept.  An E8M0 NaN records MOE_ERR_NAN_SCALE and skips the block.
+__global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __restrict__ fp4,
+                                                           const uint8_t* __restrict__ e8m0, int N, int K,
+                                                           uint8_t* __restrict__ out,
+                                                           float* __restrict__ scale_inv) {
+  __shared__ int s_key[4];
+  __shared__ int s_nan[4];
+  const int KB = K / 128, NB = N / 128;
+  const int64_t blk = blockIdx.x;
+  const int kb = (int)(blk % KB);
+  const int64_t t = blk / KB;
+  const int nb = (int)(t % NB);
+  const int64_t mat = t / NB;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int j = tid & 3;                       // sub-block (32 columns) of this thread's chunks
+  const int64_t row0 = mat * N + (int64_t)nb * 128;
+  // pass p: row (p * 32 + tid / 4), sub-block j
+  uint4 in[4];
+  int b[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int64_t row = row0 + p * 32 + (tid >> 2);
+    in[p] = __ldg(reinterpret_cast<const uint4*>(fp4 + row * (K / 2) + (int64_t)kb * 64) + j);
+    b[p] = (int)__ldg(e8m0 + row * (K / 32) + (int64_t)kb * 4 + j);
+  }
+  // floor(log2) and mantissa bit of E2M1 magnitude codes 0..7 (0.5, 1, 1.5, 2, 3, 4, 6)
+  const int kFl[8] = {0, -1, 0, 0, 1, 1, 2, 2};
+  const int kHalf[8] = {0, 0, 0, 1, 0, 1, 0, 1};
+  int key = INT_MIN;
+  int nan = 0;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    nan |= b[p] == 255;
+    uint32_t mw = __vmaxu4(__vmaxu4(in[p].x & 0x07070707u, (in[p].x >> 4) & 0x07070707u),
+                           __vmaxu4(in[p].y & 0x07070707u, (in[p].y >> 4) & 0x07070707u));
+    mw = __vmaxu4(mw, __vmaxu4(__vmaxu4(in[p].z & 0x07070707u, (in[p].z >> 4) & 0x07070707u),
+                               __vmaxu4(in[p].w & 0x07070707u, (in[p].w >> 4) & 0x07070707u)));
+    mw = __vmaxu4(mw, mw >> 16);
+    const int mc = (int)max(mw & 0xFFu, (mw >> 8) & 0xFFu);
+    if (mc > 0) key = max(key, 2 * (b[p] - 127 + kFl[mc]) + kHalf[mc]);
+  }
+  key = __reduce_max_sync(0xFFFFFFFFu, key);
+  nan = __reduce_or_sync(0xFFFFFFFFu, nan);
+  if (lane == 0) { s_key[wid] = key; s_nan[wid] = nan; }
+  __syncthreads();
+  key = max(max(s_key[0], s_key[1]), max(s_key[2], s_key[3]));
+  nan = s_nan[0] | s_nan[1] | s_nan[2] | s_nan[3];
+  if (nan) {
+    if (tid == 0) record_error(MOE_ERR_NAN_SCALE);
+    return;
+  }
+  const int s = key == INT_MIN ? 0 : max(-127, min(127, (key >> 1) - 8));   // key >> 1 = floor(key / 2) = E
+  if (tid == 0) scale_inv[(mat * NB + nb) * KB + kb] = exp2_int(s);
+  const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  bool inexact = false;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int d = b[p] - 127 - s;
+    // values below 2^-10 round to 0 in E4M3 whatever their float32 form, so
+    // the scale factor is clamped into float32's range
+    const float sc = exp2_int(max(d, -149));
+    const uint32_t t0 = e4m3x4(0.0f, kE2M1[1] * sc, kE2M1[2] * sc, kE2M1[3] * sc);
+    const uint32_t t1 = e4m3x4(kE2M1[4] * sc, kE2M1[5] * sc, kE2M1[6] * sc, kE2M1[7] * sc);
+    const uint32_t w[4] = {in[p].x, in[p].y, in[p].z, in[p].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = (w[k] >> (16 * h)) & 0xFFFFu;          // four nibbles
+        const uint32_t sgn = __byte_perm(0x00008000u, 0u, (sel >> 3) & 0x1111u);
+        o[2 * k + h] = __byte_perm(t0, t1, sel) | sgn;
+      }
+    }
+    const int64_t row = row0 + p * 32 + (tid >> 2);
+    uint4* dst = reinterpret_cast<uint4*>(out + row * K + (int64_t)kb * 128 + j * 32);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    if (d < -8) {
+      // exact iff every present nonzero code c has d >= -9 - lsb(c)
+      const int kMin[8] = {INT_MIN, -8, -9, -8, -10, -9, -11, -10};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int n = 0; n < 8; ++n) inexact |= d < kMin[(w[k] >> (4 * n)) & 7u];
+    }
+  }
+  if (inexact) record_error(MOE_ERR_RANGE);
 }
 
 }  // namespace moe

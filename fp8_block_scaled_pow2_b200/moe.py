@@ -164,3 +164,11 @@ def repack_mxfp4_to_int4g128(fp4, e8m0, out_int4, out_scale_inv, stream=None):
     n_mats, N, k2 = fp4.shape
     _check("repack_mxfp4_to_int4g128", _lib().repack_mxfp4_to_int4g128(
         _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_int4), _ptr(out_scale_inv), _stream(stream)))
+
+
+def repack_mxfp4_to_fp8_block128(fp4, e8m0, out_e4m3, out_scale_inv, stream=None):
+    """MXFP4 [n_mats, N, K/2] + E8M0 [n_mats, N, K/32] -> E4M3 [n_mats, N, K] and
+    float32 scale_inv [n_mats, N/128, K/128] (power-of-two block scales)."""
+    n_mats, N, k2 = fp4.shape
+    _check("repack_mxfp4_to_fp8_block128", _lib().repack_mxfp4_to_fp8_block128(
+        _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_e4m3), _ptr(out_scale_inv), _stream(stream)))

@@ -288,6 +288,24 @@ int repack_mxfp4_to_nvfp4(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mat
 int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N,
                              int K, int8_t* out_int4, float* out_scale_inv, void* stream);
 
+/*
+ * f1 -- MXFP4 -> FP8 E4M3 with a [128, 128] block scale [NVFP4 关于 MXFP4 的无损
+ * 种子: cast_e2m1fn_to_e4m3fn rewrites the scale per 128 block; SI 模型训练:
+ * weight block size [128, 128]].  Per (128-row, 128-column) block of each
+ * matrix: amax = exact block maximum; s = ceil(log2(amax / 448)) clamped to
+ * [-127, 127] (0 when amax == 0), the a1 rule; out_scale_inv = 2^s (the
+ * dequant multiplier: w = e4m3 * scale_inv); out = E4M3(w / 2^s), nearest
+ * even, sign kept.  Exact unless a nonzero element falls below E4M3's 2^-9
+ * (exponents spread by more than 14 inside a block); then the rounded codes
+ * are written and MOE_ERR_RANGE is recorded.  A block with an E8M0 NaN
+ * (byte 255) records MOE_ERR_NAN_SCALE and is not written.
+ *   fp4 uint8 [n_mats, N, K/2] (16-byte aligned); e8m0 [n_mats, N, K/32]
+ *   (4-byte aligned); out_e4m3 uint8 [n_mats, N, K] (16-byte aligned);
+ *   out_scale_inv float32 [n_mats, N/128, K/128];  N % 128 == 0, K % 128 == 0
+ */
+int repack_mxfp4_to_fp8_block128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                                 uint8_t* out_e4m3, float* out_scale_inv, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

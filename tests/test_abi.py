@@ -56,3 +56,4 @@ def test_argument_validation_without_gpu():
                                       ctypes.c_float(10), 48, None, None, None, 0, None) == -2
     assert lib.moe_prepared_weights_size(3, 256, 512) == 3 * 2 * 4 * 8704
     assert lib.repack_mxfp4_to_int4g128(None, None, 1, 8, 96, None, None, None) == -1
+    assert lib.repack_mxfp4_to_fp8_block128(None, None, 1, 100, 128, None, None, None) == -1   # N % 128

@@ -343,6 +343,56 @@ def test_repack_int4_errors(lib):
     assert lib.moe_get_device_error() == -4
 
 
+# ------------------------------- f1 ---------------------------------------
+def _fp8_cast(lib, fp4, e8):
+    M, N, k2 = fp4.shape
+    q = torch.empty((M, N, 2 * k2), dtype=torch.uint8, device="cuda")
+    si = torch.empty((M, N // 128, 2 * k2 // 128), dtype=torch.float32, device="cuda")
+    lib.repack_mxfp4_to_fp8_block128(dev(fp4), dev(e8), q, si)
+    torch.cuda.synchronize()
+    return host(q), host(si)
+
+
+@pytest.mark.parametrize("lo,hi,exact", [(118, 126, True), (1, 254, False)])
+def test_fp8_block_cast_bit_exact(lib, lo, hi, exact):
+    """Codes and block scales equal the oracle's bit for bit; exponents over
+    the whole E8M0 range (maxima up to 6 * 2^127, beyond float32) make many
+    blocks inexact, which is reported as MOE_ERR_RANGE."""
+    M, N, K = 2, 256, 512
+    fp4 = synth.random_bytes(8, 1, (M, N, K // 2))
+    e8 = synth.random_bytes(8, 2, (M, N, K // 32), lo, hi)
+    q, si = _fp8_cast(lib, fp4, e8)
+    q_ref, si_ref, ex_ref = Rp.repack_mxfp4_to_fp8_block128(fp4, e8)
+    assert ex_ref == exact
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(si.view(np.uint32), si_ref.view(np.uint32))
+    assert lib.moe_get_device_error() == (0 if exact else -4)
+
+
+def test_fp8_block_cast_edges(lib):
+    """Spread 14 (exact) and 15 (rounded, flagged) inside one block, an
+    all-zero block with negative zeros, and an E8M0 NaN."""
+    N, K = 128, 384
+    codes = np.zeros((N, K), np.uint8)
+    codes[:, 0:32], codes[:, 32:64], codes[:, 64:96] = 7, 1, 3       # block 0: spread 14
+    codes[:, 128:160], codes[:, 160:192], codes[:, 192:224] = 7, 1, 3  # block 1: spread 15
+    codes[:, 256::2] = 8                                                # block 2: zeros and -0
+    fp4 = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)[None]
+    e8 = np.full((1, N, K // 32), 126, np.uint8)
+    e8[0, :, 0] = 140
+    e8[0, :, 4] = 140
+    e8[0, :, 5:8] = 125
+    q, si = _fp8_cast(lib, fp4, e8)
+    q_ref, si_ref, ex_ref = Rp.repack_mxfp4_to_fp8_block128(fp4, e8)
+    assert not ex_ref
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(si, si_ref)
+    assert lib.moe_get_device_error() == -4
+    e8[0, 7, 3] = 255
+    _fp8_cast(lib, fp4, e8)
+    assert lib.moe_get_device_error() == -3
+
+
 # ------------------------------- a10 --------------------------------------
 def _w4a_inputs(seed, sizes, N, K, integer):
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
