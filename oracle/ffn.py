@@ -9,6 +9,11 @@ Passages:
     projections are named w1, w2, w3; weights are [N, K] with K the input
     dimension; the W4AFP8 form holds INT4 weights with a float32
     weight_scale_inv of shape [N, K/128] and dynamic E4M3 activations.
+  * FP8 shared expert: "DeepSeek-V4-Pro-0813-nvfp4-DSpark" walkthrough (only-
+    experts section: the shared experts stay FP8) and the "DeepSeek-V4-Flash-SI"
+    model card (模型训练: weight block size [128, 128]).  Reading: E4M3 weights
+    [N, K] with a float32 weight_scale_inv [N/128, K/128] per [128, 128] block
+    (w = e4m3 * scale_inv), the same dynamic E4M3 activations.
 
 Readings: w1 = gate, w3 = up, w2 = down; both gate and up are clamped to
 [-limit, limit] before silu(gate) * up (which tensors the clamp applies to is
@@ -23,7 +28,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import decode_e2m1_packed, decode_e8m0
+from .formats import decode_e2m1_packed, decode_e4m3, decode_e8m0
 from .permute import gather_rows, permute
 from .quant import dequantize_fp8_pow2, quantize_act_fp8, quantize_fp8_pow2
 from .route import route_topk
@@ -89,6 +94,20 @@ def grouped_gemm_w4afp8(a_q, a_s, offsets, w_int4, w_scale_inv):
     return out if out.shape[1] else np.zeros((a_q.shape[0], N))
 
 
+def dequant_fp8_block128(q: np.ndarray, scale_inv: np.ndarray) -> np.ndarray:
+    """E4M3 [N, K] + float32 scale_inv [N/128, K/128] -> float64 [N, K]."""
+    v = decode_e4m3(q)
+    s = np.asarray(scale_inv, dtype=np.float32).astype(np.float64)
+    return v * np.repeat(np.repeat(s, 128, axis=-2), 128, axis=-1)
+
+
+def grouped_gemm_fp8_block128(a_q, a_s, offsets, w_q, w_scale_inv):
+    """FP8 rows x FP8 [128, 128]-block weights [G, N, K] -> float64 [R, N]."""
+    N = w_q.shape[1]
+    out = grouped_gemm(a_q, a_s, offsets, lambda g: dequant_fp8_block128(w_q[g], w_scale_inv[g]), w_q.shape[0])
+    return out if out.shape[1] else np.zeros((a_q.shape[0], N))
+
+
 def silu(g: np.ndarray) -> np.ndarray:
     return g / (1.0 + np.exp(-g))
 
@@ -123,10 +142,16 @@ def combine(o: np.ndarray, inv: np.ndarray, w: np.ndarray, offsets: np.ndarray,
 
 def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
               swiglu_limit=10.0, has_shared=1, route_norm=1, weights="mxfp4",
-              w13_int4=None, w13_sinv=None, w2_int4=None, w2_sinv=None, tokens=None):
+              w13_int4=None, w13_sinv=None, w2_int4=None, w2_sinv=None, tokens=None,
+              shared_fp8=None):
     """The whole expert path (a1 -> a7) for the tokens listed in ``tokens``
     (all tokens when None).  Token outputs are independent given the routing,
     so a subset gives exactly those rows of the full result.
+
+    shared_fp8: optional (w13_q, w13_scale_inv, w2_q, w2_scale_inv) of the
+    shared expert in FP8 with [128, 128] block scales ([2I, H], [2I/128,
+    H/128], [H, I], [H/128, I/128]); the shared group then uses these instead
+    of group E of the routed weight arrays.
 
     Returns a dict of the intermediates (indices refer to the subset)."""
     x_bf16 = np.asarray(x_bf16)
@@ -145,11 +170,18 @@ def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
         gu = grouped_gemm_mxfp4(xq_p, sx_p, offsets, w13, w13_e8m0)
     else:
         gu = grouped_gemm_w4afp8(xq_p, sx_p, offsets, w13_int4, w13_sinv)
+    shared = shared_fp8 is not None and has_shared
+    r0, r1 = (int(offsets[E]), int(offsets[E + 1])) if shared else (0, 0)
+    if r1 > r0:      # the shared group with its FP8 weights
+        gu[r0:r1] = dequantize_fp8_pow2(xq_p[r0:r1], sx_p[r0:r1]) @ \
+            dequant_fp8_block128(shared_fp8[0], shared_fp8[1]).T
     hq, sh = swiglu_quant(gu, I, swiglu_limit)
     if weights == "mxfp4":
         o = grouped_gemm_mxfp4(hq, sh, offsets, w2, w2_e8m0)
     else:
         o = grouped_gemm_w4afp8(hq, sh, offsets, w2_int4, w2_sinv)
+    if r1 > r0:
+        o[r0:r1] = dequantize_fp8_pow2(hq[r0:r1], sh[r0:r1]) @ dequant_fp8_block128(shared_fp8[2], shared_fp8[3]).T
     y = combine(o, inv, w, offsets, has_shared)
     return dict(xq=xq, sx=sx, idx=idx, w=w, counts=counts, offsets=offsets, perm=perm,
                 inv=inv, xq_perm=xq_p, sx_perm=sx_p, gu=gu, hq=hq, sh=sh, o=o, y=y)

@@ -98,3 +98,59 @@ def test_w4afp8_dequant_loop():
     q = np.array([[0x7F, 0x98] + [0] * 62], np.uint8).view(np.int8)   # nibbles 15,7,8,9
     d = ffn.dequant_int4g128(q, np.array([[0.5]], np.float32))
     assert d[0, :4].tolist() == [-0.5, 3.5, -4.0, -3.5]
+
+
+# ------------------------- FP8 [128, 128]-block weights (shared expert) -------------------------
+def test_fp8_block_dequant_closed_forms():
+    """Code 0x38 is 1.0; every [128, 128] block takes its own scale_inv."""
+    q = np.full((256, 256), 0x38, np.uint8)
+    sinv = np.array([[1.0, 2.0], [0.25, 8.0]], np.float32)
+    w = ffn.dequant_fp8_block128(q, sinv)
+    assert (w[:128, :128] == 1.0).all() and (w[:128, 128:] == 2.0).all()
+    assert (w[128:, :128] == 0.25).all() and (w[128:, 128:] == 8.0).all()
+
+
+def test_fp8_gemm_matches_mxfp4_gemm_after_lossless_cast():
+    """Weights cast losslessly to FP8 [128, 128] blocks give the MXFP4 GEMM's
+    result exactly (an independent path to the same dequantised weights)."""
+    from oracle import repack as Rp
+    G, N, K = 2, 256, 384
+    w = synth.random_bytes(12, 1, (G, N, K // 2))
+    ws = synth.random_bytes(12, 2, (G, N, K // 32), 119, 126)
+    q, sinv, exact = Rp.repack_mxfp4_to_fp8_block128(w, ws)
+    assert exact
+    offsets = np.array([0, 5, 40], np.int32)
+    a = synth.random_e4m3(12, 3, (40, K))
+    asc = synth.random_bytes(12, 4, (40, K // 128), 120, 130)
+    np.testing.assert_array_equal(ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv),
+                                  ffn.grouped_gemm_mxfp4(a, asc, offsets, w, ws))
+
+
+def test_layer_shared_fp8_equals_mxfp4_shared_after_cast():
+    """The tiny layer with its shared expert cast losslessly to FP8 gives the
+    same output as with the MXFP4 shared expert."""
+    from oracle import repack as Rp
+    wl = synth.tiny_layer(4)
+    E = wl.E
+    q13, s13, ok13 = Rp.repack_mxfp4_to_fp8_block128(wl.w13[E:E + 1], wl.w13_e8m0[E:E + 1])
+    q2, s2, ok2 = Rp.repack_mxfp4_to_fp8_block128(wl.w2[E:E + 1], wl.w2_e8m0[E:E + 1])
+    assert ok13 and ok2
+    ref = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    got = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk,
+                        shared_fp8=(q13[0], s13[0], q2[0], s2[0]))
+    np.testing.assert_array_equal(got["y"], ref["y"])
+
+
+def test_fp8_block_scale_is_linear_per_block():
+    """Doubling one block's scale_inv doubles exactly that block's contribution."""
+    K = 256
+    q = synth.small_int_e4m3(13, 1, (128, K))
+    a = synth.small_int_e4m3(13, 2, (8, K))
+    asc = np.full((8, K // 128), 127, np.uint8)
+    off = np.array([0, 8], np.int32)
+    s1 = np.array([[1.0, 1.0]], np.float32)
+    s2 = np.array([[1.0, 2.0]], np.float32)
+    base = ffn.grouped_gemm_fp8_block128(a, asc, off, q[None], s1[None])
+    twice = ffn.grouped_gemm_fp8_block128(a, asc, off, q[None], s2[None])
+    hi = ffn.grouped_gemm_fp8_block128(a[:, :], asc, off, np.where(np.arange(K) >= 128, q, 0)[None], s1[None])
+    np.testing.assert_array_equal(twice, base + hi)
