@@ -33,12 +33,14 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s or HBM GB/s vs B200 roofline"
-def kernels_per_step(wl: dict) -> int:
+def kernels_per_step(wl: dict, shared: str = "mxfp4") -> int:
     """Library kernels one layer step launches: quant 1, route 1, grouping 2
     (one block for <= 2048 routed pairs, then the gather) or 4 (chunked), two
-    GEMM calls of 2 (prep + GEMM), combine 1."""
+    GEMM calls of 2 (prep + GEMM; two more with the FP8 shared expert),
+    combine 1."""
     grouping = 2 if wl["T"] * wl["k"] <= 2048 else 4
-    return 1 + 1 + grouping + 2 * 2 + 1
+    gemm_calls = 4 if shared == "fp8" else 2
+    return 1 + 1 + grouping + gemm_calls * 2 + 1
 
 WORKLOADS = {
     "repack": dict(T=0, H=4096, I=2048, E=256, k=6, logits="uniform"),
@@ -217,9 +219,15 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
     H, I = wl["H"], wl["I"]
     w13 = 2 * I * H // 2 + 2 * I * H // 32
     w2 = H * I // 2 + H * I // 32
+    w13_bytes = active * w13
+    w2_bytes = active * w2
+    if getattr(layer, "shared", "mxfp4") == "fp8" and counts[-1] > 0:
+        # the shared expert streams E4M3 bytes and float32 [128, 128] block scales instead
+        w13_bytes += 2 * I * H + 4 * (2 * I // 128) * (H // 128) - w13
+        w2_bytes += H * I + 4 * (H // 128) * (I // 128) - w2
     return dict(active_experts=active, rows=R,
-                w13=active * w13 + R * (H + H // 128) + R * (I + I // 128),
-                w2=active * w2 + R * (I + I // 128) + R * H * 4,
+                w13=w13_bytes + R * (H + H // 128) + R * (I + I // 128),
+                w2=w2_bytes + R * (I + I // 128) + R * H * 4,
                 flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
 
 
@@ -327,7 +335,7 @@ def run_ours(args, wl):
 
     rank, world, local, pg = dist_setup(args.gpus)
     x, logits, (w13, s13, w2, s2) = make_inputs(wl, args.seed, rank)
-    layer = MoeLayer(w13, s13, w2, s2, wl["k"], weights=args.weights)
+    layer = MoeLayer(w13, s13, w2, s2, wl["k"], weights=args.weights, shared=args.shared)
     T = wl["T"]
     buf = layer.alloc(T)
     xd = torch.from_numpy(x.view(np.int16)).cuda()
@@ -438,7 +446,7 @@ def run_ours(args, wl):
         "data": "synthetic",
         "config": {"workload": f"{args.workload} layer: hidden {wl['H']}, intermediate {wl['I']}, "
                                f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {T} tokens per GPU",
-                   "weights": args.weights,
+                   "weights": args.weights, "shared_expert": args.shared,
                    "tokens_per_gpu": T, "parallelism": f"replicas x{world} (data parallel, no collective)",
                    "cuda_graph": use_graph,
                    "l2": f"inputs larger than L2: {ab['active_experts']} active experts stream "
@@ -453,7 +461,7 @@ def run_ours(args, wl):
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xh.numel() * 2 + lh.numel() * 4),
                 "d2h_bytes_per_step": int(yh.numel() * 2)},
-        "gpu_launches": kernels_per_step(wl) * args.steps,
+        "gpu_launches": kernels_per_step(wl, args.shared) * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
@@ -571,6 +579,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--weights", choices=["mxfp4", "w4afp8"], default="mxfp4")
+    ap.add_argument("--shared", choices=["mxfp4", "fp8"], default="mxfp4",
+                    help="shared expert weights: MXFP4 (group E of the grouped GEMM) or FP8 [128, 128] blocks")
     ap.add_argument("--graph", choices=["on", "off"], default="on",
                     help="replay the layer step as four CUDA graphs (off: eager library calls)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -33,6 +33,7 @@ SIGNATURES = {
     "moe_gemm_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "moe_grouped_gemm_mxfp4": (_I, [_P, _P, _I, _P, _I, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_grouped_gemm_w4afp8": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
+    "moe_grouped_gemm_fp8_block128": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_swiglu_clamp": (_I, [_P, _I, _I, _F, _P, _P, _P]),
     "moe_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P]),
     "repack_mxfp4_to_nvfp4": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P, _P]),

@@ -163,9 +163,10 @@ constexpr int kPrepPerThread = (kMaxGroups + kPrepThreads) / kPrepThreads;   // 
 // holds its scales of the K steps 4g .. 4g+3, one per byte (the MMA of K step
 // kt selects byte kt % 4); rows past the tile and K steps past K are 0.
 // Block 0 writes the plan.  Unless the offsets are nondecreasing from
-// offsets[0] = 0 to offsets[G] <= a_rows, the plan has no work and
+// offsets[0] >= 0 to offsets[G] <= a_rows, the plan has no work and
 // MOE_ERR_INVALID is recorded, so no tile ever addresses rows outside the
-// operands or the workspace.
+// operands or the workspace.  (offsets[0] > 0 lets a caller run a subset of
+// groups, e.g. one group of a larger grouping.)
 __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* __restrict__ offsets, int G,
                                                                  int a_rows, int BN, int n_ft,
                                                                  const uint8_t* __restrict__ sx, int KT,
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
   __syncthreads();
   bool bad = false;
   for (int g = tid; g < G; g += kPrepThreads)
-    bad |= s_off[g + 1] < s_off[g] || (g == 0 && s_off[0] != 0) || (g == G - 1 && s_off[G] > a_rows);
+    bad |= s_off[g + 1] < s_off[g] || (g == 0 && s_off[0] < 0) || (g == G - 1 && s_off[G] > a_rows);
   bad = __syncthreads_or(bad);
   // exclusive scan of the tile counts; thread tid owns groups [tid*P, tid*P + P)
   const int g0 = tid * kPrepPerThread;

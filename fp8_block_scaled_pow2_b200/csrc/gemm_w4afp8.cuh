@@ -17,6 +17,13 @@
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, then CONV_WARPS
 // converters (8 for narrow token tiles, where transcoding is the critical
 // path, else 4), then 4 promotion + epilogue warps.
+//
+// W8 = true is the same GEMM for FP8 E4M3 weights with a float32 scale_inv
+// per [128, 128] block (the FP8 shared expert: "DeepSeek-V4-Pro-0813-nvfp4-
+// DSpark" walkthrough, only-experts section; "DeepSeek-V4-Flash-SI" model
+// card, weight block size [128, 128]): the producer copies the E4M3 tiles
+// straight into the MMA layout (128-byte swizzle), there are no converters,
+// and the promotion multiplies by the tile's block scale.
 #pragma once
 
 #include "gemm_mxfp4.cuh"
@@ -28,15 +35,15 @@ using namespace sm100;
 using gemm::Item;
 using gemm::decode_item;
 
-template <int BN, bool DUAL>
+template <int BN, bool DUAL, bool W8 = false>
 struct Cfg {
-  static constexpr int CONV_WARPS = BN <= 32 ? 8 : 4;
+  static constexpr int CONV_WARPS = W8 ? 0 : (BN <= 32 ? 8 : 4);
   static constexpr int PROMO_FIRST = 2 + CONV_WARPS;      // first promotion warp
   static constexpr int THREADS = (PROMO_FIRST + 4) * 32;
   static constexpr int CONV_THREADS = CONV_WARPS * 32;
   static constexpr int NA = (BN + 127) / 128;
   static constexpr int NUM_A = DUAL ? 2 : 1;
-  static constexpr int RAW_BYTES = 128 * 64;          // INT4 tile as loaded (64 B per row)
+  static constexpr int RAW_BYTES = W8 ? 0 : 128 * 64;   // INT4 tile as loaded (64 B per row)
   static constexpr int A_BYTES = 128 * 128;           // E4M3 tile for the MMA
   static constexpr int B_BYTES = BN * 128;
   static constexpr int A_OFF = 0;                      // NUM_A E4M3 tiles (1024-aligned)
@@ -47,7 +54,7 @@ struct Cfg {
   static constexpr int STAGE = (STAGE_RAW + 1023) / 1024 * 1024;
   static constexpr int STAGES_FIT = (196 * 1024) / STAGE;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int TX = NUM_A * RAW_BYTES + B_BYTES;   // + NA * 512 every 4th K step
+  static constexpr int TX = NUM_A * (W8 ? A_BYTES : RAW_BYTES) + B_BYTES;   // + NA * 512 every 4th K step
   // TMEM: two partial buffers of NUM_A * BN columns, then scale factors
   static constexpr int P_COLS = NUM_A * BN;
   static constexpr int SFA_COL = 2 * P_COLS;
@@ -80,7 +87,7 @@ __device__ __forceinline__ uint32_t int4x4_to_e4m3x4(uint32_t h) {
 }
 
 struct W4Args {
-  const float* w_sinv;     // [G, N, K/128]
+  const float* w_sinv;     // [G, N, K/128] (INT4) or [G, N/128, K/128] (FP8)
   const uint8_t* a_sf;     // per-tile activation scales (as in the MXFP4 GEMM)
   const int* header;
   const int* prefix;
@@ -92,11 +99,11 @@ struct W4Args {
   float limit;
 };
 
-template <int BN, bool DUAL, int EPI>
-__global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
+template <int BN, bool DUAL, int EPI, bool W8 = false>
+__global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     gemm_w4afp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const W4Args args) {
-  using C = Cfg<BN, DUAL>;
+  using C = Cfg<BN, DUAL, W8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -120,7 +127,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], C::CONV_THREADS);
+      mbar_init(&conv[s], C::CONV_THREADS > 0 ? C::CONV_THREADS : 1);   // unused with FP8 weights
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -161,8 +168,13 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
           uint8_t* st = smem + stage * C::STAGE;
           const bool new_group = (kt & 3) == 0;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
-          tma_load_2d(st + C::RAW_OFF, &tmA, kt * 64, rb0 * 128, &full[stage]);
-          if (DUAL) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, &tmA, kt * 64, rb1 * 128, &full[stage]);
+          if constexpr (W8) {
+            tma_load_2d(st + C::A_OFF, &tmA, kt * 128, rb0 * 128, &full[stage]);
+            if (DUAL) tma_load_2d(st + C::A_OFF + C::A_BYTES, &tmA, kt * 128, rb1 * 128, &full[stage]);
+          } else {
+            tma_load_2d(st + C::RAW_OFF, &tmA, kt * 64, rb0 * 128, &full[stage]);
+            if (DUAL) tma_load_2d(st + C::RAW_OFF + C::RAW_BYTES, &tmA, kt * 64, rb1 * 128, &full[stage]);
+          }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
         }
@@ -186,7 +198,8 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
       bool ok = true;
       for (int kt = 0; kt < KT && ok; ++kt) {
         if (!mbar_wait_warp(&pempty[pb], ((pbits >> pb) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-        if (!mbar_wait_warp(&conv[stage], phase, abort_flag)) { ok = false; break; }
+        // FP8 weights are MMA-ready when they land; INT4 after the converters
+        if (!mbar_wait_warp(W8 ? &full[stage] : &conv[stage], phase, abort_flag)) { ok = false; break; }
         tc_fence_after();     // orders the MMA after the promotion warps' release of the partial buffer
         const uint32_t st = smem_u32(smem + stage * C::STAGE);
         const uint32_t dcol = tmem + pb * C::P_COLS;
@@ -218,7 +231,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
       }
       if (!ok) break;
     }
-  } else if (warp < C::PROMO_FIRST) {
+  } else if (!W8 && warp < C::PROMO_FIRST) {
     // ------------------------------ converters ----------------------------
     // thread layout: converter warp w (0..CONV_WARPS-1), lane l -> 16-byte
     // input chunk (l & 3) of rows w*8 + (l >> 2) + 8*CONV_WARPS*j;
@@ -269,8 +282,12 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL>::THREADS, 1)
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb_per_g = N / 128;
-      const float* s0 = args.w_sinv + ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT;
-      const float* s1 = args.w_sinv + ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT;
+      // scale_inv of this thread's weight row per K step: [G, N, K/128] (INT4,
+      // per row) or [G, N/128, K/128] (FP8, one value per 128-row block)
+      const float* s0 = args.w_sinv + (W8 ? (size_t)(it.g * rb_per_g + it.ft) * KT
+                                          : ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT);
+      const float* s1 = args.w_sinv + (W8 ? (size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * KT
+                                          : ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT);
       float acc0[BN], acc1[DUAL ? BN : 1];
 #pragma unroll
       for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;

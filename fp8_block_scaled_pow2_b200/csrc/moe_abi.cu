@@ -104,14 +104,89 @@ int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const g
   }
 }
 
-template <int BN, bool DUAL, int EPI>
+template <int BN, bool DUAL, int EPI, bool W8>
 int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& a, cudaStream_t st) {
-  using C = w4a::Cfg<BN, DUAL>;
-  auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI>;
+  using C = w4a::Cfg<BN, DUAL, W8>;
+  auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI, W8>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
   k<<<sm_count(), C::THREADS, C::SMEM_ALLOC, st>>>(ta, tb, a);
   return launch_status();
+}
+
+// Grouped GEMM whose weight scale is applied by promotion warps: INT4 group-128
+// weights (W8 = false, transcoded to E4M3 in shared memory) or FP8 E4M3 weights
+// with [128, 128] block scales (W8 = true).
+template <bool W8>
+int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets, int n_groups,
+                  const void* w, const float* w_scale_inv, int N, int K, int epilogue, float swiglu_limit, int block_n,
+                  void* out, uint8_t* out_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
+    return MOE_ERR_INVALID;
+  if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
+  const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
+  if (dual && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
+  if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
+  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual)) return MOE_ERR_UNSUPPORTED;
+  if (a_rows == 0) return MOE_OK;
+  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
+  if (!aligned(a_e4m3, 16) || !aligned(w, 16) || !aligned(w_scale_inv, 4) || !aligned(workspace, 256))
+    return MOE_ERR_INVALID;
+  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
+  if (workspace_bytes < L.total) return MOE_ERR_INVALID;
+  CUtensorMap ta, tb;
+  // INT4: raw [rows, K/2] tiles of 64 x 128 bytes; FP8: [rows, K] tiles of 128 x 128 bytes
+  // written straight into the 128-byte-swizzled MMA layout
+  if (W8 ? !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K, (uint64_t)n_groups * N, (uint64_t)K, 128,
+                     128)
+         : !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K / 2, (uint64_t)n_groups * N,
+                     (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MOE_ERR_LAUNCH;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
+                (uint32_t)block_n))
+    return MOE_ERR_LAUNCH;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  w4a::W4Args args;
+  args.w_sinv = w_scale_inv;
+  args.a_sf = ws + L.a_sf;
+  args.header = reinterpret_cast<const int*>(ws + L.header);
+  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
+  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
+  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
+  args.G = n_groups;
+  args.N = N;
+  args.K = K;
+  args.out = out;
+  args.out_scale = out_scale;
+  args.limit = swiglu_limit;
+  cudaStream_t st = S(stream);
+  const int n_ft = dual ? N / 256 : N / 128;
+  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+      offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
+      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  if (dual) {
+    switch (block_n) {
+      case 16: return launch_w4a<16, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
+      case 32: return launch_w4a<32, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
+      default: return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
+    }
+  }
+  if (epilogue == MOE_EPI_STORE_F32) {
+    switch (block_n) {
+      case 16: return launch_w4a<16, false, MOE_EPI_STORE_F32, W8>(ta, tb, args, st);
+      case 32: return launch_w4a<32, false, MOE_EPI_STORE_F32, W8>(ta, tb, args, st);
+      case 64: return launch_w4a<64, false, MOE_EPI_STORE_F32, W8>(ta, tb, args, st);
+      default: return launch_w4a<128, false, MOE_EPI_STORE_F32, W8>(ta, tb, args, st);
+    }
+  }
+  switch (block_n) {
+    case 16: return launch_w4a<16, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
+    case 32: return launch_w4a<32, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
+    case 64: return launch_w4a<64, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
+    default: return launch_w4a<128, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
+  }
 }
 
 // Self-test of the bounded waits: one thread waits on an mbarrier that no
@@ -331,68 +406,17 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
                             int n_groups, const int8_t* w_int4, const float* w_scale_inv, int N, int K,
                             int epilogue, float swiglu_limit, int block_n, void* out, uint8_t* out_scale,
                             void* workspace, size_t workspace_bytes, void* stream) {
-  if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
-    return MOE_ERR_INVALID;
-  if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
-  const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
-  if (dual && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
-  if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
-  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual)) return MOE_ERR_UNSUPPORTED;
-  if (a_rows == 0) return MOE_OK;
-  if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_int4 || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
-  if (!aligned(a_e4m3, 16) || !aligned(w_int4, 16) || !aligned(w_scale_inv, 4) || !aligned(workspace, 256))
-    return MOE_ERR_INVALID;
-  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
-  if (workspace_bytes < L.total) return MOE_ERR_INVALID;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_int4, (uint64_t)K / 2, (uint64_t)n_groups * N,
-                (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return MOE_ERR_LAUNCH;
-  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
-                (uint32_t)block_n))
-    return MOE_ERR_LAUNCH;
-  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  w4a::W4Args args;
-  args.w_sinv = w_scale_inv;
-  args.a_sf = ws + L.a_sf;
-  args.header = reinterpret_cast<const int*>(ws + L.header);
-  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
-  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
-  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
-  args.G = n_groups;
-  args.N = N;
-  args.K = K;
-  args.out = out;
-  args.out_scale = out_scale;
-  args.limit = swiglu_limit;
-  cudaStream_t st = S(stream);
-  const int n_ft = dual ? N / 256 : N / 128;
-  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
-      offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
-      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
-  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  if (dual) {
-    switch (block_n) {
-      case 16: return launch_w4a<16, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
-      case 32: return launch_w4a<32, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
-      default: return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT>(ta, tb, args, st);
-    }
-  }
-  if (epilogue == MOE_EPI_STORE_F32) {
-    switch (block_n) {
-      case 16: return launch_w4a<16, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
-      case 32: return launch_w4a<32, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
-      case 64: return launch_w4a<64, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
-      default: return launch_w4a<128, false, MOE_EPI_STORE_F32>(ta, tb, args, st);
-    }
-  }
-  switch (block_n) {
-    case 16: return launch_w4a<16, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
-    case 32: return launch_w4a<32, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
-    case 64: return launch_w4a<64, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
-    default: return launch_w4a<128, false, MOE_EPI_STORE_BF16>(ta, tb, args, st);
-  }
+  return promoted_gemm<false>(a_e4m3, a_e8m0_128, a_rows, offsets, n_groups, w_int4, w_scale_inv, N, K, epilogue,
+                              swiglu_limit, block_n, out, out_scale, workspace, workspace_bytes, stream);
+}
+
+int moe_grouped_gemm_fp8_block128(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
+                                  const int32_t* offsets, int n_groups, const uint8_t* w_e4m3,
+                                  const float* w_scale_inv, int N, int K, int epilogue, float swiglu_limit,
+                                  int block_n, void* out, uint8_t* out_scale, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return promoted_gemm<true>(a_e4m3, a_e8m0_128, a_rows, offsets, n_groups, w_e4m3, w_scale_inv, N, K, epilogue,
+                             swiglu_limit, block_n, out, out_scale, workspace, workspace_bytes, stream);
 }
 
 int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq, uint8_t* sh, void* stream) {

@@ -53,13 +53,36 @@ class Buffers:
 class MoeLayer:
     def __init__(self, w13, w13_e8m0, w2, w2_e8m0, topk: int, route_scale: float = 1.5,
                  swiglu_limit: float = 10.0, has_shared: int = 1, route_norm: int = 1, device="cuda",
-                 weights: str = "mxfp4"):
+                 weights: str = "mxfp4", shared: str = "mxfp4"):
         """weights="mxfp4" runs the block-scaled MXFP4 GEMMs; weights="w4afp8"
         repacks the experts once on the GPU to symmetric INT4 group-128
-        (repack_mxfp4_to_int4g128) and runs the W4AFP8 GEMMs."""
+        (repack_mxfp4_to_int4g128) and runs the W4AFP8 GEMMs.  shared="fp8"
+        casts the shared expert (group E of the arrays) once on the GPU to FP8
+        E4M3 with [128, 128] block scales (repack_mxfp4_to_fp8_block128) and
+        runs it through moe_grouped_gemm_fp8_block128."""
         self.device = torch.device(device)
         self.G = w13.shape[0]                      # routed experts + shared expert
         self.E = self.G - (1 if has_shared else 0)
+        if shared not in ("mxfp4", "fp8") or (shared == "fp8" and not has_shared):
+            raise ValueError(shared)
+        self.shared = shared
+        if shared == "fp8":
+            d = self.device
+            E = self.E
+            I2, H = w13.shape[1], w13.shape[2] * 2
+            self.ws13_q = torch.empty((1, I2, H), dtype=torch.uint8, device=d)
+            self.ws13_s = torch.empty((1, I2 // 128, H // 128), dtype=torch.float32, device=d)
+            self.ws2_q = torch.empty((1, H, I2 // 2), dtype=torch.uint8, device=d)
+            self.ws2_s = torch.empty((1, H // 128, I2 // 256), dtype=torch.float32, device=d)
+            moe.repack_mxfp4_to_fp8_block128(_dev(w13[E:E + 1], d), _dev(w13_e8m0[E:E + 1], d), self.ws13_q,
+                                             self.ws13_s)
+            moe.repack_mxfp4_to_fp8_block128(_dev(w2[E:E + 1], d), _dev(w2_e8m0[E:E + 1], d), self.ws2_q, self.ws2_s)
+            err = moe.moe_get_device_error()
+            if err != 0:
+                raise moe.MoeError("repack_mxfp4_to_fp8_block128", err)
+            # the routed GEMMs cover groups 0 .. E-1 only
+            w13, w13_e8m0, w2, w2_e8m0 = w13[:E], w13_e8m0[:E], w2[:E], w2_e8m0[:E]
+        self.GR = w13.shape[0]                     # groups of the routed-weight GEMMs
         self.I = w13.shape[1] // 2
         self.H = w13.shape[2] * 2
         assert w2.shape[1] == self.H and w2.shape[2] * 2 == self.I
@@ -71,19 +94,19 @@ class MoeLayer:
             # prepared blocks (nibbles + tensor-memory-order scales); the raw
             # MXFP4 arrays are not kept
             w13_d, s13_d = _dev(w13, d), _dev(w13_e8m0, d)
-            self.w13_p = torch.empty(moe.moe_prepared_weights_size(self.G, 2 * self.I, self.H), dtype=torch.uint8,
+            self.w13_p = torch.empty(moe.moe_prepared_weights_size(self.GR, 2 * self.I, self.H), dtype=torch.uint8,
                                      device=d)
             moe.moe_prepare_weights(w13_d, s13_d, self.w13_p, paired=True)
             del w13_d, s13_d
             w2_d, s2_d = _dev(w2, d), _dev(w2_e8m0, d)
-            self.w2_p = torch.empty(moe.moe_prepared_weights_size(self.G, self.H, self.I), dtype=torch.uint8, device=d)
+            self.w2_p = torch.empty(moe.moe_prepared_weights_size(self.GR, self.H, self.I), dtype=torch.uint8, device=d)
             moe.moe_prepare_weights(w2_d, s2_d, self.w2_p)
             del w2_d, s2_d
         elif weights == "w4afp8":
-            self.w13_q = torch.empty((self.G, 2 * self.I, self.H // 2), dtype=torch.int8, device=d)
-            self.w13_sinv = torch.empty((self.G, 2 * self.I, self.H // 128), dtype=torch.float32, device=d)
-            self.w2_q = torch.empty((self.G, self.H, self.I // 2), dtype=torch.int8, device=d)
-            self.w2_sinv = torch.empty((self.G, self.H, self.I // 128), dtype=torch.float32, device=d)
+            self.w13_q = torch.empty((self.GR, 2 * self.I, self.H // 2), dtype=torch.int8, device=d)
+            self.w13_sinv = torch.empty((self.GR, 2 * self.I, self.H // 128), dtype=torch.float32, device=d)
+            self.w2_q = torch.empty((self.GR, self.H, self.I // 2), dtype=torch.int8, device=d)
+            self.w2_sinv = torch.empty((self.GR, self.H, self.I // 128), dtype=torch.float32, device=d)
             moe.repack_mxfp4_to_int4g128(_dev(w13, d), _dev(w13_e8m0, d), self.w13_q, self.w13_sinv)
             moe.repack_mxfp4_to_int4g128(_dev(w2, d), _dev(w2_e8m0, d), self.w2_q, self.w2_sinv)
             if moe.moe_get_device_error() != 0:
@@ -100,7 +123,7 @@ class MoeLayer:
         R = T * k + (T if self.has_shared else 0)
         u8, i32, f32 = torch.uint8, torch.int32, torch.float32
         # the W4AFP8 w1/w3 GEMM may use narrower token tiles than block_n
-        bns = (block_n, 16) if self.weights == "w4afp8" else (block_n,)
+        bns = (block_n, 16) if (self.weights == "w4afp8" or self.shared == "fp8") else (block_n,)
         ws_g = max([moe.moe_gemm_workspace_size(R, self.G, K, bn) for bn in bns for K in (H, I)] + [256])
         return Buffers(
             T=T,
@@ -121,7 +144,8 @@ class MoeLayer:
         Each only enqueues library calls, so each can be captured in a CUDA
         graph; forward() runs them eagerly."""
         b = buf
-        g_off = b.offsets if self.has_shared else b.offsets[: self.G + 1]
+        g_off = b.offsets[: self.GR + 1]          # the groups of the routed-weight GEMMs
+        s_off = b.offsets[self.E:]                 # the shared group alone (FP8 shared expert)
 
         def pre():
             moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
@@ -129,26 +153,38 @@ class MoeLayer:
             moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
                             b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
 
+        bn_dual = min(b.block_n, 64) if b.block_n else 0
         if self.weights == "mxfp4":
-            def gemm13():
-                moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13_p, self.G, 2 * self.I,
+            def routed13():
+                moe.moe_grouped_gemm_mxfp4(b.xq_perm, b.sx_perm, g_off, self.w13_p, self.GR, 2 * self.I,
                                            moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
                                            b.block_n, stream=stream)
 
-            def gemm2():
-                moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.G, self.H, moe.MOE_EPI_STORE_F32,
+            def routed2():
+                moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.GR, self.H, moe.MOE_EPI_STORE_F32,
                                            b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
         else:
-            bn = min(b.block_n, 64) if b.block_n else 0
-
-            def gemm13():
+            def routed13():
                 moe.moe_grouped_gemm_w4afp8(b.xq_perm, b.sx_perm, g_off, self.w13_q, self.w13_sinv,
                                             moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm, self.swiglu_limit,
-                                            bn, stream=stream)
+                                            bn_dual, stream=stream)
 
-            def gemm2():
+            def routed2():
                 moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
                                             b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        if self.shared == "fp8":
+            def gemm13():
+                routed13()
+                moe.moe_grouped_gemm_fp8_block128(b.xq_perm, b.sx_perm, s_off, self.ws13_q, self.ws13_s,
+                                                  moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm,
+                                                  self.swiglu_limit, bn_dual, stream=stream)
+
+            def gemm2():
+                routed2()
+                moe.moe_grouped_gemm_fp8_block128(b.hq, b.sh, s_off, self.ws2_q, self.ws2_s, moe.MOE_EPI_STORE_F32,
+                                                  b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        else:
+            gemm13, gemm2 = routed13, routed2
 
         def post():
             moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)

@@ -140,6 +140,19 @@ def moe_grouped_gemm_w4afp8(a, a_scale, offsets, w_int4, w_scale_inv, epilogue, 
         _stream(stream)))
 
 
+def moe_grouped_gemm_fp8_block128(a, a_scale, offsets, w_e4m3, w_scale_inv, epilogue, out, out_scale=None,
+                                  workspace=None, swiglu_limit=10.0, block_n=0, stream=None):
+    """FP8 rows x FP8 weights [G, N, K] with float32 scale_inv [G, N/128, K/128];
+    offsets [G+1] may start above 0 (a view into a larger grouping)."""
+    a_rows, K = a.shape
+    G, N = w_e4m3.shape[0], w_e4m3.shape[1]
+    _check("moe_grouped_gemm_fp8_block128", _lib().moe_grouped_gemm_fp8_block128(
+        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_e4m3), _ptr(w_scale_inv), N, K,
+        int(epilogue), ctypes.c_float(swiglu_limit), int(block_n), _ptr(out), _ptr(out_scale),
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
 def moe_swiglu_clamp(gu, hq, sh, limit=10.0, stream=None):
     rows, two_i = gu.shape
     _check("moe_swiglu_clamp", _lib().moe_swiglu_clamp(_ptr(gu), rows, two_i // 2, ctypes.c_float(limit),

@@ -191,10 +191,11 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
  *                                          * w[g, n, k] * 2^(sw[g, n, k/32]-127)
  *   a_e4m3       uint8 [a_rows, K] (16-byte aligned), a_rows >= offsets[G]
  *   a_e8m0_128   uint8 [a_rows, K/128]
- *   offsets      int32 [G+1] device, non-decreasing, offsets[0] == 0,
- *                offsets[G] <= a_rows; otherwise the call does no work, leaves
- *                out untouched and records MOE_ERR_INVALID in the device error
- *                word (moe_get_device_error)
+ *   offsets      int32 [G+1] device, non-decreasing, offsets[0] >= 0,
+ *                offsets[G] <= a_rows (rows outside [offsets[0], offsets[G])
+ *                are neither read nor written); otherwise the call does no
+ *                work, leaves out untouched and records MOE_ERR_INVALID in the
+ *                device error word (moe_get_device_error)
  *   w_prepared   output of moe_prepare_weights for the MXFP4 weights [G, N, K/2]
  *                and scales [G, N, K/32] (paired order for
  *                MOE_EPI_SWIGLU_QUANT, plain otherwise)
@@ -239,6 +240,24 @@ int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, in
                             int epilogue, float swiglu_limit, int block_n,
                             void* out, uint8_t* out_scale,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * f3 -- grouped GEMM with FP8 E4M3 weights and a float32 scale_inv per
+ * [128, 128] block (the FP8 shared expert [NVFP4 只量化专家: shared experts
+ * stay FP8; SI 模型训练: weight block size [128, 128]]).  For every group g:
+ * acc[r, n] = sum over 128-wide K steps kt of scale_inv[g, n/128, kt] *
+ * (sum_{k in kt} a[r, k] * 2^(sa[r, kt]-127) * w[g, n, k]); each step is one
+ * block-scaled MMA with unit weight scales whose float32 partial is scaled
+ * and summed in ascending kt.
+ *   w_e4m3       uint8 [G, N, K] (16-byte aligned); w_scale_inv float32
+ *                [G, N/128, K/128]
+ *   other arguments, layouts and epilogues as moe_grouped_gemm_w4afp8.
+ */
+int moe_grouped_gemm_fp8_block128(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
+                                  const int32_t* offsets, int n_groups, const uint8_t* w_e4m3,
+                                  const float* w_scale_inv, int N, int K, int epilogue, float swiglu_limit,
+                                  int block_n, void* out, uint8_t* out_scale, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /*
  * a5 standalone -- SwiGLU with clamp and per-128 power-of-two requantisation

@@ -74,15 +74,15 @@ def test_out_of_range_expert_id_is_flagged(lib, T):
     assert lib.moe_get_device_error() == 0
 
 
-@pytest.mark.parametrize("bad", ["past_rows", "decreasing", "nonzero_start"])
+@pytest.mark.parametrize("bad", ["past_rows", "decreasing", "negative_start"])
 def test_invalid_group_offsets_plan_no_work(lib, bad):
-    """Offsets that are not nondecreasing from 0 up to at most a_rows (device
+    """Offsets that are not nondecreasing from >= 0 up to at most a_rows (device
     data the host cannot check) are caught by the GEMM's plan: it records
     MOE_ERR_INVALID and plans no work, so the output keeps its contents and
     no tile reads or writes outside the operands."""
     G, N, K, R = 3, 256, 256, 40
     offsets = {"past_rows": [0, 10, 20, 41], "decreasing": [0, 30, 10, 40],
-               "nonzero_start": [5, 10, 20, 40]}[bad]
+               "negative_start": [-5, 10, 20, 40]}[bad]
     a = torch.zeros((R, K), dtype=torch.uint8, device="cuda")
     asc = torch.full((R, K // 128), 127, dtype=torch.uint8, device="cuda")
     w = torch.zeros((G, N, K // 2), dtype=torch.uint8, device="cuda")

@@ -460,3 +460,90 @@ def test_w4afp8_swiglu_epilogue_matches_standalone(lib):
     np.testing.assert_array_equal(host(hq), host(hq2))
     np.testing.assert_array_equal(host(sh), host(sh2))
     _swiglu_ok(host(hq), host(sh), ffn.grouped_gemm_w4afp8(a, asc, offsets, q, sinv), I)
+
+
+# ------------------------------- f3 ---------------------------------------
+def _fp8w_inputs(seed, sizes, N, K, integer):
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Rn, G = int(offsets[-1]), len(sizes)
+    if integer:
+        a = synth.small_int_e4m3(seed, 1, (Rn, K))
+        asc = np.full((Rn, K // 128), 127, np.uint8)
+        q = synth.small_int_e4m3(seed, 2, (G, N, K))
+        # power-of-two block scales keep every partial product exact
+        sinv = np.exp2((synth.splitmix64(seed, 3, G * (N // 128) * (K // 128)) % np.uint64(5)).astype(np.float64) - 2)
+        sinv = sinv.astype(np.float32).reshape(G, N // 128, K // 128)
+    else:
+        a = synth.random_e4m3(seed, 1, (Rn, K))
+        asc = synth.random_bytes(seed, 2, (Rn, K // 128), 118, 130)
+        q = synth.random_e4m3(seed, 3, (G, N, K))
+        sinv = (synth.uniform(seed, 4, G * (N // 128) * (K // 128)) * 0.01 + 1e-4).astype(np.float32)
+        sinv = sinv.reshape(G, N // 128, K // 128)
+    return a, asc, offsets, q, sinv
+
+
+def _run_fp8w(lib, a, asc, offsets, q, sinv, epi, block_n, out=None):
+    G, N, K = q.shape
+    Rn = a.shape[0]
+    ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
+    osc = None
+    if epi == lib.MOE_EPI_SWIGLU_QUANT:
+        out = torch.empty((Rn, N // 2), dtype=torch.uint8, device="cuda")
+        osc = torch.empty((Rn, N // 256), dtype=torch.uint8, device="cuda")
+    elif out is None:
+        out = torch.empty((Rn, N), dtype=torch.float32, device="cuda")
+    off = offsets if isinstance(offsets, torch.Tensor) else dev(offsets)
+    lib.moe_grouped_gemm_fp8_block128(dev(a), dev(asc), off, dev(q), dev(sinv), epi, out, osc, ws, 10.0, block_n)
+    torch.cuda.synchronize()
+    return out, osc
+
+
+@pytest.mark.parametrize("block_n", [16, 32, 64, 128])
+def test_fp8_block_gemm_integer_exact(lib, block_n):
+    a, asc, offsets, q, sinv = _fp8w_inputs(14, GROUPS, 256, 512, True)
+    out, _ = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("block_n", [16, 64])
+def test_fp8_block_gemm_random(lib, block_n):
+    a, asc, offsets, q, sinv = _fp8w_inputs(15, [3, 0, 40, 130, 1], 384, 1024, False)
+    out, _ = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv)
+    av = Q.dequantize_fp8_pow2(a, asc)
+    bound = np.zeros_like(ref)
+    for g in range(len(offsets) - 1):
+        r0, r1 = offsets[g], offsets[g + 1]
+        if r1 > r0:
+            bound[r0:r1] = np.abs(av[r0:r1]) @ np.abs(ffn.dequant_fp8_block128(q[g], sinv[g])).T
+    got = out.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= 1024 * 2.0 ** -24 * bound + 1e-30).all()
+
+
+def test_fp8_block_gemm_swiglu_matches_standalone(lib):
+    I = 256
+    a, asc, offsets, q, sinv = _fp8w_inputs(16, [5, 0, 33, 70], 2 * I, 512, False)
+    gu, _ = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, 32)
+    hq, sh = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_SWIGLU_QUANT, 32)
+    hq2, sh2 = torch.empty_like(hq), torch.empty_like(sh)
+    lib.moe_swiglu_clamp(gu, hq2, sh2, 10.0)
+    np.testing.assert_array_equal(host(hq), host(hq2))
+    np.testing.assert_array_equal(host(sh), host(sh2))
+    _swiglu_ok(host(hq), host(sh), ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv), I)
+
+
+def test_fp8_block_gemm_group_view(lib):
+    """offsets may start above 0: a one-group view [offsets[2], offsets[3]) of
+    a larger grouping computes exactly those rows and leaves the rest."""
+    a, asc, offsets, q, sinv = _fp8w_inputs(17, [7, 20, 19, 5], 256, 256, True)
+    off_d = dev(offsets)
+    out = torch.full((a.shape[0], 256), -1.0, dtype=torch.float32, device="cuda")
+    _run_fp8w(lib, a, asc, off_d[2:], q[2:3], sinv[2:3], lib.MOE_EPI_STORE_F32, 16, out=out)
+    got = out.cpu().numpy()
+    r0, r1 = int(offsets[2]), int(offsets[3])
+    ref = ffn.grouped_gemm_fp8_block128(a[r0:r1], asc[r0:r1], np.array([0, r1 - r0], np.int32), q[2:3], sinv[2:3])
+    np.testing.assert_array_equal(got[r0:r1], ref.astype(np.float32))
+    assert (got[:r0] == -1.0).all() and (got[r1:] == -1.0).all()
+    no_device_error(lib)

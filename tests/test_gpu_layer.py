@@ -161,3 +161,53 @@ def test_segment_graphs_match_eager(lib):
         assert torch.equal(y_graph.view(torch.int16), buf.y.view(torch.int16))
     assert lib.moe_get_device_error() == 0
     del graphs
+
+
+def _shared_fp8_ref(x, logits, w13, s13, w2, s2, k, tokens=None):
+    """Oracle layer with the shared expert (group E) cast to FP8 [128, 128]
+    blocks by the oracle's cast."""
+    from oracle import repack as Rp
+    E = w13.shape[0] - 1
+    q13, i13, _ = Rp.repack_mxfp4_to_fp8_block128(w13[E:E + 1], s13[E:E + 1])
+    q2, i2, _ = Rp.repack_mxfp4_to_fp8_block128(w2[E:E + 1], s2[E:E + 1])
+    return ffn.moe_layer(x, logits, w13, s13, w2, s2, k, tokens=tokens, shared_fp8=(q13[0], i13[0], q2[0], i2[0]))
+
+
+@pytest.mark.parametrize("weights", ["mxfp4", "w4afp8"])
+def test_tiny_layer_shared_fp8(lib, weights):
+    """Routed experts in MXFP4 (or W4AFP8), the shared expert as FP8 with
+    [128, 128] block scales through moe_grouped_gemm_fp8_block128."""
+    wl = synth.tiny_layer(5)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk, weights=weights, shared="fp8")
+    buf = layer.alloc(wl.T)
+    y = layer.forward(torch.from_numpy(wl.x_bf16.view(np.int16)).cuda(), torch.from_numpy(wl.logits).cuda(), buf)
+    if weights == "mxfp4":
+        ref = _shared_fp8_ref(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    else:
+        from oracle import repack as Rp
+        E = wl.E
+        q13, i13 = Rp.repack_mxfp4_to_int4g128(wl.w13, wl.w13_e8m0)
+        q2, i2 = Rp.repack_mxfp4_to_int4g128(wl.w2, wl.w2_e8m0)
+        f13, g13, _ = Rp.repack_mxfp4_to_fp8_block128(wl.w13[E:E + 1], wl.w13_e8m0[E:E + 1])
+        f2, g2, _ = Rp.repack_mxfp4_to_fp8_block128(wl.w2[E:E + 1], wl.w2_e8m0[E:E + 1])
+        ref = ffn.moe_layer(wl.x_bf16, wl.logits, None, None, None, None, wl.topk, weights="w4afp8",
+                            w13_int4=q13, w13_sinv=i13, w2_int4=q2, w2_sinv=i2,
+                            shared_fp8=(f13[0], g13[0], f2[0], g2[0]))
+    check_y(y.float().cpu().numpy(), ref["y"])
+    assert lib.moe_get_device_error() == 0
+
+
+def test_decode_layer_shared_fp8_full_size(lib):
+    """Decode configuration (64 tokens, 256 + 1 experts) with the FP8 shared
+    expert; sampled tokens against the oracle."""
+    T, H, I, E, k = 64, 4096, 2048, 256, 6
+    w13, s13, w2, s2 = synth.expert_weights(0, E + 1, H, I, n_proto=4)
+    x = synth.decode_activations(0, T, H)
+    logits = synth.uniform_logits(0, T, E)
+    layer = MoeLayer(w13, s13, w2, s2, k, shared="fp8")
+    buf = layer.alloc(T)
+    y = layer.forward(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(logits).cuda(), buf)
+    toks = np.sort((synth.splitmix64(0, 79, 8) % np.uint64(T)).astype(np.int64))
+    ref = _shared_fp8_ref(x, logits, w13, s13, w2, s2, k, tokens=toks)
+    check_y(y.float().cpu().numpy()[toks], ref["y"])
+    assert lib.moe_get_device_error() == 0
