@@ -14,6 +14,16 @@ Passages:
     model card (模型训练: weight block size [128, 128]).  Reading: E4M3 weights
     [N, K] with a float32 weight_scale_inv [N/128, K/128] per [128, 128] block
     (w = e4m3 * scale_inv), the same dynamic E4M3 activations.
+  * PTPC-FP8: "DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough, 核心参数
+    (quant_scheme ptpc_fp8): E4M3 everywhere; weights per output channel with
+    a static scale (ch_axis 0, min-max observer), activations per token with a
+    dynamic scale, symmetric, half_even rounding; the routed and shared
+    experts are both quantised, from the dequantised base weights.  Readings:
+    scale = amax / 448 (float32 IEEE divide; 1.0 when amax == 0); q =
+    E4M3(x / scale) with a float32 IEEE divide, nearest even, saturating; the
+    GEMM accumulates sum q_a * q_w and multiplies by scale_a[token] *
+    scale_w[channel]; h after SwiGLU is requantised per token over its I
+    columns.
 
 Readings: w1 = gate, w3 = up, w2 = down; both gate and up are clamped to
 [-limit, limit] before silu(gate) * up (which tensors the clamp applies to is
@@ -28,7 +38,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .formats import decode_e2m1_packed, decode_e4m3, decode_e8m0
+from .formats import decode_bf16_bits, decode_e2m1_packed, decode_e4m3, decode_e8m0, encode_e4m3_rne_sat
 from .permute import gather_rows, permute
 from .quant import dequantize_fp8_pow2, quantize_act_fp8, quantize_fp8_pow2
 from .route import route_topk
@@ -106,6 +116,62 @@ def grouped_gemm_fp8_block128(a_q, a_s, offsets, w_q, w_scale_inv):
     N = w_q.shape[1]
     out = grouped_gemm(a_q, a_s, offsets, lambda g: dequant_fp8_block128(w_q[g], w_scale_inv[g]), w_q.shape[0])
     return out if out.shape[1] else np.zeros((a_q.shape[0], N))
+
+
+def quantize_fp8_per_row(x: np.ndarray):
+    """float32 [rows, cols] -> (E4M3 [rows, cols], float32 scale [rows]):
+    scale = amax / 448 (float32 divide, 1 when amax == 0), q = E4M3(x / scale)
+    with a float32 divide (PTPC-FP8 per-token / per-channel rule)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x32).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    q = encode_e4m3_rne_sat((x32 / scale[..., None]).astype(np.float64))
+    return q, scale
+
+
+def ptpc_weights(fp4: np.ndarray, e8m0: np.ndarray):
+    """MXFP4 [G, N, K/2] + E8M0 -> (E4M3 [G, N, K], float32 per-channel scale [G, N]):
+    the per-row rule applied to the exact float32 dequantisation."""
+    w = dequant_mxfp4(fp4, e8m0).astype(np.float32)
+    return quantize_fp8_per_row(w)
+
+
+def grouped_gemm_ptpc(a_q, a_scale, offsets, w_q, w_scale):
+    """E4M3 rows [R, K] with per-row scales [R] x E4M3 weights [G, N, K] with
+    per-channel scales [G, N] -> float64 [R, N]."""
+    a = decode_e4m3(a_q) * np.asarray(a_scale, np.float32).astype(np.float64)[:, None]
+    N = w_q.shape[1]
+    out = np.zeros((a.shape[0], N), np.float64)
+    for g in range(w_q.shape[0]):
+        r0, r1 = int(offsets[g]), int(offsets[g + 1])
+        if r1 > r0:
+            w = decode_e4m3(w_q[g]) * np.asarray(w_scale[g], np.float32).astype(np.float64)[:, None]
+            out[r0:r1] = a[r0:r1] @ w.T
+    return out
+
+
+def moe_layer_ptpc(x_bf16, logits, w13_q, w13_scale, w2_q, w2_scale, topk, route_scale=1.5,
+                   swiglu_limit=10.0, has_shared=1, route_norm=1, tokens=None):
+    """The expert path with PTPC-FP8 weights (w13_q [G, 2I, H] + [G, 2I], w2_q
+    [G, H, I] + [G, H]; G = E + has_shared) and per-token dynamic activations."""
+    x_bf16 = np.asarray(x_bf16)
+    logits = np.asarray(logits, dtype=np.float32)
+    if tokens is not None:
+        x_bf16 = x_bf16[tokens]
+        logits = logits[tokens]
+    T, H = x_bf16.shape
+    E = logits.shape[1]
+    I = w2_q.shape[2]
+    xq, sx = quantize_fp8_per_row(decode_bf16_bits(x_bf16))
+    idx, w = route_topk(logits, topk, route_scale, route_norm)
+    counts, offsets, perm, inv, src = permute(idx, E, has_shared)
+    xq_p, sx_p = xq[src], sx[src]
+    gu = grouped_gemm_ptpc(xq_p, sx_p, offsets, w13_q, w13_scale)
+    h = swiglu_clamp(gu, I, swiglu_limit).astype(np.float32)
+    hq, sh = quantize_fp8_per_row(h)
+    o = grouped_gemm_ptpc(hq, sh, offsets, w2_q, w2_scale)
+    y = combine(o, inv, w, offsets, has_shared)
+    return dict(xq=xq, sx=sx, idx=idx, w=w, offsets=offsets, inv=inv, gu=gu, h=h, hq=hq, sh=sh, o=o, y=y)
 
 
 def silu(g: np.ndarray) -> np.ndarray:

@@ -154,3 +154,57 @@ def test_fp8_block_scale_is_linear_per_block():
     twice = ffn.grouped_gemm_fp8_block128(a, asc, off, q[None], s2[None])
     hi = ffn.grouped_gemm_fp8_block128(a[:, :], asc, off, np.where(np.arange(K) >= 128, q, 0)[None], s1[None])
     np.testing.assert_array_equal(twice, base + hi)
+
+
+# --------------------------------- PTPC-FP8 ---------------------------------------
+def test_ptpc_per_row_closed_forms():
+    # amax 3.5 -> scale 3.5 / 448 = 2^-7 exactly; 3.5 -> 448 (0x7E), 1.0 -> 128 (0x70)
+    q, s = ffn.quantize_fp8_per_row(np.array([[3.5, 1.0, -1.0, 0.0]], np.float32))
+    assert s[0] == np.float32(2.0 ** -7)
+    assert list(q[0]) == [0x7E, 0x70, 0xF0, 0x00]
+    # an all-zero row: scale 1, codes 0
+    q, s = ffn.quantize_fp8_per_row(np.zeros((1, 8), np.float32))
+    assert s[0] == 1.0 and (q == 0).all()
+
+
+def test_ptpc_per_row_error_bound():
+    """|dequant - x| <= 2^-4 |x| for normal E4M3 codes, <= 2^-10 * scale below."""
+    x = (synth.normal(21, 1, 64 * 512) * 3).astype(np.float32).reshape(64, 512)
+    q, s = ffn.quantize_fp8_per_row(x)
+    back = F.decode_e4m3(q) * s[:, None].astype(np.float64)
+    err = np.abs(back - x)
+    assert (err <= np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * s[:, None])).all()
+    # the row maximum lands on 448 up to the float32 divide
+    assert (np.abs(F.decode_e4m3(q)).max(axis=1) == 448.0).all()
+
+
+def test_ptpc_gemm_integer_case():
+    """Unit scales and small-integer E4M3 codes: the result is the integer
+    matmul, computed here in int64."""
+    a = synth.small_int_e4m3(22, 1, (30, 256))
+    w = synth.small_int_e4m3(22, 2, (2, 128, 256))
+    off = np.array([0, 11, 30], np.int32)
+    got = ffn.grouped_gemm_ptpc(a, np.ones(30, np.float32), off, w, np.ones((2, 128), np.float32))
+    ai = F.decode_e4m3(a).astype(np.int64)
+    wi = F.decode_e4m3(w).astype(np.int64)
+    ref = np.concatenate([ai[:11] @ wi[0].T, ai[11:] @ wi[1].T])
+    np.testing.assert_array_equal(got, ref.astype(np.float64))
+
+
+def test_ptpc_scale_is_pow2_equivariant():
+    """Scaling a row by 2^j scales its per-row scale by 2^j and keeps the codes."""
+    x = (synth.normal(23, 1, 4 * 256) * 0.7).astype(np.float32).reshape(4, 256)
+    q, s = ffn.quantize_fp8_per_row(x)
+    q2, s2 = ffn.quantize_fp8_per_row(x * np.float32(8.0))
+    np.testing.assert_array_equal(q, q2)
+    np.testing.assert_array_equal(s2, s * np.float32(8.0))
+
+
+def test_ptpc_layer_token_subset():
+    wl = synth.tiny_layer(6)
+    q13, s13 = ffn.ptpc_weights(wl.w13, wl.w13_e8m0)
+    q2, s2 = ffn.ptpc_weights(wl.w2, wl.w2_e8m0)
+    full = ffn.moe_layer_ptpc(wl.x_bf16, wl.logits, q13, s13, q2, s2, wl.topk)
+    toks = np.array([1, 4, 9])
+    sub = ffn.moe_layer_ptpc(wl.x_bf16, wl.logits, q13, s13, q2, s2, wl.topk, tokens=toks)
+    np.testing.assert_allclose(sub["y"], full["y"][toks], rtol=0, atol=1e-12 * np.abs(full["y"]).max())
