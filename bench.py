@@ -33,14 +33,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s or HBM GB/s vs B200 roofline"
-def kernels_per_step(wl: dict, shared: str = "mxfp4") -> int:
+def kernels_per_step(wl: dict, shared: str = "mxfp4", weights: str = "mxfp4") -> int:
     """Library kernels one layer step launches: quant 1, route 1, grouping 2
     (one block for <= 2048 routed pairs, then the gather) or 4 (chunked), two
     GEMM calls of 2 (prep + GEMM; two more with the FP8 shared expert),
-    combine 1."""
+    combine 1.  PTPC-FP8 adds the row-scale gather and the per-token
+    quantisation of h."""
     grouping = 2 if wl["T"] * wl["k"] <= 2048 else 4
     gemm_calls = 4 if shared == "fp8" else 2
-    return 1 + 1 + grouping + gemm_calls * 2 + 1
+    extra = 2 if weights == "ptpc" else 0
+    return 1 + 1 + grouping + gemm_calls * 2 + 1 + extra
 
 WORKLOADS = {
     "repack": dict(T=0, H=4096, I=2048, E=256, k=6, logits="uniform"),
@@ -60,8 +62,11 @@ def read_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
+GEMM_ENTRY = {"mxfp4": "moe_grouped_gemm_mxfp4", "w4afp8": "moe_grouped_gemm_w4afp8",
+              "ptpc": "moe_grouped_gemm_fp8_ptpc"}
 GEMM_SOURCES = {"mxfp4": ("common.cuh", "gemm_mxfp4.cuh", "sm100.cuh"),
-                "w4afp8": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh")}
+                "w4afp8": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh"),
+                "ptpc": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh")}
 
 
 def source_digest(weights: str = "mxfp4") -> str:
@@ -225,6 +230,14 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
         # the shared expert streams E4M3 bytes and float32 [128, 128] block scales instead
         w13_bytes += 2 * I * H + 4 * (2 * I // 128) * (H // 128) - w13
         w2_bytes += H * I + 4 * (H // 128) * (I // 128) - w2
+    if getattr(layer, "weights", "mxfp4") == "ptpc":
+        # E4M3 weights with one float32 scale per channel; activations E4M3
+        # with one float32 scale per row (the float32 h round trip between
+        # the GEMM and its per-token requantisation is not counted)
+        return dict(active_experts=active, rows=R,
+                    w13=active * (2 * I * H + 4 * 2 * I) + R * (H + 4) + R * (I + 4),
+                    w2=active * (H * I + 4 * H) + R * (I + 4) + R * H * 4,
+                    flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
     return dict(active_experts=active, rows=R,
                 w13=w13_bytes + R * (H + H // 128) + R * (I + I // 128),
                 w2=w2_bytes + R * (I + I // 128) + R * H * 4,
@@ -430,19 +443,20 @@ def run_ours(args, wl):
         achieved = ab["w13"] / (g13 / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm"], 4), "traffic": recorded_traffic(args.workload, args.weights),
-                "kernel": f"moe_grouped_gemm_{args.weights} (w1/w3, SwiGLU epilogue)",
+                "kernel": f"{GEMM_ENTRY[args.weights]} (w1/w3, SwiGLU epilogue)",
                 "peak_source": f"{peaks['src']} HBM copy"}
     else:
         fp8_peak = 2.0 * peaks["bf16_sustained"]
         achieved = ab["flops13"] / (g13 / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": round(achieved / fp8_peak, 4), "traffic": recorded_traffic(args.workload, args.weights),
-                "kernel": f"moe_grouped_gemm_{args.weights} (w1/w3, SwiGLU epilogue)",
+                "kernel": f"{GEMM_ENTRY[args.weights]} (w1/w3, SwiGLU epilogue)",
                 "peak_source": f"{peaks['src']} bf16 sustained x 2 (FP8 rate)"}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe2m1->f32" if args.weights == "mxfp4" else "e4m3xint4->f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": {"mxfp4": "e4m3xe2m1->f32", "w4afp8": "e4m3xint4->f32",
+                                                                                 "ptpc": "e4m3xe4m3->f32"}[args.weights],
         "data": "synthetic",
         "config": {"workload": f"{args.workload} layer: hidden {wl['H']}, intermediate {wl['I']}, "
                                f"{wl['E']} routed + 1 shared experts, top-{wl['k']}, {T} tokens per GPU",
@@ -461,7 +475,7 @@ def run_ours(args, wl):
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xh.numel() * 2 + lh.numel() * 4),
                 "d2h_bytes_per_step": int(yh.numel() * 2)},
-        "gpu_launches": kernels_per_step(wl, args.shared) * args.steps,
+        "gpu_launches": kernels_per_step(wl, args.shared, args.weights) * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
@@ -578,7 +592,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--weights", choices=["mxfp4", "w4afp8"], default="mxfp4")
+    ap.add_argument("--weights", choices=["mxfp4", "w4afp8", "ptpc"], default="mxfp4")
     ap.add_argument("--shared", choices=["mxfp4", "fp8"], default="mxfp4",
                     help="shared expert weights: MXFP4 (group E of the grouped GEMM) or FP8 [128, 128] blocks")
     ap.add_argument("--graph", choices=["on", "off"], default="on",

@@ -39,6 +39,10 @@ SIGNATURES = {
     "repack_mxfp4_to_nvfp4": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P, _P]),
     "repack_mxfp4_to_int4g128": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P]),
     "repack_mxfp4_to_fp8_block128": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P]),
+    "moe_quantize_fp8_per_token": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_gather_row_scales": (_I, [_P, _I, _I, _P, _I, _P, _P, _P]),
+    "moe_grouped_gemm_fp8_ptpc": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _SZ, _P]),
+    "repack_mxfp4_to_fp8_per_channel": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P]),
 }
 
 _lib = None

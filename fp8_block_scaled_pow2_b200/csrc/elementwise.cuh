@@ -122,6 +122,75 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
+// ------------------------- per-token FP8 (PTPC) ----------------------------
+// PTPC-FP8 ("DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough, 核心参数):
+// per-row (per-token) dynamic scale = amax / 448 (float32 IEEE divide, 1 for
+// a zero row); q = E4M3(x / scale), float32 IEEE divide, nearest even,
+// saturating.  One block of 256 threads per row; cols % 8 == 0.
+template <bool F32_IN>
+__global__ void __launch_bounds__(256) quant_fp8_per_row_kernel(const void* __restrict__ x, int cols,
+                                                                uint8_t* __restrict__ q, float* __restrict__ scale) {
+  __shared__ float s_max[8];
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  auto load8 = [&](int c8, float (&v)[8]) {
+    if constexpr (F32_IN) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + row * cols) + 2 * c8;
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + row * cols) + c8);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = bf16_lo(u[j]);
+        v[2 * j + 1] = bf16_hi(u[j]);
+      }
+    }
+  };
+  float m = 0.0f;
+  for (int c8 = tid; c8 < cols / 8; c8 += blockDim.x) {
+    float v[8];
+    load8(c8, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+  m = warp_max_nonneg(m);
+  if (lane == 0) s_max[wid] = m;
+  __syncthreads();
+  m = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+  const float sc = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  if (tid == 0) scale[row] = sc;
+  for (int c8 = tid; c8 < cols / 8; c8 += blockDim.x) {
+    float v[8];
+    load8(c8, v);
+    const uint32_t lo = e4m3x4(__fdiv_rn(v[0], sc), __fdiv_rn(v[1], sc), __fdiv_rn(v[2], sc), __fdiv_rn(v[3], sc));
+    const uint32_t hi = e4m3x4(__fdiv_rn(v[4], sc), __fdiv_rn(v[5], sc), __fdiv_rn(v[6], sc), __fdiv_rn(v[7], sc));
+    reinterpret_cast<uint2*>(q + row * cols)[c8] = make_uint2(lo, hi);
+  }
+}
+
+// Per-row float32 scales of the grouped rows: row r takes the scale of its
+// source token (perm[r] / k for a routed pair, perm[r] - T*k for a shared
+// row).  Rows past offsets[E + 1] (pairs the grouping rejected) are skipped.
+__global__ void __launch_bounds__(256) gather_row_scales_kernel(const int32_t* __restrict__ perm, int T, int k,
+                                                                const int32_t* __restrict__ offsets, int E,
+                                                                const float* __restrict__ src,
+                                                                float* __restrict__ dst) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int P = T * k;
+  if (r >= offsets[E + 1] || r >= (int64_t)P + T) return;
+  const int p = perm[r];
+  if (p < 0 || p >= P + T) {
+    record_error(MOE_ERR_INVALID);
+    dst[r] = 0.0f;
+    return;
+  }
+  dst[r] = src[p < P ? p / k : p - P];
+}
+
 // ------------------------------- a3 ---------------------------------------
 // Grouping in deterministic passes:
 //   count:   per chunk of kChunk pairs, a histogram over experts

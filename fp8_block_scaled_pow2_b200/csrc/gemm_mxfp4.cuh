@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
     }
   }
   const int t = blockIdx.x;
-  if (t >= n_tiles) return;
+  if (t >= n_tiles || sx == nullptr) return;     // sx == nullptr: the plan only
   // the group of tile t: the last g with s_t0[g] <= t (empty groups share
   // their successor's first tile and sort before it)
   int lo = 0, hi = G - 1;

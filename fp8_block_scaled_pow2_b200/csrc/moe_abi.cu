@@ -10,6 +10,7 @@
 #include "elementwise.cuh"
 #include "gemm_mxfp4.cuh"
 #include "gemm_w4afp8.cuh"
+#include "gemm_ptpc.cuh"
 #include "repack.cuh"
 
 using namespace moe;
@@ -186,6 +187,26 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
     case 32: return launch_w4a<32, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
     case 64: return launch_w4a<64, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
     default: return launch_w4a<128, false, MOE_EPI_STORE_BF16, W8>(ta, tb, args, st);
+  }
+}
+
+template <int BN, bool DUAL, int EPI>
+int launch_ptpc(const CUtensorMap& ta, const CUtensorMap& tb, const ptpc::Args& a, cudaStream_t st) {
+  using C = ptpc::Cfg<BN, DUAL>;
+  auto k = ptpc::gemm_ptpc_kernel<BN, DUAL, EPI>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  k<<<sm_count(), ptpc::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  return launch_status();
+}
+
+template <bool DUAL, int EPI>
+int launch_ptpc_bn(int block_n, const CUtensorMap& ta, const CUtensorMap& tb, const ptpc::Args& a, cudaStream_t st) {
+  switch (block_n) {
+    case 16: return launch_ptpc<16, DUAL, EPI>(ta, tb, a, st);
+    case 32: return launch_ptpc<32, DUAL, EPI>(ta, tb, a, st);
+    case 64: return launch_ptpc<64, DUAL, EPI>(ta, tb, a, st);
+    default: return launch_ptpc<128, DUAL, EPI>(ta, tb, a, st);
   }
 }
 
@@ -419,6 +440,82 @@ int moe_grouped_gemm_fp8_block128(const uint8_t* a_e4m3, const uint8_t* a_e8m0_1
                              swiglu_limit, block_n, out, out_scale, workspace, workspace_bytes, stream);
 }
 
+int moe_grouped_gemm_fp8_ptpc(const uint8_t* a_e4m3, const float* a_scale, int a_rows, const int32_t* offsets,
+                              int n_groups, const uint8_t* w_e4m3, const float* w_scale, int N, int K, int epilogue,
+                              float swiglu_limit, int block_n, void* out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
+    return MOE_ERR_INVALID;
+  if (epilogue != MOE_EPI_STORE_F32 && epilogue != MOE_EPI_STORE_BF16 && epilogue != MOE_EPI_SWIGLU_F32)
+    return MOE_ERR_INVALID;
+  const bool dual = epilogue == MOE_EPI_SWIGLU_F32;
+  if (dual && N % 256) return MOE_ERR_INVALID;
+  if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
+  if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128) return MOE_ERR_UNSUPPORTED;
+  if (a_rows == 0) return MOE_OK;
+  if (!a_e4m3 || !a_scale || !offsets || !w_e4m3 || !w_scale || !out || !workspace) return MOE_ERR_INVALID;
+  if (!aligned(a_e4m3, 16) || !aligned(w_e4m3, 16) || !aligned(a_scale, 4) || !aligned(w_scale, 4) ||
+      !aligned(workspace, 256))
+    return MOE_ERR_INVALID;
+  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
+  if (workspace_bytes < L.total) return MOE_ERR_INVALID;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_e4m3, (uint64_t)K, (uint64_t)n_groups * N, (uint64_t)K, 128,
+                128))
+    return MOE_ERR_LAUNCH;
+  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
+                (uint32_t)block_n))
+    return MOE_ERR_LAUNCH;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  ptpc::Args args;
+  args.w_scale = w_scale;
+  args.a_scale = a_scale;
+  args.header = reinterpret_cast<const int*>(ws + L.header);
+  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
+  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
+  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
+  args.G = n_groups;
+  args.N = N;
+  args.K = K;
+  args.out = out;
+  args.limit = swiglu_limit;
+  cudaStream_t st = S(stream);
+  const int n_ft = dual ? N / 256 : N / 128;
+  // the plan only: no per-tile activation scale blocks (sx == nullptr)
+  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+      offsets, n_groups, (int)a_rows, block_n, n_ft, nullptr, K / 128, reinterpret_cast<int*>(ws + L.header),
+      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  if (dual) return launch_ptpc_bn<true, MOE_EPI_SWIGLU_F32>(block_n, ta, tb, args, st);
+  if (epilogue == MOE_EPI_STORE_F32) return launch_ptpc_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
+  return launch_ptpc_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
+}
+
+int moe_quantize_fp8_per_token(const void* x, int x_is_f32, int rows, int cols, uint8_t* q, float* scale,
+                               void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 8) return MOE_ERR_INVALID;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !scale || !aligned(x, 16) || !aligned(q, 8) || !aligned(scale, 4)) return MOE_ERR_INVALID;
+  if (x_is_f32)
+    quant_fp8_per_row_kernel<true><<<(unsigned)rows, 256, 0, S(stream)>>>(x, cols, q, scale);
+  else
+    quant_fp8_per_row_kernel<false><<<(unsigned)rows, 256, 0, S(stream)>>>(x, cols, q, scale);
+  return launch_status();
+}
+
+int moe_gather_row_scales(const int32_t* perm, int T, int k, const int32_t* offsets, int E, const float* src,
+                          float* dst, void* stream) {
+  if (T < 0 || k < 0 || E < 0) return MOE_ERR_INVALID;
+  const int64_t max_rows = (int64_t)T * (k + 1);
+  if (max_rows > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (max_rows == 0) return MOE_OK;
+  if (!perm || !offsets || !src || !dst || !aligned(src, 4) || !aligned(dst, 4)) return MOE_ERR_INVALID;
+  gather_row_scales_kernel<<<(unsigned)((max_rows + 255) / 256), 256, 0, S(stream)>>>(perm, T, k, offsets, E, src,
+                                                                                        dst);
+  return launch_status();
+}
+
 int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq, uint8_t* sh, void* stream) {
   if (rows < 0 || I <= 0 || I % 128) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
@@ -499,6 +596,18 @@ int repack_mxfp4_to_fp8_block128(const uint8_t* fp4, const uint8_t* e8m0, int64_
   const int64_t blocks = n_mats * (int64_t)(N / 128) * (K / 128);
   if (blocks > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
   fp8_block128_kernel<<<(unsigned)blocks, 128, 0, S(stream)>>>(fp4, e8m0, N, K, out_e4m3, out_scale_inv);
+  return launch_status();
+}
+
+int repack_mxfp4_to_fp8_per_channel(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                                    uint8_t* out_e4m3, float* out_scale, void* stream) {
+  if (n_mats < 0 || N <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID;
+  if (n_mats == 0) return MOE_OK;
+  if (!fp4 || !e8m0 || !out_e4m3 || !out_scale) return MOE_ERR_INVALID;
+  if (!aligned(fp4, 4) || !aligned(out_e4m3, 8) || !aligned(out_scale, 4)) return MOE_ERR_INVALID;
+  const int64_t rows = n_mats * (int64_t)N;
+  if (rows > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  fp8_per_channel_kernel<<<(unsigned)rows, 256, 0, S(stream)>>>(fp4, e8m0, K, out_e4m3, out_scale);
   return launch_status();
 }
 

@@ -342,4 +342,71 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
   if (inexact) record_error(MOE_ERR_RANGE);
 }
 
+// MXFP4 -> PTPC-FP8 weights ("DeepSeek-V4.1-Flash-Quark-PTPC-FP8"
+// walkthrough, 核心参数: per output channel, static, symmetric, half_even):
+// one block of 256 threads per row of K elements; w = exact float32
+// dequantisation; scale = amax / 448 (float32 IEEE divide, 1 for a zero row);
+// q = E4M3(w / scale) with a float32 IEEE divide.  A float32 overflow of w
+// records MOE_ERR_RANGE; an E8M0 NaN records MOE_ERR_NAN_SCALE and skips the
+// row.  K % 32 == 0.
+__global__ void __launch_bounds__(256) fp8_per_channel_kernel(const uint8_t* __restrict__ fp4,
+                                                              const uint8_t* __restrict__ e8m0, int K,
+                                                              uint8_t* __restrict__ out, float* __restrict__ scale) {
+  __shared__ float s_max[8];
+  __shared__ int s_bad[8];
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  // thread t owns 8-element chunks t, t + 256, ...: 4 bytes of nibbles each
+  auto load8 = [&](int c8, float (&v)[8], int& bad) {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(fp4 + row * (K / 2)) + c8);
+    const int b = __ldg(e8m0 + row * (K / 32) + c8 / 4);
+    bad |= b == 255;
+    const float sc = exp2_int(b - 127);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t nib = (w >> (4 * j)) & 0xFu;
+      const float mag = __fmul_rn(kE2M1[nib & 7u], sc);
+      v[j] = (nib & 8u) ? -mag : mag;
+    }
+  };
+  float m = 0.0f;
+  int bad = 0;
+  for (int c8 = tid; c8 < K / 8; c8 += blockDim.x) {
+    float v[8];
+    load8(c8, v, bad);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+  m = warp_max_nonneg(m);
+  bad = __reduce_or_sync(0xFFFFFFFFu, bad);
+  if (lane == 0) { s_max[wid] = m; s_bad[wid] = bad; }
+  __syncthreads();
+  m = s_max[0];
+  bad = s_bad[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) {
+    m = fmaxf(m, s_max[w]);
+    bad |= s_bad[w];
+  }
+  if (bad) {
+    if (tid == 0) record_error(MOE_ERR_NAN_SCALE);
+    return;
+  }
+  if (isinf(m)) {
+    if (tid == 0) record_error(MOE_ERR_RANGE);
+    return;
+  }
+  const float sc = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+  if (tid == 0) scale[row] = sc;
+  for (int c8 = tid; c8 < K / 8; c8 += blockDim.x) {
+    float v[8];
+    int unused = 0;
+    load8(c8, v, unused);
+    const uint32_t lo = e4m3x4(__fdiv_rn(v[0], sc), __fdiv_rn(v[1], sc), __fdiv_rn(v[2], sc), __fdiv_rn(v[3], sc));
+    const uint32_t hi = e4m3x4(__fdiv_rn(v[4], sc), __fdiv_rn(v[5], sc), __fdiv_rn(v[6], sc), __fdiv_rn(v[7], sc));
+    reinterpret_cast<uint2*>(out + row * K)[c8] = make_uint2(lo, hi);
+  }
+}
+
 }  // namespace moe

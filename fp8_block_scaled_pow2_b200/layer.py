@@ -11,6 +11,15 @@ fixed sequence of library calls on one stream, with no host synchronisation:
 
 The shared expert is group E, fed every token with weight 1 ("DeepSeek-V4-
 Flash-SI" model card, 架构特性: one shared expert per layer, always active).
+
+weights="ptpc" runs the PTPC-FP8 form of the same layer ("DeepSeek-V4.1-Flash-
+Quark-PTPC-FP8" walkthrough, 核心参数): per-channel FP8 weights cast once on
+the GPU, per-token dynamic FP8 activations:
+
+    moe_quantize_fp8_per_token -> moe_route_topk -> moe_permute
+    -> moe_gather_row_scales -> moe_grouped_gemm_fp8_ptpc(w13, SwiGLU float32)
+    -> moe_quantize_fp8_per_token(h) -> moe_grouped_gemm_fp8_ptpc(w2, float32)
+    -> moe_combine
 """
 from __future__ import annotations
 
@@ -48,6 +57,11 @@ class Buffers:
     ws_permute: torch.Tensor
     ws_gemm: torch.Tensor
     block_n: int
+    # PTPC-FP8 only: float32 per-row scales and the float32 SwiGLU output
+    sxf: torch.Tensor | None = None
+    sxf_perm: torch.Tensor | None = None
+    hf: torch.Tensor | None = None
+    shf: torch.Tensor | None = None
 
 
 class MoeLayer:
@@ -59,11 +73,14 @@ class MoeLayer:
         (repack_mxfp4_to_int4g128) and runs the W4AFP8 GEMMs.  shared="fp8"
         casts the shared expert (group E of the arrays) once on the GPU to FP8
         E4M3 with [128, 128] block scales (repack_mxfp4_to_fp8_block128) and
-        runs it through moe_grouped_gemm_fp8_block128."""
+        runs it through moe_grouped_gemm_fp8_block128.  weights="ptpc" casts
+        every expert (the shared one included) once on the GPU to PTPC-FP8
+        (repack_mxfp4_to_fp8_per_channel) and quantises the activations per
+        token."""
         self.device = torch.device(device)
         self.G = w13.shape[0]                      # routed experts + shared expert
         self.E = self.G - (1 if has_shared else 0)
-        if shared not in ("mxfp4", "fp8") or (shared == "fp8" and not has_shared):
+        if shared not in ("mxfp4", "fp8") or (shared == "fp8" and (not has_shared or weights == "ptpc")):
             raise ValueError(shared)
         self.shared = shared
         if shared == "fp8":
@@ -111,6 +128,16 @@ class MoeLayer:
             moe.repack_mxfp4_to_int4g128(_dev(w2, d), _dev(w2_e8m0, d), self.w2_q, self.w2_sinv)
             if moe.moe_get_device_error() != 0:
                 raise moe.MoeError("repack_mxfp4_to_int4g128", -4)
+        elif weights == "ptpc":
+            self.w13_q = torch.empty((self.GR, 2 * self.I, self.H), dtype=torch.uint8, device=d)
+            self.w13_s = torch.empty((self.GR, 2 * self.I), dtype=torch.float32, device=d)
+            self.w2_q = torch.empty((self.GR, self.H, self.I), dtype=torch.uint8, device=d)
+            self.w2_s = torch.empty((self.GR, self.H), dtype=torch.float32, device=d)
+            moe.repack_mxfp4_to_fp8_per_channel(_dev(w13, d), _dev(w13_e8m0, d), self.w13_q, self.w13_s)
+            moe.repack_mxfp4_to_fp8_per_channel(_dev(w2, d), _dev(w2_e8m0, d), self.w2_q, self.w2_s)
+            err = moe.moe_get_device_error()
+            if err != 0:
+                raise moe.MoeError("repack_mxfp4_to_fp8_per_channel", err)
         else:
             raise ValueError(weights)
 
@@ -123,7 +150,7 @@ class MoeLayer:
         R = T * k + (T if self.has_shared else 0)
         u8, i32, f32 = torch.uint8, torch.int32, torch.float32
         # the W4AFP8 w1/w3 GEMM may use narrower token tiles than block_n
-        bns = (block_n, 16) if (self.weights == "w4afp8" or self.shared == "fp8") else (block_n,)
+        bns = (block_n, 16) if (self.weights in ("w4afp8", "ptpc") or self.shared == "fp8") else (block_n,)
         ws_g = max([moe.moe_gemm_workspace_size(R, self.G, K, bn) for bn in bns for K in (H, I)] + [256])
         return Buffers(
             T=T,
@@ -136,7 +163,11 @@ class MoeLayer:
             hq=torch.empty((R, I), dtype=u8, device=d), sh=torch.empty((R, I // 128), dtype=u8, device=d),
             o=torch.empty((R, H), dtype=f32, device=d), y=torch.empty((T, H), dtype=torch.bfloat16, device=d),
             ws_permute=torch.empty(moe.moe_permute_workspace_size(T, self.E, k), dtype=u8, device=d),
-            ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n)
+            ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n,
+            **(dict(sxf=torch.empty(max(T, 1), dtype=f32, device=d),
+                    sxf_perm=torch.zeros(max(R, 1), dtype=f32, device=d),
+                    hf=torch.zeros((R, I), dtype=f32, device=d),
+                    shf=torch.empty(max(R, 1), dtype=f32, device=d)) if self.weights == "ptpc" else {}))
 
     def segments(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers, stream=None):
         """The forward pass as four callables run in order on `stream`:
@@ -147,11 +178,21 @@ class MoeLayer:
         g_off = b.offsets[: self.GR + 1]          # the groups of the routed-weight GEMMs
         s_off = b.offsets[self.E:]                 # the shared group alone (FP8 shared expert)
 
+        ptpc = self.weights == "ptpc"
+
         def pre():
-            moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
+            if ptpc:
+                moe.moe_quantize_fp8_per_token(x, b.xq, b.sxf, stream=stream)
+            else:
+                moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
             moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
+            # (PTPC: the E8M0 rows moved alongside are unused; the float32
+            # per-token scales follow the rows through moe_gather_row_scales)
             moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
                             b.xq_perm, b.sx_perm, b.ws_permute, stream=stream)
+            if ptpc:
+                moe.moe_gather_row_scales(b.perm, b.T, self.topk, b.offsets, self.E, b.sxf, b.sxf_perm,
+                                          stream=stream)
 
         bn_dual = min(b.block_n, 64) if b.block_n else 0
         if self.weights == "mxfp4":
@@ -163,6 +204,16 @@ class MoeLayer:
             def routed2():
                 moe.moe_grouped_gemm_mxfp4(b.hq, b.sh, g_off, self.w2_p, self.GR, self.H, moe.MOE_EPI_STORE_F32,
                                            b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+        elif ptpc:
+            def routed13():
+                moe.moe_grouped_gemm_fp8_ptpc(b.xq_perm, b.sxf_perm, g_off, self.w13_q, self.w13_s,
+                                              moe.MOE_EPI_SWIGLU_F32, b.hf, b.ws_gemm, self.swiglu_limit, bn_dual,
+                                              stream=stream)
+                moe.moe_quantize_fp8_per_token(b.hf, b.hq, b.shf, stream=stream)
+
+            def routed2():
+                moe.moe_grouped_gemm_fp8_ptpc(b.hq, b.shf, g_off, self.w2_q, self.w2_s, moe.MOE_EPI_STORE_F32,
+                                              b.o, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
         else:
             def routed13():
                 moe.moe_grouped_gemm_w4afp8(b.xq_perm, b.sx_perm, g_off, self.w13_q, self.w13_sinv,

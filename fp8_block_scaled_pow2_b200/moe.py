@@ -16,6 +16,7 @@ from ._lib import load
 MOE_EPI_STORE_F32 = 0
 MOE_EPI_STORE_BF16 = 1
 MOE_EPI_SWIGLU_QUANT = 2
+MOE_EPI_SWIGLU_F32 = 3
 
 
 class MoeError(RuntimeError):
@@ -153,6 +154,32 @@ def moe_grouped_gemm_fp8_block128(a, a_scale, offsets, w_e4m3, w_scale_inv, epil
         _stream(stream)))
 
 
+def moe_grouped_gemm_fp8_ptpc(a, a_scale, offsets, w_e4m3, w_scale, epilogue, out, workspace=None,
+                              swiglu_limit=10.0, block_n=0, stream=None):
+    """PTPC-FP8: E4M3 rows [R, K] with float32 per-row scales [R] x E4M3 weights
+    [G, N, K] with float32 per-channel scales [G, N]."""
+    a_rows, K = a.shape
+    G, N = w_e4m3.shape[0], w_e4m3.shape[1]
+    _check("moe_grouped_gemm_fp8_ptpc", _lib().moe_grouped_gemm_fp8_ptpc(
+        _ptr(a), _ptr(a_scale), a_rows, _ptr(offsets), G, _ptr(w_e4m3), _ptr(w_scale), N, K,
+        int(epilogue), ctypes.c_float(swiglu_limit), int(block_n), _ptr(out),
+        _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def moe_quantize_fp8_per_token(x, q, scale, stream=None):
+    """bfloat16 or float32 [rows, cols] -> E4M3 [rows, cols] + float32 scale [rows]."""
+    rows, cols = x.shape
+    is_f32 = 1 if x.element_size() == 4 else 0
+    _check("moe_quantize_fp8_per_token", _lib().moe_quantize_fp8_per_token(
+        _ptr(x), is_f32, rows, cols, _ptr(q), _ptr(scale), _stream(stream)))
+
+
+def moe_gather_row_scales(perm, T, k, offsets, E, src, dst, stream=None):
+    _check("moe_gather_row_scales", _lib().moe_gather_row_scales(
+        _ptr(perm), T, k, _ptr(offsets), E, _ptr(src), _ptr(dst), _stream(stream)))
+
+
 def moe_swiglu_clamp(gu, hq, sh, limit=10.0, stream=None):
     rows, two_i = gu.shape
     _check("moe_swiglu_clamp", _lib().moe_swiglu_clamp(_ptr(gu), rows, two_i // 2, ctypes.c_float(limit),
@@ -185,3 +212,11 @@ def repack_mxfp4_to_fp8_block128(fp4, e8m0, out_e4m3, out_scale_inv, stream=None
     n_mats, N, k2 = fp4.shape
     _check("repack_mxfp4_to_fp8_block128", _lib().repack_mxfp4_to_fp8_block128(
         _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_e4m3), _ptr(out_scale_inv), _stream(stream)))
+
+
+def repack_mxfp4_to_fp8_per_channel(fp4, e8m0, out_e4m3, out_scale, stream=None):
+    """MXFP4 [n_mats, N, K/2] + E8M0 [n_mats, N, K/32] -> E4M3 [n_mats, N, K] and
+    float32 per-channel scales [n_mats, N]."""
+    n_mats, N, k2 = fp4.shape
+    _check("repack_mxfp4_to_fp8_per_channel", _lib().repack_mxfp4_to_fp8_per_channel(
+        _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, _ptr(out_e4m3), _ptr(out_scale), _stream(stream)))

@@ -40,6 +40,16 @@
  *   [W4A]   "DeepSeek-V4-Flash-0731-W4AFP8-mt" model card: 量化方式 and
  *           权重约定 (FP4 -> signed INT4, group 128, two INT4 per int8,
  *           float32 weight_scale_inv [N, K/128], dynamic E4M3 activations).
+ *   [PTPC]  "DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough: 核心参数 (FP8
+ *           E4M3 weights, per-channel static symmetric scales; activations
+ *           per-token dynamic symmetric; round half to even).
+ *
+ * Step labels used below
+ *   a1 activation quantisation    a2 routing          a3 grouping (permute)
+ *   a4 gate/up GEMM               a5 SwiGLU + requant a6 down GEMM
+ *   a7 weighted combine           a8 MXFP4 -> NVFP4   a9 MXFP4 -> INT4 g128
+ *   a10 W4AFP8 GEMM               f1 MXFP4 -> FP8 [128, 128] blocks
+ *   f3 FP8 block-scaled GEMM (shared expert)   f4 PTPC-FP8 expert path
  */
 #ifndef MOE_FP8_POW2_H
 #define MOE_FP8_POW2_H
@@ -63,6 +73,7 @@ extern "C" {
 #define MOE_EPI_STORE_F32 0    /* out: float32 [rows, N]                                   */
 #define MOE_EPI_STORE_BF16 1   /* out: bfloat16 [rows, N]                                  */
 #define MOE_EPI_SWIGLU_QUANT 2 /* out: E4M3 h [rows, N/2]; out_scale: E8M0 [rows, N/256] */
+#define MOE_EPI_SWIGLU_F32 3   /* out: float32 h [rows, N/2] (PTPC GEMM only)               */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_string(int status);
@@ -260,6 +271,53 @@ int moe_grouped_gemm_fp8_block128(const uint8_t* a_e4m3, const uint8_t* a_e8m0_1
                                   size_t workspace_bytes, void* stream);
 
 /*
+ * f4 -- PTPC-FP8 per-token activation quantisation [PTPC 核心参数: activations
+ * per-token, dynamic, symmetric, half_even].  Per row: amax = max |x|;
+ * scale = amax / 448 (float32 IEEE divide; 1.0 when amax == 0);
+ * q = E4M3(x / scale) with a float32 IEEE divide, nearest even, saturating
+ * at +-448.  x holding NaN or inf gives unspecified codes for that row.
+ *   x      bfloat16 (x_is_f32 == 0) or float32 [rows, cols], 16-byte aligned
+ *   q      uint8 E4M3 [rows, cols] (8-byte aligned);  scale float32 [rows]
+ *   cols % 8 == 0
+ */
+int moe_quantize_fp8_per_token(const void* x, int x_is_f32, int rows, int cols, uint8_t* q, float* scale,
+                               void* stream);
+
+/*
+ * f4 -- per-row scales of the grouped rows: dst[r] = src[perm[r] / k] for a
+ * routed row (perm[r] < T*k), src[perm[r] - T*k] for a shared-expert row,
+ * for r < offsets[E+1]; rows past it are untouched.  perm and offsets are the
+ * outputs of moe_permute; a perm entry outside [0, T*(k+1)) writes 0 and
+ * records MOE_ERR_INVALID.
+ *   perm int32 [T*(k+1)];  offsets int32 [E+2];  src float32 [T];
+ *   dst float32 [T*(k+1)]
+ */
+int moe_gather_row_scales(const int32_t* perm, int T, int k, const int32_t* offsets, int E, const float* src,
+                          float* dst, void* stream);
+
+/*
+ * f4 -- grouped GEMM in PTPC-FP8 [PTPC 核心参数]: E4M3 weights with one
+ * float32 scale per output channel, E4M3 activations with one float32 scale
+ * per row.  For every group g and row r in [offsets[g], offsets[g+1]):
+ *   acc[r, n] = (sum_k a[r, k] * w[g, n, k]) * a_scale[r] * w_scale[g, n]
+ * (the sum over all of K accumulated by the tensor cores in float32; then
+ * two float32 multiplies, a_scale first).
+ *   a_e4m3 uint8 [a_rows, K] (16-byte aligned);  a_scale float32 [a_rows]
+ *   w_e4m3 uint8 [G, N, K] (16-byte aligned);  w_scale float32 [G, N]
+ *   offsets as moe_grouped_gemm_mxfp4;  N % 128 == 0, K % 128 == 0
+ *   epilogue MOE_EPI_STORE_F32 / MOE_EPI_STORE_BF16: out = acc [a_rows, N];
+ *            MOE_EPI_SWIGLU_F32 (N % 256 == 0): columns [0, N/2) gate,
+ *            [N/2, N) up; out = float32 h [a_rows, N/2],
+ *            h = silu(clamp(g, +-limit)) * clamp(u, +-limit)
+ *   block_n token rows per tile: 16, 32, 64 or 128 (0 = choose)
+ *   workspace moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
+ */
+int moe_grouped_gemm_fp8_ptpc(const uint8_t* a_e4m3, const float* a_scale, int a_rows, const int32_t* offsets,
+                              int n_groups, const uint8_t* w_e4m3, const float* w_scale, int N, int K, int epilogue,
+                              float swiglu_limit, int block_n, void* out, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * a5 standalone -- SwiGLU with clamp and per-128 power-of-two requantisation
  * [SI 架构特性 / 低精度计算], same arithmetic as MOE_EPI_SWIGLU_QUANT.
  *   gu  float32 [rows, 2I] (gate | up), 16-byte aligned; I % 128 == 0
@@ -324,6 +382,21 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
  */
 int repack_mxfp4_to_fp8_block128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
                                  uint8_t* out_e4m3, float* out_scale_inv, void* stream);
+
+/*
+ * f4 -- MXFP4 -> PTPC-FP8 weights [PTPC 核心参数: weights FP8 E4M3,
+ * per-channel, static, symmetric, half_even].  Per output channel (row of
+ * K elements): w = exact float32 dequantisation; amax; scale = amax / 448
+ * (float32 IEEE divide; 1.0 when amax == 0); out = E4M3(w / scale), float32
+ * IEEE divide, nearest even (|w / scale| <= 448 by construction).
+ * Device errors: MOE_ERR_NAN_SCALE (row not written), MOE_ERR_RANGE (w
+ * overflows float32; row not written).
+ *   fp4 uint8 [n_mats, N, K/2] (4-byte aligned); e8m0 [n_mats, N, K/32];
+ *   out_e4m3 uint8 [n_mats, N, K] (8-byte aligned); out_scale float32
+ *   [n_mats, N];  K % 32 == 0
+ */
+int repack_mxfp4_to_fp8_per_channel(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats, int N, int K,
+                                    uint8_t* out_e4m3, float* out_scale, void* stream);
 
 #ifdef __cplusplus
 }

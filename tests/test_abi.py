@@ -57,3 +57,19 @@ def test_argument_validation_without_gpu():
     assert lib.moe_prepared_weights_size(3, 256, 512) == 3 * 2 * 4 * 8704
     assert lib.repack_mxfp4_to_int4g128(None, None, 1, 8, 96, None, None, None) == -1
     assert lib.repack_mxfp4_to_fp8_block128(None, None, 1, 100, 128, None, None, None) == -1   # N % 128
+    # PTPC-FP8 entry points
+    assert lib.moe_quantize_fp8_per_token(None, 0, 4, 100, None, None, None) == -1     # cols % 8
+    assert lib.moe_quantize_fp8_per_token(None, 1, 0, 128, None, None, None) == 0      # empty: no-op
+    assert lib.repack_mxfp4_to_fp8_per_channel(None, None, 1, 8, 48, None, None, None) == -1   # K % 32
+    assert lib.moe_gather_row_scales(None, 0, 6, None, 8, None, None, None) == 0       # no rows
+    assert lib.moe_grouped_gemm_fp8_ptpc(None, None, 4, None, 2, None, None, 256, 128, 2,
+                                         ctypes.c_float(10), 16, None, None, 0, None) == -1   # pow2 epilogue
+    assert lib.moe_grouped_gemm_fp8_ptpc(None, None, 4, None, 2, None, None, 384, 128, 3,
+                                         ctypes.c_float(10), 16, None, None, 0, None) == -1   # N % 256
+    assert lib.moe_grouped_gemm_fp8_ptpc(None, None, 4, None, 2, None, None, 256, 128, 3,
+                                         ctypes.c_float(10), 48, None, None, 0, None) == -2   # block_n 48
+    assert lib.moe_grouped_gemm_fp8_ptpc(None, None, 4, None, 2, None, None, 256, 128, 3,
+                                         ctypes.c_float(10), 128, None, None, 0, None) == -1  # null pointers
+    # the block-scaled GEMMs take no float32 SwiGLU epilogue
+    assert lib.moe_grouped_gemm_fp8_block128(None, None, 4, None, 2, None, None, 256, 128, 3,
+                                             ctypes.c_float(10), 16, None, None, None, 0, None) == -1

@@ -547,3 +547,201 @@ def test_fp8_block_gemm_group_view(lib):
     np.testing.assert_array_equal(got[r0:r1], ref.astype(np.float32))
     assert (got[:r0] == -1.0).all() and (got[r1:] == -1.0).all()
     no_device_error(lib)
+
+
+# --------------------------- PTPC-FP8 (f4) --------------------------------
+def _ptpc_quant(lib, x, is_bf16):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(max(rows, 1), dtype=torch.float32, device="cuda")
+    lib.moe_quantize_fp8_per_token(dev(x.view(np.int16) if is_bf16 else x), q, sc)
+    return host(q), host(sc)[:rows]
+
+
+@pytest.mark.parametrize("T,H", [(1, 128), (37, 520), (300, 4096)])
+def test_ptpc_quant_bf16_bit_exact(lib, T, H):
+    x = synth.decode_activations(30 + T, T, H)
+    x[0, :] = 0                                           # a zero row: scale 1
+    q, sc = _ptpc_quant(lib, x, True)
+    q_ref, s_ref = ffn.quantize_fp8_per_row(F.decode_bf16_bits(x))
+    np.testing.assert_array_equal(sc.view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q, q_ref)
+    no_device_error(lib)
+
+
+def test_ptpc_quant_every_bf16(lib):
+    """Every finite bf16 value against a row maximum that varies by row, so
+    each value meets many scales (the IEEE divide and E4M3 rounding, the
+    E4M3 subnormals and the flush to zero all exercised)."""
+    b = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    b = b[np.isfinite(F.decode_bf16_bits(b))]
+    x = np.zeros((len(b), 8), np.uint16)
+    x[:, 1] = b
+    amax = np.abs(F.decode_bf16_bits(b)).astype(np.float64) * np.exp2((np.arange(len(b)) % 23) - 3) * 1.3
+    x[:, 6] = synth.to_bf16_bits(np.clip(np.where(amax > 0, amax, 1.0), 0.0, 3.0e38))
+    q, sc = _ptpc_quant(lib, x, True)
+    q_ref, s_ref = ffn.quantize_fp8_per_row(F.decode_bf16_bits(x))
+    np.testing.assert_array_equal(sc.view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q, q_ref)
+
+
+def test_ptpc_quant_f32_wide_range(lib):
+    """float32 rows spanning 2^-140 .. 2^100 (subnormal scales included)."""
+    rows, cols = 64, 1024
+    x = synth.normal(31, 1, rows * cols).astype(np.float64).reshape(rows, cols)
+    x *= np.exp2(np.linspace(-140, 100, rows))[:, None]
+    x = x.astype(np.float32)
+    x[5] = 0.0
+    x[6] = -0.0
+    q, sc = _ptpc_quant(lib, x, False)
+    q_ref, s_ref = ffn.quantize_fp8_per_row(x)
+    np.testing.assert_array_equal(sc.view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q, q_ref)
+
+
+def _ptpc_cast(lib, fp4, e8):
+    M, N, k2 = fp4.shape
+    q = torch.full((M, N, 2 * k2), 0x11, dtype=torch.uint8, device="cuda")
+    s = torch.full((M, N), -1.0, dtype=torch.float32, device="cuda")
+    lib.repack_mxfp4_to_fp8_per_channel(dev(fp4), dev(e8), q, s)
+    return host(q), host(s)
+
+
+@pytest.mark.parametrize("N,K,lo,hi", [(256, 512, 110, 140), (48, 7168, 60, 200), (5, 96, 0, 20)])
+def test_ptpc_weight_cast_bit_exact(lib, N, K, lo, hi):
+    """Per-channel codes and scales equal the oracle's bit for bit, from
+    exponent spreads that keep every code normal to ones that push small
+    elements into E4M3 subnormals and zero (and float32 subnormal weights)."""
+    fp4 = synth.random_bytes(32, 1, (2, N, K // 2))
+    e8 = synth.random_bytes(32, 2, (2, N, K // 32), lo, hi)
+    q, s = _ptpc_cast(lib, fp4, e8)
+    q_ref, s_ref = ffn.ptpc_weights(fp4, e8)
+    np.testing.assert_array_equal(s.view(np.uint32), s_ref.view(np.uint32))
+    np.testing.assert_array_equal(q, q_ref)
+    no_device_error(lib)
+
+
+def test_ptpc_weight_cast_edges(lib):
+    """An all-zero channel with negative zeros (scale 1, codes 0x00 / 0x80); a
+    channel whose values overflow float32 (MOE_ERR_RANGE, not written); an
+    E8M0 NaN (MOE_ERR_NAN_SCALE, not written)."""
+    N, K = 4, 64
+    codes = synth.random_bytes(33, 1, (N, K), 0, 15)
+    codes[0, :] = 0
+    codes[0, 1::3] = 8
+    fp4 = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)[None]
+    e8 = np.full((1, N, K // 32), 127, np.uint8)
+    q, s = _ptpc_cast(lib, fp4, e8)
+    q_ref, s_ref = ffn.ptpc_weights(fp4, e8)
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(s, s_ref)
+    assert s[0, 0] == 1.0 and set(np.unique(q[0, 0])) <= {0x00, 0x80}
+    no_device_error(lib)
+    codes[2, 5] = 7                                       # 6 * 2^127 overflows float32
+    fp4 = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)[None]
+    e8[0, 2, 0] = 254
+    q, s = _ptpc_cast(lib, fp4, e8)
+    assert lib.moe_get_device_error() == -4
+    assert s[0, 2] == -1.0 and (q[0, 2] == 0x11).all()
+    np.testing.assert_array_equal(q[0, 3], q_ref[0, 3])
+    e8[0, 2, 0] = 127
+    e8[0, 1, 1] = 255
+    q, s = _ptpc_cast(lib, fp4, e8)
+    assert lib.moe_get_device_error() == -3
+    assert s[0, 1] == -1.0 and (q[0, 1] == 0x11).all()
+
+
+def test_gather_row_scales(lib):
+    T, E, k = 40, 9, 3
+    idx = (synth.splitmix64(34, 1, T * k) % np.uint64(E)).astype(np.int32).reshape(T, k)
+    counts, offsets, perm, inv, src = Pm.permute(idx, E, 1)
+    sx = (synth.uniform(34, 2, T) + 0.5).astype(np.float32)
+    dst = torch.full((T * (k + 1),), -1.0, dtype=torch.float32, device="cuda")
+    lib.moe_gather_row_scales(dev(perm.astype(np.int32)), T, k, dev(offsets.astype(np.int32)), E, dev(sx), dst)
+    np.testing.assert_array_equal(host(dst), sx[src])
+    no_device_error(lib)
+    bad = perm.astype(np.int32).copy()
+    bad[7] = T * (k + 1)
+    lib.moe_gather_row_scales(dev(bad), T, k, dev(offsets.astype(np.int32)), E, dev(sx), dst)
+    assert lib.moe_get_device_error() == -1
+    assert host(dst)[7] == 0.0
+
+
+def _ptpc_inputs(seed, sizes, N, K, integer):
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Rn, G = int(offsets[-1]), len(sizes)
+    if integer:
+        a = synth.small_int_e4m3(seed, 1, (Rn, K))
+        q = synth.small_int_e4m3(seed, 2, (G, N, K))
+        # power-of-two scales keep the epilogue multiplies exact
+        sa = np.exp2((synth.splitmix64(seed, 3, Rn) % np.uint64(7)).astype(np.float64) - 3).astype(np.float32)
+        sw = np.exp2((synth.splitmix64(seed, 4, G * N) % np.uint64(5)).astype(np.float64) - 2)
+        sw = sw.astype(np.float32).reshape(G, N)
+    else:
+        a = synth.random_e4m3(seed, 1, (Rn, K))
+        q = synth.random_e4m3(seed, 2, (G, N, K))
+        sa = (synth.uniform(seed, 3, Rn) * 0.01 + 1e-4).astype(np.float32)
+        sw = (synth.uniform(seed, 4, G * N) * 0.01 + 1e-4).astype(np.float32).reshape(G, N)
+    return a, sa, offsets, q, sw
+
+
+def _run_ptpc(lib, a, sa, offsets, q, sw, epi, block_n):
+    G, N, K = q.shape
+    Rn = a.shape[0]
+    ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
+    cols = N // 2 if epi == lib.MOE_EPI_SWIGLU_F32 else N
+    out = torch.full((Rn, cols), -7.0, dtype=torch.float32, device="cuda")
+    lib.moe_grouped_gemm_fp8_ptpc(dev(a), dev(sa), dev(offsets), dev(q), dev(sw), epi, out, ws, 10.0, block_n)
+    return host(out)
+
+
+@pytest.mark.parametrize("block_n", [16, 32, 64, 128])
+def test_ptpc_gemm_integer_exact(lib, block_n):
+    a, sa, offsets, q, sw = _ptpc_inputs(35, GROUPS, 256, 512, True)
+    out = _run_ptpc(lib, a, sa, offsets, q, sw, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_ptpc(a, sa, offsets, q, sw)
+    np.testing.assert_array_equal(out, ref.astype(np.float32))
+    no_device_error(lib)
+
+
+def _ptpc_bound(a, sa, offsets, q, sw):
+    av = F.decode_e4m3(a) * sa.astype(np.float64)[:, None]
+    bound = np.zeros((a.shape[0], q.shape[1]))
+    for g in range(len(offsets) - 1):
+        r0, r1 = offsets[g], offsets[g + 1]
+        if r1 > r0:
+            bound[r0:r1] = np.abs(av[r0:r1]) @ np.abs(F.decode_e4m3(q[g]) * sw[g].astype(np.float64)[:, None]).T
+    return bound
+
+
+@pytest.mark.parametrize("block_n", [16, 64, 128])
+def test_ptpc_gemm_random(lib, block_n):
+    """float32 tensor-core sums over K and two epilogue multiplies: within
+    1024 float32 ulps of sum |a||w|."""
+    a, sa, offsets, q, sw = _ptpc_inputs(36, [3, 0, 40, 130, 1], 384, 1024, False)
+    out = _run_ptpc(lib, a, sa, offsets, q, sw, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_ptpc(a, sa, offsets, q, sw)
+    bound = _ptpc_bound(a, sa, offsets, q, sw)
+    assert (np.abs(out.astype(np.float64) - ref) <= 1024 * 2.0 ** -24 * bound + 1e-30).all()
+
+
+@pytest.mark.parametrize("block_n", [16, 32, 64, 128])
+def test_ptpc_gemm_swiglu_f32(lib, block_n):
+    """The float32 SwiGLU epilogue equals the clamp and silu of the same
+    kernel's float32 gate/up sums within the silu bound (24 ulp of |h|), and
+    the oracle's h within the GEMM bound carried through the clamp."""
+    I = 256
+    a, sa, offsets, q, sw = _ptpc_inputs(37, [5, 0, 33, 70], 2 * I, 512, False)
+    sa *= 0.4
+    gu = _run_ptpc(lib, a, sa, offsets, q, sw, lib.MOE_EPI_STORE_F32, block_n)
+    h = _run_ptpc(lib, a, sa, offsets, q, sw, lib.MOE_EPI_SWIGLU_F32, block_n)
+    h_same = ffn.swiglu_clamp(gu, I)
+    assert (np.abs(h - h_same) <= 24 * np.spacing(np.abs(h_same).astype(np.float32)).astype(np.float64)
+            + 1e-37).all()
+    assert np.abs(gu).max() < 30 and (np.abs(gu) > 10).any()       # the clamp is reached
+    ref = ffn.swiglu_clamp(ffn.grouped_gemm_ptpc(a, sa, offsets, q, sw), I)
+    bound = _ptpc_bound(a, sa, offsets, q, sw)
+    # |d h| <= (|silu'| <= 1.1) * 10 * |d g| + 10 * |d u| + silu rounding
+    tol = 1024 * 2.0 ** -24 * (11 * bound[:, :I] + 10 * bound[:, I:]) + 32 * np.spacing(np.abs(ref).astype(np.float32))
+    assert (np.abs(h - ref) <= tol).all()
+    no_device_error(lib)

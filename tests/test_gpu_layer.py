@@ -211,3 +211,59 @@ def test_decode_layer_shared_fp8_full_size(lib):
     ref = _shared_fp8_ref(x, logits, w13, s13, w2, s2, k, tokens=toks)
     check_y(y.float().cpu().numpy()[toks], ref["y"])
     assert lib.moe_get_device_error() == 0
+
+
+class _ProtoWeights:
+    """[G, ...] view whose entry g is prototype g % n_proto of a smaller array
+    (the synthetic weights repeat n_proto experts), so the oracle repacks only
+    the prototypes."""
+
+    def __init__(self, protos, G):
+        self.protos, self.shape = protos, (G,) + protos.shape[1:]
+
+    def __getitem__(self, g):
+        return self.protos[g % len(self.protos)]
+
+
+def _ptpc_ref(x, logits, w13, s13, w2, s2, k, tokens=None, n_proto=None):
+    """Oracle PTPC-FP8 layer: the oracle's per-channel cast of the experts,
+    then its FFN with per-token activations."""
+    G = w13.shape[0]
+    n = G if n_proto is None else n_proto
+    q13, i13 = ffn.ptpc_weights(w13[:n], s13[:n])
+    q2, i2 = ffn.ptpc_weights(w2[:n], s2[:n])
+    return ffn.moe_layer_ptpc(x, logits, _ProtoWeights(q13, G), _ProtoWeights(i13, G), _ProtoWeights(q2, G),
+                              _ProtoWeights(i2, G), k, tokens=tokens)
+
+
+@pytest.mark.parametrize("block_n", [0, 16, 128])
+def test_tiny_layer_ptpc(lib, block_n):
+    """PTPC-FP8: experts cast per channel on the GPU, activations quantised
+    per token; the per-token quantisation of x is bit-exact."""
+    wl = synth.tiny_layer(6)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk, weights="ptpc")
+    buf = layer.alloc(wl.T, block_n)
+    y = layer.forward(torch.from_numpy(wl.x_bf16.view(np.int16)).cuda(), torch.from_numpy(wl.logits).cuda(), buf)
+    ref = _ptpc_ref(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(buf.xq.cpu().numpy(), ref["xq"])
+    np.testing.assert_array_equal(buf.sxf.cpu().numpy().view(np.uint32), ref["sx"].view(np.uint32))
+    np.testing.assert_array_equal(buf.idx.cpu().numpy(), ref["idx"])
+    check_y(y.float().cpu().numpy(), ref["y"])
+    assert lib.moe_get_device_error() == 0
+
+
+def test_decode_layer_ptpc_full_size(lib):
+    """Decode configuration (64 tokens, hidden 4096, intermediate 2048, 256 + 1
+    experts, top-6) in PTPC-FP8; sampled tokens against the oracle."""
+    T, H, I, E, k = 64, 4096, 2048, 256, 6
+    w13, s13, w2, s2 = synth.expert_weights(0, E + 1, H, I, n_proto=2)
+    x = synth.decode_activations(0, T, H)
+    logits = synth.uniform_logits(0, T, E)
+    layer = MoeLayer(w13, s13, w2, s2, k, weights="ptpc")
+    buf = layer.alloc(T)
+    y = layer.forward(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(logits).cuda(), buf)
+    toks = np.sort((synth.splitmix64(0, 80, 8) % np.uint64(T)).astype(np.int64))
+    ref = _ptpc_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
+    check_y(y.float().cpu().numpy()[toks], ref["y"])
+    assert lib.moe_get_device_error() == 0

@@ -208,3 +208,19 @@ def test_ptpc_layer_token_subset():
     toks = np.array([1, 4, 9])
     sub = ffn.moe_layer_ptpc(wl.x_bf16, wl.logits, q13, s13, q2, s2, wl.topk, tokens=toks)
     np.testing.assert_allclose(sub["y"], full["y"][toks], rtol=0, atol=1e-12 * np.abs(full["y"]).max())
+
+
+def test_ptpc_weights_per_output_channel():
+    """The weight scale is per output channel (row of [N, K]): rows with very
+    different magnitudes each reach code 448 and dequantise within the E4M3
+    bound of their own scale; the scale is amax/448 of the exact MXFP4 values."""
+    N, K = 6, 64
+    fp4 = synth.random_bytes(24, 1, (1, N, K // 2))
+    e8 = np.repeat((np.arange(N, dtype=np.uint8) * 9 + 100)[:, None], K // 32, axis=1)[None]
+    q, s = ffn.ptpc_weights(fp4, e8)
+    w = ffn.dequant_mxfp4(fp4, e8)[0]
+    amax = np.abs(w).max(axis=1)
+    np.testing.assert_array_equal(s[0], (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32))
+    assert (np.abs(F.decode_e4m3(q[0])).max(axis=1) == 448.0).all()
+    back = F.decode_e4m3(q[0]) * s[0][:, None].astype(np.float64)
+    assert (np.abs(back - w) <= np.maximum(2.0 ** -4 * np.abs(w), 2.0 ** -10 * s[0][:, None])).all()
