@@ -74,15 +74,19 @@ struct Cfg {
   static_assert(BN <= 128, "register accumulators: BN <= 128");
 };
 
-// Eight INT4 (two's complement nibbles, element 0 in the low nibble) ->
-// eight E4M3 bytes, by byte-permute table lookups.
-__device__ __forceinline__ uint32_t int4x4_to_e4m3x4(uint32_t h) {
+// Four INT4 (two's complement nibbles, element 0 in the low nibble) from
+// bit s of w -> four E4M3 bytes, by byte-permute table lookups.  A byte
+// permute reads the low 3 bits of each selector nibble of the low 16 bits.
+__device__ __forceinline__ uint32_t int4x4_to_e4m3x4(uint32_t w, int s) {
   // codes of 0..7 and of -8..-1
   const uint32_t P0 = 0x44403800u, P1 = 0x4E4C4A48u;
   const uint32_t N0 = 0xCACCCED0u, N1 = 0xB8C0C4C8u;
+  const uint32_t h = w >> s;
   const uint32_t pos = __byte_perm(P0, P1, h);
   const uint32_t neg = __byte_perm(N0, N1, h);
-  const uint32_t mask = __byte_perm(0x0000FF00u, 0u, (h >> 3) & 0x1111u);
+  // selector nibble i of h >> 3 is odd exactly when element i is negative
+  // (its sign bit, plus higher bits times 2): odd table bytes are 0xFF
+  const uint32_t mask = __byte_perm(0xFF00FF00u, 0xFF00FF00u, h >> 3);
   return (pos & ~mask) | (neg & mask);
 }
 
@@ -254,14 +258,14 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
             const int r = w * 8 + (lane >> 2) + 8 * C::CONV_WARPS * j;
             const uint4 in = *reinterpret_cast<const uint4*>(raw + r * 64 + chunk * 16);
             uint4 o0, o1;
-            o0.x = int4x4_to_e4m3x4(in.x & 0xFFFFu);
-            o0.y = int4x4_to_e4m3x4(in.x >> 16);
-            o0.z = int4x4_to_e4m3x4(in.y & 0xFFFFu);
-            o0.w = int4x4_to_e4m3x4(in.y >> 16);
-            o1.x = int4x4_to_e4m3x4(in.z & 0xFFFFu);
-            o1.y = int4x4_to_e4m3x4(in.z >> 16);
-            o1.z = int4x4_to_e4m3x4(in.w & 0xFFFFu);
-            o1.w = int4x4_to_e4m3x4(in.w >> 16);
+            o0.x = int4x4_to_e4m3x4(in.x, 0);
+            o0.y = int4x4_to_e4m3x4(in.x, 16);
+            o0.z = int4x4_to_e4m3x4(in.y, 0);
+            o0.w = int4x4_to_e4m3x4(in.y, 16);
+            o1.x = int4x4_to_e4m3x4(in.z, 0);
+            o1.y = int4x4_to_e4m3x4(in.z, 16);
+            o1.z = int4x4_to_e4m3x4(in.w, 0);
+            o1.w = int4x4_to_e4m3x4(in.w, 16);
             const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
             *reinterpret_cast<uint4*>(dst + r * 128 + ((c0 ^ (r & 7)) << 4)) = o0;
             *reinterpret_cast<uint4*>(dst + r * 128 + ((c1 ^ (r & 7)) << 4)) = o1;
