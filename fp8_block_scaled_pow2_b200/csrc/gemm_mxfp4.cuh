@@ -28,7 +28,8 @@
 //                 copies)
 //   warp 1        TMEM owner and MMA issuer 0: scale factors shared -> TMEM
 //                 (tcgen05.cp), 4 MMAs of K = 32 per 128-wide K step
-//   warp 10       MMA issuer 1 (narrow token tiles, see Cfg::ISSUERS)
+//   warp 10       MMA issuer 1 (tile 1 of a pair, or alternate K steps of a
+//                 single tile; see Cfg::ISSUERS)
 //   warps 2..9    epilogue: TMEM -> registers -> global (float32 / bf16 /
 //                 SwiGLU + per-128 FP8 requantisation)
 // The producer and issuer loops run converged on their whole warp and one
@@ -85,18 +86,16 @@ struct Cfg {
   // transaction bytes of a step (the TMA counts the packed weight bytes);
   // steps that also load token scales add NA * 512
   static constexpr int TX = NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;
-  // MMA issue: one warp issuing small-N MMAs is bound by its own issue
-  // latency, so narrow tiles use two issuing warps.  With a tile pair issuer
-  // 0 computes tile 0 and issuer 1 tile 1; with one tile they take alternate
-  // K steps into two partial accumulators the epilogue adds.  Wide pairs keep
-  // one issuer (its two MMAs per K block share the token operand back to
-  // back).
+  // MMA issue: one warp issuing block-scaled MMAs is bound by its own issue
+  // latency (about 60 cycles per instruction, the tensor work of N = 128),
+  // so two warps issue.  With a tile pair issuer 0 computes tile 0 and
+  // issuer 1 tile 1; with one tile they take alternate K steps into two
+  // partial accumulators the epilogue adds.
   // tensor-memory columns: ACC_BUFS accumulators of 2 * BN columns, then one
   // scale set (weight + token scales) per issuer
-  static constexpr int ISSUERS = (PAIR && BN >= 64) ? 1 : 2;
-  static constexpr int TILES_PER_ISSUER = (PAIR && ISSUERS == 1) ? 2 : 1;
+  static constexpr int ISSUERS = 2;
   static constexpr int ACC_COLS = 2 * BN;
-  static constexpr int SF_SET = 4 * TILES_PER_ISSUER + 4 * NA;
+  static constexpr int SF_SET = 4 + 4 * NA;
   static constexpr int SF_COLS = 2 * SF_SET;
   static constexpr int ACC_BUFS = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
   static constexpr int SF_COL = ACC_BUFS * ACC_COLS;      // issuer i: SF_COL + i * SF_SET
@@ -421,7 +420,7 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
   using C = Cfg<BN, PAIR>;
   const uint32_t ring0 = smem_u32(smem);
   const uint32_t sfa_t = tmem + C::SF_COL + iss * C::SF_SET;     // 4 columns per weight tile
-  const uint32_t sfb_t = sfa_t + 4 * C::TILES_PER_ISSUER;
+  const uint32_t sfb_t = sfa_t + 4;
   uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const Item it = decode_item(item, plan, args.G, n_ft, BN);
@@ -434,7 +433,7 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
     tc_fence_after();
     const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
     for (int kt = 0; kt < KT; ++kt) {
-      const bool mine = PAIR || C::ISSUERS == 1 || (kt & 1) == iss;
+      const bool mine = PAIR || (kt & 1) == iss;
       if (mine) {
         if (!mbar_wait_warp(&full[stage], phase, abort_flag)) return;
         const uint32_t st = ring0 + stage * C::STAGE;
@@ -444,11 +443,10 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
         const uint64_t da = sdesc_kmajor_sw128(a_base);
         const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
         // this issuer's first step of the item starts a fresh accumulator
-        const uint32_t first = (PAIR || C::ISSUERS == 1) ? (kt != 0) : (kt > 1);
+        const uint32_t first = PAIR ? (kt != 0) : (kt > 1);
         if (elect_one()) {
           tmem_cp_32x128b_warpx4(sfa_t, sdesc_sf(st + C::SFA_OFF + (PAIR ? iss * C::SF_BYTES : 0)));
-          if (C::TILES_PER_ISSUER == 2) tmem_cp_32x128b_warpx4(sfa_t + 4, sdesc_sf(st + C::SFA_OFF + C::SF_BYTES));
-          if ((kt & 3) == (PAIR || C::ISSUERS == 1 ? 0 : iss)) {
+          if ((kt & 3) == (PAIR ? 0 : iss)) {
 #pragma unroll
             for (int a = 0; a < C::NA; ++a) tmem_cp_32x128b_warpx4(sfb_t + 4 * a, sdesc_sf(st + C::SFB_OFF + 512 * a));
           }
@@ -456,9 +454,6 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
           for (int kb = 0; kb < 4; ++kb) {
             mma_mxf8f6f4(d, da + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4), sfa_t | ((uint32_t)kb << 30), sfb,
                          kb ? 1u : first);
-            if (C::TILES_PER_ISSUER == 2)
-              mma_mxf8f6f4(d + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, id_kb[kb] | (bsel << 4),
-                           (sfa_t + 4) | ((uint32_t)kb << 30), sfb, kb ? 1u : first);
           }
           tc_commit(&empty[stage]);
         }
@@ -552,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + stage * C::STAGE;
           // token scales: one block per 4 K steps, read by each issuer at its
           // first step of the group (issuers alternate steps without PAIR)
-          const bool new_group = (PAIR || C::ISSUERS == 1) ? (kt & 3) == 0 : (kt & 3) < 2;
+          const bool new_group = PAIR ? (kt & 3) == 0 : (kt & 3) < 2;
           mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
 #pragma unroll
           for (int a = 0; a < C::NUM_A; ++a) {
@@ -574,9 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                          n_items, KT, n_ft);
   } else if (warp == kThreads / 32 - 1) {
     // ------------------------------ MMA issuer 1 ---------------------------
-    if (C::ISSUERS == 2)
-      mma_issuer<BN, PAIR>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan,
-                           args, n_items, KT, n_ft);
+    mma_issuer<BN, PAIR>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
+                         n_items, KT, n_ft);
   } else {
     // ------------------------------ epilogue ------------------------------
     const int e = warp - C::EPI_FIRST;

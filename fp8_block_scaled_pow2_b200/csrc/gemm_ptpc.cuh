@@ -13,8 +13,11 @@
 // channels) x BN token rows; with DUAL (the SwiGLU epilogue) a tile holds the
 // gate rows [ft*128, ft*128+128) and the matching up rows N/2 further, so
 // one accumulator pair gives both halves of h for 128 channels.
-// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..9 epilogue (two warps
-// per tensor-memory lane quadrant, each on half of the token columns).
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (gate, or the only tile),
+// 2..9 epilogue (two warps per tensor-memory lane quadrant, each on half of
+// the token columns), 10 MMA issuer of the up tile (DUAL): one warp issuing
+// MMAs is bound by its own issue latency, so the two tiles of a pair are
+// issued from two warps.
 // Tensor memory holds two accumulators (the epilogue of one tile overlaps the
 // main loop of the next).
 #pragma once
@@ -29,7 +32,7 @@ using gemm::Item;
 using gemm::decode_item;
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+constexpr int kThreads = (3 + kEpiWarps) * 32;
 
 __host__ __device__ constexpr int tmem_cols_for(int used) {
   return used <= 32 ? 32 : used <= 64 ? 64 : used <= 128 ? 128 : used <= 256 ? 256 : 512;
@@ -99,10 +102,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], C::NUM_A);            // one commit per issuer
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], C::NUM_A);
       mbar_init(&acc_empty[b], 32 * kEpiWarps);
     }
     *abort_flag = 0;
@@ -141,41 +144,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ----------------------------
-    const uint32_t ring0 = smem_u32(smem);
-    uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = decode_item(item, plan, G, n_ft, BN);
-      const int n_mma = max(16, (it.rows + 15) & ~15);
-      const uint32_t idesc = idesc_f8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
-      if (!mbar_wait_warp(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) break;
-      tc_fence_after();
-      const uint32_t d = tmem + ab * C::ACC_COLS;
-      bool ok = true;
-      for (int kt = 0; kt < KT; ++kt) {
-        if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
+  } else if (warp == 1 || warp == kThreads / 32 - 1) {
+    // ------------------------------ MMA issuers ---------------------------
+    // issuer 0 (warp 1): tile 0; issuer 1 (last warp): tile 1 of a pair
+    const int iss = warp == 1 ? 0 : 1;
+    if (iss < C::NUM_A) {
+      const uint32_t ring0 = smem_u32(smem);
+      uint32_t stage = 0, phase = 0, ab = 0, acc_bits = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const Item it = decode_item(item, plan, G, n_ft, BN);
+        const int n_mma = max(16, (it.rows + 15) & ~15);
+        const uint32_t idesc = idesc_f8f6f4(0u /*E4M3*/, 0u /*E4M3*/, 128, n_mma);
+        if (!mbar_wait_warp(&acc_empty[ab], ((acc_bits >> ab) & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
-        const uint32_t st = ring0 + stage * C::STAGE;
-        const uint64_t da = sdesc_kmajor_sw128(st);
-        const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
-        if (elect_one()) {
+        const uint32_t d = tmem + ab * C::ACC_COLS + iss * BN;
+        bool ok = true;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = ring0 + stage * C::STAGE;
+          const uint64_t da = sdesc_kmajor_sw128(st + iss * C::A_BYTES);
+          const uint64_t db = sdesc_kmajor_sw128(st + C::B_OFF);
+          if (elect_one()) {
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint32_t accumulate = (kt > 0 || kb > 0) ? 1u : 0u;
-            mma_f8f6f4(d, da + 2 * kb, db + 2 * kb, idesc, accumulate);
-            if (DUAL) mma_f8f6f4(d + BN, da + (C::A_BYTES >> 4) + 2 * kb, db + 2 * kb, idesc, accumulate);
+            for (int kb = 0; kb < 4; ++kb)
+              mma_f8f6f4(d, da + 2 * kb, db + 2 * kb, idesc, (kt > 0 || kb > 0) ? 1u : 0u);
+            tc_commit(&empty[stage]);
           }
-          tc_commit(&empty[stage]);
+          __syncwarp();
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (!ok) break;
+        if (elect_one()) tc_commit(&acc_full[ab]);
         __syncwarp();
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        acc_bits ^= 1u << ab;
+        ab ^= 1u;
       }
-      if (!ok) break;
-      if (elect_one()) tc_commit(&acc_full[ab]);
-      __syncwarp();
-      acc_bits ^= 1u << ab;
-      ab ^= 1u;
     }
   } else {
     // ------------------------------ epilogue ------------------------------
