@@ -230,15 +230,26 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
         # the shared expert streams E4M3 bytes and float32 [128, 128] block scales instead
         w13_bytes += 2 * I * H + 4 * (2 * I // 128) * (H // 128) - w13
         w2_bytes += H * I + 4 * (H // 128) * (I // 128) - w2
-    if getattr(layer, "weights", "mxfp4") == "ptpc":
+    T, E, k = wl["T"], wl["E"], wl["k"]
+    ptpc = getattr(layer, "weights", "mxfp4") == "ptpc"
+    # quantise (bf16 in, E4M3 + scales out), route (logits in, ids + weights
+    # out), group (ids in, perm + inv out, rows and scales gathered), plus the
+    # row-scale gather of PTPC; combine (k routed rows + the shared row in,
+    # bf16 out, ids + weights in)
+    quant = T * H * 2 + T * H + (4 * T if ptpc else T * H // 128)
+    route = T * E * 4 + T * k * 8
+    group = T * k * 4 + R * 4 + T * k * 4 + 2 * R * (H + H // 128)
+    pre = quant + route + group + (3 * 4 * R if ptpc else 0)
+    post = R * H * 4 + T * k * 8 + T * H * 2
+    if ptpc:
         # E4M3 weights with one float32 scale per channel; activations E4M3
         # with one float32 scale per row (the float32 h round trip between
         # the GEMM and its per-token requantisation is not counted)
-        return dict(active_experts=active, rows=R,
+        return dict(active_experts=active, rows=R, pre=pre, post=post,
                     w13=active * (2 * I * H + 4 * 2 * I) + R * (H + 4) + R * (I + 4),
                     w2=active * (H * I + 4 * H) + R * (I + 4) + R * H * 4,
                     flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
-    return dict(active_experts=active, rows=R,
+    return dict(active_experts=active, rows=R, pre=pre, post=post,
                 w13=w13_bytes + R * (H + H // 128) + R * (I + I // 128),
                 w2=w2_bytes + R * (I + I // 128) + R * H * 4,
                 flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
@@ -375,10 +386,13 @@ def run_ours(args, wl):
         runners = list(segs)
 
     def step(ev=None):
+        # events: before pre, w1/w3, w2 and combine, and after combine
         for i, run in enumerate(runners):
-            if ev and i > 0:
-                ev[i - 1].record(stream)
+            if ev:
+                ev[i].record(stream)
             run()
+        if ev:
+            ev[len(runners)].record(stream)
 
     clk = ClockSampler(local).start()
     for _ in range(args.warmup):
@@ -387,7 +401,7 @@ def run_ours(args, wl):
     assert moe.moe_get_device_error() == 0
     ab = algorithmic_bytes(layer, buf, wl)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg)
     torch.cuda.synchronize()
@@ -402,8 +416,10 @@ def run_ours(args, wl):
     barrier(pg)
     ms = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms, pg)
-    g13 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    g2 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    g13 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    g2 = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    post_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
 
     # end to end through the public API with host buffers: pinned x / logits
     # in, y out, copies inside the timed region
@@ -472,6 +488,10 @@ def run_ours(args, wl):
                  "w13_TFLOPs": round(ab["flops13"] / (g13 / 1e3) / 1e12, 2),
                  "w2_TFLOPs": round(ab["flops2"] / (g2 / 1e3) / 1e12, 2),
                  "active_experts": ab["active_experts"], "rows": ab["rows"]},
+        "segments": {"pre_ms": round(pre_ms, 4), "pre_GBps": round(ab["pre"] / (pre_ms / 1e3) / 1e9, 1),
+                     "post_ms": round(post_ms, 4), "post_GBps": round(ab["post"] / (post_ms / 1e3) / 1e9, 1),
+                     "pre": "quantise + route + group (+ row-scale gather)", "post": "combine",
+                     "bytes": "algorithmic: each input read once, each output written once"},
         "e2e": {"value": round(tokens / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xh.numel() * 2 + lh.numel() * 4),
                 "d2h_bytes_per_step": int(yh.numel() * 2)},

@@ -16,8 +16,17 @@ _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 _F = ctypes.c_float
 
+
+
+class MoeConfig(ctypes.Structure):
+    """The C struct MoeConfig (one layer's configuration)."""
+    _fields_ = [("T", _I), ("H", _I), ("I", _I), ("E", _I), ("topk", _I), ("route_scale", _F),
+                ("swiglu_limit", _F), ("has_shared", _I), ("route_norm", _I)]
+
+
 # name -> (restype, argtypes)
 SIGNATURES = {
+    "moe_workspace_size": (_SZ, [ctypes.POINTER(MoeConfig), _I]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_version": (_I, []),
     "moe_get_device_error": (_I, [ctypes.POINTER(_I), _P]),

@@ -360,6 +360,20 @@ size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n) {
   return gemm::ws_layout(a_rows, n_groups, K, block_n).total;
 }
 
+size_t moe_workspace_size(const MoeConfig* cfg, int path) {
+  if (!cfg || path < MOE_PATH_MXFP4 || path > MOE_PATH_PTPC) return 0;
+  const MoeConfig& c = *cfg;
+  if (c.T < 0 || c.H <= 0 || c.I <= 0 || c.H % 128 || c.I % 128 || c.E < 1 || c.topk < 1 || c.topk > c.E)
+    return 0;
+  const int64_t R = (int64_t)c.T * c.topk + (c.has_shared ? c.T : 0);
+  if (R > (int64_t)INT32_MAX) return 0;
+  const int G = c.E + (c.has_shared ? 1 : 0);
+  size_t need = moe_permute_workspace_size(c.T, c.E, c.topk);
+  for (int bn : {16, 32, 64, 128})
+    for (int K : {c.H, c.I}) need = std::max(need, moe_gemm_workspace_size((int)R, G, K, bn));
+  return (need + 255) / 256 * 256;
+}
+
 int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets,
                            int n_groups, const uint8_t* w_prepared, int N, int K, int epilogue, float swiglu_limit,
                            int block_n, void* out, uint8_t* out_scale, void* workspace, size_t workspace_bytes,

@@ -115,6 +115,17 @@ def moe_prepare_weights(fp4, e8m0, prepared, paired=False, stream=None):
         _ptr(fp4), _ptr(e8m0), n_mats, N, k2 * 2, int(bool(paired)), _ptr(prepared), _stream(stream)))
 
 
+MOE_PATH_MXFP4, MOE_PATH_W4AFP8, MOE_PATH_PTPC = 0, 1, 2
+
+
+def moe_workspace_size(T: int, H: int, I: int, E: int, topk: int, has_shared: int = 1, path: int = 0,
+                       route_scale: float = 1.5, swiglu_limit: float = 10.0, route_norm: int = 1) -> int:
+    """Scratch bytes for moe_permute and every grouped GEMM of one layer step."""
+    from ._lib import MoeConfig
+    cfg = MoeConfig(T, H, I, E, topk, route_scale, swiglu_limit, int(has_shared), int(route_norm))
+    return int(_lib().moe_workspace_size(ctypes.byref(cfg), int(path)))
+
+
 def moe_gemm_workspace_size(a_rows: int, n_groups: int, K: int, block_n: int = 0) -> int:
     return int(_lib().moe_gemm_workspace_size(a_rows, n_groups, K, block_n))
 

@@ -223,6 +223,34 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
  *   workspace scratch of moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
  */
 size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n);
+
+/*
+ * One layer's configuration [SI 架构特性: top-k 6, routing scale 1.5, SwiGLU
+ * clamp 10, one shared expert].  T tokens, hidden H, expert intermediate I,
+ * E routed experts, topk experts per token.
+ */
+typedef struct {
+  int T, H, I, E, topk;
+  float route_scale;   /* 1.5 */
+  float swiglu_limit;  /* 10.0 */
+  int has_shared;      /* 1: the shared expert is group E and sees every token */
+  int route_norm;      /* 1: routing weights normalised to sum 1 before the scale */
+} MoeConfig;
+
+#define MOE_PATH_MXFP4 0
+#define MOE_PATH_W4AFP8 1
+#define MOE_PATH_PTPC 2
+
+/*
+ * Scratch bytes of one layer step (host call, no CUDA call): one buffer of
+ * this size, 256-byte aligned, can serve as the `workspace` of moe_permute
+ * and of every grouped GEMM of the step (w1/w3 and w2, any block_n), since
+ * they run in order on one stream.  path: MOE_PATH_MXFP4, MOE_PATH_W4AFP8 or
+ * MOE_PATH_PTPC.  Returns 0 for a NULL or invalid configuration (T < 0,
+ * H or I not a positive multiple of 128, E < 1, topk < 1 or > E, unknown
+ * path).
+ */
+size_t moe_workspace_size(const MoeConfig* cfg, int path);
 int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
                            const int32_t* offsets, int n_groups,
                            const uint8_t* w_prepared, int N, int K,

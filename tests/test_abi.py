@@ -73,3 +73,21 @@ def test_argument_validation_without_gpu():
     # the block-scaled GEMMs take no float32 SwiGLU epilogue
     assert lib.moe_grouped_gemm_fp8_block128(None, None, 4, None, 2, None, None, 256, 128, 3,
                                              ctypes.c_float(10), 16, None, None, None, 0, None) == -1
+
+
+def test_layer_workspace_size_without_gpu():
+    """moe_workspace_size covers moe_permute and every grouped GEMM of the
+    step, for every token tile, and rejects invalid configurations."""
+    from fp8_block_scaled_pow2_b200 import moe
+    lib = moe._lib()
+    T, H, I, E, k = 4096, 4096, 2048, 256, 6
+    ws = moe.moe_workspace_size(T, H, I, E, k)
+    R, G = T * k + T, E + 1
+    need = [lib.moe_permute_workspace_size(T, E, k)]
+    need += [lib.moe_gemm_workspace_size(R, G, K, bn) for K in (H, I) for bn in (16, 32, 64, 128)]
+    assert ws >= max(need) and ws % 256 == 0
+    assert moe.moe_workspace_size(T, H, I, E, k, path=moe.MOE_PATH_PTPC) == ws
+    assert moe.moe_workspace_size(T, 100, I, E, k) == 0            # H % 128
+    assert moe.moe_workspace_size(T, H, I, E, 7, path=3) == 0      # unknown path
+    assert moe.moe_workspace_size(T, H, I, 4, 6) == 0              # topk > E
+    assert moe.moe_workspace_size(0, H, I, E, k) > 0               # empty batch still valid

@@ -267,3 +267,19 @@ def test_decode_layer_ptpc_full_size(lib):
     ref = _ptpc_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
     check_y(y.float().cpu().numpy()[toks], ref["y"])
     assert lib.moe_get_device_error() == 0
+
+
+@pytest.mark.parametrize("weights", ["mxfp4", "w4afp8", "ptpc"])
+def test_empty_batch(lib, weights):
+    """Zero tokens: every call of the step is a no-op that returns MOE_OK (the
+    grouping still writes all-zero counts and offsets), y is [0, H]."""
+    wl = synth.tiny_layer(7)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk, weights=weights)
+    buf = layer.alloc(0)
+    x = torch.empty((0, layer.H), dtype=torch.int16, device="cuda")
+    lg = torch.empty((0, wl.E), dtype=torch.float32, device="cuda")
+    y = layer.forward(x, lg, buf)
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (0, layer.H)
+    assert (buf.counts.cpu().numpy() == 0).all() and (buf.offsets.cpu().numpy() == 0).all()
+    assert lib.moe_get_device_error() == 0
