@@ -126,11 +126,12 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
     return MOE_ERR_INVALID;
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
   const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
-  if (dual && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
+  if (dual && N % 256) return MOE_ERR_INVALID;
   if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
   if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual)) return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
+  if (dual && !out_scale) return MOE_ERR_INVALID;
   if (!aligned(a_e4m3, 16) || !aligned(w, 16) || !aligned(w_scale_inv, 4) || !aligned(workspace, 256))
     return MOE_ERR_INVALID;
   const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
@@ -381,11 +382,12 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   if (a_rows < 0 || n_groups < 1 || n_groups > 1024 || N <= 0 || K <= 0 || N % 128 || K % 128)
     return MOE_ERR_INVALID;
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
-  if (epilogue == MOE_EPI_SWIGLU_QUANT && (N % 256 || !out_scale)) return MOE_ERR_INVALID;
+  if (epilogue == MOE_EPI_SWIGLU_QUANT && N % 256) return MOE_ERR_INVALID;
   if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
   if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128) return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_prepared || !out || !workspace) return MOE_ERR_INVALID;
+  if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_scale) return MOE_ERR_INVALID;
   if (!aligned(a_e4m3, 16) || !aligned(w_prepared, 32) || !aligned(workspace, 256)) return MOE_ERR_INVALID;
   const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
