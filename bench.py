@@ -23,6 +23,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -122,7 +123,9 @@ class ClockSampler:
             pass
         self.proc = None
         self.window = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # MOE_CLOCKS_DIR: where the sampled clock log is kept (default: a temp dir)
+        self.path = os.path.join(os.environ.get("MOE_CLOCKS_DIR") or tempfile.gettempdir(),
+                                 f"moe_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:

@@ -22,16 +22,24 @@ Modules and the passages they follow:
               架构特性, Mixture of Experts paragraph)
   permute  -- grouping routed (token, slot) pairs by expert
   ffn      -- grouped expert GEMMs w1/w3 and w2, SwiGLU with the +-10 clamp,
-              weighted combine, and the W4AFP8 variant
-              ("DeepSeek-V4-Flash-0731-W4AFP8-mt" model card, 量化方式 / 权重约定)
-  repack   -- MXFP4 -> NVFP4 (DeepSeek-V4-Pro-0813-nvfp4-DSpark, 阶段三 storage table)
-              and MXFP4 -> symmetric INT4 group 128 (W4AFP8-mt, 量化方式 / 权重约定)
+              weighted combine, the W4AFP8 variant
+              ("DeepSeek-V4-Flash-0731-W4AFP8-mt" model card, 量化方式 / 权重约定),
+              the FP8 [128, 128]-block shared expert (DeepSeek-V4-Pro-0813-nvfp4-DSpark,
+              只量化专家; DeepSeek-V4-Flash-SI, 模型训练) and the PTPC-FP8 path
+              ("DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough, 核心参数)
+  repack   -- MXFP4 -> NVFP4 (DeepSeek-V4-Pro-0813-nvfp4-DSpark, 阶段三 storage table),
+              MXFP4 -> symmetric INT4 group 128 (W4AFP8-mt, 量化方式 / 权重约定) and
+              MXFP4 -> FP8 E4M3 with [128, 128] block scales (nvfp4-DSpark, 关于 MXFP4 的无损种子)
 
 Parity pins (tests/test_oracle_*.py) tie each function to something other than
 itself: the E2M1 value set, exhaustive E8M0 / E4M3 code tables, hand-derived
 rounding cases, closed forms, brute force on tiny inputs, the INT4 shape
 example of the W4AFP8 card and the lossless property of the NVFP4 cast.
-Readings of points the pages leave open are listed in the design doc; two of them
-are "parity unpinned" because no page fixes them: the nibble order inside a
-byte and the exact INT4 scale rule (amax / 7).
+Where the pages leave a point open the oracle takes the plainest reading and
+says so at the function.  Five readings are "parity unpinned" because no page
+fixes them: the nibble order inside a byte (element 2i in the low nibble), the
+exact INT4 scale rule (amax / 7), the PTPC-FP8 scale rule (amax / 448), the
+normalisation of the routing weights before the 1.5 scale (flag route_norm),
+and the clamp of both the gate and the up projection to +-10 before
+silu(g) * u.
 """

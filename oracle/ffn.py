@@ -121,7 +121,10 @@ def grouped_gemm_fp8_block128(a_q, a_s, offsets, w_q, w_scale_inv):
 def quantize_fp8_per_row(x: np.ndarray):
     """float32 [rows, cols] -> (E4M3 [rows, cols], float32 scale [rows]):
     scale = amax / 448 (float32 divide, 1 when amax == 0), q = E4M3(x / scale)
-    with a float32 divide (PTPC-FP8 per-token / per-channel rule)."""
+    with a float32 divide, nearest even (PTPC-FP8 per-token / per-channel rule,
+    "DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough, 核心参数: symmetric,
+    half_even).  Parity unpinned: the page names the scheme, not the scale
+    formula; amax / 448 is the plain symmetric reading."""
     x32 = np.asarray(x, dtype=np.float32)
     amax = np.abs(x32).max(axis=-1)
     scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
