@@ -101,3 +101,39 @@ def test_invalid_group_offsets_plan_no_work(lib, bad):
     torch.cuda.synchronize()
     assert lib.moe_get_device_error() == 0
     assert (out == 0.0).all()
+
+
+@pytest.mark.parametrize("gemm", ["w4afp8", "fp8_block128", "fp8_ptpc"])
+@pytest.mark.parametrize("bad", ["past_rows", "decreasing"])
+def test_invalid_group_offsets_other_gemms(lib, gemm, bad):
+    """The same plan check guards the INT4, FP8-block and PTPC-FP8 GEMMs:
+    invalid offsets record MOE_ERR_INVALID and leave the output untouched."""
+    G, N, K, R = 3, 256, 256, 40
+    offsets = {"past_rows": [0, 10, 20, 41], "decreasing": [0, 30, 10, 40]}[bad]
+    a = torch.zeros((R, K), dtype=torch.uint8, device="cuda")
+    asc = torch.full((R, K // 128), 127, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(lib.moe_gemm_workspace_size(R, G, K, 16), dtype=torch.uint8, device="cuda")
+    out = torch.full((R, N), 7.0, dtype=torch.float32, device="cuda")
+
+    def run(off):
+        if gemm == "w4afp8":
+            q = torch.zeros((G, N, K // 2), dtype=torch.int8, device="cuda")
+            s = torch.ones((G, N, K // 128), dtype=torch.float32, device="cuda")
+            lib.moe_grouped_gemm_w4afp8(a, asc, off, q, s, lib.MOE_EPI_STORE_F32, out, None, ws, 10.0, 16)
+        elif gemm == "fp8_block128":
+            q = torch.zeros((G, N, K), dtype=torch.uint8, device="cuda")
+            s = torch.ones((G, N // 128, K // 128), dtype=torch.float32, device="cuda")
+            lib.moe_grouped_gemm_fp8_block128(a, asc, off, q, s, lib.MOE_EPI_STORE_F32, out, None, ws, 10.0, 16)
+        else:
+            q = torch.zeros((G, N, K), dtype=torch.uint8, device="cuda")
+            s = torch.ones((G, N), dtype=torch.float32, device="cuda")
+            sa = torch.ones(R, dtype=torch.float32, device="cuda")
+            lib.moe_grouped_gemm_fp8_ptpc(a, sa, off, q, s, lib.MOE_EPI_STORE_F32, out, ws, 10.0, 16)
+        torch.cuda.synchronize()
+
+    run(torch.tensor(offsets, dtype=torch.int32, device="cuda"))
+    assert lib.moe_get_device_error() == -1
+    assert (out == 7.0).all()
+    run(torch.tensor([0, 10, 20, 40], dtype=torch.int32, device="cuda"))
+    assert lib.moe_get_device_error() == 0
+    assert (out == 0.0).all()

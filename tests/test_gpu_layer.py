@@ -283,3 +283,27 @@ def test_empty_batch(lib, weights):
     assert tuple(y.shape) == (0, layer.H)
     assert (buf.counts.cpu().numpy() == 0).all() and (buf.offsets.cpu().numpy() == 0).all()
     assert lib.moe_get_device_error() == 0
+
+
+@pytest.mark.parametrize("graphs", [True, False])
+def test_step_runner_overlapped_copies(lib, graphs):
+    """StepRunner (host copies overlapped with the neighbouring steps on a
+    second stream) gives, step after step with changing inputs, the eager
+    forward's y bit for bit."""
+    from fp8_block_scaled_pow2_b200.runner import StepRunner, pinned_inputs
+    wl = synth.tiny_layer(8)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    runner = StepRunner(layer, wl.T, graphs=graphs)
+    steps = [synth.tiny_layer(20 + i) for i in range(4)]
+    hosts = [pinned_inputs(s.x_bf16, s.logits) for s in steps]
+    for xh, lh, yh in hosts:
+        runner.submit(xh, lh, yh)
+    runner.synchronize()
+    ref_buf = layer.alloc(wl.T)
+    for s, (xh, lh, yh) in zip(steps, hosts):
+        y = layer.forward(torch.from_numpy(s.x_bf16.view(np.int16)).cuda(), torch.from_numpy(s.logits).cuda(),
+                          ref_buf)
+        torch.cuda.synchronize()
+        assert torch.equal(yh.view(torch.int16), y.cpu().view(torch.int16))
+    runner.close()
+    assert lib.moe_get_device_error() == 0
