@@ -509,7 +509,8 @@ def run_ours(args, wl):
         "gpu_launches": kernels_per_step(wl, args.shared, args.weights) * args.steps,
         "clocks": clocks,
     }
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:
+        # the oracle on the host cores, at N = 1 only (rank 0 is the only rank)
         line["cpu_baseline"] = cpu_baseline(wl, args.seed, budget_s=args.cpu_seconds)
     print(json.dumps(line), flush=True)
     if pg is not None:
