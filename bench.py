@@ -1,7 +1,7 @@
 """Benchmark of the routed-expert MoE layer (MXFP4 experts, FP8 activations).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|long_prefill]
+                    [--workload decode|prefill|long_prefill|decode_small|prefill_small]
 
 A step is one pass of the whole expert path (quantise, route, group, w1/w3
 GEMM + SwiGLU + requantise, w2 GEMM, combine) over one batch of synthetic
@@ -50,6 +50,9 @@ WORKLOADS = {
     "decode": dict(T=64, H=4096, I=2048, E=256, k=6, logits="uniform"),
     "prefill": dict(T=4096, H=4096, I=2048, E=256, k=6, logits="zipf"),
     "long_prefill": dict(T=16384, H=4096, I=2048, E=384, k=6, logits="zipf"),
+    # small cases of the same shapes, for kernel profiles (a few hundred MB on the device)
+    "decode_small": dict(T=64, H=4096, I=2048, E=32, k=6, logits="uniform"),
+    "prefill_small": dict(T=1024, H=4096, I=2048, E=32, k=6, logits="zipf"),
 }
 
 
