@@ -224,16 +224,21 @@ class MoeLayer:
                 moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
                                             b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
         if self.shared == "fp8":
+            # the shared expert is one group of T rows: narrow token tiles for
+            # small T spread its weight tiles over more SMs
+            bn_sh = b.block_n or (16 if b.T <= 256 else 0)
+            bn_sh_dual = min(bn_sh, 64) if bn_sh else 0
+
             def gemm13():
                 routed13()
                 moe.moe_grouped_gemm_fp8_block128(b.xq_perm, b.sx_perm, s_off, self.ws13_q, self.ws13_s,
                                                   moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm,
-                                                  self.swiglu_limit, bn_dual, stream=stream)
+                                                  self.swiglu_limit, bn_sh_dual, stream=stream)
 
             def gemm2():
                 routed2()
                 moe.moe_grouped_gemm_fp8_block128(b.hq, b.sh, s_off, self.ws2_q, self.ws2_s, moe.MOE_EPI_STORE_F32,
-                                                  b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
+                                                  b.o, None, b.ws_gemm, self.swiglu_limit, bn_sh, stream=stream)
         else:
             gemm13, gemm2 = routed13, routed2
 
