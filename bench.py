@@ -1,7 +1,7 @@
 """Benchmark of the routed-expert MoE layer (MXFP4 experts, FP8 activations).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|prefill|long_prefill|decode_small|prefill_small]
+                    [--workload decode|prefill|long_prefill|repack|decode_small|prefill_small|repack_small]
 
 A step is one pass of the whole expert path (quantise, route, group, w1/w3
 GEMM + SwiGLU + requantise, w2 GEMM, combine) over one batch of synthetic
@@ -53,6 +53,7 @@ WORKLOADS = {
     # small cases of the same shapes, for kernel profiles (a few hundred MB on the device)
     "decode_small": dict(T=64, H=4096, I=2048, E=32, k=6, logits="uniform"),
     "prefill_small": dict(T=1024, H=4096, I=2048, E=32, k=6, logits="zipf"),
+    "repack_small": dict(T=0, H=4096, I=2048, E=16, k=6, logits="uniform"),
 }
 
 
@@ -589,7 +590,7 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    if args.workload == "repack":
+    if args.workload.startswith("repack"):
         return run_reference_repack(args, wl)
     import synth
     from oracle import ffn
@@ -640,7 +641,7 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
-    elif args.workload == "repack":
+    elif args.workload.startswith("repack"):
         run_repack(args, wl)
     else:
         run_ours(args, wl)

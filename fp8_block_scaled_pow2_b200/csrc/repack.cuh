@@ -230,8 +230,9 @@ __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__
     const uint32_t lo = words[w] & 0x0F0F0F0Fu, hi = (words[w] >> 4) & 0x0F0F0F0Fu;
     const uint32_t sel_e = __byte_perm(lo | (lo >> 4), 0u, 0x0020u);
     const uint32_t sel_o = __byte_perm(hi | (hi >> 4), 0u, 0x0020u);
-    const uint32_t m_e = __byte_perm(0x0000FF00u, 0u, (sel_e >> 3) & 0x1111u);
-    const uint32_t m_o = __byte_perm(0x0000FF00u, 0u, (sel_o >> 3) & 0x1111u);
+    // sign masks: in sel >> 3 a selector nibble is odd exactly for a set sign bit
+    const uint32_t m_e = __byte_perm(0xFF00FF00u, 0xFF00FF00u, sel_e >> 3);
+    const uint32_t m_o = __byte_perm(0xFF00FF00u, 0xFF00FF00u, sel_o >> 3);
     const uint32_t r_e = (__byte_perm(tp[0], tp[1], sel_e) & ~m_e) | (__byte_perm(tn[0], tn[1], sel_e) & m_e);
     const uint32_t r_o = (__byte_perm(tp[0], tp[1], sel_o) & ~m_o) | (__byte_perm(tn[0], tn[1], sel_o) & m_o);
     ow[w] = r_e | (r_o << 4);
@@ -277,9 +278,8 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
     in[p] = __ldg(reinterpret_cast<const uint4*>(fp4 + row * (K / 2) + (int64_t)kb * 64) + j);
     b[p] = (int)__ldg(e8m0 + row * (K / 32) + (int64_t)kb * 4 + j);
   }
-  // floor(log2) and mantissa bit of E2M1 magnitude codes 0..7 (0.5, 1, 1.5, 2, 3, 4, 6)
-  const int kFl[8] = {0, -1, 0, 0, 1, 1, 2, 2};
-  const int kHalf[8] = {0, 0, 0, 1, 0, 1, 0, 1};
+  // E2M1 magnitude code c = 1..7 (0.5, 1, 1.5, 2, 3, 4, 6): floor(log2) = (c >> 1) - 1,
+  // mantissa bit = c & 1 for c >= 2 (0 for c = 1)
   int key = INT_MIN;
   int nan = 0;
 #pragma unroll
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
                                __vmaxu4(in[p].w & 0x07070707u, (in[p].w >> 4) & 0x07070707u)));
     mw = __vmaxu4(mw, mw >> 16);
     const int mc = (int)max(mw & 0xFFu, (mw >> 8) & 0xFFu);
-    if (mc > 0) key = max(key, 2 * (b[p] - 127 + kFl[mc]) + kHalf[mc]);
+    if (mc > 0) key = max(key, 2 * (b[p] - 127 + (mc >> 1) - 1) + ((mc >> 1) != 0 ? (mc & 1) : 0));
   }
   key = __reduce_max_sync(0xFFFFFFFFu, key);
   nan = __reduce_or_sync(0xFFFFFFFFu, nan);
@@ -321,8 +321,12 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
     for (int k = 0; k < 4; ++k) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t sel = (w[k] >> (16 * h)) & 0xFFFFu;          // four nibbles
-        const uint32_t sgn = __byte_perm(0x00008000u, 0u, (sel >> 3) & 0x1111u);
+        // a byte permute reads the low 3 bits of the four selector nibbles of
+        // its low 16 bits: the nibbles pick the magnitude codes, and in
+        // w >> 3 the selector is odd exactly for a set sign bit (odd table
+        // bytes are 0x80)
+        const uint32_t sel = w[k] >> (16 * h);
+        const uint32_t sgn = __byte_perm(0x80008000u, 0x80008000u, sel >> 3);
         o[2 * k + h] = __byte_perm(t0, t1, sel) | sgn;
       }
     }
