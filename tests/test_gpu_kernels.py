@@ -745,3 +745,49 @@ def test_ptpc_gemm_swiglu_f32(lib, block_n):
     tol = 1024 * 2.0 ** -24 * (11 * bound[:, :I] + 10 * bound[:, I:]) + 32 * np.spacing(np.abs(ref).astype(np.float32))
     assert (np.abs(h - ref) <= tol).all()
     no_device_error(lib)
+
+
+def _random_sizes(seed, n_groups, max_rows):
+    """Group sizes with zeros and ragged tails (about a third empty)."""
+    r = synth.splitmix64(seed, 0, n_groups)
+    sizes = (r % np.uint64(max_rows + 1)).astype(np.int64)
+    sizes[(r >> np.uint64(40)) % np.uint64(3) == 0] = 0
+    sizes[-1] = max(int(sizes[-1]), 1)
+    return sizes.tolist()
+
+
+@pytest.mark.parametrize("gemm", ["w4afp8", "fp8_block128", "ptpc"])
+def test_promoted_and_ptpc_gemms_max_groups(lib, gemm):
+    """1024 groups (the plan limit) with empty groups through the INT4, FP8-block
+    and PTPC GEMMs: integer-exact data, bit-exact against the oracle."""
+    sizes = _random_sizes(40, 1024, 5)
+    if gemm == "w4afp8":
+        a, asc, offsets, q, sinv = _w4a_inputs(41, sizes, 256, 128, True)
+        out, _ = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, 16)
+        ref = ffn.grouped_gemm_w4afp8(a, asc, offsets, q, sinv)
+        np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    elif gemm == "fp8_block128":
+        a, asc, offsets, q, sinv = _fp8w_inputs(42, sizes, 256, 128, True)
+        out, _ = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, 16)
+        ref = ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv)
+        np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    else:
+        a, sa, offsets, q, sw = _ptpc_inputs(43, sizes, 256, 128, True)
+        out = _run_ptpc(lib, a, sa, offsets, q, sw, lib.MOE_EPI_STORE_F32, 16)
+        np.testing.assert_array_equal(out, ffn.grouped_gemm_ptpc(a, sa, offsets, q, sw).astype(np.float32))
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("seed", [50, 51, 52])
+@pytest.mark.parametrize("block_n", [0, 32, 128])
+def test_gemm_random_group_mixes(lib, seed, block_n):
+    """Seeded random group-size mixes (empty groups, ragged tails, a few large
+    groups) through the MXFP4 GEMM, single tiles (N = 384) and pairs (N = 512),
+    integer-exact data: bit-exact against the oracle."""
+    sizes = _random_sizes(seed, 24, 300)
+    for N in (384, 512):
+        a, asc, offsets, w, wsc = _gemm_inputs(seed, sizes, N, 256, True)
+        out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
+        ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
+        np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
