@@ -68,14 +68,15 @@ class StepRunner:
             self.x.copy_(x_host, non_blocking=True)
             self.logits.copy_(logits_host, non_blocking=True)
             self.in_ready.record(self.h2d)
-        self.compute.wait_event(self.in_ready)
-        pre()
-        self.pre_done.record(self.compute)
-        gemm13()
-        gemm2()
-        self.compute.wait_event(self.y_copied)           # the previous y has left
-        post()
-        self.post_done.record(self.compute)
+        with torch.cuda.stream(self.compute):          # the segments run on the compute stream
+            self.compute.wait_event(self.in_ready)
+            pre()
+            self.pre_done.record(self.compute)
+            gemm13()
+            gemm2()
+            self.compute.wait_event(self.y_copied)       # the previous y has left
+            post()
+            self.post_done.record(self.compute)
         with torch.cuda.stream(self.d2h):
             self.d2h.wait_event(self.post_done)
             y_host.copy_(self.buf.y, non_blocking=True)
