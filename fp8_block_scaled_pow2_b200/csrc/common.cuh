@@ -47,6 +47,16 @@ __device__ __forceinline__ int pow2_scale_exponent(float amax) {
 }
 
 // 2^e as a float for e in [-149, 127], built from the bit pattern (exact).
+// Programmatic dependent launch (every kernel of this library is launched
+// with programmatic stream serialization): pdl_trigger lets the next kernel
+// on the stream be scheduled now, so its launch and local set-up overlap this
+// kernel; pdl_wait blocks until the previous kernel on the stream has
+// completed and its writes are visible.  Every kernel calls pdl_wait before
+// its first read or write of global memory.  Both are no-ops for a kernel
+// launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ float exp2_int(int e) {
   if (e >= -126) return __uint_as_float((uint32_t)(e + 127) << 23);
   return __uint_as_float(1u << (e + 149));

@@ -15,6 +15,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict__ x, int64_t n_groups,
                                                         int gpr, uint32_t* __restrict__ xq,
                                                         uint8_t* __restrict__ sx) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t grp = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (grp >= n_groups) return;
@@ -34,6 +36,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict_
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const float4* __restrict__ gu, int rows, int I,
                                                            float limit, uint32_t* __restrict__ hq,
                                                            uint8_t* __restrict__ sh) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int gpr = I / 128;
   const int64_t grp = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -63,6 +67,8 @@ template <int V>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E,
                                                          int k, float route_scale, int route_norm,
                                                          int32_t* __restrict__ idx, float* __restrict__ w) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -130,6 +136,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 template <bool F32_IN>
 __global__ void __launch_bounds__(256) quant_fp8_per_row_kernel(const void* __restrict__ x, int cols,
                                                                 uint8_t* __restrict__ q, float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_max[8];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -179,6 +187,8 @@ __global__ void __launch_bounds__(256) gather_row_scales_kernel(const int32_t* _
                                                                 const int32_t* __restrict__ offsets, int E,
                                                                 const float* __restrict__ src,
                                                                 float* __restrict__ dst) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int P = T * k;
   if (r >= offsets[E + 1] || r >= (int64_t)P + T) return;
@@ -206,6 +216,8 @@ constexpr int kChunk = 2048;
 
 __global__ void __launch_bounds__(256) permute_count_kernel(const int32_t* __restrict__ idx, int P, int E,
                                                             int32_t* __restrict__ chunk_hist) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[1024];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -223,6 +235,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
                                                             int E, int T, int has_shared,
                                                             int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int warp_sums[32];
   const int e = threadIdx.x;          // E + 1 <= 1024 groups
   int c = 0;
@@ -293,6 +307,8 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
                                                               const int32_t* __restrict__ offsets,
                                                               int32_t* __restrict__ perm,
                                                               int32_t* __restrict__ inv) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int ctr[1024];
   __shared__ int sidx[kChunk];
   const int p0 = blockIdx.x * kChunk;
@@ -313,6 +329,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(const int32_t* __re
                                                              int32_t* __restrict__ offsets,
                                                              int32_t* __restrict__ perm,
                                                              int32_t* __restrict__ inv) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[1024];
   __shared__ int sidx[kChunk];
   __shared__ int warp_sums[32];
@@ -370,6 +388,8 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
                                                              int E, int32_t* __restrict__ perm,
                                                              uint4* __restrict__ xq_perm,
                                                              uint8_t* __restrict__ sx_perm) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int R = offsets[E + 1];
@@ -397,6 +417,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
                                                       const float* __restrict__ w, int T, int k, int H,
                                                       int has_shared, const int32_t* __restrict__ offsets,
                                                       int E, uint2* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int h4 = H / 4;
   if (i >= (int64_t)T * h4) return;

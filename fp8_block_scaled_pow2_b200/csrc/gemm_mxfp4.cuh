@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
                                                                  int* __restrict__ header, int* __restrict__ prefix,
                                                                  int* __restrict__ tstart, int2* __restrict__ groups,
                                                                  uint8_t* __restrict__ a_sf) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_off[kMaxGroups + 1];
   __shared__ int s_t0[kMaxGroups + 1];      // first tile of each group; s_t0[G] = tiles in all
   __shared__ int s_warp[kPrepThreads / 32];
@@ -493,9 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KT = K / 128;
   const int n_ft = PAIR ? N / 256 : N / 128;
   const int rb_per_g = N / 128;
-  const int n_items = args.header[0];
-  plan.load(args.prefix, args.tstart, args.groups, G);
-
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -514,6 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // the set-up above is local; the plan and the operands come from earlier kernels
+  pdl_wait();
+  const int n_items = args.header[0];
+  plan.load(args.prefix, args.tstart, args.groups, G);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -608,6 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(128) prepare_weights_kernel(const uint8_t* __restrict__ fp4,
                                                               const uint8_t* __restrict__ e8m0, int N, int K,
                                                               int paired, uint8_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int KT = K / 128, RB = N / 128;
   const int64_t ob = blockIdx.x;            // output block index
   int64_t mat, rb;

@@ -96,9 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KT = K / 128;
   const int n_ft = DUAL ? N / 256 : N / 128;
   const int rb_per_g = N / 128;
-  const int n_items = args.header[0];
-  plan.load(args.prefix, args.tstart, args.groups, G);
-
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -117,6 +115,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // the set-up above is local; the plan and the operands come from earlier kernels
+  pdl_wait();
+  const int n_items = args.header[0];
+  plan.load(args.prefix, args.tstart, args.groups, G);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -125,9 +125,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
   const int G = args.G, N = args.N, K = args.K;
   const int KT = K / 128;
   const int n_ft = DUAL ? N / 256 : N / 128;
-  const int n_items = args.header[0];
-  plan.load(args.prefix, args.tstart, args.groups, G);
-
+  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -150,6 +148,10 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
+  // the set-up above is local; the plan and the operands come from earlier kernels
+  pdl_wait();
+  const int n_items = args.header[0];
+  plan.load(args.prefix, args.tstart, args.groups, G);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -254,7 +256,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
           const uint8_t* raw = st + C::RAW_OFF + a * C::RAW_BYTES;
           uint8_t* dst = st + C::A_OFF + a * C::A_BYTES;
 #pragma unroll
-          for (int j = 0; j < 128 / (8 * C::CONV_WARPS); ++j) {
+          for (int j = 0; j < 128 / (8 * (C::CONV_WARPS > 0 ? C::CONV_WARPS : 1)); ++j) {
             const int r = w * 8 + (lane >> 2) + 8 * C::CONV_WARPS * j;
             const uint4 in = *reinterpret_cast<const uint4*>(raw + r * 64 + chunk * 16);
             uint4 o0, o1;

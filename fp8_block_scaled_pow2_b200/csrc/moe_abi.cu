@@ -75,6 +75,25 @@ bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// Every kernel is launched with programmatic stream serialization: it may be
+// scheduled while the previous kernel on the stream is still running, and
+// waits for it (pdl_wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int pick_block_n(int a_rows, int G) {
   const double avg = (double)a_rows / (G > 0 ? G : 1);
   if (avg <= 12) return 16;
@@ -89,7 +108,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmAr
   auto k = gemm::gemm_mxfp4_kernel<BN, PAIR, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
-  k<<<sm_count(), gemm::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  launch(k, dim3(sm_count()), dim3(gemm::kThreads), C::SMEM_ALLOC, st, ta, tb, a);
   return launch_status();
 }
 
@@ -111,7 +130,7 @@ int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& 
   auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI, W8>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
-  k<<<sm_count(), C::THREADS, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  launch(k, dim3(sm_count()), dim3(C::THREADS), C::SMEM_ALLOC, st, ta, tb, a);
   return launch_status();
 }
 
@@ -163,7 +182,7 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   args.limit = swiglu_limit;
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
-  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+  launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
       reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
@@ -197,7 +216,7 @@ int launch_ptpc(const CUtensorMap& ta, const CUtensorMap& tb, const ptpc::Args& 
   auto k = ptpc::gemm_ptpc_kernel<BN, DUAL, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
-  k<<<sm_count(), ptpc::kThreads, C::SMEM_ALLOC, st>>>(ta, tb, a);
+  launch(k, dim3(sm_count()), dim3(ptpc::kThreads), C::SMEM_ALLOC, st, ta, tb, a);
   return launch_status();
 }
 
@@ -271,7 +290,7 @@ int moe_quantize_act_fp8(const void* x, int rows, int cols, uint8_t* xq, uint8_t
   if (rows == 0) return MOE_OK;
   if (!x || !xq || !sx || !aligned(x, 8) || !aligned(xq, 4)) return MOE_ERR_INVALID;
   const int64_t n_groups = (int64_t)rows * (cols / 128);
-  quant_act_kernel<<<(unsigned)((n_groups + 7) / 8), 256, 0, S(stream)>>>(
+  launch(quant_act_kernel, dim3((unsigned)((n_groups + 7) / 8)), dim3(256), 0, S(stream), 
       reinterpret_cast<const uint2*>(x), n_groups, cols / 128, reinterpret_cast<uint32_t*>(xq), sx);
   return launch_status();
 }
@@ -284,12 +303,12 @@ int moe_route_topk(const float* logits, int T, int E, int k, float route_scale, 
   const int V = (E + 31) / 32;
   const dim3 grid((T + 7) / 8);
   cudaStream_t st = S(stream);
-  if (V <= 1) route_topk_kernel<1><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
-  else if (V <= 2) route_topk_kernel<2><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
-  else if (V <= 4) route_topk_kernel<4><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
-  else if (V <= 8) route_topk_kernel<8><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
-  else if (V <= 16) route_topk_kernel<16><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
-  else route_topk_kernel<32><<<grid, 256, 0, st>>>(logits, T, E, k, route_scale, route_norm, idx, w);
+  if (V <= 1) launch(route_topk_kernel<1>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 2) launch(route_topk_kernel<2>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 4) launch(route_topk_kernel<4>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 8) launch(route_topk_kernel<8>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
+  else if (V <= 16) launch(route_topk_kernel<16>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
+  else launch(route_topk_kernel<32>, dim3(grid), dim3(256), 0, st, logits, T, E, k, route_scale, route_norm, idx, w);
   return launch_status();
 }
 
@@ -301,15 +320,15 @@ static void launch_permute(const int32_t* idx, int T, int E, int k, int has_shar
   const int P = T * k;
   const int n_chunks = (P + kChunk - 1) / kChunk;
   if (n_chunks <= 1) {
-    permute_small_kernel<<<1, 1024, 0, st>>>(idx, P, E, T, has_shared ? 1 : 0, counts, offsets, perm, inv);
+    launch(permute_small_kernel, dim3(1), dim3(1024), 0, st, idx, P, E, T, has_shared ? 1 : 0, counts, offsets, perm, inv);
   } else {
-    permute_count_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist);
-    permute_scan_kernel<<<1, 1024, 0, st>>>(hist, n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
-    permute_scatter_kernel<<<n_chunks, 256, 0, st>>>(idx, P, E, hist, offsets, perm, inv);
+    launch(permute_count_kernel, dim3(n_chunks), dim3(256), 0, st, idx, P, E, hist);
+    launch(permute_scan_kernel, dim3(1), dim3(1024), 0, st, hist, n_chunks, E, T, has_shared ? 1 : 0, counts, offsets);
+    launch(permute_scatter_kernel, dim3(n_chunks), dim3(256), 0, st, idx, P, E, hist, offsets, perm, inv);
   }
   const int64_t R = (int64_t)P + (has_shared ? T : 0);
   if (R > 0)
-    permute_gather_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(
+    launch(permute_gather_kernel, dim3((unsigned)((R + 7) / 8)), dim3(256), 0, st, 
         reinterpret_cast<const uint4*>(xq), sx, H, T, k, offsets, E, perm, reinterpret_cast<uint4*>(xq_perm),
         sx_perm);
 }
@@ -351,7 +370,7 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
     return MOE_ERR_INVALID;
   const int64_t blocks = n_mats * (N / 128) * (K / 128);
   if (blocks > 0x7FFFFFFFLL) return MOE_ERR_UNSUPPORTED;
-  gemm::prepare_weights_kernel<<<(unsigned)blocks, 128, 0, S(stream)>>>(fp4, e8m0, N, K, paired ? 1 : 0, prepared);
+  launch(gemm::prepare_weights_kernel, dim3((unsigned)blocks), dim3(128), 0, S(stream), fp4, e8m0, N, K, paired ? 1 : 0, prepared);
   return launch_status();
 }
 
@@ -423,7 +442,7 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   // SwiGLU, which requires N % 256 == 0)
   const bool pair = epilogue == MOE_EPI_SWIGLU_QUANT || N % 256 == 0;
   const int n_ft = pair ? N / 256 : N / 128;
-  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+  launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
       reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
@@ -498,7 +517,7 @@ int moe_grouped_gemm_fp8_ptpc(const uint8_t* a_e4m3, const float* a_scale, int a
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
   // the plan only: no per-tile activation scale blocks (sx == nullptr)
-  gemm::gemm_prep_kernel<<<L.max_tiles, gemm::kPrepThreads, 0, st>>>(
+  launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, nullptr, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
       reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
@@ -514,9 +533,9 @@ int moe_quantize_fp8_per_token(const void* x, int x_is_f32, int rows, int cols, 
   if (rows == 0) return MOE_OK;
   if (!x || !q || !scale || !aligned(x, 16) || !aligned(q, 8) || !aligned(scale, 4)) return MOE_ERR_INVALID;
   if (x_is_f32)
-    quant_fp8_per_row_kernel<true><<<(unsigned)rows, 256, 0, S(stream)>>>(x, cols, q, scale);
+    launch(quant_fp8_per_row_kernel<true>, dim3((unsigned)rows), dim3(256), 0, S(stream), x, cols, q, scale);
   else
-    quant_fp8_per_row_kernel<false><<<(unsigned)rows, 256, 0, S(stream)>>>(x, cols, q, scale);
+    launch(quant_fp8_per_row_kernel<false>, dim3((unsigned)rows), dim3(256), 0, S(stream), x, cols, q, scale);
   return launch_status();
 }
 
@@ -527,7 +546,7 @@ int moe_gather_row_scales(const int32_t* perm, int T, int k, const int32_t* offs
   if (max_rows > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
   if (max_rows == 0) return MOE_OK;
   if (!perm || !offsets || !src || !dst || !aligned(src, 4) || !aligned(dst, 4)) return MOE_ERR_INVALID;
-  gather_row_scales_kernel<<<(unsigned)((max_rows + 255) / 256), 256, 0, S(stream)>>>(perm, T, k, offsets, E, src,
+  launch(gather_row_scales_kernel, dim3((unsigned)((max_rows + 255) / 256)), dim3(256), 0, S(stream), perm, T, k, offsets, E, src,
                                                                                         dst);
   return launch_status();
 }
@@ -537,7 +556,7 @@ int moe_swiglu_clamp(const float* gu, int rows, int I, float limit, uint8_t* hq,
   if (rows == 0) return MOE_OK;
   if (!gu || !hq || !sh || !aligned(gu, 16) || !aligned(hq, 4)) return MOE_ERR_INVALID;
   const int64_t groups = (int64_t)rows * (I / 128);
-  swiglu_quant_kernel<<<(unsigned)((groups + 7) / 8), 256, 0, S(stream)>>>(
+  launch(swiglu_quant_kernel, dim3((unsigned)((groups + 7) / 8)), dim3(256), 0, S(stream), 
       reinterpret_cast<const float4*>(gu), rows, I, limit, reinterpret_cast<uint32_t*>(hq), sh);
   return launch_status();
 }
@@ -549,7 +568,7 @@ int moe_combine(const float* o, const int32_t* inv, const float* w, int T, int k
   if (!o || !y || (k > 0 && (!inv || !w)) || (has_shared && !offsets)) return MOE_ERR_INVALID;
   if (!aligned(o, 16) || !aligned(y, 8)) return MOE_ERR_INVALID;
   const int64_t n = (int64_t)T * (H / 4);
-  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, S(stream)>>>(
+  launch(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, S(stream), 
       reinterpret_cast<const float4*>(o), inv, w, T, k, H, has_shared ? 1 : 0, offsets, E,
       reinterpret_cast<uint2*>(y));
   return launch_status();
@@ -570,19 +589,19 @@ int repack_mxfp4_to_nvfp4(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mat
   // 16 scale bytes at a time when the scale arrays allow it
   const bool vec = per_mat % 16 == 0 && aligned(e8m0, 16) && aligned(out_e4m3, 16);
   if (vec) {
-    nvfp4_global_vec_kernel<<<(unsigned)n_mats, 512, 0, st>>>(reinterpret_cast<const uint4*>(e8m0), per_mat / 16,
+    launch(nvfp4_global_vec_kernel, dim3((unsigned)n_mats), dim3(512), 0, st, reinterpret_cast<const uint4*>(e8m0), per_mat / 16,
                                                              out_global);
     const int64_t work = std::max<int64_t>(n_scale / 16, alias ? 0 : fp4_bytes / 16);
     const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
-    nvfp4_convert_vec_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
+    launch(nvfp4_convert_vec_kernel, dim3((unsigned)std::max<int64_t>(grid, 1)), dim3(256), 0, st, 
         reinterpret_cast<const uint4*>(e8m0), n_scale / 16, per_mat / 16, out_global,
         reinterpret_cast<uint4*>(out_e4m3), reinterpret_cast<const uint4*>(fp4),
         alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
   } else {
-    nvfp4_global_kernel<<<(unsigned)n_mats, 256, 0, st>>>(e8m0, per_mat, out_global);
+    launch(nvfp4_global_kernel, dim3((unsigned)n_mats), dim3(256), 0, st, e8m0, per_mat, out_global);
     const int64_t work = std::max<int64_t>(n_scale, alias ? 0 : fp4_bytes / 16);
     const int64_t grid = std::min<int64_t>((work + 255) / 256, (int64_t)sm_count() * 16);
-    nvfp4_convert_kernel<<<(unsigned)std::max<int64_t>(grid, 1), 256, 0, st>>>(
+    launch(nvfp4_convert_kernel, dim3((unsigned)std::max<int64_t>(grid, 1)), dim3(256), 0, st, 
         e8m0, n_scale, per_mat, out_global, out_e4m3, reinterpret_cast<const uint4*>(fp4),
         alias ? nullptr : reinterpret_cast<uint4*>(out_fp4), fp4_bytes / 16);
   }
@@ -597,7 +616,7 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
   if (!aligned(fp4, 16) || !aligned(out_int4, 16) || !aligned(e8m0, 4) || !aligned(out_scale_inv, 4))
     return MOE_ERR_INVALID;
   const int64_t blocks = n_mats * (int64_t)N * (K / 32);     // 32-element blocks, 4 per group
-  int4g128_kernel<<<(unsigned)((blocks + 255) / 256), 256, 0, S(stream)>>>(
+  launch(int4g128_kernel, dim3((unsigned)((blocks + 255) / 256)), dim3(256), 0, S(stream), 
       reinterpret_cast<const uint4*>(fp4), e8m0, blocks, reinterpret_cast<uint4*>(out_int4), out_scale_inv);
   return launch_status();
 }
@@ -611,7 +630,7 @@ int repack_mxfp4_to_fp8_block128(const uint8_t* fp4, const uint8_t* e8m0, int64_
     return MOE_ERR_INVALID;
   const int64_t blocks = n_mats * (int64_t)(N / 128) * (K / 128);
   if (blocks > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
-  fp8_block128_kernel<<<(unsigned)blocks, 128, 0, S(stream)>>>(fp4, e8m0, N, K, out_e4m3, out_scale_inv);
+  launch(fp8_block128_kernel, dim3((unsigned)blocks), dim3(128), 0, S(stream), fp4, e8m0, N, K, out_e4m3, out_scale_inv);
   return launch_status();
 }
 
@@ -623,7 +642,7 @@ int repack_mxfp4_to_fp8_per_channel(const uint8_t* fp4, const uint8_t* e8m0, int
   if (!aligned(fp4, 4) || !aligned(out_e4m3, 8) || !aligned(out_scale, 4)) return MOE_ERR_INVALID;
   const int64_t rows = n_mats * (int64_t)N;
   if (rows > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
-  fp8_per_channel_kernel<<<(unsigned)rows, 256, 0, S(stream)>>>(fp4, e8m0, K, out_e4m3, out_scale);
+  launch(fp8_per_channel_kernel, dim3((unsigned)rows), dim3(256), 0, S(stream), fp4, e8m0, K, out_e4m3, out_scale);
   return launch_status();
 }
 

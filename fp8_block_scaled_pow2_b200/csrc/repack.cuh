@@ -25,6 +25,8 @@ namespace moe {
 // in out_global[m] (float32, possibly subnormal).
 __global__ void __launch_bounds__(256) nvfp4_global_kernel(const uint8_t* __restrict__ e8m0, int64_t per_mat,
                                                            float* __restrict__ out_global) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t m = blockIdx.x;
   const uint8_t* s = e8m0 + m * per_mat;
   int lo = 255, hi = 0, nan = 0;
@@ -81,6 +83,8 @@ __global__ void __launch_bounds__(256) nvfp4_convert_kernel(const uint8_t* __res
                                                             uint8_t* __restrict__ out_e4m3,
                                                             const uint4* __restrict__ fp4, uint4* __restrict__ out_fp4,
                                                             int64_t n_fp4_16) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   for (int64_t i = tid; i < n_scale; i += stride) {
@@ -101,6 +105,8 @@ __global__ void __launch_bounds__(256) nvfp4_convert_kernel(const uint8_t* __res
 // NaN scale shows as max == 255).
 __global__ void __launch_bounds__(512) nvfp4_global_vec_kernel(const uint4* __restrict__ e8m0, int64_t per_mat16,
                                                                float* __restrict__ out_global) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t m = blockIdx.x;
   const uint4* s = e8m0 + m * per_mat16;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
@@ -152,6 +158,8 @@ __global__ void __launch_bounds__(256) nvfp4_convert_vec_kernel(const uint4* __r
                                                                 uint4* __restrict__ out_e4m3,
                                                                 const uint4* __restrict__ fp4,
                                                                 uint4* __restrict__ out_fp4, int64_t n_fp4_16) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   for (int64_t i = tid; i < n16; i += stride) {
@@ -182,6 +190,8 @@ __global__ void __launch_bounds__(256) nvfp4_convert_vec_kernel(const uint4* __r
 __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__ fp4,
                                                        const uint8_t* __restrict__ e8m0, int64_t n_blocks,
                                                        uint4* __restrict__ out, float* __restrict__ scale_inv) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const bool live = blk < n_blocks;
   const uint4 in = live ? __ldg(fp4 + blk) : make_uint4(0u, 0u, 0u, 0u);
@@ -258,6 +268,8 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
                                                            const uint8_t* __restrict__ e8m0, int N, int K,
                                                            uint8_t* __restrict__ out,
                                                            float* __restrict__ scale_inv) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_key[4];
   __shared__ int s_nan[4];
   const int KB = K / 128, NB = N / 128;
@@ -356,6 +368,8 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
 __global__ void __launch_bounds__(256) fp8_per_channel_kernel(const uint8_t* __restrict__ fp4,
                                                               const uint8_t* __restrict__ e8m0, int K,
                                                               uint8_t* __restrict__ out, float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_max[8];
   __shared__ int s_bad[8];
   const int64_t row = blockIdx.x;
