@@ -26,6 +26,12 @@
  *   - Packed FP4 / INT4: element 2i is the LOW nibble of byte i, 2i+1 the high.
  *   - No exceptions cross this boundary; calls on different streams may run
  *     concurrently when their buffers are disjoint.
+ *   - Kernels are launched with programmatic dependent launch: each may be
+ *     scheduled while the previous kernel on the stream runs, and waits for
+ *     it before touching memory, so stream order is kept.  A caller kernel
+ *     that follows on the same stream and is itself launched with
+ *     programmatic stream serialization must wait for its predecessor
+ *     (cudaGridDependencySynchronize) before reading these outputs.
  *
  * Sources (web pages describing the method; cited by title and section)
  *   [SI]    "DeepSeek-V4-Flash-SI" model card: 架构特性 (Mixture of Experts
