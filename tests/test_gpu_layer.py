@@ -307,3 +307,20 @@ def test_step_runner_overlapped_copies(lib, graphs):
         assert torch.equal(yh.view(torch.int16), y.cpu().view(torch.int16))
     runner.close()
     assert lib.moe_get_device_error() == 0
+
+
+def test_prefill_layer_ptpc_sampled(lib):
+    """Prefill configuration (4096 tokens, Zipf loads, 256 + 1 experts) in
+    PTPC-FP8, the launch configuration the benchmark times (128-token tiles
+    with gate and up pairs); sampled tokens against the oracle."""
+    T, H, I, E, k = 4096, 4096, 2048, 256, 6
+    w13, s13, w2, s2 = synth.expert_weights(0, E + 1, H, I, n_proto=2)
+    x = synth.decode_activations(0, T, H)
+    logits = synth.zipf_logits(0, T, E)
+    layer = MoeLayer(w13, s13, w2, s2, k, weights="ptpc")
+    buf = layer.alloc(T)
+    y = layer.forward(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(logits).cuda(), buf)
+    toks = np.sort((synth.splitmix64(0, 81, 6) % np.uint64(T)).astype(np.int64))
+    ref = _ptpc_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
+    check_y(y.float().cpu().numpy()[toks], ref["y"])
+    assert lib.moe_get_device_error() == 0
