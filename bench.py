@@ -233,10 +233,18 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
     w2 = H * I // 2 + H * I // 32
     w13_bytes = active * w13
     w2_bytes = active * w2
+    shared_fp8 = 0
+    Rg = R                                       # rows of the grouped (segment-timed) GEMMs
     if getattr(layer, "shared", "mxfp4") == "fp8" and counts[-1] > 0:
-        # the shared expert streams E4M3 bytes and float32 [128, 128] block scales instead
-        w13_bytes += 2 * I * H + 4 * (2 * I // 128) * (H // 128) - w13
-        w2_bytes += H * I + 4 * (H // 128) * (I // 128) - w2
+        # the FP8 shared expert runs beside the grouping (pre-GEMM segment): its
+        # E4M3 weights with float32 [128, 128] block scales, its rows in and out
+        w13_bytes -= w13
+        w2_bytes -= w2
+        Ts = int(counts[-1])
+        Rg = R - Ts
+        active -= 1
+        shared_fp8 = (2 * I * H + 4 * (2 * I // 128) * (H // 128) + H * I + 4 * (H // 128) * (I // 128)
+                      + Ts * (H + H // 128) + 2 * Ts * (I + I // 128) + 4 * Ts * H)
     T, E, k = wl["T"], wl["E"], wl["k"]
     ptpc = getattr(layer, "weights", "mxfp4") == "ptpc"
     # quantise (bf16 in, E4M3 + scales out), route (logits in, ids + weights
@@ -246,7 +254,7 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
     quant = T * H * 2 + T * H + (4 * T if ptpc else T * H // 128)
     route = T * E * 4 + T * k * 8
     group = T * k * 4 + R * 4 + T * k * 4 + 2 * R * (H + H // 128)
-    pre = quant + route + group + (3 * 4 * R if ptpc else 0)
+    pre = quant + route + group + (3 * 4 * R if ptpc else 0) + shared_fp8
     post = R * H * 4 + T * k * 8 + T * H * 2
     if ptpc:
         # E4M3 weights with one float32 scale per channel; activations E4M3
@@ -256,10 +264,10 @@ def algorithmic_bytes(layer, buf, wl) -> dict:
                     w13=active * (2 * I * H + 4 * 2 * I) + R * (H + 4) + R * (I + 4),
                     w2=active * (H * I + 4 * H) + R * (I + 4) + R * H * 4,
                     flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
-    return dict(active_experts=active, rows=R, pre=pre, post=post,
-                w13=w13_bytes + R * (H + H // 128) + R * (I + I // 128),
-                w2=w2_bytes + R * (I + I // 128) + R * H * 4,
-                flops13=2.0 * R * 2 * I * H, flops2=2.0 * R * H * I)
+    return dict(active_experts=active, rows=Rg, pre=pre, post=post,
+                w13=w13_bytes + Rg * (H + H // 128) + Rg * (I + I // 128),
+                w2=w2_bytes + Rg * (I + I // 128) + Rg * H * 4,
+                flops13=2.0 * Rg * 2 * I * H, flops2=2.0 * Rg * H * I)
 
 
 def run_repack(args, wl):

@@ -57,6 +57,9 @@ class Buffers:
     ws_permute: torch.Tensor
     ws_gemm: torch.Tensor
     block_n: int
+    # FP8 shared expert only: offsets [0, T] of its one group and its own GEMM workspace
+    shared_off: torch.Tensor | None = None
+    ws_shared: torch.Tensor | None = None
     # PTPC-FP8 only: float32 per-row scales and the float32 SwiGLU output
     sxf: torch.Tensor | None = None
     sxf_perm: torch.Tensor | None = None
@@ -164,6 +167,11 @@ class MoeLayer:
             o=torch.empty((R, H), dtype=f32, device=d), y=torch.empty((T, H), dtype=torch.bfloat16, device=d),
             ws_permute=torch.empty(moe.moe_permute_workspace_size(T, self.E, k), dtype=u8, device=d),
             ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n,
+            **(dict(shared_off=torch.tensor([0, T], dtype=i32, device=d),
+                    ws_shared=torch.empty(max([moe.moe_gemm_workspace_size(max(T, 1), 1, K, bn)
+                                               for bn in (0, 16, block_n) for K in (H, I)] + [256]),
+                                          dtype=u8, device=d))
+               if self.shared == "fp8" else {}),
             **(dict(sxf=torch.empty(max(T, 1), dtype=f32, device=d),
                     sxf_perm=torch.zeros(max(R, 1), dtype=f32, device=d),
                     hf=torch.zeros((R, I), dtype=f32, device=d),
@@ -176,15 +184,41 @@ class MoeLayer:
         graph; forward() runs them eagerly."""
         b = buf
         g_off = b.offsets[: self.GR + 1]          # the groups of the routed-weight GEMMs
-        s_off = b.offsets[self.E:]                 # the shared group alone (FP8 shared expert)
 
         ptpc = self.weights == "ptpc"
 
+        shared_fp8 = self.shared == "fp8"
+        if shared_fp8:
+            # The shared expert sees every token in token order, so its GEMMs read
+            # xq / sx directly (one group [0, T)) and write rows T*k .. T*k+T of
+            # hq / sh / o, where the grouping places the shared group (all T*k
+            # routed pairs carry valid expert ids: the routing produces them).
+            # They run on a side stream while routing and grouping run.
+            Tk = b.T * self.topk
+            bn_sh = b.block_n or (16 if b.T <= 256 else 0)
+            bn_sh_dual = min(bn_sh, 64) if bn_sh else 0
+            if getattr(self, "_side", None) is None:
+                self._side = torch.cuda.Stream(self.device)
+            side = self._side
+
+            def shared_gemms():
+                moe.moe_grouped_gemm_fp8_block128(b.xq, b.sx, b.shared_off, self.ws13_q, self.ws13_s,
+                                                  moe.MOE_EPI_SWIGLU_QUANT, b.hq[Tk:], b.sh[Tk:], b.ws_shared,
+                                                  self.swiglu_limit, bn_sh_dual)
+                moe.moe_grouped_gemm_fp8_block128(b.hq[Tk:], b.sh[Tk:], b.shared_off, self.ws2_q, self.ws2_s,
+                                                  moe.MOE_EPI_STORE_F32, b.o[Tk:], None, b.ws_shared,
+                                                  self.swiglu_limit, bn_sh)
+
         def pre():
+            main = stream if stream is not None else torch.cuda.current_stream(self.device)
             if ptpc:
                 moe.moe_quantize_fp8_per_token(x, b.xq, b.sxf, stream=stream)
             else:
                 moe.moe_quantize_act_fp8(x, b.xq, b.sx, stream=stream)
+            if shared_fp8 and b.T > 0:
+                side.wait_stream(main)                   # xq, sx are ready
+                with torch.cuda.stream(side):
+                    shared_gemms()
             moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
             # (PTPC: the E8M0 rows moved alongside are unused; the float32
             # per-token scales follow the rows through moe_gather_row_scales)
@@ -193,6 +227,8 @@ class MoeLayer:
             if ptpc:
                 moe.moe_gather_row_scales(b.perm, b.T, self.topk, b.offsets, self.E, b.sxf, b.sxf_perm,
                                           stream=stream)
+            if shared_fp8 and b.T > 0:
+                main.wait_stream(side)                   # the shared rows of hq, sh and o are written
 
         bn_dual = min(b.block_n, 64) if b.block_n else 0
         if self.weights == "mxfp4":
@@ -223,24 +259,7 @@ class MoeLayer:
             def routed2():
                 moe.moe_grouped_gemm_w4afp8(b.hq, b.sh, g_off, self.w2_q, self.w2_sinv, moe.MOE_EPI_STORE_F32,
                                             b.o, None, b.ws_gemm, self.swiglu_limit, b.block_n, stream=stream)
-        if self.shared == "fp8":
-            # the shared expert is one group of T rows: narrow token tiles for
-            # small T spread its weight tiles over more SMs
-            bn_sh = b.block_n or (16 if b.T <= 256 else 0)
-            bn_sh_dual = min(bn_sh, 64) if bn_sh else 0
-
-            def gemm13():
-                routed13()
-                moe.moe_grouped_gemm_fp8_block128(b.xq_perm, b.sx_perm, s_off, self.ws13_q, self.ws13_s,
-                                                  moe.MOE_EPI_SWIGLU_QUANT, b.hq, b.sh, b.ws_gemm,
-                                                  self.swiglu_limit, bn_sh_dual, stream=stream)
-
-            def gemm2():
-                routed2()
-                moe.moe_grouped_gemm_fp8_block128(b.hq, b.sh, s_off, self.ws2_q, self.ws2_s, moe.MOE_EPI_STORE_F32,
-                                                  b.o, None, b.ws_gemm, self.swiglu_limit, bn_sh, stream=stream)
-        else:
-            gemm13, gemm2 = routed13, routed2
+        gemm13, gemm2 = routed13, routed2
 
         def post():
             moe.moe_combine(b.o, b.inv, b.w, self.has_shared, b.offsets, self.E, b.y, stream=stream)

@@ -129,12 +129,14 @@ def test_long_prefill_w4afp8_sampled(lib):
     check_y(y.float().cpu().numpy()[toks], ref["y"])
 
 
-def test_segment_graphs_match_eager(lib):
+@pytest.mark.parametrize("shared", ["mxfp4", "fp8"])
+def test_segment_graphs_match_eager(lib, shared):
     """The forward pass captured as four CUDA graphs (one per segment, as the
     decode benchmark replays it) gives the eager result bit for bit, also
-    after new inputs are copied into the captured buffers."""
+    after new inputs are copied into the captured buffers; with the FP8
+    shared expert the capture holds its side-stream GEMMs too."""
     wl = synth.tiny_layer(2)
-    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk, shared=shared)
     buf = layer.alloc(wl.T)
     x = torch.from_numpy(wl.x_bf16.view(np.int16)).cuda()
     lg = torch.from_numpy(wl.logits).cuda()
