@@ -196,13 +196,18 @@ __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__
   const bool live = blk < n_blocks;
   const uint4 in = live ? __ldg(fp4 + blk) : make_uint4(0u, 0u, 0u, 0u);
   const int b = live ? (int)__ldg(e8m0 + blk) : 0;
-  // largest magnitude code of the block: max over the 32 three-bit fields
-  uint32_t mw = __vmaxu4(__vmaxu4(in.x & 0x07070707u, (in.x >> 4) & 0x07070707u),
-                         __vmaxu4(in.y & 0x07070707u, (in.y >> 4) & 0x07070707u));
-  mw = __vmaxu4(mw, __vmaxu4(__vmaxu4(in.z & 0x07070707u, (in.z >> 4) & 0x07070707u),
-                             __vmaxu4(in.w & 0x07070707u, (in.w >> 4) & 0x07070707u)));
-  mw = __vmaxu4(mw, mw >> 16);
-  const uint32_t mc = max(mw & 0xFFu, (mw >> 8) & 0xFFu);
+  // largest magnitude code of the block, by a three-step binary search: some
+  // nibble m (0..7) reaches t exactly when m + 8 - t sets the nibble's bit 3
+  // (the sums stay below 16, so no carry crosses nibbles)
+  const uint32_t m0 = in.x & 0x77777777u, m1 = in.y & 0x77777777u;
+  const uint32_t m2 = in.z & 0x77777777u, m3 = in.w & 0x77777777u;
+  auto any_ge = [&](uint32_t t) {
+    const uint32_t k = (8u - t) * 0x11111111u;
+    return (((m0 + k) | (m1 + k) | (m2 + k) | (m3 + k)) & 0x88888888u) != 0u;
+  };
+  uint32_t mc = any_ge(4u) ? 4u : 0u;
+  mc += any_ge(mc + 2u) ? 2u : 0u;
+  mc += any_ge(mc + 1u) ? 1u : 0u;
   const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
   const float sc = exp2_int(b - 127);
   float bm = __fmul_rn(kE2M1[mc], sc);
@@ -225,11 +230,14 @@ __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__
   const float d3 = __fdiv_rn(__fmul_rn(3.0f, sc), sinv);
   const float qv[8] = {0.0f, 0.5f * d1, d1, 0.5f * d3, 2.0f * d1, d3, 4.0f * d1, 2.0f * d3};
   // byte tables over the magnitude code: tp = q, tn = (16 - q) & 15 (q <= 7, so
-  // the byte-wise subtraction never borrows)
-  uint32_t tp[2] = {0u, 0u};
+  // the byte-wise subtraction never borrows).  For 0 <= v <= 7 the float v + 2^23
+  // holds rint(v) (round half to even) in its low byte, and its byte 1 is zero.
+  uint32_t u[8];
 #pragma unroll
-  for (int c = 1; c < 8; ++c)
-    tp[c >> 2] |= __float2uint_rn(fminf(qv[c], 7.0f)) << (8 * (c & 3));   // round half to even
+  for (int c = 1; c < 8; ++c) u[c] = __float_as_uint(__fadd_rn(fminf(qv[c], 7.0f), 8388608.0f));
+  const uint32_t tp[2] = {__byte_perm(__byte_perm(u[1], u[2], 0x1401u), u[3], 0x4210u),     // 0, q1, q2, q3
+                          __byte_perm(__byte_perm(u[4], u[5], 0x0040u), __byte_perm(u[6], u[7], 0x0040u),
+                                      0x5410u)};                                              // q4 .. q7
   const uint32_t tn[2] = {(0x10101010u - tp[0]) & 0x0F0F0F0Fu, (0x10101010u - tp[1]) & 0x0F0F0F0Fu};
   const uint32_t words[4] = {in.x, in.y, in.z, in.w};
   uint32_t ow[4];
