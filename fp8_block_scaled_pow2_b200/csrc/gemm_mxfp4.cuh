@@ -131,7 +131,7 @@ struct Cfg {
 //   a_sf     uint8[max_tiles * KG * NA * 512]: per-tile activation scales, interleaved
 //            for tensor memory, four 128-wide K steps per 512-byte block (KG = ceil(KT/4))
 struct WsLayout {
-  size_t header, prefix, tstart, groups, a_sf, total;
+  size_t header, prefix, tstart, groups, a_sf, a_corr, total;
   int max_tiles;
 };
 
@@ -146,8 +146,26 @@ inline WsLayout ws_layout(int a_rows, int G, int K, int BN) {
   L.tstart = L.prefix + align256(4 * (size_t)(G + 1));
   L.groups = L.tstart + align256(4 * (size_t)G);
   L.a_sf = L.groups + align256(8 * (size_t)G);
-  L.total = L.a_sf + align256((size_t)L.max_tiles * ((KT + 3) / 4) * NA * 512);
+  L.a_corr = L.a_sf + align256((size_t)L.max_tiles * ((KT + 3) / 4) * NA * 512);
+  L.total = L.a_corr + align256(4 * (size_t)a_rows * KT);
   return L;
+}
+
+// Sum of sixteen E4M3 values (bytes of v, any order) in float32; each pair is
+// converted exactly to half precision first.
+__device__ __forceinline__ float sum_e4m3x16(const uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> (16 * h)), __NV_E4M3);
+      const float2 f = __half22float2(__half2(r));
+      s += f.x + f.y;
+    }
+  }
+  return s;
 }
 
 constexpr int kPrepThreads = 128;
@@ -166,12 +184,20 @@ constexpr int kPrepPerThread = (kMaxGroups + kPrepThreads) / kPrepThreads;   // 
 // MOE_ERR_INVALID is recorded, so no tile ever addresses rows outside the
 // operands or the workspace.  (offsets[0] > 0 lets a caller run a subset of
 // groups, e.g. one group of a larger grouping.)
+//
+// With a_corr (the INT4 weight GEMM on narrow token tiles), each block also
+// writes, for every row r of its tile and K step kt, a_corr[r * KT + kt] =
+// 8 * 2^(sx - 127) * (sum of the row's 128 E4M3 values in that step): the GEMM
+// multiplies the activations by the weights offset by +8 (codes 0..15) and
+// subtracts this term.
 __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* __restrict__ offsets, int G,
                                                                  int a_rows, int BN, int n_ft,
                                                                  const uint8_t* __restrict__ sx, int KT,
                                                                  int* __restrict__ header, int* __restrict__ prefix,
                                                                  int* __restrict__ tstart, int2* __restrict__ groups,
-                                                                 uint8_t* __restrict__ a_sf) {
+                                                                 uint8_t* __restrict__ a_sf,
+                                                                 const uint8_t* __restrict__ aq,
+                                                                 float* __restrict__ a_corr) {
   pdl_trigger();
   pdl_wait();
   __shared__ int s_off[kMaxGroups + 1];
@@ -253,6 +279,26 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
       }
       uint8_t* blk = a_sf + ((size_t)(t * KG + kg) * NA + a) * 512;
       *reinterpret_cast<uint32_t*>(blk + (n & 31) * 16 + (n >> 5) * 4) = w;
+    }
+  }
+  if (a_corr == nullptr) return;
+  // eight threads per (row, K step), 16 bytes each; the loop count is uniform
+  // over the block so that the shuffles see full warps
+  const int sub = tid & 7, n_pairs = rows * KT;
+  for (int p0 = 0; p0 < n_pairs; p0 += kPrepThreads / 8) {
+    const int p = p0 + (tid >> 3);
+    const int r = p / KT, kt = p - r * KT;
+    float s = 0.0f;
+    if (p < n_pairs) {
+      const uint4 v = *reinterpret_cast<const uint4*>(aq + ((size_t)(row0 + r) * KT + kt) * 128 + sub * 16);
+      s = sum_e4m3x16(v);
+    }
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, 4);
+    if (p < n_pairs && sub == 0) {
+      const size_t o = (size_t)(row0 + r) * KT + kt;
+      a_corr[o] = 8.0f * s * exp2_int((int)sx[o] - 127);
     }
   }
 }

@@ -6,14 +6,26 @@
 // The weight scale is an arbitrary float32 per (row, 128-column group), so it
 // cannot ride in the MMA's E8M0 scale slots.  Each 128-wide K step is one
 // weight group:
-//   * converter warps transcode the INT4 tile to E4M3 in shared memory (every
-//     integer -8..7 is an exact E4M3 value) in the 128-byte-swizzled K-major
-//     layout the tensor core reads;
-//   * the MMA (kind::mxf8f6f4, E4M3 x E4M3, unit weight scales, per-128
-//     activation scales) writes the group's partial sum into one of two
-//     tensor-memory buffers;
+//   * converter warps transcode the INT4 tile to E4M3 in shared memory in the
+//     128-byte-swizzled K-major layout the tensor core reads;
+//   * the MMA (kind::mxf8f6f4, E4M3 x E4M3, per-128 activation scales)
+//     writes the group's partial sum into one of two tensor-memory buffers;
 //   * promotion warps multiply each partial by the row's scale_inv and add it
 //     into float32 registers, then run the same epilogues as the MXFP4 GEMM.
+// Two transcodes:
+//   * narrow token tiles (BN <= 32, decode), where the transcode is the
+//     critical path: each code n becomes u = n + 8 (0..15) by flipping its top
+//     bit, and the byte u is the E4M3 encoding of u * 2^-9 (0..7 subnormal,
+//     8..15 with exponent field 1): a mask, an exclusive or and a byte
+//     interleave, five operations per eight weights.  The weight scale slots
+//     hold 2^9, so the MMA sums x * u; the promotion subtracts 8 * (the token
+//     row's scaled activation sum over the step, computed once per call by
+//     the plan kernel).  sum(x * u) - 8 * sum(x) = sum(x * n) exactly; in
+//     float32 the rounding is relative to sum(|x| * u) rather than
+//     sum(|x * n|);
+//   * wider tiles (prefill), bound by the operand ring rather than the
+//     transcode: byte-permute table lookups of the exact E4M3 codes of
+//     -8..7, unit weight scales, no correction.
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, then CONV_WARPS
 // converters (8 for narrow token tiles, where transcoding is the critical
 // path, else 4), then 4 promotion + epilogue warps.
@@ -35,8 +47,13 @@ using namespace sm100;
 using gemm::Item;
 using gemm::decode_item;
 
+// INT4 token tiles of at most 32 rows use the offset codes (and the plan
+// kernel's activation sums)
+__host__ __device__ constexpr bool offset_codes(int bn) { return bn <= 32; }
+
 template <int BN, bool DUAL, bool W8 = false>
 struct Cfg {
+  static constexpr bool OFFS = !W8 && offset_codes(BN);
   static constexpr int CONV_WARPS = W8 ? 0 : (BN <= 32 ? 8 : 4);
   static constexpr int PROMO_FIRST = 2 + CONV_WARPS;      // first promotion warp
   static constexpr int THREADS = (PROMO_FIRST + 4) * 32;
@@ -64,7 +81,8 @@ struct Cfg {
   static constexpr int SFA_SMEM_OFF = STAGES * STAGE;  // 512 bytes of unit scales
   static constexpr int BAR_OFF = SFA_SMEM_OFF + 512;
   static constexpr int RED_OFF = BAR_OFF + 512;
-  static constexpr int PLAN_OFF = RED_OFF + 5 * BN * 4;      // after [4][BN] maxima + [BN] scales
+  static constexpr int CORR_OFF = RED_OFF + 5 * BN * 4;      // after [4][BN] maxima + [BN] scales
+  static constexpr int PLAN_OFF = CORR_OFF + 2 * BN * 4;     // after [2][BN] offset terms
   static constexpr int SMEM_USED = PLAN_OFF + gemm::kPlanSmemBytes;
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
@@ -90,9 +108,19 @@ __device__ __forceinline__ uint32_t int4x4_to_e4m3x4(uint32_t w, int s) {
   return (pos & ~mask) | (neg & mask);
 }
 
+// Eight INT4 (two's complement nibbles, element 0 in the low nibble) ->
+// eight E4M3 bytes of (n + 8) * 2^-9: lo4 holds elements 0..3, hi4 4..7.
+__device__ __forceinline__ void int4x8_to_e4m3_offset(uint32_t w, uint32_t& lo4, uint32_t& hi4) {
+  const uint32_t ev = (w & 0x0F0F0F0Fu) ^ 0x08080808u;            // elements 0, 2, 4, 6
+  const uint32_t od = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;     // elements 1, 3, 5, 7
+  lo4 = __byte_perm(ev, od, 0x5140u);
+  hi4 = __byte_perm(ev, od, 0x7362u);
+}
+
 struct W4Args {
   const float* w_sinv;     // [G, N, K/128] (INT4) or [G, N/128, K/128] (FP8)
   const uint8_t* a_sf;     // per-tile activation scales (as in the MXFP4 GEMM)
+  const float* a_corr;     // offset codes: [a_rows][K/128] terms from the plan kernel
   const int* header;
   const int* prefix;
   const int* tstart;
@@ -141,8 +169,10 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
   }
-  // unit weight scales (E8M0 127 = 2^0) for every row and sub-block
-  if (threadIdx.x < 128) reinterpret_cast<uint32_t*>(smem + C::SFA_SMEM_OFF)[threadIdx.x] = 0x7F7F7F7Fu;
+  // weight scale slots for every row and sub-block: 2^9 (E8M0 136) for the
+  // offset codes stored as u * 2^-9, else 2^0 (E8M0 127)
+  if (threadIdx.x < 128)
+    reinterpret_cast<uint32_t*>(smem + C::SFA_SMEM_OFF)[threadIdx.x] = C::OFFS ? 0x88888888u : 0x7F7F7F7Fu;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -260,14 +290,21 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
             const int r = w * 8 + (lane >> 2) + 8 * C::CONV_WARPS * j;
             const uint4 in = *reinterpret_cast<const uint4*>(raw + r * 64 + chunk * 16);
             uint4 o0, o1;
-            o0.x = int4x4_to_e4m3x4(in.x, 0);
-            o0.y = int4x4_to_e4m3x4(in.x, 16);
-            o0.z = int4x4_to_e4m3x4(in.y, 0);
-            o0.w = int4x4_to_e4m3x4(in.y, 16);
-            o1.x = int4x4_to_e4m3x4(in.z, 0);
-            o1.y = int4x4_to_e4m3x4(in.z, 16);
-            o1.z = int4x4_to_e4m3x4(in.w, 0);
-            o1.w = int4x4_to_e4m3x4(in.w, 16);
+            if constexpr (C::OFFS) {
+              int4x8_to_e4m3_offset(in.x, o0.x, o0.y);
+              int4x8_to_e4m3_offset(in.y, o0.z, o0.w);
+              int4x8_to_e4m3_offset(in.z, o1.x, o1.y);
+              int4x8_to_e4m3_offset(in.w, o1.z, o1.w);
+            } else {
+              o0.x = int4x4_to_e4m3x4(in.x, 0);
+              o0.y = int4x4_to_e4m3x4(in.x, 16);
+              o0.z = int4x4_to_e4m3x4(in.y, 0);
+              o0.w = int4x4_to_e4m3x4(in.y, 16);
+              o1.x = int4x4_to_e4m3x4(in.z, 0);
+              o1.y = int4x4_to_e4m3x4(in.z, 16);
+              o1.z = int4x4_to_e4m3x4(in.w, 0);
+              o1.w = int4x4_to_e4m3x4(in.w, 16);
+            }
             const int c0 = 2 * chunk, c1 = 2 * chunk + 1;
             *reinterpret_cast<uint4*>(dst + r * 128 + ((c0 ^ (r & 7)) << 4)) = o0;
             *reinterpret_cast<uint4*>(dst + r * 128 + ((c1 ^ (r & 7)) << 4)) = o1;
@@ -302,10 +339,26 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
       const int nchunks = (it.rows + 15) >> 4;
       bool ok = true;
       float sc0 = __ldg(s0), sc1 = DUAL ? __ldg(s1) : 0.0f;
+      // offset codes: thread f < rows fetches token column f's term of each
+      // K step; the 128 promotion threads swap them through shared memory
+      const bool has_c = C::OFFS && f < it.rows;
+      const float* cf = has_c ? args.a_corr + (size_t)(it.row0 + f) * KT : nullptr;
+      float cv = has_c ? __ldg(cf) : 0.0f;
       for (int kt = 0; kt < KT; ++kt) {
         const float nx0 = (kt + 1 < KT) ? __ldg(s0 + kt + 1) : 0.0f;
         const float nx1 = (DUAL && kt + 1 < KT) ? __ldg(s1 + kt + 1) : 0.0f;
-        if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag)) { ok = false; break; }
+        const float* cs = reinterpret_cast<const float*>(smem + C::CORR_OFF) + (kt & 1) * BN;
+        if constexpr (C::OFFS) {
+          const float nc = (has_c && kt + 1 < KT) ? __ldg(cf + kt + 1) : 0.0f;
+          if (f < BN) reinterpret_cast<float*>(smem + C::CORR_OFF)[(kt & 1) * BN + f] = cv;
+          cv = nc;
+          // the barrier publishes the terms and makes the give-up decision the
+          // same in all 128 threads (the epilogue has more barriers)
+          const bool got = mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag);
+          if (!named_bar_and(1, 128, got)) { ok = false; break; }
+        } else {
+          if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag)) { ok = false; break; }
+        }
         tc_fence_after();
         const uint32_t base = lane_addr + pb * C::P_COLS;
 #pragma unroll
@@ -319,13 +372,17 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
               tmem_wait_ld(r0, r1);
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]), acc0[ch * 16 + j]);
-                acc1[ch * 16 + j] = fmaf(sc1, __uint_as_float(r1[j]), acc1[ch * 16 + j]);
+                const float c = C::OFFS ? cs[ch * 16 + j] : 0.0f;
+                acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]) - c, acc0[ch * 16 + j]);
+                acc1[ch * 16 + j] = fmaf(sc1, __uint_as_float(r1[j]) - c, acc1[ch * 16 + j]);
               }
             } else {
               tmem_wait_ld(r0);
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]), acc0[ch * 16 + j]);
+              for (int j = 0; j < 16; ++j) {
+                const float c = C::OFFS ? cs[ch * 16 + j] : 0.0f;
+                acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]) - c, acc0[ch * 16 + j]);
+              }
             }
           }
         }

@@ -180,12 +180,16 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   args.out = out;
   args.out_scale = out_scale;
   args.limit = swiglu_limit;
+  // INT4 weights on narrow token tiles: per (row, K step) activation sums for
+  // the +8 weight offset
+  float* a_corr = (!W8 && w4a::offset_codes(block_n)) ? reinterpret_cast<float*>(ws + L.a_corr) : nullptr;
+  args.a_corr = a_corr;
   cudaStream_t st = S(stream);
   const int n_ft = dual ? N / 256 : N / 128;
   launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, a_e4m3, a_corr);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   if (dual) {
     switch (block_n) {
@@ -445,7 +449,7 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   switch (epilogue) {
     case MOE_EPI_STORE_F32:
@@ -520,7 +524,7 @@ int moe_grouped_gemm_fp8_ptpc(const uint8_t* a_e4m3, const float* a_scale, int a
   launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, nullptr, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf);
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   if (dual) return launch_ptpc_bn<true, MOE_EPI_SWIGLU_F32>(block_n, ta, tb, args, st);
   if (epilogue == MOE_EPI_STORE_F32) return launch_ptpc_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);

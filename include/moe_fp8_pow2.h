@@ -271,9 +271,15 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
  * FP8 activations as moe_grouped_gemm_mxfp4:
  *   acc[r, n] = sum_g scale_inv[g', n, g] * sum_{k in group g}
  *               a[r, k] * 2^(sa[r, g]-127) * q[g', n, k]        (g' = r's group)
- * Each 128-wide group is one block-scaled MMA (INT4 transcoded exactly to
- * E4M3 in shared memory) whose float32 partial is scaled and summed in
- * registers, groups in ascending order.
+ * Each 128-wide group is one block-scaled MMA whose float32 partial is
+ * scaled and summed in registers, groups in ascending order.  Token tiles of
+ * at most 32 rows run the MMA on the offset codes q + 8 (exact E4M3 values
+ * of (q + 8) * 2^-9, with weight scale slots 2^9) and subtract 8 x the row's
+ * scaled activation sum over the group (computed once per call into the
+ * workspace) from each partial: an exact identity, whose float32 rounding is
+ * relative to sum |a| * 2^(sa-127) * (q + 8) per group rather than
+ * sum |a * q|.  Wider tiles transcode q exactly to E4M3 (unit weight scale
+ * slots).
  *   w_int4       int8 [G, N, K/2] (16-byte aligned); w_scale_inv float32 [G, N, K/128]
  *   other arguments, layouts and epilogues as moe_grouped_gemm_mxfp4;
  *   block_n: 16, 32, 64 (SWIGLU_QUANT) or up to 128 (STORE_F32 / STORE_BF16);
