@@ -322,6 +322,9 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     const int f = q * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t pb = 0, pbits = 0;
+    // offset-term slot, alternating per K step across items: the barrier of
+    // step s + 1 separates the reads of step s from the writes of step s + 2
+    uint32_t cslot = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb_per_g = N / 128;
@@ -347,11 +350,12 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const float nx0 = (kt + 1 < KT) ? __ldg(s0 + kt + 1) : 0.0f;
         const float nx1 = (DUAL && kt + 1 < KT) ? __ldg(s1 + kt + 1) : 0.0f;
-        const float* cs = reinterpret_cast<const float*>(smem + C::CORR_OFF) + (kt & 1) * BN;
+        const float* cs = reinterpret_cast<const float*>(smem + C::CORR_OFF) + cslot * BN;
         if constexpr (C::OFFS) {
           const float nc = (has_c && kt + 1 < KT) ? __ldg(cf + kt + 1) : 0.0f;
-          if (f < BN) reinterpret_cast<float*>(smem + C::CORR_OFF)[(kt & 1) * BN + f] = cv;
+          if (f < BN) reinterpret_cast<float*>(smem + C::CORR_OFF)[cslot * BN + f] = cv;
           cv = nc;
+          cslot ^= 1u;
           // the barrier publishes the terms and makes the give-up decision the
           // same in all 128 threads (the epilogue has more barriers)
           const bool got = mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag);
