@@ -435,6 +435,20 @@ def test_w4afp8_integer_exact(lib, block_n):
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("block_n", [16, 32])
+@pytest.mark.parametrize("N", [4096, 3968])
+def test_w4afp8_odd_k_steps_many_items(lib, block_n, N):
+    """Three K steps per item and more work items than SMs (each block runs
+    several in a row), gate/up tile pairs (N % 256 == 0) and single tiles:
+    the promotion's per-step offset terms must not leak between items.
+    Integer-exact inputs, so the output must equal the oracle bit for bit."""
+    a, asc, offsets, q, sinv = _w4a_inputs(12, [5, 17, 1, 33, 2, 40, 9, 16], N, 384, True)
+    out, _ = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_w4afp8(a, asc, offsets, q, sinv)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
+
+
 @pytest.mark.parametrize("block_n", [16, 64])
 def test_w4afp8_random(lib, block_n):
     a, asc, offsets, q, sinv = _w4a_inputs(8, [3, 0, 40, 130, 1], 384, 1024, False)
