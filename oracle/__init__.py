@@ -18,8 +18,9 @@ Modules and the passages they follow:
                "DeepSeek-V4-Pro-0813-nvfp4-DSpark" walkthrough, 关于 MXFP4 的无损种子)
   quant    -- online FP8 E4M3 activation quantisation, one power-of-two scale
               per 128 elements (DeepSeek-V4-Flash-SI, 低精度计算 and 模型训练 table)
-  route    -- sqrtsoftplus top-k routing with route scale 1.5 (DeepSeek-V4-Flash-SI,
-              架构特性, Mixture of Experts paragraph)
+  route    -- sqrtsoftplus top-k routing with route scale 1.5, and the hash routing
+              of the first layers read as a token-id -> experts table lookup
+              (DeepSeek-V4-Flash-SI, 架构特性, Mixture of Experts paragraph)
   permute  -- grouping routed (token, slot) pairs by expert
   ffn      -- grouped expert GEMMs w1/w3 and w2, SwiGLU with the +-10 clamp,
               weighted combine, the W4AFP8 variant
@@ -36,10 +37,11 @@ itself: the E2M1 value set, exhaustive E8M0 / E4M3 code tables, hand-derived
 rounding cases, closed forms, brute force on tiny inputs, the INT4 shape
 example of the W4AFP8 card and the lossless property of the NVFP4 cast.
 Where the pages leave a point open the oracle takes the plainest reading and
-says so at the function.  Five readings are "parity unpinned" because no page
+says so at the function.  Six readings are "parity unpinned" because no page
 fixes them: the nibble order inside a byte (element 2i in the low nibble), the
 exact INT4 scale rule (amax / 7), the PTPC-FP8 scale rule (amax / 448), the
 normalisation of the routing weights before the 1.5 scale (flag route_norm),
-and the clamp of both the gate and the up projection to +-10 before
-silu(g) * u.
+the clamp of both the gate and the up projection to +-10 before
+silu(g) * u, and hash routing as a lookup in a caller-supplied table (the
+page names hash routing by token ID but gives no hash).
 """

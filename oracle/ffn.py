@@ -41,7 +41,7 @@ import numpy as np
 from .formats import decode_bf16_bits, decode_e2m1_packed, decode_e4m3, decode_e8m0, encode_e4m3_rne_sat
 from .permute import gather_rows, permute
 from .quant import dequantize_fp8_pow2, quantize_act_fp8, quantize_fp8_pow2
-from .route import route_topk
+from .route import route_hash, route_topk
 
 
 def dequant_mxfp4(packed: np.ndarray, e8m0: np.ndarray) -> np.ndarray:
@@ -212,10 +212,13 @@ def combine(o: np.ndarray, inv: np.ndarray, w: np.ndarray, offsets: np.ndarray,
 def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
               swiglu_limit=10.0, has_shared=1, route_norm=1, weights="mxfp4",
               w13_int4=None, w13_sinv=None, w2_int4=None, w2_sinv=None, tokens=None,
-              shared_fp8=None):
+              shared_fp8=None, token_ids=None, tid2eid=None):
     """The whole expert path (a1 -> a7) for the tokens listed in ``tokens``
     (all tokens when None).  Token outputs are independent given the routing,
     so a subset gives exactly those rows of the full result.
+
+    tid2eid / token_ids: hash routing (oracle.route.route_hash) in place of
+    the top-k router: the experts of token t are tid2eid[token_ids[t]].
 
     shared_fp8: optional (w13_q, w13_scale_inv, w2_q, w2_scale_inv) of the
     shared expert in FP8 with [128, 128] block scales ([2I, H], [2I/128,
@@ -228,11 +231,17 @@ def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
     if tokens is not None:
         x_bf16 = x_bf16[tokens]
         logits = logits[tokens]
+        if token_ids is not None:
+            token_ids = np.asarray(token_ids)[tokens]
     T, H = x_bf16.shape
     E = logits.shape[1]
     I = (w2 if weights == "mxfp4" else w2_int4).shape[2] * 2
     xq, sx = quantize_act_fp8(x_bf16)
-    idx, w = route_topk(logits, topk, route_scale, route_norm)
+    if tid2eid is not None:
+        assert np.asarray(tid2eid).shape[1] == topk
+        idx, w = route_hash(token_ids, tid2eid, logits, route_scale, route_norm)
+    else:
+        idx, w = route_topk(logits, topk, route_scale, route_norm)
     counts, offsets, perm, inv, src = permute(idx, E, has_shared)
     xq_p, sx_p = gather_rows(xq, sx, src)
     if weights == "mxfp4":

@@ -299,3 +299,24 @@ def small_int_fp4(seed: int, stream: int, shape_packed) -> np.ndarray:
     lo = codes[(r % np.uint64(11)).astype(np.int64)]
     hi = codes[((r >> np.uint64(8)) % np.uint64(11)).astype(np.int64)]
     return (lo | (hi << 4)).astype(np.uint8).reshape(shape_packed)
+
+
+def hash_table(seed: int, vocab: int, E: int, k: int) -> np.ndarray:
+    """A token-id -> expert table int32 [vocab, k]: k distinct expert ids per
+    entry, drawn uniformly without replacement (a partial Fisher-Yates shuffle
+    of 0..E-1 per entry, one 64-bit draw per swap).  It stands in for the
+    table a checkpoint carries for the hash-routed layers."""
+    assert 1 <= k <= E
+    r = splitmix64(seed, 6, vocab * k).reshape(vocab, k)
+    perm = np.tile(np.arange(E, dtype=np.int64), (vocab, 1))
+    rows = np.arange(vocab)
+    for j in range(k):
+        pick = j + (r[:, j] % np.uint64(E - j)).astype(np.int64)
+        a, b = perm[rows, j].copy(), perm[rows, pick].copy()
+        perm[rows, j], perm[rows, pick] = b, a
+    return perm[:, :k].astype(np.int32)
+
+
+def token_ids(seed: int, T: int, vocab: int) -> np.ndarray:
+    """T token ids uniform over [0, vocab), int32."""
+    return (splitmix64(seed, 7, T) % np.uint64(vocab)).astype(np.int32)

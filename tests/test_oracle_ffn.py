@@ -85,6 +85,40 @@ def test_single_expert_reduction():
     np.testing.assert_allclose(r["y"], 1.5 * dense(0) + dense(1), rtol=1e-12, atol=1e-15)
 
 
+def test_combine_k3_hand_built():
+    """Combine at k = 3 with the shared expert and a grouping whose inv is not
+    the identity, checked against values worked out by hand.  Tokens 0, 1 pick
+    experts [2, 0, 3] and [0, 1, 2] (E = 4), so pairs p = 0..5 go to experts
+    2, 0, 3, 0, 1, 2; grouped in ascending pair id per expert, the rows are
+    e0: p1, p3 | e1: p4 | e2: p0, p5 | e3: p2 | shared: t0, t1, hence
+    inv = [3, 0, 5, 1, 2, 4] and perm = [1, 3, 4, 0, 5, 2, 6, 7].
+    With o[r] = [r + 1, 10 (r + 1)]:
+      y[0] = 0.5 o[3] + 0.25 o[0] + 0.75 o[5] + o[6] = 2 + 0.25 + 4.5 + 7
+      y[1] = 1.0 o[1] + 0.125 o[2] + 0.375 o[4] + o[7] = 2 + 0.375 + 1.875 + 8
+    (indexing o by perm gives 12.75 for y[0, 0]; reversing the slot weights
+    of token 0 gives 13.25)."""
+    from oracle import permute as Pm
+    idx = np.array([[2, 0, 3], [0, 1, 2]], np.int32)
+    counts, offsets, perm, inv, src = Pm.permute(idx, 4, 1)
+    assert counts.tolist() == [2, 1, 2, 1, 2] and offsets.tolist() == [0, 2, 3, 5, 6, 8]
+    assert inv.tolist() == [3, 0, 5, 1, 2, 4] and perm.tolist() == [1, 3, 4, 0, 5, 2, 6, 7]
+    assert src.tolist() == [0, 1, 1, 0, 1, 0, 0, 1]
+    o = np.array([[r + 1, 10.0 * (r + 1)] for r in range(8)])
+    w = np.array([[0.5, 0.25, 0.75], [1.0, 0.125, 0.375]])
+    y = ffn.combine(o, inv, w, offsets, has_shared=1)
+    assert y.tolist() == [[13.75, 137.5], [12.25, 122.5]]
+    # the same sum as a plain loop over tokens, slots and columns
+    for t in range(2):
+        for c in range(2):
+            acc = o[offsets[4] + t, c]
+            for j in range(3):
+                acc += w[t, j] * o[inv[t * 3 + j], c]
+            assert y[t, c] == acc
+    # without the shared expert the shared rows are not added
+    y0 = ffn.combine(o[:6], inv, w, np.array([0, 2, 3, 5, 6, 6]), has_shared=0)
+    assert y0.tolist() == [[6.75, 67.5], [4.25, 42.5]]
+
+
 def test_token_subset_equals_full_rows():
     wl = synth.tiny_layer(0)
     full = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
@@ -92,6 +126,22 @@ def test_token_subset_equals_full_rows():
     part = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk,
                          tokens=sub)
     np.testing.assert_array_equal(part["y"], full["y"][sub])
+
+
+def test_layer_hash_routing_with_topk_table_equals_topk_layer():
+    """The hash-routed layer whose table rows hold each token's top-k experts
+    (one vocabulary entry per token) is the top-k routed layer, bit for bit."""
+    from oracle import route as R
+    wl = synth.tiny_layer(7)
+    idx, _ = R.route_topk(wl.logits, wl.topk)
+    ref = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
+    got = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk,
+                        token_ids=np.arange(wl.T), tid2eid=idx)
+    np.testing.assert_array_equal(got["y"], ref["y"])
+    sub = [2, 9]
+    part = ffn.moe_layer(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk,
+                         token_ids=np.arange(wl.T), tid2eid=idx, tokens=sub)
+    np.testing.assert_array_equal(part["y"], ref["y"][sub])
 
 
 def test_w4afp8_dequant_loop():

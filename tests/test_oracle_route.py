@@ -56,3 +56,59 @@ def test_weights_sum_to_route_scale():
 def test_softplus_monotone_so_logit_order_is_score_order():
     z = np.linspace(-40, 40, 20001)
     assert (np.diff(R.sqrtsoftplus(z)) > 0).all()
+
+
+# ------------------------------ hash routing ------------------------------
+def test_hash_route_is_the_table_lookup():
+    """idx[t, j] is entry j of the token's table row, checked element by element."""
+    V, E, k, T = 50, 16, 4, 40
+    table = synth.hash_table(3, V, E, k)
+    tok = synth.token_ids(3, T, V)
+    z = synth.uniform_logits(3, T, E)
+    idx, w = R.route_hash(tok, table, z)
+    for t in range(T):
+        for j in range(k):
+            assert idx[t, j] == table[tok[t], j]
+    assert idx.dtype == np.int32
+
+
+def test_hash_route_weights_closed_forms():
+    """Equal logits at the chosen experts give 1.5 / k each; logit 0 scores
+    sqrt(ln 2); unnormalised weights are 1.5 * sqrt(softplus(z))."""
+    table = np.array([[2, 0, 3], [1, 3, 0]], np.int32)
+    z = np.array([[0.0, 9.0, 0.0, 0.0], [0.0, 30.0, -7.0, 0.0]], np.float32)
+    idx, w = R.route_hash(np.array([0, 0]), table, z)
+    assert idx.tolist() == [[2, 0, 3], [2, 0, 3]]
+    np.testing.assert_allclose(w[0], [0.5, 0.5, 0.5], rtol=1e-15)
+    _, w0 = R.route_hash(np.array([1]), table, z[1:], route_norm=0)
+    np.testing.assert_allclose(w0[0], 1.5 * np.array([np.sqrt(30.0), np.sqrt(np.log(2.0)), np.sqrt(np.log(2.0))]),
+                               rtol=1e-12)
+
+
+def test_hash_route_ignores_unchosen_logits():
+    """Only the logits of the looked-up experts enter the weights."""
+    V, E, k, T = 30, 12, 3, 20
+    table = synth.hash_table(4, V, E, k)
+    tok = synth.token_ids(4, T, V)
+    z = synth.uniform_logits(4, T, E)
+    idx, w = R.route_hash(tok, table, z)
+    z2 = z.copy()
+    mask = np.ones_like(z2, bool)
+    np.put_along_axis(mask, idx.astype(np.int64), False, axis=1)
+    z2[mask] = 99.0
+    idx2, w2 = R.route_hash(tok, table, z2)
+    np.testing.assert_array_equal(idx, idx2)
+    np.testing.assert_array_equal(w, w2)
+    np.testing.assert_allclose(w.sum(1), 1.5, rtol=1e-14)
+
+
+def test_hash_route_equals_topk_when_table_holds_the_topk():
+    """A table whose row for token t lists that token's k largest logits in
+    order gives exactly the top-k router's result (pinned by brute force)."""
+    T, E, k = 10, 9, 3
+    z = synth.uniform_logits(5, T, E)
+    table = np.array([_brute_topk(z[t], k) for t in range(T)], np.int32)
+    idx_h, w_h = R.route_hash(np.arange(T), table, z)
+    idx_t, w_t = R.route_topk(z, k)
+    np.testing.assert_array_equal(idx_h, idx_t)
+    np.testing.assert_array_equal(w_h, w_t)

@@ -36,3 +36,16 @@ def test_zipf_loads_are_skewed():
     top = np.argsort(-z, axis=1, kind="stable")[:, :6]
     load = np.bincount(top.reshape(-1), minlength=256)
     assert load[0] > 3000 and load[-1] < 40 and load.sum() == 4096 * 6
+
+
+def test_hash_table_rows_distinct_and_in_range():
+    t = synth.hash_table(0, 2000, 256, 6)
+    assert t.shape == (2000, 6) and t.dtype == np.int32
+    assert ((t >= 0) & (t < 256)).all()
+    assert all(len(set(r)) == 6 for r in t.tolist())
+    # every expert is used, roughly uniformly (12000 draws over 256 experts)
+    c = np.bincount(t.reshape(-1), minlength=256)
+    assert c.min() > 15 and c.max() < 80
+    np.testing.assert_array_equal(t, synth.hash_table(0, 2000, 256, 6))
+    ids = synth.token_ids(0, 1000, 2000)
+    assert ids.dtype == np.int32 and ids.min() >= 0 and ids.max() < 2000
