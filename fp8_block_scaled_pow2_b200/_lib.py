@@ -33,6 +33,7 @@ SIGNATURES = {
     "moe_selftest_wait_timeout": (_I, [_I64, _P]),
     "moe_quantize_act_fp8": (_I, [_P, _I, _I, _P, _P, _P]),
     "moe_route_topk": (_I, [_P, _I, _I, _I, _F, _I, _P, _P, _P]),
+    "moe_route_hash": (_I, [_P, _I, _P, _I, _P, _I, _I, _F, _I, _P, _P, _P]),
     "moe_permute_workspace_size": (_SZ, [_I, _I, _I]),
     "moe_permute": (_I, [_P, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute_noalloc_max_counters": (_I64, []),

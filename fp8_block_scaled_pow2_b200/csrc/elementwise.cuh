@@ -128,6 +128,60 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
+// ---------------------------- hash routing --------------------------------
+// "DeepSeek-V4-Flash-SI", 架构特性: the first layers route by hash, chosen
+// deterministically from the token ID.  The experts of token t are the k
+// entries of its row in a caller-supplied table (tid2eid[token_ids[t]]); the
+// weights follow the scored layers' rule at those experts: sqrtsoftplus of
+// the gate logits, normalised in slot order and scaled.  One thread per
+// token.  An out-of-range token id or table entry records MOE_ERR_INVALID;
+// the token's row (bad id) or that slot (bad entry) gets idx -1 and weight 0.
+__global__ void __launch_bounds__(256) route_hash_kernel(const int32_t* __restrict__ token_ids, int T,
+                                                         const int32_t* __restrict__ tid2eid, int vocab,
+                                                         const float* __restrict__ logits, int E, int k,
+                                                         float route_scale, int route_norm,
+                                                         int32_t* __restrict__ idx, float* __restrict__ w) {
+  pdl_trigger();
+  pdl_wait();
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int id = __ldg(token_ids + t);
+  int32_t* irow = idx + (int64_t)t * k;
+  float* wrow = w + (int64_t)t * k;
+  if (id < 0 || id >= vocab) {
+    record_error(MOE_ERR_INVALID);
+    for (int j = 0; j < k; ++j) { irow[j] = -1; wrow[j] = 0.0f; }
+    return;
+  }
+  const int32_t* trow = tid2eid + (int64_t)id * k;
+  const float* lrow = logits + (int64_t)t * E;
+  int e_sel[16];
+  float s_sel[16];
+  float sum = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    e_sel[j] = -1;
+    s_sel[j] = 0.0f;
+    if (j < k) {
+      const int e = __ldg(trow + j);
+      if (e >= 0 && e < E) {
+        e_sel[j] = e;
+        s_sel[j] = sqrtf(softplus_f(__ldg(lrow + e)));
+        sum += s_sel[j];
+      } else {
+        record_error(MOE_ERR_INVALID);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    if (j < k) {
+      irow[j] = e_sel[j];
+      wrow[j] = e_sel[j] < 0 ? 0.0f : (route_norm ? route_scale * __fdiv_rn(s_sel[j], sum) : route_scale * s_sel[j]);
+    }
+  }
+}
+
 // ------------------------- per-token FP8 (PTPC) ----------------------------
 // PTPC-FP8 ("DeepSeek-V4.1-Flash-Quark-PTPC-FP8" walkthrough, 核心参数):
 // per-row (per-token) dynamic scale = amax / 448 (float32 IEEE divide, 1 for

@@ -316,6 +316,16 @@ int moe_route_topk(const float* logits, int T, int E, int k, float route_scale, 
   return launch_status();
 }
 
+int moe_route_hash(const int32_t* token_ids, int T, const int32_t* tid2eid, int vocab, const float* logits, int E,
+                   int k, float route_scale, int route_norm, int32_t* idx, float* w, void* stream) {
+  if (T < 0 || vocab < 1 || E < 1 || k < 1 || k > 16) return MOE_ERR_INVALID;
+  if (T == 0) return MOE_OK;
+  if (!token_ids || !tid2eid || !logits || !idx || !w) return MOE_ERR_INVALID;
+  launch(route_hash_kernel, dim3((T + 255) / 256), dim3(256), 0, S(stream), token_ids, T, tid2eid, vocab, logits, E,
+         k, route_scale, route_norm, idx, w);
+  return launch_status();
+}
+
 // The a3 passes on one stream (arguments already validated).  hist: per-chunk
 // expert counters, unused when all pairs fit in one chunk.
 static void launch_permute(const int32_t* idx, int T, int E, int k, int has_shared, const uint8_t* xq,

@@ -12,6 +12,17 @@ fixed sequence of library calls on one stream, with no host synchronisation:
 The shared expert is group E, fed every token with weight 1 ("DeepSeek-V4-
 Flash-SI" model card, 架构特性: one shared expert per layer, always active).
 
+tid2eid (int [vocab, topk]) makes it a hash-routed layer (the same card's
+first three layers: experts chosen from the token ID): moe_route_hash looks
+the experts up by token id in place of moe_route_topk, and forward() /
+segments() then take the token ids.
+
+A step whose inputs make a kernel record a device error (an expert id or
+token id out of range, see moe_get_device_error) leaves y unspecified: with
+the FP8 shared expert, for instance, a rejected pair shifts the shared group
+below row T*k, where the side-stream shared GEMMs wrote.  Check the device
+error word before using y from untrusted inputs.
+
 weights="ptpc" runs the PTPC-FP8 form of the same layer ("DeepSeek-V4.1-Flash-
 Quark-PTPC-FP8" walkthrough, 核心参数): per-channel FP8 weights cast once on
 the GPU, per-token dynamic FP8 activations:
@@ -70,7 +81,7 @@ class Buffers:
 class MoeLayer:
     def __init__(self, w13, w13_e8m0, w2, w2_e8m0, topk: int, route_scale: float = 1.5,
                  swiglu_limit: float = 10.0, has_shared: int = 1, route_norm: int = 1, device="cuda",
-                 weights: str = "mxfp4", shared: str = "mxfp4"):
+                 weights: str = "mxfp4", shared: str = "mxfp4", tid2eid=None):
         """weights="mxfp4" runs the block-scaled MXFP4 GEMMs; weights="w4afp8"
         repacks the experts once on the GPU to symmetric INT4 group-128
         (repack_mxfp4_to_int4g128) and runs the W4AFP8 GEMMs.  shared="fp8"
@@ -81,6 +92,9 @@ class MoeLayer:
         (repack_mxfp4_to_fp8_per_channel) and quantises the activations per
         token."""
         self.device = torch.device(device)
+        self.tid2eid = None if tid2eid is None else _dev(np.asarray(tid2eid, np.int32), self.device)
+        if self.tid2eid is not None and self.tid2eid.shape[1] != topk:
+            raise ValueError("tid2eid must be [vocab, topk]")
         self.G = w13.shape[0]                      # routed experts + shared expert
         self.E = self.G - (1 if has_shared else 0)
         if shared not in ("mxfp4", "fp8") or (shared == "fp8" and (not has_shared or weights == "ptpc")):
@@ -177,12 +191,15 @@ class MoeLayer:
                     hf=torch.zeros((R, I), dtype=f32, device=d),
                     shf=torch.empty(max(R, 1), dtype=f32, device=d)) if self.weights == "ptpc" else {}))
 
-    def segments(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers, stream=None):
+    def segments(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers, stream=None, token_ids=None):
         """The forward pass as four callables run in order on `stream`:
         (quantise + route + group, w1/w3 GEMM with SwiGLU, w2 GEMM, combine).
         Each only enqueues library calls, so each can be captured in a CUDA
-        graph; forward() runs them eagerly."""
+        graph; forward() runs them eagerly.  token_ids (int32 [T], device):
+        required by a hash-routed layer."""
         b = buf
+        if self.tid2eid is not None and (token_ids is None or token_ids.dtype != torch.int32):
+            raise ValueError("a hash-routed layer needs int32 token_ids")
         g_off = b.offsets[: self.GR + 1]          # the groups of the routed-weight GEMMs
 
         ptpc = self.weights == "ptpc"
@@ -219,7 +236,11 @@ class MoeLayer:
                 side.wait_stream(main)                   # xq, sx are ready
                 with torch.cuda.stream(side):
                     shared_gemms()
-            moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
+            if self.tid2eid is not None:
+                moe.moe_route_hash(token_ids, self.tid2eid, logits, b.idx, b.w, self.route_scale, self.route_norm,
+                                   stream=stream)
+            else:
+                moe.moe_route_topk(logits, self.topk, b.idx, b.w, self.route_scale, self.route_norm, stream=stream)
             # (PTPC: the E8M0 rows moved alongside are unused; the float32
             # per-token scales follow the rows through moe_gather_row_scales)
             moe.moe_permute(b.idx, self.E, self.has_shared, b.xq, b.sx, b.counts, b.offsets, b.perm, b.inv,
@@ -267,8 +288,9 @@ class MoeLayer:
         return pre, gemm13, gemm2, post
 
     def forward(self, x: torch.Tensor, logits: torch.Tensor, buf: Buffers | None = None,
-                stream=None, marks=None) -> torch.Tensor:
+                stream=None, marks=None, token_ids=None) -> torch.Tensor:
         """x bfloat16 [T, H] (or its uint16 bits), logits float32 [T, E] -> y bfloat16 [T, H].
+        token_ids int32 [T] (device): the token ids of a hash-routed layer.
 
         marks: optional three torch.cuda.Event recorded on the stream before the
         w1/w3 GEMM, between the GEMMs and after the w2 GEMM (for timing)."""
@@ -276,7 +298,7 @@ class MoeLayer:
         if buf is None or buf.T != T:
             buf = self.alloc(T)
         ev_stream = stream if stream is not None else torch.cuda.current_stream()
-        for i, seg in enumerate(self.segments(x, logits, buf, stream)):
+        for i, seg in enumerate(self.segments(x, logits, buf, stream, token_ids=token_ids)):
             if marks and i > 0:
                 marks[i - 1].record(ev_stream)
             seg()

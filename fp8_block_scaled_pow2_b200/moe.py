@@ -73,6 +73,16 @@ def moe_route_topk(logits, k, idx, w, route_scale=1.5, route_norm=1, stream=None
                                                    int(route_norm), _ptr(idx), _ptr(w), _stream(stream)))
 
 
+def moe_route_hash(token_ids, tid2eid, logits, idx, w, route_scale=1.5, route_norm=1, stream=None):
+    T, E = logits.shape
+    vocab, k = tid2eid.shape
+    if token_ids.shape != (T,):
+        raise ValueError("token_ids must be [T]")
+    _check("moe_route_hash", _lib().moe_route_hash(_ptr(token_ids), T, _ptr(tid2eid), vocab, _ptr(logits), E, k,
+                                                   ctypes.c_float(route_scale), int(route_norm), _ptr(idx),
+                                                   _ptr(w), _stream(stream)))
+
+
 def moe_permute_workspace_size(T: int, E: int, k: int) -> int:
     return int(_lib().moe_permute_workspace_size(T, E, k))
 

@@ -55,7 +55,8 @@
  *   a4 gate/up GEMM               a5 SwiGLU + requant a6 down GEMM
  *   a7 weighted combine           a8 MXFP4 -> NVFP4   a9 MXFP4 -> INT4 g128
  *   a10 W4AFP8 GEMM               f1 MXFP4 -> FP8 [128, 128] blocks
- *   f3 FP8 block-scaled GEMM (shared expert)   f4 PTPC-FP8 expert path
+ *   f2 hash routing               f3 FP8 block-scaled GEMM (shared expert)
+ *   f4 PTPC-FP8 expert path
  */
 #ifndef MOE_FP8_POW2_H
 #define MOE_FP8_POW2_H
@@ -129,6 +130,29 @@ int moe_quantize_act_fp8(const void* x, int rows, int cols, uint8_t* xq, uint8_t
  */
 int moe_route_topk(const float* logits, int T, int E, int k, float route_scale,
                    int route_norm, int32_t* idx, float* w, void* stream);
+
+/*
+ * f2 -- hash routing of the first layers [SI 架构特性: the first 3 layers
+ * choose experts by hash, deterministically from the token ID].  The page
+ * gives no hash function; the choice is read as a lookup in a table of k
+ * expert ids per vocabulary entry that the caller supplies (a checkpoint
+ * carries it): idx[t, j] = tid2eid[token_ids[t], j], in table order.  The
+ * weights take the scored layers' rule at those experts:
+ * s_j = sqrt(softplus(logits[t, idx[t, j]])),
+ * w[t, j] = route_scale * s_j / sum_j s_j   (route_norm != 0)
+ *         = route_scale * s_j               (route_norm == 0),
+ * the sum taken in slot order in float32 (device expf/log1pf/sqrtf, as
+ * moe_route_topk).
+ *   token_ids int32 [T];  tid2eid int32 [vocab, k] (expert ids in [0, E));
+ *   logits float32 [T, E];  idx int32 [T, k];  w float32 [T, k];
+ *   1 <= k <= 16
+ * A token id outside [0, vocab) records MOE_ERR_INVALID in the device error
+ * word and gives that token idx -1 and weight 0 in every slot; a table entry
+ * outside [0, E) does the same for its slot only (moe_permute then gives
+ * such a pair no row and moe_combine skips it).
+ */
+int moe_route_hash(const int32_t* token_ids, int T, const int32_t* tid2eid, int vocab, const float* logits,
+                   int E, int k, float route_scale, int route_norm, int32_t* idx, float* w, void* stream);
 
 /*
  * a3 -- grouping by expert.  Groups g = 0..E-1 are the routed experts,

@@ -50,6 +50,11 @@ def test_argument_validation_without_gpu():
     assert lib.moe_quantize_act_fp8(None, 4, 100, None, None, None) == -1      # cols % 128
     assert lib.moe_quantize_act_fp8(None, 0, 128, None, None, None) == 0       # empty: no-op
     assert lib.moe_route_topk(None, 4, 8, 9, ctypes.c_float(1.5), 1, None, None, None) == -1
+    # hash routing: k > 16, an empty vocabulary and null pointers are rejected; T = 0 is a no-op
+    assert lib.moe_route_hash(None, 4, None, 100, None, 256, 17, ctypes.c_float(1.5), 1, None, None, None) == -1
+    assert lib.moe_route_hash(None, 4, None, 0, None, 256, 6, ctypes.c_float(1.5), 1, None, None, None) == -1
+    assert lib.moe_route_hash(None, 4, None, 100, None, 256, 6, ctypes.c_float(1.5), 1, None, None, None) == -1
+    assert lib.moe_route_hash(None, 0, None, 100, None, 256, 6, ctypes.c_float(1.5), 1, None, None, None) == 0
     assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 256, 100, 0,
                                       ctypes.c_float(10), 0, None, None, None, 0, None) == -1
     assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 256, 128, 0,
