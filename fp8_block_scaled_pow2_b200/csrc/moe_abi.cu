@@ -671,24 +671,53 @@ namespace {
 constexpr int64_t kNoAllocScratchInts = 65536;   // 256 KiB: n_chunks * E int32 counters
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocScratchInts];
 
-// Device address of g_permute_scratch, looked up once per device with that
-// device current (the host-side symbol is not a device address).
+// Device address of g_permute_scratch, looked up with the device current
+// (the host-side symbol is not a device address) and cached per device
+// together with the context it was found in: after a device reset the
+// primary context, and with it the module and the array's address, is new,
+// so a changed context triggers a fresh lookup.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 int32_t* permute_scratch_ptr(int* status) {
   static std::mutex mu;
   static int32_t* ptrs[128] = {};
+  static CUcontext ctxs[128] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (!get_ctx || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    *status = MOE_ERR_LAUNCH;
+    return nullptr;
+  }
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) {
     *status = MOE_ERR_LAUNCH;
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev] || !ctx || ctxs[dev] != ctx) {
+    // the lookup also makes the device's primary context current when no
+    // context was yet (it allocates nothing)
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p) {
+    if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess || !p || get_ctx(&ctx) != CUDA_SUCCESS ||
+        !ctx) {
       *status = MOE_ERR_LAUNCH;
       return nullptr;
     }
     ptrs[dev] = static_cast<int32_t*>(p);
+    ctxs[dev] = ctx;
   }
   *status = MOE_OK;
   return ptrs[dev];

@@ -192,7 +192,10 @@ int moe_permute(const int32_t* idx, int T, int E, int k, int has_shared,
  * cudaFree or allocating library routine.
  *   - The first call on each device looks up the array's device address with
  *     that device current (cudaGetSymbolAddress); make that first call before
- *     any stream capture on the device.
+ *     any stream capture on the device.  The address is cached with the CUDA
+ *     context it was found in; a device reset (cudaDeviceReset) ends that
+ *     context and invalidates the address, so the first call after a reset
+ *     looks it up again (and should likewise precede any capture).
  *   - All calls share the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero (each call writes every counter it
  *     reads).  Calls whose executions overlap on the GPU (different streams,
