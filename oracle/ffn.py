@@ -88,19 +88,34 @@ def grouped_gemm(a_q, a_s, offsets, w_deq_fn, n_groups):
     return out
 
 
-def grouped_gemm_mxfp4(a_q, a_s, offsets, w_fp4, w_e8m0):
+def _memo(cache, arrays, fn):
+    """fn() -- or, with a cache dict, its value stored under the memory
+    address and shape of the source arrays: groups whose weights occupy the
+    same memory dequantise once (a saving of time, not a change of values)."""
+    if cache is None:
+        return fn()
+    key = tuple((np.asarray(a).__array_interface__["data"][0], np.asarray(a).shape) for a in arrays)
+    if key not in cache:
+        cache[key] = fn()
+    return cache[key]
+
+
+def grouped_gemm_mxfp4(a_q, a_s, offsets, w_fp4, w_e8m0, cache=None):
     """Steps a4 / a6: FP8 rows x MXFP4 weights [G, N, K/2] -> float64 [R, N]."""
     N = w_fp4.shape[1]
-    out = grouped_gemm(a_q, a_s, offsets, lambda g: dequant_mxfp4(w_fp4[g], w_e8m0[g]),
+    out = grouped_gemm(a_q, a_s, offsets,
+                       lambda g: _memo(cache, (w_fp4[g], w_e8m0[g]), lambda: dequant_mxfp4(w_fp4[g], w_e8m0[g])),
                        w_fp4.shape[0])
     return out if out.shape[1] else np.zeros((a_q.shape[0], N))
 
 
-def grouped_gemm_w4afp8(a_q, a_s, offsets, w_int4, w_scale_inv):
+def grouped_gemm_w4afp8(a_q, a_s, offsets, w_int4, w_scale_inv, cache=None):
     """Step a10: FP8 rows x INT4-g128 weights [G, N, K/2] -> float64 [R, N]."""
     N = w_int4.shape[1]
     out = grouped_gemm(a_q, a_s, offsets,
-                       lambda g: dequant_int4g128(w_int4[g], w_scale_inv[g]), w_int4.shape[0])
+                       lambda g: _memo(cache, (w_int4[g], w_scale_inv[g]),
+                                       lambda: dequant_int4g128(w_int4[g], w_scale_inv[g])),
+                       w_int4.shape[0])
     return out if out.shape[1] else np.zeros((a_q.shape[0], N))
 
 
@@ -212,13 +227,17 @@ def combine(o: np.ndarray, inv: np.ndarray, w: np.ndarray, offsets: np.ndarray,
 def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
               swiglu_limit=10.0, has_shared=1, route_norm=1, weights="mxfp4",
               w13_int4=None, w13_sinv=None, w2_int4=None, w2_sinv=None, tokens=None,
-              shared_fp8=None, token_ids=None, tid2eid=None):
+              shared_fp8=None, token_ids=None, tid2eid=None, cache=None):
     """The whole expert path (a1 -> a7) for the tokens listed in ``tokens``
     (all tokens when None).  Token outputs are independent given the routing,
     so a subset gives exactly those rows of the full result.
 
     tid2eid / token_ids: hash routing (oracle.route.route_hash) in place of
     the top-k router: the experts of token t are tid2eid[token_ids[t]].
+
+    cache: optional dict in which dequantised expert weights are kept, keyed
+    by the memory of their source arrays (experts sharing memory dequantise
+    once; the arithmetic is unchanged).
 
     shared_fp8: optional (w13_q, w13_scale_inv, w2_q, w2_scale_inv) of the
     shared expert in FP8 with [128, 128] block scales ([2I, H], [2I/128,
@@ -245,9 +264,9 @@ def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
     counts, offsets, perm, inv, src = permute(idx, E, has_shared)
     xq_p, sx_p = gather_rows(xq, sx, src)
     if weights == "mxfp4":
-        gu = grouped_gemm_mxfp4(xq_p, sx_p, offsets, w13, w13_e8m0)
+        gu = grouped_gemm_mxfp4(xq_p, sx_p, offsets, w13, w13_e8m0, cache)
     else:
-        gu = grouped_gemm_w4afp8(xq_p, sx_p, offsets, w13_int4, w13_sinv)
+        gu = grouped_gemm_w4afp8(xq_p, sx_p, offsets, w13_int4, w13_sinv, cache)
     shared = shared_fp8 is not None and has_shared
     r0, r1 = (int(offsets[E]), int(offsets[E + 1])) if shared else (0, 0)
     if r1 > r0:      # the shared group with its FP8 weights
@@ -255,9 +274,9 @@ def moe_layer(x_bf16, logits, w13, w13_e8m0, w2, w2_e8m0, topk, route_scale=1.5,
             dequant_fp8_block128(shared_fp8[0], shared_fp8[1]).T
     hq, sh = swiglu_quant(gu, I, swiglu_limit)
     if weights == "mxfp4":
-        o = grouped_gemm_mxfp4(hq, sh, offsets, w2, w2_e8m0)
+        o = grouped_gemm_mxfp4(hq, sh, offsets, w2, w2_e8m0, cache)
     else:
-        o = grouped_gemm_w4afp8(hq, sh, offsets, w2_int4, w2_sinv)
+        o = grouped_gemm_w4afp8(hq, sh, offsets, w2_int4, w2_sinv, cache)
     if r1 > r0:
         o[r0:r1] = dequantize_fp8_pow2(hq[r0:r1], sh[r0:r1]) @ dequant_fp8_block128(shared_fp8[2], shared_fp8[3]).T
     y = combine(o, inv, w, offsets, has_shared)

@@ -207,6 +207,57 @@ class MoeWorkload:
     swiglu_limit: float = 10.0
 
 
+class RepeatedExperts:
+    """Read-only [E1, ...] view of per-expert arrays in which expert e holds
+    prototype e % n (the n_proto recipe of expert_weights) without copying:
+    indexing by an expert gives its prototype, a slice gives a stacked copy,
+    materialize() the whole array."""
+
+    def __init__(self, protos: np.ndarray, E1: int):
+        self.protos = protos
+        self.shape = (E1,) + protos.shape[1:]
+        self.dtype = protos.dtype
+        self.ndim = len(self.shape)
+
+    def __len__(self):
+        return self.shape[0]
+
+    def __getitem__(self, g):
+        n = len(self.protos)
+        if isinstance(g, (int, np.integer)):
+            if not -self.shape[0] <= g < self.shape[0]:
+                raise IndexError(g)
+            return self.protos[int(g) % self.shape[0] % n]
+        if isinstance(g, slice):
+            return self.protos[np.arange(self.shape[0])[g] % n]
+        raise TypeError("index an expert by int or slice")
+
+    def materialize(self) -> np.ndarray:
+        return self.protos[np.arange(self.shape[0]) % len(self.protos)]
+
+
+def expert_prototypes(seed: int, n: int, H: int, I: int, std: float = 0.02):
+    """The first n experts of expert_weights: MXFP4 w13 [n, 2I, H/2] + E8M0,
+    w2 [n, H, I/2] + E8M0, expert e from its own streams."""
+    w13 = np.empty((n, 2 * I, H // 2), np.uint8)
+    s13 = np.empty((n, 2 * I, H // 32), np.uint8)
+    w2 = np.empty((n, H, I // 2), np.uint8)
+    s2 = np.empty((n, H, I // 32), np.uint8)
+    for e in range(n):
+        a = normal(seed, 1000 + 2 * e, 2 * I * H).reshape(2 * I, H) * std
+        w13[e], s13[e] = quantize_mxfp4(a)
+        b = normal(seed, 1001 + 2 * e, H * I).reshape(H, I) * std
+        w2[e], s2[e] = quantize_mxfp4(b)
+    return w13, s13, w2, s2
+
+
+def expert_views(seed: int, E1: int, H: int, I: int, n_proto: int, std: float = 0.02):
+    """expert_weights(seed, E1, H, I, std, n_proto) as RepeatedExperts views
+    (the same values, drawn once per prototype, nothing repeated in memory)."""
+    protos = expert_prototypes(seed, min(E1, n_proto), H, I, std)
+    return tuple(RepeatedExperts(p, E1) for p in protos)
+
+
 def expert_weights(seed: int, E1: int, H: int, I: int, std: float = 0.02, n_proto: int | None = None):
     """MXFP4 w13 [E1, 2I, H] (w1 rows then w3 rows) and w2 [E1, H, I] from N(0, std).
 
@@ -215,19 +266,10 @@ def expert_weights(seed: int, E1: int, H: int, I: int, std: float = 0.02, n_prot
     memory, same values): full-size layers then take seconds to synthesise
     while every expert still streams its own bytes."""
     n_draw = E1 if n_proto is None else min(E1, n_proto)
-    w13 = np.empty((E1, 2 * I, H // 2), np.uint8)
-    s13 = np.empty((E1, 2 * I, H // 32), np.uint8)
-    w2 = np.empty((E1, H, I // 2), np.uint8)
-    s2 = np.empty((E1, H, I // 32), np.uint8)
-    for e in range(n_draw):
-        a = normal(seed, 1000 + 2 * e, 2 * I * H).reshape(2 * I, H) * std
-        w13[e], s13[e] = quantize_mxfp4(a)
-        b = normal(seed, 1001 + 2 * e, H * I).reshape(H, I) * std
-        w2[e], s2[e] = quantize_mxfp4(b)
-    for e in range(n_draw, E1):
-        p = e % n_draw
-        w13[e], s13[e], w2[e], s2[e] = w13[p], s13[p], w2[p], s2[p]
-    return w13, s13, w2, s2
+    protos = expert_prototypes(seed, n_draw, H, I, std)
+    if n_draw == E1:
+        return protos
+    return tuple(RepeatedExperts(p, E1).materialize() for p in protos)
 
 
 def tiny_layer(seed: int = 0) -> MoeWorkload:
@@ -243,12 +285,34 @@ def tiny_layer(seed: int = 0) -> MoeWorkload:
     return MoeWorkload("tiny", T, H, I, E, k, x, logits, w13, s13, w2, s2)
 
 
-def decode_activations(seed: int, T: int, H: int) -> np.ndarray:
-    """N(0,1) with each element scaled x20 with probability 0.001 (outliers)."""
-    x = normal(seed, 1, T * H)
-    out = uniform(seed, 3, T * H) < 0.001
+def _values_at(key: np.uint64, counters: np.ndarray) -> np.ndarray:
+    """Outputs at the given 0-based counters of the stream with this key."""
+    with np.errstate(over="ignore"):
+        z = np.asarray(counters, dtype=np.uint64) + np.uint64(1)
+        np.multiply(z, _GAMMA, out=z)
+        np.add(z, key, out=z)
+        return _mix(z)
+
+
+def decode_activations(seed: int, T: int, H: int, rows=None) -> np.ndarray:
+    """N(0,1) with each element scaled x20 with probability 0.001 (outliers).
+
+    rows: optional token indices; then only those rows of the [T, H] batch
+    are generated (the same values, from the same counters)."""
+    if rows is None:
+        x = normal(seed, 1, T * H)
+        out = uniform(seed, 3, T * H) < 0.001
+        x = np.where(out, 20.0 * x, x)
+        return to_bf16_bits(x.reshape(T, H))
+    rows = np.asarray(rows, dtype=np.int64)
+    i = (rows[:, None] * H + np.arange(H)[None, :]).reshape(-1)
+    k1 = _key(seed, 1)
+    u1 = (_values_at(k1, 2 * i) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    u2 = (_values_at(k1, 2 * i + 1) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    x = np.sqrt(-2.0 * np.log1p(-u1)) * np.cos(2.0 * np.pi * u2)
+    out = (_values_at(_key(seed, 3), i) >> np.uint64(11)).astype(np.float64) * (2.0 ** -53) < 0.001
     x = np.where(out, 20.0 * x, x)
-    return to_bf16_bits(x.reshape(T, H))
+    return to_bf16_bits(x.reshape(len(rows), H))
 
 
 def uniform_logits(seed: int, T: int, E: int) -> np.ndarray:

@@ -464,6 +464,49 @@ def test_w4afp8_random(lib, block_n):
     assert (np.abs(got - ref) <= 1024 * 2.0 ** -24 * bound + 1e-30).all()
 
 
+@pytest.mark.parametrize("block_n", [16, 32])
+def test_w4afp8_offset_codes_zero_weight_groups(lib, block_n):
+    """Token tiles of at most 32 rows run the MMA on the offset codes u = q + 8
+    and subtract 8 x the row's activation sum, so an all-zero INT4 group
+    (scale_inv 1.0, the repack's rule for a zero group) leaves a float32
+    residue instead of an exact 0.  The bound follows the MMA's magnitudes:
+    |gpu - oracle| <= 1024 * 2^-24 * sum_g scale_inv[n, g] * sum_{k in g}
+    |a_k| 2^(sa-127) (|q_nk| + 8), the test_w4afp8_random allowance with |q|
+    replaced by |u| <= |q| + 8; for rows whose every group is zero the oracle
+    is exactly 0 and the bound is 1024 * 2^-24 * 8 * sum |a| 2^(sa-127).
+    Inputs: rows with large activation scales, rows of E4M3 subnormal codes,
+    a weight row block zero in every group and one zero in a single group."""
+    N, K = 256, 512
+    sizes = [16, 3, 29, 1]
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    Rn, G = int(offsets[-1]), len(sizes)
+    a = synth.random_e4m3(31, 1, (Rn, K))
+    a[3:9] = synth.random_bytes(31, 2, (6, K), 0, 7) | (synth.random_bytes(31, 3, (6, K), 0, 1) << 7)  # subnormals
+    asc = synth.random_bytes(31, 4, (Rn, K // 128), 120, 134)
+    asc[10:14] = 150                                                  # large |x| rows
+    q = synth.random_bytes(31, 5, (G, N, K // 2)).view(np.int8).copy()
+    sinv = (synth.uniform(31, 6, G * N * (K // 128)) * 0.01 + 1e-4).astype(np.float32).reshape(G, N, K // 128)
+    q[0, :64] = 0                                                     # every group of rows 0..63 zero
+    sinv[0, :64] = 1.0
+    q[2, 100:130, 128:192] = 0                                        # K group 2 of rows 100..129 zero
+    sinv[2, 100:130, 2] = 1.0
+    out, _ = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, block_n)
+    ref = ffn.grouped_gemm_w4afp8(a, asc, offsets, q, sinv)
+    assert (ref[0:16, :64] == 0).all()
+    av = np.abs(Q.dequantize_fp8_pow2(a, asc))
+    qv = np.abs(ffn.dequant_int4g128(q, np.ones_like(sinv)))            # |q| per element
+    bound = np.zeros_like(ref)
+    for g in range(G):
+        r0, r1 = offsets[g], offsets[g + 1]
+        for kg in range(K // 128):
+            ks = slice(128 * kg, 128 * kg + 128)
+            bound[r0:r1] += (av[r0:r1, ks] @ (qv[g][:, ks] + 8.0).T) * sinv[g][:, kg].astype(np.float64)[None, :]
+    bound *= 1024 * 2.0 ** -24
+    got = out.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= bound).all(), np.max(np.abs(got - ref) / np.maximum(bound, 1e-300))
+    no_device_error(lib)
+
+
 def test_w4afp8_swiglu_epilogue_matches_standalone(lib):
     I = 256
     a, asc, offsets, q, sinv = _w4a_inputs(10, [5, 0, 33, 70], 2 * I, 512, False)

@@ -6,7 +6,8 @@ Tolerance (the layer's floating-point output): max |gpu - oracle| <=
 Intermediates that are integer decisions on exact data (quantised x, routing
 indices, grouping) must match bit for bit.  At full sizes the oracle
 evaluates a seeded sample of tokens; token outputs are independent given the
-routing, so the sample is exact.
+routing, so the sample is exact.  The benchmark's full-size MXFP4 and W4AFP8
+layers are checked in test_gpu_full_size.py.
 """
 import numpy as np
 import pytest
@@ -54,28 +55,6 @@ def test_layer_deterministic(lib):
     np.testing.assert_array_equal(y1, y2)
 
 
-def _full_size(T, logits_fn, E=256, n_proto=4, sample=12, seed=0):
-    H, I, k = 4096, 2048, 6
-    w13, s13, w2, s2 = synth.expert_weights(seed, E + 1, H, I, n_proto=n_proto)
-    x = synth.decode_activations(seed, T, H)
-    logits = logits_fn(seed, T, E)
-    layer, buf, y = run_layer(x, logits, w13, s13, w2, s2, k)
-    toks = np.sort((synth.splitmix64(seed, 77, sample) % np.uint64(T)).astype(np.int64))
-    ref = ffn.moe_layer(x, logits, w13, s13, w2, s2, k, tokens=toks)
-    np.testing.assert_array_equal(buf.idx.cpu().numpy()[toks], ref["idx"])
-    check_y(y[toks], ref["y"])
-
-
-def test_decode_layer_full_size(lib):
-    """Hidden 4096, intermediate 2048, 256 routed + 1 shared, top-6, 64 tokens."""
-    _full_size(64, synth.uniform_logits)
-
-
-def test_prefill_layer_full_size(lib):
-    """Same shapes, 4096 tokens with Zipf(1.1) expert loads."""
-    _full_size(4096, synth.zipf_logits, sample=8)
-
-
 def _w4a_ref(x, logits, w13, s13, w2, s2, k, tokens=None, n_proto=None):
     """Oracle W4AFP8 layer: the oracle's INT4 repack of the experts, then its FFN.
     With n_proto set (expert e holds the values of expert e % n_proto) only
@@ -112,21 +91,6 @@ def test_tiny_layer_w4afp8(lib, block_n):
     ref = _w4a_ref(wl.x_bf16, wl.logits, wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
     check_y(y.float().cpu().numpy(), ref["y"])
     assert lib.moe_get_device_error() == 0
-
-
-def test_long_prefill_w4afp8_sampled(lib):
-    """Hidden 4096, intermediate 2048, 384 routed + 1 shared, top-6, 16384 tokens
-    with Zipf loads, W4AFP8 path; sampled tokens against the oracle."""
-    T, H, I, E, k = 16384, 4096, 2048, 384, 6
-    w13, s13, w2, s2 = synth.expert_weights(0, E + 1, H, I, n_proto=2)
-    x = synth.decode_activations(0, T, H)
-    logits = synth.zipf_logits(0, T, E)
-    layer = MoeLayer(w13, s13, w2, s2, k, weights="w4afp8")
-    buf = layer.alloc(T)
-    y = layer.forward(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(logits).cuda(), buf)
-    toks = np.sort((synth.splitmix64(0, 78, 4) % np.uint64(T)).astype(np.int64))
-    ref = _w4a_ref(x, logits, w13, s13, w2, s2, k, tokens=toks, n_proto=2)
-    check_y(y.float().cpu().numpy()[toks], ref["y"])
 
 
 @pytest.mark.parametrize("shared", ["mxfp4", "fp8"])

@@ -274,3 +274,18 @@ def test_ptpc_weights_per_output_channel():
     assert (np.abs(F.decode_e4m3(q[0])).max(axis=1) == 448.0).all()
     back = F.decode_e4m3(q[0]) * s[0][:, None].astype(np.float64)
     assert (np.abs(back - w) <= np.maximum(2.0 ** -4 * np.abs(w), 2.0 ** -10 * s[0][:, None])).all()
+
+
+def test_dequant_cache_changes_no_value():
+    """The optional dequantisation memo gives the uncached result bit for bit,
+    on experts that share memory (repeated prototypes) and on distinct ones."""
+    wl = synth.tiny_layer(8)
+    views = synth.expert_views(8, wl.E + 1, wl.H, wl.I, n_proto=3)
+    full = [v.materialize() for v in views]
+    cache = {}
+    a = ffn.moe_layer(wl.x_bf16, wl.logits, *views, wl.topk, cache=cache)
+    b = ffn.moe_layer(wl.x_bf16, wl.logits, *full, wl.topk)
+    np.testing.assert_array_equal(a["y"], b["y"])
+    assert 0 < len(cache) <= 6            # at most 3 prototypes x (w13, w2)
+    c = ffn.moe_layer(wl.x_bf16, wl.logits, *full, wl.topk, cache={})
+    np.testing.assert_array_equal(c["y"], b["y"])

@@ -49,3 +49,19 @@ def test_hash_table_rows_distinct_and_in_range():
     np.testing.assert_array_equal(t, synth.hash_table(0, 2000, 256, 6))
     ids = synth.token_ids(0, 1000, 2000)
     assert ids.dtype == np.int32 and ids.min() >= 0 and ids.max() < 2000
+
+
+def test_activation_rows_equal_full_batch_rows():
+    full = synth.decode_activations(5, 40, 256)
+    rows = np.array([0, 17, 39, 17])
+    np.testing.assert_array_equal(synth.decode_activations(5, 40, 256, rows=rows), full[rows])
+
+
+def test_repeated_expert_views_equal_repeated_arrays():
+    full = synth.expert_weights(1, 7, 256, 128, n_proto=3)
+    views = synth.expert_views(1, 7, 256, 128, n_proto=3)
+    for f, v in zip(full, views):
+        assert v.shape == f.shape
+        np.testing.assert_array_equal(v.materialize(), f)
+        np.testing.assert_array_equal(v[5], f[5])
+        np.testing.assert_array_equal(v[2:6], f[2:6])
