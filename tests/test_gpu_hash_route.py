@@ -57,7 +57,7 @@ def test_route_hash_rejects_out_of_range_ids(lib):
     s = R.sqrtsoftplus(z[2, [table[5, 0], table[5, 2]]])
     np.testing.assert_allclose(ww[2, [0, 2]], 1.5 * s / s.sum(), rtol=1e-6)
     for t, v in ((0, 0), (3, 3)):
-        i_ref, w_ref = R.route_hash(np.array([v]), table[[v]].clip(0, E - 1), z[[t]])
+        i_ref, w_ref = R.route_hash(np.array([0]), table[[v]], z[[t]])
         assert i[t].tolist() == i_ref[0].tolist()
         np.testing.assert_allclose(ww[t], w_ref[0], rtol=1e-6)
     assert lib.moe_get_device_error() == 0            # the word was cleared by the read
