@@ -41,6 +41,7 @@ SIGNATURES = {
     "moe_prepared_weights_size": (_SZ, [_I64, _I, _I]),
     "moe_prepare_weights": (_I, [_P, _P, _I64, _I, _I, _I, _P, _P]),
     "moe_gemm_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "moe_w4afp8_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_grouped_gemm_mxfp4": (_I, [_P, _P, _I, _P, _I, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_grouped_gemm_w4afp8": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),
     "moe_grouped_gemm_fp8_block128": (_I, [_P, _P, _I, _P, _I, _P, _P, _I, _I, _I, _F, _I, _P, _P, _P, _SZ, _P]),

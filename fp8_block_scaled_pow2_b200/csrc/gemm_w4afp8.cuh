@@ -131,7 +131,10 @@ struct W4Args {
   float limit;
 };
 
-template <int BN, bool DUAL, int EPI, bool W8 = false>
+// ROWS (with W8): E4M3 weights with the INT4 layout's per-row scales
+// [G, N, K/128] -- the E4M3 copy of INT4 weights that transcode_int4_kernel
+// writes once per call for wide token tiles.
+template <int BN, bool DUAL, int EPI, bool W8 = false, bool ROWS = false>
 __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     gemm_w4afp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const W4Args args) {
@@ -328,12 +331,14 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
       const int rb_per_g = N / 128;
-      // scale_inv of this thread's weight row per K step: [G, N, K/128] (INT4,
-      // per row) or [G, N/128, K/128] (FP8, one value per 128-row block)
-      const float* s0 = args.w_sinv + (W8 ? (size_t)(it.g * rb_per_g + it.ft) * KT
-                                          : ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT);
-      const float* s1 = args.w_sinv + (W8 ? (size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * KT
-                                          : ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT);
+      // scale_inv of this thread's weight row per K step: [G, N, K/128] (INT4
+      // and its E4M3 copy, per row) or [G, N/128, K/128] (FP8, one value per
+      // 128-row block)
+      constexpr bool BLOCK_SCALE = W8 && !ROWS;
+      const float* s0 = args.w_sinv + (BLOCK_SCALE ? (size_t)(it.g * rb_per_g + it.ft) * KT
+                                                   : ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT);
+      const float* s1 = args.w_sinv + (BLOCK_SCALE ? (size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * KT
+                                                   : ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT);
       float acc0[BN], acc1[DUAL ? BN : 1];
 #pragma unroll
       for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
@@ -447,6 +452,36 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// INT4 [G, N, K/2] -> E4M3 [G, N, K] (the exact codes of -8..7), once per
+// call, for the wide-token-tile path: the GEMM then streams E4M3 tiles with
+// TMA instead of transcoding every weight tile once per token tile.  Grid
+// (chunks of 256 x 16 input bytes, G); groups without rows (offsets[g + 1] <=
+// offsets[g]) are skipped, their copy is never read.  Offsets are only read
+// here; the plan kernel validates them.
+__global__ void __launch_bounds__(256) transcode_int4_kernel(const uint4* __restrict__ q,
+                                                             const int32_t* __restrict__ offsets,
+                                                             int64_t chunks_per_group, uint4* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  const int g = blockIdx.y;
+  if (__ldg(offsets + g + 1) <= __ldg(offsets + g)) return;
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= chunks_per_group) return;
+  const int64_t i = (int64_t)g * chunks_per_group + c;
+  const uint4 in = __ldg(q + i);
+  uint4 o0, o1;
+  o0.x = int4x4_to_e4m3x4(in.x, 0);
+  o0.y = int4x4_to_e4m3x4(in.x, 16);
+  o0.z = int4x4_to_e4m3x4(in.y, 0);
+  o0.w = int4x4_to_e4m3x4(in.y, 16);
+  o1.x = int4x4_to_e4m3x4(in.z, 0);
+  o1.y = int4x4_to_e4m3x4(in.z, 16);
+  o1.z = int4x4_to_e4m3x4(in.w, 0);
+  o1.w = int4x4_to_e4m3x4(in.w, 16);
+  out[2 * i] = o0;
+  out[2 * i + 1] = o1;
 }
 
 }  // namespace w4a

@@ -124,19 +124,30 @@ int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const g
   }
 }
 
-template <int BN, bool DUAL, int EPI, bool W8>
+template <int BN, bool DUAL, int EPI, bool W8, bool ROWS = false>
 int launch_w4a(const CUtensorMap& ta, const CUtensorMap& tb, const w4a::W4Args& a, cudaStream_t st) {
   using C = w4a::Cfg<BN, DUAL, W8>;
-  auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI, W8>;
+  auto k = w4a::gemm_w4afp8_kernel<BN, DUAL, EPI, W8, ROWS>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
   launch(k, dim3(sm_count()), dim3(C::THREADS), C::SMEM_ALLOC, st, ta, tb, a);
   return launch_status();
 }
 
+// Bytes of the E4M3 copy of INT4 weights [G, N, K/2] that the W4AFP8 GEMM
+// writes into its workspace (after the plan) for token tiles of 64 rows or
+// more.
+size_t w4a_scratch_bytes(int G, int N, int K) { return gemm::align256((size_t)G * N * K); }
+
+bool w4a_uses_scratch(int block_n) { return block_n >= 64; }
+
 // Grouped GEMM whose weight scale is applied by promotion warps: INT4 group-128
-// weights (W8 = false, transcoded to E4M3 in shared memory) or FP8 E4M3 weights
-// with [128, 128] block scales (W8 = true).
+// weights (W8 = false) or FP8 E4M3 weights with [128, 128] block scales (W8 =
+// true).  INT4 on token tiles of 64 rows or more, when the workspace holds
+// w4a_scratch_bytes after the plan: transcoded once per call to an E4M3 copy
+// in the workspace, then streamed like FP8 weights with per-row scales;
+// otherwise transcoded to E4M3 in shared memory, once per weight tile and
+// token tile.
 template <bool W8>
 int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets, int n_groups,
                   const void* w, const float* w_scale_inv, int N, int K, int epilogue, float swiglu_limit, int block_n,
@@ -155,13 +166,17 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
     return MOE_ERR_INVALID;
   const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
+  const bool scratch = !W8 && w4a_uses_scratch(block_n) &&
+                       workspace_bytes >= L.total + w4a_scratch_bytes(n_groups, N, K);
+  uint8_t* e4m3_copy = scratch ? reinterpret_cast<uint8_t*>(workspace) + L.total : nullptr;
   CUtensorMap ta, tb;
-  // INT4: raw [rows, K/2] tiles of 64 x 128 bytes; FP8: [rows, K] tiles of 128 x 128 bytes
-  // written straight into the 128-byte-swizzled MMA layout
-  if (W8 ? !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K, (uint64_t)n_groups * N, (uint64_t)K, 128,
-                     128)
-         : !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K / 2, (uint64_t)n_groups * N,
-                     (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+  // INT4: raw [rows, K/2] tiles of 64 x 128 bytes; FP8 (and the E4M3 copy of
+  // INT4): [rows, K] tiles of 128 x 128 bytes written straight into the
+  // 128-byte-swizzled MMA layout
+  if ((W8 || scratch) ? !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, scratch ? e4m3_copy : w, (uint64_t)K,
+                                  (uint64_t)n_groups * N, (uint64_t)K, 128, 128)
+                      : !make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)K / 2, (uint64_t)n_groups * N,
+                                  (uint64_t)K / 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
     return MOE_ERR_LAUNCH;
   if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
                 (uint32_t)block_n))
@@ -191,6 +206,18 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
       reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, a_e4m3, a_corr);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  if (scratch) {
+    const int64_t chunks = (int64_t)N * K / 32;     // 16 input bytes (32 INT4) per thread
+    launch(w4a::transcode_int4_kernel, dim3((unsigned)((chunks + 255) / 256), (unsigned)n_groups), dim3(256), 0, st,
+           reinterpret_cast<const uint4*>(w), offsets, chunks, reinterpret_cast<uint4*>(e4m3_copy));
+    if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+    if (dual) return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT, true, true>(ta, tb, args, st);
+    if (epilogue == MOE_EPI_STORE_F32)
+      return block_n == 64 ? launch_w4a<64, false, MOE_EPI_STORE_F32, true, true>(ta, tb, args, st)
+                           : launch_w4a<128, false, MOE_EPI_STORE_F32, true, true>(ta, tb, args, st);
+    return block_n == 64 ? launch_w4a<64, false, MOE_EPI_STORE_BF16, true, true>(ta, tb, args, st)
+                         : launch_w4a<128, false, MOE_EPI_STORE_BF16, true, true>(ta, tb, args, st);
+  }
   if (dual) {
     switch (block_n) {
       case 16: return launch_w4a<16, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
@@ -394,6 +421,20 @@ size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n) {
   return gemm::ws_layout(a_rows, n_groups, K, block_n).total;
 }
 
+size_t moe_w4afp8_workspace_size(int a_rows, int n_groups, int N, int K, int block_n) {
+  if (a_rows < 0 || n_groups <= 0 || N <= 0 || K <= 0) return 0;
+  size_t plan = 0;
+  if (block_n == 0) {
+    // the call caps its own choice at 64 rows for the SwiGLU epilogue: cover
+    // the plan of every tile width it may pick
+    for (int bn : {16, 32, 64, 128}) plan = std::max(plan, gemm::ws_layout(a_rows, n_groups, K, bn).total);
+    block_n = pick_block_n(a_rows, n_groups);
+  } else {
+    plan = gemm::ws_layout(a_rows, n_groups, K, block_n).total;
+  }
+  return plan + (w4a_uses_scratch(block_n) ? w4a_scratch_bytes(n_groups, N, K) : 0);
+}
+
 size_t moe_workspace_size(const MoeConfig* cfg, int path) {
   if (!cfg || path < MOE_PATH_MXFP4 || path > MOE_PATH_PTPC) return 0;
   const MoeConfig& c = *cfg;
@@ -405,6 +446,10 @@ size_t moe_workspace_size(const MoeConfig* cfg, int path) {
   size_t need = moe_permute_workspace_size(c.T, c.E, c.topk);
   for (int bn : {16, 32, 64, 128})
     for (int K : {c.H, c.I}) need = std::max(need, moe_gemm_workspace_size((int)R, G, K, bn));
+  if (path == MOE_PATH_W4AFP8) {   // the E4M3 copy of the weights for wide token tiles
+    need = std::max(need, moe_w4afp8_workspace_size((int)R, G, 2 * c.I, c.H, 0));
+    need = std::max(need, moe_w4afp8_workspace_size((int)R, G, c.H, c.I, 0));
+  }
   return (need + 255) / 256 * 256;
 }
 

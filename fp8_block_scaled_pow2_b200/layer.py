@@ -169,6 +169,10 @@ class MoeLayer:
         # the W4AFP8 w1/w3 GEMM may use narrower token tiles than block_n
         bns = (block_n, 16) if (self.weights in ("w4afp8", "ptpc") or self.shared == "fp8") else (block_n,)
         ws_g = max([moe.moe_gemm_workspace_size(R, self.G, K, bn) for bn in bns for K in (H, I)] + [256])
+        if self.weights == "w4afp8":
+            # room for the E4M3 copy of the INT4 weights that wide token tiles stream
+            ws_g = max([ws_g] + [moe.moe_w4afp8_workspace_size(R, self.GR, N, K, bn) for bn in bns
+                                 for N, K in ((2 * I, H), (H, I))])
         return Buffers(
             T=T,
             xq=torch.empty((T, H), dtype=u8, device=d), sx=torch.empty((T, H // 128), dtype=u8, device=d),

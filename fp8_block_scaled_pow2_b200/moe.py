@@ -140,6 +140,10 @@ def moe_gemm_workspace_size(a_rows: int, n_groups: int, K: int, block_n: int = 0
     return int(_lib().moe_gemm_workspace_size(a_rows, n_groups, K, block_n))
 
 
+def moe_w4afp8_workspace_size(a_rows: int, n_groups: int, N: int, K: int, block_n: int = 0) -> int:
+    return int(_lib().moe_w4afp8_workspace_size(a_rows, n_groups, N, K, block_n))
+
+
 def moe_grouped_gemm_mxfp4(a, a_scale, offsets, w_prepared, G, N, epilogue, out, out_scale=None,
                            workspace=None, swiglu_limit=10.0, block_n=0, stream=None):
     """w_prepared: moe_prepare_weights output for G matrices [N, K] (K = a.shape[1])."""

@@ -278,7 +278,8 @@ typedef struct {
  * Scratch bytes of one layer step (host call, no CUDA call): one buffer of
  * this size, 256-byte aligned, can serve as the `workspace` of moe_permute
  * and of every grouped GEMM of the step (w1/w3 and w2, any block_n), since
- * they run in order on one stream.  path: MOE_PATH_MXFP4, MOE_PATH_W4AFP8 or
+ * they run in order on one stream; for MOE_PATH_W4AFP8 it includes the E4M3
+ * weight copy of moe_w4afp8_workspace_size.  path: MOE_PATH_MXFP4, MOE_PATH_W4AFP8 or
  * MOE_PATH_PTPC.  Returns 0 for a NULL or invalid configuration (T < 0,
  * H or I not a positive multiple of 128, E < 1, topk < 1 or > E, unknown
  * path).
@@ -310,8 +311,16 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
  *   w_int4       int8 [G, N, K/2] (16-byte aligned); w_scale_inv float32 [G, N, K/128]
  *   other arguments, layouts and epilogues as moe_grouped_gemm_mxfp4;
  *   block_n: 16, 32, 64 (SWIGLU_QUANT) or up to 128 (STORE_F32 / STORE_BF16);
- *   workspace: moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
+ *   workspace: at least moe_gemm_workspace_size(a_rows, G, K, block_n) bytes.
+ *   Token tiles of 64 rows or more, given the larger workspace that
+ *   moe_w4afp8_workspace_size(a_rows, G, N, K, block_n) returns: the call
+ *   first writes an E4M3 copy of the INT4 weights of every group that has
+ *   rows (G * N * K bytes, after the plan) and the GEMM streams that copy,
+ *   instead of transcoding each weight tile in shared memory once per token
+ *   tile.  The arithmetic is the same (exact E4M3 codes of q, unit weight
+ *   scale slots, the same promotion), so both give the same result.
  */
+size_t moe_w4afp8_workspace_size(int a_rows, int n_groups, int N, int K, int block_n);
 int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows,
                             const int32_t* offsets, int n_groups,
                             const int8_t* w_int4, const float* w_scale_inv, int N, int K,

@@ -96,3 +96,18 @@ def test_layer_workspace_size_without_gpu():
     assert moe.moe_workspace_size(T, H, I, E, 7, path=3) == 0      # unknown path
     assert moe.moe_workspace_size(T, H, I, 4, 6) == 0              # topk > E
     assert moe.moe_workspace_size(0, H, I, E, k) > 0               # empty batch still valid
+
+
+def test_w4afp8_workspace_sizes_without_gpu():
+    """The E4M3 weight copy is G * N * K bytes on top of the plan for token
+    tiles of 64 rows or more, nothing for narrower ones; the layer's W4AFP8
+    workspace covers the copy of w1/w3 [2I, H] and of w2 [H, I]."""
+    from fp8_block_scaled_pow2_b200 import moe
+    plan = moe.moe_gemm_workspace_size(1000, 9, 4096, 64)
+    assert moe.moe_w4afp8_workspace_size(1000, 9, 4096, 4096, 64) == plan + 9 * 4096 * 4096
+    assert moe.moe_w4afp8_workspace_size(1000, 9, 4096, 4096, 32) == moe.moe_gemm_workspace_size(1000, 9, 4096, 32)
+    T, H, I, E, k = 16384, 4096, 2048, 384, 6
+    R, G = T * k + T, E + 1
+    ws = moe.moe_workspace_size(T, H, I, E, k, path=moe.MOE_PATH_W4AFP8)
+    assert ws >= moe.moe_w4afp8_workspace_size(R, G, 2 * I, H, 0) >= G * 2 * I * H
+    assert moe.moe_workspace_size(T, H, I, E, k, path=moe.MOE_PATH_MXFP4) < G * 2 * I * H

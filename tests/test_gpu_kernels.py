@@ -412,15 +412,21 @@ def _w4a_inputs(seed, sizes, N, K, integer):
     return a, asc, offsets, q, sinv
 
 
-def _run_w4a(lib, a, asc, offsets, q, sinv, epi, block_n):
+def _run_w4a(lib, a, asc, offsets, q, sinv, epi, block_n, scratch=False):
+    """scratch: size the workspace for the E4M3 weight copy (token tiles of
+    64 rows or more then stream it); otherwise the plan alone (every tile
+    transcoded in shared memory)."""
     G, N, K = q.shape[0], q.shape[1], q.shape[2] * 2
     Rn = a.shape[0]
-    ws = torch.empty(max(lib.moe_gemm_workspace_size(Rn, G, K, block_n), 256), dtype=torch.uint8, device="cuda")
+    size = (lib.moe_w4afp8_workspace_size(Rn, G, N, K, block_n) if scratch
+            else lib.moe_gemm_workspace_size(Rn, G, K, block_n))
+    ws = torch.full((max(size, 256),), 0xA5, dtype=torch.uint8, device="cuda")
     if epi == lib.MOE_EPI_SWIGLU_QUANT:
-        out = torch.empty((Rn, N // 2), dtype=torch.uint8, device="cuda")
-        osc = torch.empty((Rn, N // 256), dtype=torch.uint8, device="cuda")
+        out = torch.zeros((Rn, N // 2), dtype=torch.uint8, device="cuda")
+        osc = torch.zeros((Rn, N // 256), dtype=torch.uint8, device="cuda")
     else:
-        out, osc = torch.empty((Rn, N), dtype=torch.float32, device="cuda"), None
+        dt = torch.bfloat16 if epi == lib.MOE_EPI_STORE_BF16 else torch.float32
+        out, osc = torch.zeros((Rn, N), dtype=dt, device="cuda"), None
     lib.moe_grouped_gemm_w4afp8(dev(a), dev(asc), dev(offsets), dev(q), dev(sinv), epi, out, osc, ws, 10.0, block_n)
     torch.cuda.synchronize()
     return out, osc
@@ -504,6 +510,26 @@ def test_w4afp8_offset_codes_zero_weight_groups(lib, block_n):
     bound *= 1024 * 2.0 ** -24
     got = out.cpu().numpy().astype(np.float64)
     assert (np.abs(got - ref) <= bound).all(), np.max(np.abs(got - ref) / np.maximum(bound, 1e-300))
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("block_n,epi", [(64, 2), (64, 0), (128, 0), (128, 1)])
+def test_w4afp8_e4m3_copy_path(lib, block_n, epi):
+    """Wide token tiles with a workspace that holds the E4M3 weight copy:
+    the result equals the in-shared-memory transcode bit for bit (the same
+    codes, scales and promotion order), on random scaled data with empty and
+    ragged groups; integer-exact inputs equal the oracle bit for bit."""
+    N = 512
+    a, asc, offsets, q, sinv = _w4a_inputs(14, [70, 0, 129, 1, 300, 64], N, 1024, False)
+    got, gsc = _run_w4a(lib, a, asc, offsets, q, sinv, epi, block_n, scratch=True)
+    ref, rsc = _run_w4a(lib, a, asc, offsets, q, sinv, epi, block_n, scratch=False)
+    assert torch.equal(got.view(torch.uint8), ref.view(torch.uint8))
+    if gsc is not None:
+        assert torch.equal(gsc, rsc)
+    if epi == lib.MOE_EPI_STORE_F32:
+        ai, aa, ao, aq, asv = _w4a_inputs(15, [5, 0, 130, 64], N, 512, True)
+        out, _ = _run_w4a(lib, ai, aa, ao, aq, asv, epi, block_n, scratch=True)
+        np.testing.assert_array_equal(out.cpu().numpy(), ffn.grouped_gemm_w4afp8(ai, aa, ao, aq, asv).astype(np.float32))
     no_device_error(lib)
 
 
