@@ -511,7 +511,7 @@ def bench_layer(args, name: str, weights: str, shared: str, steps: int, warmup: 
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     T = wl["T"]
-    buf = layer.alloc(T)
+    buf = layer.alloc(T, args.block_n)
     xd = torch.from_numpy(x.view(np.int16)).cuda()
     ld = torch.from_numpy(logits).cuda()
     stream = torch.cuda.current_stream()
@@ -584,7 +584,7 @@ def bench_layer(args, name: str, weights: str, shared: str, steps: int, warmup: 
         # region; StepRunner overlaps those copies with the neighbouring steps'
         # compute on a second stream
         from fp8_block_scaled_pow2_b200.runner import StepRunner, pinned_inputs
-        runner = StepRunner(layer, T, graphs=use_graph)
+        runner = StepRunner(layer, T, block_n=args.block_n, graphs=use_graph)
         xh, lh, yh = pinned_inputs(x, logits)
         for _ in range(max(1, warmup)):
             runner.submit(xh, lh, yh)
@@ -857,6 +857,8 @@ def main(argv=None):
                     help="shared expert weights: MXFP4 (group E of the grouped GEMM) or FP8 [128, 128] blocks")
     ap.add_argument("--graph", choices=["on", "off"], default="on",
                     help="replay the layer step as four CUDA graphs (off: eager library calls)")
+    ap.add_argument("--block-n", type=int, default=0,
+                    help="token rows per GEMM tile (0: the library's choice)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extras", choices=["default", "none"], default="default",

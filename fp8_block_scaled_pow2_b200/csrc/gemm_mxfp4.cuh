@@ -120,6 +120,9 @@ struct Cfg {
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
   static_assert(SMEM_ALLOC > 116 * 1024, "one CTA per SM keeps tensor-memory allocation uncontended");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "bad token tile");
+  // epilogue loads of 16 (or, for CW = 8, 8) columns start on a multiple of
+  // their width: each warp's column slice starts at a multiple of CW
+  static_assert(CW == 8 || CW % 16 == 0, "epilogue column slices must be whole 16-column loads");
 };
 
 // ----------------------- plan (work decomposition) -------------------------
@@ -381,10 +384,11 @@ __device__ __forceinline__ void epilogue_item(const Item& it, uint32_t src, int 
   const bool use_v1 = PAIR || KT > 1;
   uint32_t v0[CW];
   uint32_t v1[CW];
+  // 16-column loads, and an 8-column load for a remainder (CW % 16 == 8)
 #pragma unroll
-  for (int c = 0; c < CW; c += (CW >= 16 ? 16 : 8)) {
+  for (int c = 0; c < CW; c += (c + 16 <= CW ? 16 : 8)) {
     if (c < my_cols) {
-      if constexpr (CW >= 16) {
+      if (c + 16 <= CW) {
         tmem_ld16(src + c, *reinterpret_cast<uint32_t(*)[16]>(v0 + c));
         if (use_v1) tmem_ld16(src + BN + c, *reinterpret_cast<uint32_t(*)[16]>(v1 + c));
       } else {

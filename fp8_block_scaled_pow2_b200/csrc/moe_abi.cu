@@ -462,7 +462,8 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
   if (epilogue == MOE_EPI_SWIGLU_QUANT && N % 256) return MOE_ERR_INVALID;
   if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
-  if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128) return MOE_ERR_UNSUPPORTED;
+  if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128)
+    return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_prepared || !out || !workspace) return MOE_ERR_INVALID;
   if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_scale) return MOE_ERR_INVALID;
