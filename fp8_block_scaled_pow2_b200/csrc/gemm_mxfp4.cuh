@@ -44,7 +44,9 @@ namespace gemm {
 
 using namespace sm100;
 
-constexpr int kThreads = 352;                   // 11 warps: producer, 2 MMA issuers, 8 workers
+constexpr int kThreads = 384;                   // 12 warps: producer, 2 MMA issuers, 8 workers, L2 prefetcher
+constexpr int kIssuer1Warp = 10;
+constexpr int kPrefetchWarp = 11;
 
 // Prepared weights (moe_prepare_weights): one 8704-byte block per (128-row
 // block, 128-wide K step): 128 rows x 64 bytes of packed E2M1 nibbles, then
@@ -116,7 +118,7 @@ struct Cfg {
   static constexpr int SMEM_ALLOC = SMEM_USED + 1024;     // slack for 1024-byte alignment
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few pipeline stages");
-  static_assert(2 * STAGES + 4 + 1 <= 64, "barrier area overflow");
+  static_assert(2 * STAGES + 4 + 2 <= 64, "barrier area overflow");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
   static_assert(SMEM_ALLOC > 116 * 1024, "one CTA per SM keeps tensor-memory allocation uncontended");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "bad token tile");
@@ -365,6 +367,7 @@ struct GemmArgs {
   void* out;
   uint8_t* out_scale;
   float limit;
+  int pf_steps;            // K steps the L2 prefetcher runs ahead of the producer (0: off)
 };
 
 // Epilogue of one work item for one epilogue warp: copy the warp's slice of
@@ -537,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;           // [ACC_BUFS]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* produced = reinterpret_cast<volatile int*>(tmem_slot + 2);   // K steps issued so far
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
   SmemPlan plan(smem + C::PLAN_OFF);
 
@@ -556,6 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], 32 * C::EPI_WARPS);
     }
     *abort_flag = 0;
+    *produced = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
@@ -611,17 +616,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
+          *produced = *produced + 1;
         }
         __syncwarp();
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
     }
+  } else if (warp == kPrefetchWarp) {
+    // ------------------------------ L2 prefetcher --------------------------
+    // Walks the producer's sequence of K steps pf_steps ahead of it and
+    // prefetches each step's weight blocks and token tile into L2, so more of
+    // the HBM stream is in flight than the shared-memory ring holds.  A hint
+    // only: it gives up quietly when the CTA aborts or after the wait bound.
+    if (args.pf_steps > 0 && lane == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      int pf = 0;
+      bool go = true;
+      for (int item = blockIdx.x; item < n_items && go; item += gridDim.x) {
+        const Item it = decode_item(item, plan, G, n_ft, BN);
+        size_t blk0, kt_step, a_step;
+        if (PAIRED_ORDER) {
+          blk0 = (size_t)(it.g * n_ft + it.ft) * KT * 2;
+          kt_step = 2;
+          a_step = 1;
+        } else {
+          blk0 = (size_t)(it.g * rb_per_g + (PAIR ? 2 * it.ft : it.ft)) * KT;
+          kt_step = 1;
+          a_step = KT;
+        }
+        for (int kt = 0; kt < KT && go; ++kt) {
+          while (pf >= *produced + args.pf_steps) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitTimeoutNs) { go = false; break; }
+            __nanosleep(128);
+          }
+          if (!go) break;
+          const size_t blk = blk0 + (size_t)kt * kt_step;
+          if (PAIRED_ORDER) {
+            bulk_prefetch(args.w + blk * kWBlock, 2 * kWBlock);
+          } else {
+#pragma unroll
+            for (int a = 0; a < C::NUM_A; ++a) bulk_prefetch(args.w + (blk + (size_t)a * a_step) * kWBlock, kWBlock);
+          }
+          tma_prefetch_2d(&tmB, kt * 128, it.row0);
+          ++pf;
+        }
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer 0 ---------------------------
     mma_issuer<BN, PAIR>(0, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
                          n_items, KT, n_ft);
-  } else if (warp == kThreads / 32 - 1) {
+  } else if (warp == kIssuer1Warp) {
     // ------------------------------ MMA issuer 1 ---------------------------
     mma_issuer<BN, PAIR>(1, smem, tmem, full, empty, acc_full, acc_empty, abort_flag, plan, args,
                          n_items, KT, n_ft);

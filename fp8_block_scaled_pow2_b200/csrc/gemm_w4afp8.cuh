@@ -28,7 +28,9 @@
 //     -8..7, unit weight scales, no correction.
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, then CONV_WARPS
 // converters (8 for narrow token tiles, where transcoding is the critical
-// path, else 4), then 4 promotion + epilogue warps.
+// path, else 4), then 4 promotion + epilogue warps, then an L2 prefetcher
+// that runs pf_steps K steps ahead of the producer (weight tile, token tile,
+// and once per item the tile's weight-scale rows and activation sums).
 //
 // W8 = true is the same GEMM for FP8 E4M3 weights with a float32 scale_inv
 // per [128, 128] block (the FP8 shared expert: "DeepSeek-V4-Pro-0813-nvfp4-
@@ -56,7 +58,8 @@ struct Cfg {
   static constexpr bool OFFS = !W8 && offset_codes(BN);
   static constexpr int CONV_WARPS = W8 ? 0 : (BN <= 32 ? 8 : 4);
   static constexpr int PROMO_FIRST = 2 + CONV_WARPS;      // first promotion warp
-  static constexpr int THREADS = (PROMO_FIRST + 4) * 32;
+  static constexpr int PF_WARP = PROMO_FIRST + 4;          // L2 prefetcher
+  static constexpr int THREADS = (PF_WARP + 1) * 32;
   static constexpr int CONV_THREADS = CONV_WARPS * 32;
   static constexpr int NA = (BN + 127) / 128;
   static constexpr int NUM_A = DUAL ? 2 : 1;
@@ -129,6 +132,7 @@ struct W4Args {
   void* out;
   uint8_t* out_scale;
   float limit;
+  int pf_steps;            // K steps the L2 prefetcher runs ahead of the producer (0: off)
 };
 
 // ROWS (with W8): E4M3 weights with the INT4 layout's per-row scales
@@ -149,6 +153,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
   uint64_t* pempty = pfull + 2;             // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* produced = reinterpret_cast<volatile int*>(tmem_slot + 2);   // K steps issued so far
   float* red = reinterpret_cast<float*>(smem + C::RED_OFF);
   gemm::SmemPlan plan(smem + C::PLAN_OFF);
 
@@ -168,6 +173,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
       mbar_init(&pempty[b], 128);
     }
     *abort_flag = 0;
+    *produced = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
@@ -216,11 +222,60 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
           }
           tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
+          *produced = *produced + 1;
         }
         __syncwarp();
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
+    }
+  } else if (warp == C::PF_WARP) {
+    // ------------------------------ L2 prefetcher --------------------------
+    // A hint only: gives up quietly when the CTA aborts or after the wait bound.
+    if (args.pf_steps > 0 && lane == 0) {
+      const int rb_per_g = N / 128;
+      const uint64_t t0 = globaltimer_ns();
+      int pf = 0;
+      bool go = true;
+      for (int item = blockIdx.x; item < n_items && go; item += gridDim.x) {
+        const Item it = decode_item(item, plan, G, n_ft, BN);
+        const int rb0 = it.g * rb_per_g + it.ft;
+        const int rb1 = rb0 + rb_per_g / 2;
+        for (int kt = 0; kt < KT && go; ++kt) {
+          while (pf >= *produced + args.pf_steps) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitTimeoutNs) { go = false; break; }
+            __nanosleep(128);
+          }
+          if (!go) break;
+          if (kt == 0) {
+            // the per-row weight scales of the tile(s) and the token rows'
+            // activation sums, once per item (16-byte aligned ranges only)
+            if constexpr (!(W8 && !ROWS)) {
+              const float* s0 = args.w_sinv + (size_t)rb0 * 128 * KT;
+              const uint32_t bytes = 128u * KT * 4u;
+              if ((reinterpret_cast<uintptr_t>(s0) & 15u) == 0) bulk_prefetch(s0, bytes);
+              if (DUAL) {
+                const float* s1 = args.w_sinv + (size_t)rb1 * 128 * KT;
+                if ((reinterpret_cast<uintptr_t>(s1) & 15u) == 0) bulk_prefetch(s1, bytes);
+              }
+            }
+            if (C::OFFS && args.a_corr != nullptr) {
+              const float* c0 = args.a_corr + (size_t)it.row0 * KT;
+              const uint32_t bytes = (uint32_t)(it.rows * KT * 4) & ~15u;
+              if ((reinterpret_cast<uintptr_t>(c0) & 15u) == 0 && bytes > 0) bulk_prefetch(c0, bytes);
+            }
+          }
+          if constexpr (W8) {
+            tma_prefetch_2d(&tmA, kt * 128, rb0 * 128);
+            if (DUAL) tma_prefetch_2d(&tmA, kt * 128, rb1 * 128);
+          } else {
+            tma_prefetch_2d(&tmA, kt * 64, rb0 * 128);
+            if (DUAL) tma_prefetch_2d(&tmA, kt * 64, rb1 * 128);
+          }
+          tma_prefetch_2d(&tmB, kt * 128, it.row0);
+          ++pf;
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ----------------------------
