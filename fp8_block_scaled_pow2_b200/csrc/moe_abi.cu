@@ -684,7 +684,9 @@ int repack_mxfp4_to_int4g128(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_
   if (!aligned(fp4, 16) || !aligned(out_int4, 16) || !aligned(e8m0, 4) || !aligned(out_scale_inv, 4))
     return MOE_ERR_INVALID;
   const int64_t blocks = n_mats * (int64_t)N * (K / 32);     // 32-element blocks, 4 per group
-  launch(int4g128_kernel, dim3((unsigned)((blocks + 255) / 256)), dim3(256), 0, S(stream), 
+  // grid-stride: each block of threads builds its code tables once
+  const int64_t grid = std::min<int64_t>((blocks + 255) / 256, (int64_t)sm_count() * 8);
+  launch(int4g128_kernel, dim3((unsigned)grid), dim3(256), 0, S(stream), 
       reinterpret_cast<const uint4*>(fp4), e8m0, blocks, reinterpret_cast<uint4*>(out_int4), out_scale_inv);
   return launch_status();
 }

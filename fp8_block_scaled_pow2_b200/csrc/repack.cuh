@@ -181,81 +181,164 @@ __global__ void __launch_bounds__(256) nvfp4_convert_vec_kernel(const uint4* __r
 
 // INT4 group-128: one thread per 32-element block (one 16-byte chunk of
 // nibbles and its E8M0 byte), four consecutive threads per 128-group, so the
-// loads and stores of a warp are contiguous.  The group maximum is reduced over
-// the four threads by shuffles.  Every E2M1 magnitude is 1 or 3 times a power of
-// two, so the seven quotients x / scale_inv of a block come from two IEEE
-// divisions (2^e / s and 3 * 2^e / s) scaled by powers of two, which is exact
-// in the normal range; below it the quotient is far under 0.5 and rounds to 0
-// either way.  Lanes of a warp must all be present (n_blocks % 4 == 0 holds).
-__global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__ fp4,
-                                                       const uint8_t* __restrict__ e8m0, int64_t n_blocks,
-                                                       uint4* __restrict__ out, float* __restrict__ scale_inv) {
-  pdl_trigger();
-  pdl_wait();
-  const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool live = blk < n_blocks;
-  const uint4 in = live ? __ldg(fp4 + blk) : make_uint4(0u, 0u, 0u, 0u);
-  const int b = live ? (int)__ldg(e8m0 + blk) : 0;
-  // largest magnitude code of the block, by a three-step binary search: some
-  // nibble m (0..7) reaches t exactly when m + 8 - t sets the nibble's bit 3
-  // (the sums stay below 16, so no carry crosses nibbles)
-  const uint32_t m0 = in.x & 0x77777777u, m1 = in.y & 0x77777777u;
-  const uint32_t m2 = in.z & 0x77777777u, m3 = in.w & 0x77777777u;
-  auto any_ge = [&](uint32_t t) {
-    const uint32_t k = (8u - t) * 0x11111111u;
-    return (((m0 + k) | (m1 + k) | (m2 + k) | (m3 + k)) & 0x88888888u) != 0u;
-  };
-  uint32_t mc = any_ge(4u) ? 4u : 0u;
-  mc += any_ge(mc + 2u) ? 2u : 0u;
-  mc += any_ge(mc + 1u) ? 1u : 0u;
-  const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
-  const float sc = exp2_int(b - 127);
-  float bm = __fmul_rn(kE2M1[mc], sc);
-  const bool nan = b == 255;
-  if (live && !nan && isinf(bm)) record_error(MOE_ERR_RANGE);
-  if (nan) bm = 0.0f;
-  float amax = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-  // a NaN scale anywhere in the group (its four lanes) skips the group
-  const bool gnan = ((__ballot_sync(0xFFFFFFFFu, nan) >> (threadIdx.x & 28)) & 0xFu) != 0u;
-  if (!live) return;
-  if (gnan) {
-    if (nan) record_error(MOE_ERR_NAN_SCALE);
-    return;
-  }
-  const float sinv = amax > 0.0f ? __fdiv_rn(amax, 7.0f) : 1.0f;
-  if ((threadIdx.x & 3) == 0) scale_inv[blk >> 2] = sinv;
-  // q of magnitude codes 1..7 (E2M1 0.5, 1, 1.5, 2, 3, 4, 6)
-  const float d1 = __fdiv_rn(sc, sinv);
-  const float d3 = __fdiv_rn(__fmul_rn(3.0f, sc), sinv);
-  const float qv[8] = {0.0f, 0.5f * d1, d1, 0.5f * d3, 2.0f * d1, d3, 4.0f * d1, 2.0f * d3};
-  // byte tables over the magnitude code: tp = q, tn = (16 - q) & 15 (q <= 7, so
-  // the byte-wise subtraction never borrows).  For 0 <= v <= 7 the float v + 2^23
-  // holds rint(v) (round half to even) in its low byte, and its byte 1 is zero.
-  uint32_t u[8];
-#pragma unroll
-  for (int c = 1; c < 8; ++c) u[c] = __float_as_uint(__fadd_rn(fminf(qv[c], 7.0f), 8388608.0f));
-  const uint32_t tp[2] = {__byte_perm(__byte_perm(u[1], u[2], 0x1401u), u[3], 0x4210u),     // 0, q1, q2, q3
-                          __byte_perm(__byte_perm(u[4], u[5], 0x0040u), __byte_perm(u[6], u[7], 0x0040u),
-                                      0x5410u)};                                              // q4 .. q7
-  const uint32_t tn[2] = {(0x10101010u - tp[0]) & 0x0F0F0F0Fu, (0x10101010u - tp[1]) & 0x0F0F0F0Fu};
+// loads and stores of a warp are contiguous; blocks of 256 threads walk the
+// matrix grid-stride.  The group maximum is reduced over the four threads by
+// shuffles.
+//
+// Codes from a table.  The group maximum is amax = A * 2^F with A = 1 or 1.5
+// (every E2M1 value is 1 or 1.5 times a power of two), so while amax is a
+// normal float32 (F >= -96 here), scale_inv = fl(amax / 7) = 2^F * fl(A / 7),
+// and the quotient of a code of value v in a block of exponent e is
+// fl(v 2^e / scale_inv) = 2^(e - F) * fl(v / fl(A / 7)): exact power-of-two
+// scalings of the IEEE results, until the quotient is far below 0.5 (e - F <
+// -8), where every code rounds to 0.  A block with a nonzero code has e - F
+// <= 1.  So the eight codes of a block depend only on (A, e - F): each block
+// of threads first computes those 2 x 10 tables with the same IEEE divides,
+// multiplies and round-to-nearest-even the per-element rule uses (and an
+// all-zero table for e - F < -8), then every 32-element block looks its table
+// up instead of dividing.  Groups with a maximum below 2^-96 take the direct
+// path: two IEEE divisions per block (2^e / s and 3 * 2^e / s, scaled by
+// powers of two).
+__device__ __forceinline__ float e2m1_magnitude(uint32_t m) {     // code 0..7 -> 0, .5, 1, 1.5, 2, 3, 4, 6
+  const uint32_t bits = m >= 2u ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22)) : (m ? 126u << 23 : 0u);
+  return __uint_as_float(bits);
+}
+
+// Byte tables over the magnitude code from the eight codes c[0..7] (c[0] = 0):
+// t.x, t.y = q (codes 0..3, 4..7), t.z, t.w = (16 - q) & 15, the two's
+// complement nibble of -q (q <= 7, so the byte-wise subtraction never borrows).
+__device__ __forceinline__ uint4 int4_code_tables(const uint32_t (&c)[8]) {
+  const uint32_t p0 = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+  const uint32_t p1 = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+  return make_uint4(p0, p1, (0x10101010u - p0) & 0x0F0F0F0Fu, (0x10101010u - p1) & 0x0F0F0F0Fu);
+}
+
+// PTX prmt in its default mode: selector nibble i picks byte (nibble & 7) of
+// {b, a} (a = bytes 0..3); when the nibble's bit 3 is set the result byte is
+// instead that byte's sign bit replicated (0x00 or 0xFF).  (__byte_perm reads
+// only the low 3 bits of each selector nibble.)
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// 16 bytes of E2M1 nibbles -> 16 bytes of INT4 nibbles through the tables t.
+// Each E2M1 nibble (bit 3 sign, bits 0-2 magnitude m) is its own selector:
+// with sign 0 the lookup in t.x/t.y copies q(m) and the lookup in t.z/t.w
+// (selector ^ 8, sign mode) gives 0x00 (table bytes are below 0x80); with
+// sign 1 it is the other way round, so OR-ing the two lookups yields the INT4
+// code of either sign, one byte per element.  Two such bytes are then merged
+// into one output byte (element 2i in the low nibble).
+__device__ __forceinline__ uint4 int4_remap(const uint4 in, const uint4 t) {
   const uint32_t words[4] = {in.x, in.y, in.z, in.w};
   uint32_t ow[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
-    // even nibbles (0, 2, 4, 6) and odd nibbles (1, 3, 5, 7) as four 4-bit
-    // byte selectors each; the lookups land in the low nibble of each byte
-    const uint32_t lo = words[w] & 0x0F0F0F0Fu, hi = (words[w] >> 4) & 0x0F0F0F0Fu;
-    const uint32_t sel_e = __byte_perm(lo | (lo >> 4), 0u, 0x0020u);
-    const uint32_t sel_o = __byte_perm(hi | (hi >> 4), 0u, 0x0020u);
-    // sign masks: in sel >> 3 a selector nibble is odd exactly for a set sign bit
-    const uint32_t m_e = __byte_perm(0xFF00FF00u, 0xFF00FF00u, sel_e >> 3);
-    const uint32_t m_o = __byte_perm(0xFF00FF00u, 0xFF00FF00u, sel_o >> 3);
-    const uint32_t r_e = (__byte_perm(tp[0], tp[1], sel_e) & ~m_e) | (__byte_perm(tn[0], tn[1], sel_e) & m_e);
-    const uint32_t r_o = (__byte_perm(tp[0], tp[1], sel_o) & ~m_o) | (__byte_perm(tn[0], tn[1], sel_o) & m_o);
-    ow[w] = r_e | (r_o << 4);
+    const uint32_t v = words[w], vn = v ^ 0x88888888u;
+    const uint32_t a = prmt_sign(t.x, t.y, v) | prmt_sign(t.z, t.w, vn);               // elements 0..3
+    const uint32_t b = prmt_sign(t.x, t.y, v >> 16) | prmt_sign(t.z, t.w, vn >> 16);   // elements 4..7
+    const uint32_t x = a | (a >> 4), y = b | (b >> 4);   // bytes 0 and 2: two codes each
+    ow[w] = __byte_perm(x, y, 0x6420u);
   }
-  out[blk] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  return make_uint4(ow[0], ow[1], ow[2], ow[3]);
+}
+
+constexpr int kInt4TableD = 10;       // tables for e - F = -8 .. 1 (index 1 .. 10), index 0 all zero
+
+__global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__ fp4,
+                                                       const uint8_t* __restrict__ e8m0, int64_t n_blocks,
+                                                       uint4* __restrict__ out, float* __restrict__ scale_inv) {
+  __shared__ uint4 s_tab[2][kInt4TableD + 1];
+  __shared__ float s_sa[2];
+  pdl_trigger();
+  // the tables read no global memory: built before waiting for the previous kernel
+  if (threadIdx.x < 2 * (kInt4TableD + 1)) {
+    const int ai = threadIdx.x / (kInt4TableD + 1), di = threadIdx.x % (kInt4TableD + 1);
+    const float sa = __fdiv_rn(ai ? 1.5f : 1.0f, 7.0f);
+    uint32_t c[8];
+    c[0] = 0u;
+#pragma unroll
+    for (uint32_t m = 1; m < 8; ++m) {
+      const float quot = __fmul_rn(__fdiv_rn(e2m1_magnitude(m), sa), exp2_int(di - 9));
+      c[m] = di == 0 ? 0u : (uint32_t)rintf(fminf(quot, 7.0f));
+    }
+    s_tab[ai][di] = int4_code_tables(c);
+    if (di == 0) s_sa[ai] = sa;
+  }
+  __syncthreads();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // warp-uniform loop: every lane takes part in the group shuffles.  The next
+  // block's bytes are loaded before this one is worked on, so two loads per
+  // thread are in flight.
+  int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  uint4 in_next = make_uint4(0u, 0u, 0u, 0u);
+  int b_next = 0;
+  if (base + lane < n_blocks) {
+    in_next = __ldg(fp4 + base + lane);
+    b_next = (int)__ldg(e8m0 + base + lane);
+  }
+  for (; base < n_blocks; base += stride) {
+    const int64_t blk = base + lane;
+    const bool live = blk < n_blocks;
+    const uint4 in = in_next;
+    const int b = b_next;
+    if (blk + stride < n_blocks) {
+      in_next = __ldg(fp4 + blk + stride);
+      b_next = (int)__ldg(e8m0 + blk + stride);
+    }
+    // largest magnitude code of the block, by a three-step binary search: some
+    // nibble m (0..7) reaches t exactly when m + 8 - t sets the nibble's bit 3
+    // (the sums stay below 16, so no carry crosses nibbles)
+    const uint32_t m0 = in.x & 0x77777777u, m1 = in.y & 0x77777777u;
+    const uint32_t m2 = in.z & 0x77777777u, m3 = in.w & 0x77777777u;
+    auto any_ge = [&](uint32_t t) {
+      const uint32_t k = (8u - t) * 0x11111111u;
+      return (((m0 + k) | (m1 + k) | (m2 + k) | (m3 + k)) & 0x88888888u) != 0u;
+    };
+    uint32_t mc = any_ge(4u) ? 4u : 0u;
+    mc += any_ge(mc + 2u) ? 2u : 0u;
+    mc += any_ge(mc + 1u) ? 1u : 0u;
+    const float sc = exp2_int(b - 127);
+    float bm = __fmul_rn(e2m1_magnitude(mc), sc);
+    const bool nan = b == 255;
+    if (live && !nan && isinf(bm)) record_error(MOE_ERR_RANGE);
+    if (nan) bm = 0.0f;
+    float amax = fmaxf(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+    // a NaN scale anywhere in the group (its four lanes) skips the group
+    const bool gnan = ((__ballot_sync(0xFFFFFFFFu, nan) >> (lane & 28)) & 0xFu) != 0u;
+    if (!live) continue;
+    if (gnan) {
+      if (nan) record_error(MOE_ERR_NAN_SCALE);
+      continue;
+    }
+    const uint32_t ab = __float_as_uint(amax);
+    const int F = (int)((ab >> 23) & 0xFFu) - 127;
+    uint4 t;
+    float sinv;
+    if (amax > 0.0f && F >= -96 && F <= 127) {
+      const int ai = (int)((ab >> 22) & 1u);             // mantissa of the maximum: 1 or 1.5
+      sinv = __fmul_rn(s_sa[ai], exp2_int(F));
+      const int d = (b - 127) - F;
+      t = s_tab[ai][d < -8 ? 0 : min(d, 1) + 9];
+    } else {
+      sinv = amax > 0.0f ? __fdiv_rn(amax, 7.0f) : 1.0f;
+      // the seven quotients of this block: magnitudes 1, 2, 4, 6 times d1 / 2 and
+      // 1.5, 3, 6 times d3 / 3, each an exact power-of-two scaling
+      const float d1 = __fdiv_rn(sc, sinv);
+      const float d3 = __fdiv_rn(__fmul_rn(3.0f, sc), sinv);
+      const float qv[8] = {0.0f, 0.5f * d1, d1, 0.5f * d3, 2.0f * d1, d3, 4.0f * d1, 2.0f * d3};
+      uint32_t c[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) c[m] = (uint32_t)rintf(fminf(qv[m], 7.0f));
+      t = int4_code_tables(c);
+    }
+    if ((lane & 3) == 0) scale_inv[blk >> 2] = sinv;
+    out[blk] = int4_remap(in, t);
+  }
 }
 
 // FP8 cast: one block of 128 threads per (matrix, 128-row block, 128-column

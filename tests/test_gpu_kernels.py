@@ -338,11 +338,12 @@ def test_repack_nvfp4_errors(lib):
     assert lib.moe_get_device_error() == 0
 
 
-@pytest.mark.parametrize("lo,hi", [(1, 250), (120, 127)])
+@pytest.mark.parametrize("lo,hi", [(1, 250), (120, 127), (1, 30), (22, 40)])
 def test_repack_int4_bit_exact(lib, lo, hi):
-    """Scales over the whole range, and in a narrow band where a group's blocks
+    """Scales over the whole range, in a narrow band where a group's blocks
     share or neighbour the maximum exponent (many quotients near rounding
-    ties)."""
+    ties), where every group maximum is below 2^-96 (the kernel's direct
+    division path), and straddling that threshold (both paths in one call)."""
     M, N, K = 2, 256, 1024
     fp4 = synth.random_bytes(6, 1, (M, N, K // 2))
     e8 = synth.random_bytes(6, 2, (M, N, K // 32), lo, hi)
