@@ -179,6 +179,23 @@ __global__ void __launch_bounds__(256) nvfp4_convert_vec_kernel(const uint4* __r
     for (int64_t i = tid; i < n_fp4_16; i += stride) out_fp4[i] = __ldg(fp4 + i);
 }
 
+// Largest magnitude code (0..7) among the 32 E2M1 nibbles of v, by a three-
+// step binary search: some nibble m reaches t exactly when m + 8 - t sets the
+// nibble's bit 3 (the sums stay below 16, so no carry crosses nibbles); the
+// first step (m >= 4) is bit 2 itself.
+__device__ __forceinline__ uint32_t max_magnitude_code(const uint4 v) {
+  const uint32_t m0 = v.x & 0x77777777u, m1 = v.y & 0x77777777u;
+  const uint32_t m2 = v.z & 0x77777777u, m3 = v.w & 0x77777777u;
+  auto any_ge = [&](uint32_t t) {
+    const uint32_t k = (8u - t) * 0x11111111u;
+    return (((m0 + k) | (m1 + k) | (m2 + k) | (m3 + k)) & 0x88888888u) != 0u;
+  };
+  uint32_t mc = ((m0 | m1 | m2 | m3) & 0x44444444u) != 0u ? 4u : 0u;
+  mc += any_ge(mc + 2u) ? 2u : 0u;
+  mc += any_ge(mc + 1u) ? 1u : 0u;
+  return mc;
+}
+
 // INT4 group-128: one thread per 32-element block (one 16-byte chunk of
 // nibbles and its E8M0 byte), four consecutive threads per 128-group, so the
 // loads and stores of a warp are contiguous; blocks of 256 threads walk the
@@ -289,18 +306,7 @@ __global__ void __launch_bounds__(256) int4g128_kernel(const uint4* __restrict__
       in_next = __ldg(fp4 + blk + stride);
       b_next = (int)__ldg(e8m0 + blk + stride);
     }
-    // largest magnitude code of the block, by a three-step binary search: some
-    // nibble m (0..7) reaches t exactly when m + 8 - t sets the nibble's bit 3
-    // (the sums stay below 16, so no carry crosses nibbles)
-    const uint32_t m0 = in.x & 0x77777777u, m1 = in.y & 0x77777777u;
-    const uint32_t m2 = in.z & 0x77777777u, m3 = in.w & 0x77777777u;
-    auto any_ge = [&](uint32_t t) {
-      const uint32_t k = (8u - t) * 0x11111111u;
-      return (((m0 + k) | (m1 + k) | (m2 + k) | (m3 + k)) & 0x88888888u) != 0u;
-    };
-    uint32_t mc = any_ge(4u) ? 4u : 0u;
-    mc += any_ge(mc + 2u) ? 2u : 0u;
-    mc += any_ge(mc + 1u) ? 1u : 0u;
+    const uint32_t mc = max_magnitude_code(in);     // largest magnitude code of the block
     const float sc = exp2_int(b - 127);
     float bm = __fmul_rn(e2m1_magnitude(mc), sc);
     const bool nan = b == 255;
@@ -388,12 +394,7 @@ __global__ void __launch_bounds__(128) fp8_block128_kernel(const uint8_t* __rest
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     nan |= b[p] == 255;
-    uint32_t mw = __vmaxu4(__vmaxu4(in[p].x & 0x07070707u, (in[p].x >> 4) & 0x07070707u),
-                           __vmaxu4(in[p].y & 0x07070707u, (in[p].y >> 4) & 0x07070707u));
-    mw = __vmaxu4(mw, __vmaxu4(__vmaxu4(in[p].z & 0x07070707u, (in[p].z >> 4) & 0x07070707u),
-                               __vmaxu4(in[p].w & 0x07070707u, (in[p].w >> 4) & 0x07070707u)));
-    mw = __vmaxu4(mw, mw >> 16);
-    const int mc = (int)max(mw & 0xFFu, (mw >> 8) & 0xFFu);
+    const int mc = (int)max_magnitude_code(in[p]);
     if (mc > 0) key = max(key, 2 * (b[p] - 127 + (mc >> 1) - 1) + ((mc >> 1) != 0 ? (mc & 1) : 0));
   }
   key = __reduce_max_sync(0xFFFFFFFFu, key);
