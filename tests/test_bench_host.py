@@ -79,3 +79,46 @@ def test_peaks_and_traffic_bookkeeping(tmp_path):
     p = bench.read_peaks()
     assert p["hbm"] > 1000 and p["bf16"] > 100
     assert bench.source_digest("mxfp4") != bench.source_digest("w4afp8")
+
+
+def test_roofline_bookkeeping_decode_and_prefill():
+    """Decode-sized batches are reported against the measured HBM copy rate,
+    larger ones against 2 x the measured burst bf16 rate (the FP8 MMA rate)."""
+    peaks = {"hbm": 6548.2, "bf16": 1642.8, "bf16_sustained": 1402.8, "src": "measured"}
+    ab = {"w13": 1.7e9, "flops13": 9.62e11}
+    r = bench.roofline(bench.WORKLOADS["decode"], "mxfp4", ab, 0.27, peaks, "decode")
+    assert r["bound"] == "hbm" and r["peak"] == 6548.2 and abs(r["achieved"] - 1.7e9 / 0.27e-3 / 1e9) < 0.1
+    r = bench.roofline(bench.WORKLOADS["long_prefill"], "mxfp4", ab, 0.5, peaks, "long_prefill")
+    assert r["bound"] == "tensor" and r["peak"] == 3285.6 and abs(r["frac"] - 9.62e11 / 0.5e-3 / 1e12 / 3285.6) < 1e-4
+
+
+def test_default_workload_is_the_largest_layer():
+    """With no arguments the benchmark times the long-prefill layer (384 + 1
+    experts, 16384 tokens), the largest configuration that fits one GPU."""
+    seen = {}
+
+    def fake(args, wl):
+        seen["workload"], seen["extras"] = args.workload, args.extras
+
+    orig = bench.run_ours
+    bench.run_ours = fake
+    try:
+        bench.main([])
+    finally:
+        bench.run_ours = orig
+    assert seen == {"workload": "long_prefill", "extras": "default"}
+    wl = bench.WORKLOADS["long_prefill"]
+    assert (wl["T"], wl["E"], wl["H"], wl["I"], wl["k"]) == (16384, 384, 4096, 2048, 6)
+
+
+def test_repack_byte_count_matches_the_per_matrix_sum():
+    """The reference arm's bytes per expert equal the GPU line's per-matrix
+    sums for one expert (w1, w3 [I, H], w2 [H, I])."""
+    H, I = 4096, 2048
+    total = 0
+    for M, N, K in ((2, I, H), (1, H, I)):
+        fp4, e8 = M * N * K // 2, M * N * K // 32
+        total += 2 * fp4 + e8 + 2 * e8 + 4 * M                     # NVFP4
+        total += fp4 + e8 + fp4 + 4 * (M * N * K // 128)             # INT4
+        total += fp4 + e8 + 2 * fp4 + 4 * (M * (N // 128) * (K // 128))   # FP8 blocks
+    assert bench.repack_bytes_per_expert(H, I) == total
