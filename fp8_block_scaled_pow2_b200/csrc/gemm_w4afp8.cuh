@@ -58,7 +58,13 @@ struct Cfg {
   static constexpr bool OFFS = !W8 && offset_codes(BN);
   static constexpr int CONV_WARPS = W8 ? 0 : (BN <= 32 ? 8 : 4);
   static constexpr int PROMO_FIRST = 2 + CONV_WARPS;      // first promotion warp
-  static constexpr int PF_WARP = PROMO_FIRST + 4;          // L2 prefetcher
+  // promotion warps: 4 (one per tensor-memory lane quadrant, every token column
+  // in each thread), or 8 for the 96-row tiles with gate and up (two per
+  // quadrant, each on half of the token columns: 2 x 48 accumulators a thread)
+  static constexpr int PROMO_WARPS = (W8 && DUAL && BN > 64) ? 8 : 4;
+  static constexpr int HALVES = PROMO_WARPS / 4;
+  static constexpr int CB = BN / HALVES;                   // token columns per promotion thread
+  static constexpr int PF_WARP = PROMO_FIRST + PROMO_WARPS;  // L2 prefetcher
   static constexpr int THREADS = (PF_WARP + 1) * 32;
   static constexpr int CONV_THREADS = CONV_WARPS * 32;
   static constexpr int NA = (BN + 127) / 128;
@@ -91,8 +97,10 @@ struct Cfg {
   static_assert(TMEM_USED <= 512, "tensor memory overflow");
   static_assert(STAGES >= 2, "too few stages");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory overflow");
-  static_assert(!DUAL || BN <= 64, "register accumulators: BN <= 64 with gate and up");
-  static_assert(BN <= 128, "register accumulators: BN <= 128");
+  static_assert(!DUAL || CB <= 64, "register accumulators: 64 columns a thread with gate and up");
+  static_assert(CB <= 128, "register accumulators: 128 columns a thread");
+  static_assert(CB % 16 == 0 || BN <= 16, "promotion loads: whole 16-column slices");
+  static_assert(!(OFFS && HALVES > 1), "offset codes use one set of promotion warps");
 };
 
 // Four INT4 (two's complement nibbles, element 0 in the low nibble) from
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&pfull[b], 1);
-      mbar_init(&pempty[b], 128);
+      mbar_init(&pempty[b], 32 * C::PROMO_WARPS);
     }
     *abort_flag = 0;
     *produced = 0;
@@ -378,6 +386,8 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
     // --------------------------- promotion + epilogue ---------------------
     const int q = warp & 3;
     const int f = q * 32 + lane;
+    const int half = (warp - C::PROMO_FIRST) >> 2;     // token-column half (0 with 4 promotion warps)
+    const int col0 = half * C::CB;
     const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
     uint32_t pb = 0, pbits = 0;
     // offset-term slot, alternating per K step across items: the barrier of
@@ -394,12 +404,14 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
                                                    : ((size_t)(it.g * rb_per_g + it.ft) * 128 + f) * KT);
       const float* s1 = args.w_sinv + (BLOCK_SCALE ? (size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * KT
                                                    : ((size_t)(it.g * rb_per_g + rb_per_g / 2 + it.ft) * 128 + f) * KT);
-      float acc0[BN], acc1[DUAL ? BN : 1];
+      constexpr int CB = C::CB;
+      float acc0[CB], acc1[DUAL ? CB : 1];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) acc0[c] = 0.0f;
+      for (int c = 0; c < CB; ++c) acc0[c] = 0.0f;
 #pragma unroll
-      for (int c = 0; c < (DUAL ? BN : 1); ++c) acc1[c] = 0.0f;
-      const int nchunks = (it.rows + 15) >> 4;
+      for (int c = 0; c < (DUAL ? CB : 1); ++c) acc1[c] = 0.0f;
+      const int my_cols = max(0, min(CB, it.rows - col0));      // valid token columns of this thread
+      const int nchunks = (my_cols + 15) >> 4;
       bool ok = true;
       float sc0 = __ldg(s0), sc1 = DUAL ? __ldg(s1) : 0.0f;
       // offset codes: thread f < rows fetches token column f's term of each
@@ -424,9 +436,9 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
           if (!mbar_wait(&pfull[pb], (pbits >> pb) & 1u, abort_flag)) { ok = false; break; }
         }
         tc_fence_after();
-        const uint32_t base = lane_addr + pb * C::P_COLS;
+        const uint32_t base = lane_addr + pb * C::P_COLS + col0;
 #pragma unroll
-        for (int ch = 0; ch < BN / 16; ++ch) {
+        for (int ch = 0; ch < (CB + 15) / 16; ++ch) {
           if (ch < nchunks) {
             uint32_t r0[16];
             tmem_ld16(base + ch * 16, r0);
@@ -436,7 +448,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
               tmem_wait_ld(r0, r1);
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const float c = C::OFFS ? cs[ch * 16 + j] : 0.0f;
+                const float c = C::OFFS ? cs[col0 + ch * 16 + j] : 0.0f;
                 acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]) - c, acc0[ch * 16 + j]);
                 acc1[ch * 16 + j] = fmaf(sc1, __uint_as_float(r1[j]) - c, acc1[ch * 16 + j]);
               }
@@ -444,7 +456,7 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
               tmem_wait_ld(r0);
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const float c = C::OFFS ? cs[ch * 16 + j] : 0.0f;
+                const float c = C::OFFS ? cs[col0 + ch * 16 + j] : 0.0f;
                 acc0[ch * 16 + j] = fmaf(sc0, __uint_as_float(r0[j]) - c, acc0[ch * 16 + j]);
               }
             }
@@ -463,34 +475,36 @@ __global__ void __launch_bounds__(Cfg<BN, DUAL, W8>::THREADS, 1)
         const int I = N / 2;
         uint8_t* hq = reinterpret_cast<uint8_t*>(args.out);
         float* h = acc0;                    // h replaces the gate accumulators
+        // this half's [4 warps][CB] column maxima, then its [CB] scales
+        float* rr = red + half * 4 * CB;
+        float* sk = red + 4 * BN + half * CB;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
+        for (int c = 0; c < CB; ++c) {
           h[c] = swiglu_clamped(acc0[c], acc1[DUAL ? c : 0], args.limit);
           const float m = warp_max_nonneg(fabsf(h[c]));
-          if (lane == 0) red[q * BN + c] = m;
+          if (lane == 0) rr[q * CB + c] = m;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1 + half, 128);
         // one thread per token column turns the column maximum into the scale
-        float* sk = red + 4 * BN;
-        if (f < it.rows && f < BN) {
+        if (f < my_cols) {
           const int c = f;
-          const float amax = fmaxf(fmaxf(red[c], red[BN + c]), fmaxf(red[2 * BN + c], red[3 * BN + c]));
+          const float amax = fmaxf(fmaxf(rr[c], rr[CB + c]), fmaxf(rr[2 * CB + c], rr[3 * CB + c]));
           const int k = pow2_scale_exponent(amax);
           sk[c] = exp2_int(-k);
-          args.out_scale[(size_t)(it.row0 + c) * (I / 128) + it.ft] = (uint8_t)(k + 127);
+          args.out_scale[(size_t)(it.row0 + col0 + c) * (I / 128) + it.ft] = (uint8_t)(k + 127);
         }
-        named_bar_sync(1, 128);
-        uint8_t* hq_f = hq + (size_t)it.row0 * I + it.ft * 128 + f;
+        named_bar_sync(1 + half, 128);
+        uint8_t* hq_f = hq + (size_t)(it.row0 + col0) * I + it.ft * 128 + f;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          if (c < it.rows) hq_f[(size_t)c * I] = (uint8_t)(e4m3x2(__fmul_rn(h[c], sk[c]), 0.0f) & 0xFFu);
+        for (int c = 0; c < CB; ++c) {
+          if (c < my_cols) hq_f[(size_t)c * I] = (uint8_t)(e4m3x2(__fmul_rn(h[c], sk[c]), 0.0f) & 0xFFu);
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1 + half, 128);
       } else {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          if (c < it.rows) {
-            const size_t o = (size_t)(it.row0 + c) * N + it.ft * 128 + f;
+        for (int c = 0; c < CB; ++c) {
+          if (c < my_cols) {
+            const size_t o = (size_t)(it.row0 + col0 + c) * N + it.ft * 128 + f;
             if constexpr (EPI == MOE_EPI_STORE_F32)
               reinterpret_cast<float*>(args.out)[o] = acc0[c];
             else

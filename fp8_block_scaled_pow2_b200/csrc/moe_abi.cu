@@ -157,8 +157,16 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
   const bool dual = epilogue == MOE_EPI_SWIGLU_QUANT;
   if (dual && N % 256) return MOE_ERR_INVALID;
+  const bool auto_bn = block_n == 0;
   if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
-  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual)) return MOE_ERR_UNSUPPORTED;
+  // INT4 with gate and up: an automatic choice takes 96-row tiles (eight
+  // promotion warps) when the workspace holds their plan and the E4M3 copy
+  if (!W8 && dual && auto_bn && block_n == 64 &&
+      workspace_bytes >= gemm::ws_layout(a_rows, n_groups, K, 96).total + w4a_scratch_bytes(n_groups, N, K))
+    block_n = 96;
+  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual) &&
+      !(block_n == 96 && dual && !W8))
+    return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
   if (dual && !out_scale) return MOE_ERR_INVALID;
@@ -168,6 +176,7 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
   const bool scratch = !W8 && w4a_uses_scratch(block_n) &&
                        workspace_bytes >= L.total + w4a_scratch_bytes(n_groups, N, K);
+  if (block_n == 96 && !scratch) return MOE_ERR_INVALID;     // 96-row tiles stream the E4M3 copy
   uint8_t* e4m3_copy = scratch ? reinterpret_cast<uint8_t*>(workspace) + L.total : nullptr;
   CUtensorMap ta, tb;
   // INT4: raw [rows, K/2] tiles of 64 x 128 bytes; FP8 (and the E4M3 copy of
@@ -214,7 +223,9 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
     launch(w4a::transcode_int4_kernel, dim3((unsigned)((chunks + 255) / 256), (unsigned)n_groups), dim3(256), 0, st,
            reinterpret_cast<const uint4*>(w), offsets, chunks, reinterpret_cast<uint4*>(e4m3_copy));
     if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-    if (dual) return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT, true, true>(ta, tb, args, st);
+    if (dual)
+      return block_n == 96 ? launch_w4a<96, true, MOE_EPI_SWIGLU_QUANT, true, true>(ta, tb, args, st)
+                           : launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT, true, true>(ta, tb, args, st);
     if (epilogue == MOE_EPI_STORE_F32)
       return block_n == 64 ? launch_w4a<64, false, MOE_EPI_STORE_F32, true, true>(ta, tb, args, st)
                            : launch_w4a<128, false, MOE_EPI_STORE_F32, true, true>(ta, tb, args, st);
@@ -430,7 +441,7 @@ size_t moe_w4afp8_workspace_size(int a_rows, int n_groups, int N, int K, int blo
   if (block_n == 0) {
     // the call caps its own choice at 64 rows for the SwiGLU epilogue: cover
     // the plan of every tile width it may pick
-    for (int bn : {16, 32, 64, 128}) plan = std::max(plan, gemm::ws_layout(a_rows, n_groups, K, bn).total);
+    for (int bn : {16, 32, 64, 96, 128}) plan = std::max(plan, gemm::ws_layout(a_rows, n_groups, K, bn).total);
     block_n = pick_block_n(a_rows, n_groups);
   } else {
     plan = gemm::ws_layout(a_rows, n_groups, K, block_n).total;

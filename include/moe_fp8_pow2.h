@@ -310,7 +310,9 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
  * slots).
  *   w_int4       int8 [G, N, K/2] (16-byte aligned); w_scale_inv float32 [G, N, K/128]
  *   other arguments, layouts and epilogues as moe_grouped_gemm_mxfp4;
- *   block_n: 16, 32, 64 (SWIGLU_QUANT) or up to 128 (STORE_F32 / STORE_BF16);
+ *   block_n: 16, 32, 64 or 96 (SWIGLU_QUANT; 96 needs the E4M3-copy workspace
+ *   below, and with block_n = 0 is chosen instead of 64 when the workspace
+ *   holds it) or up to 128 (STORE_F32 / STORE_BF16);
  *   workspace: at least moe_gemm_workspace_size(a_rows, G, K, block_n) bytes.
  *   Token tiles of 64 rows or more, given the larger workspace that
  *   moe_w4afp8_workspace_size(a_rows, G, N, K, block_n) returns: the call

@@ -106,6 +106,8 @@ def test_w4afp8_workspace_sizes_without_gpu():
     plan = moe.moe_gemm_workspace_size(1000, 9, 4096, 64)
     assert moe.moe_w4afp8_workspace_size(1000, 9, 4096, 4096, 64) == plan + 9 * 4096 * 4096
     assert moe.moe_w4afp8_workspace_size(1000, 9, 4096, 4096, 32) == moe.moe_gemm_workspace_size(1000, 9, 4096, 32)
+    # block_n 0 covers the plan of every tile width the call may pick (96 included)
+    assert moe.moe_w4afp8_workspace_size(1000, 9, 4096, 4096, 0) >= moe.moe_gemm_workspace_size(1000, 9, 4096, 96)
     T, H, I, E, k = 16384, 4096, 2048, 384, 6
     R, G = T * k + T, E + 1
     ws = moe.moe_workspace_size(T, H, I, E, k, path=moe.MOE_PATH_W4AFP8)

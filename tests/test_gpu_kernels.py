@@ -541,6 +541,36 @@ def test_w4afp8_offset_codes_zero_weight_groups(lib, block_n):
     no_device_error(lib)
 
 
+def test_w4afp8_96_row_tiles(lib):
+    """Gate/up with 96-row token tiles (eight promotion warps, each on half of
+    the token columns), the automatic choice when the workspace holds the
+    E4M3 weight copy: integer-exact inputs equal the oracle bit for bit;
+    random scaled inputs stay within the float32 bound of the oracle and give
+    the 64-row tiles' result; empty, single-row and ragged groups."""
+    N = 512
+    sizes = [70, 0, 1, 193, 96, 300, 47]
+    ai, aa, ao, aq, asv = _w4a_inputs(16, sizes, N, 512, True)
+    gu, _ = _run_w4a(lib, ai, aa, ao, aq, asv, lib.MOE_EPI_STORE_F32, 128, scratch=True)
+    hq96, sh96 = _run_w4a(lib, ai, aa, ao, aq, asv, lib.MOE_EPI_SWIGLU_QUANT, 96, scratch=True)
+    hq0, sh0 = _run_w4a(lib, ai, aa, ao, aq, asv, lib.MOE_EPI_SWIGLU_QUANT, 0, scratch=True)
+    hq2, sh2 = torch.empty_like(hq96), torch.empty_like(sh96)
+    lib.moe_swiglu_clamp(gu, hq2, sh2, 10.0)
+    ref = ffn.grouped_gemm_w4afp8(ai, aa, ao, aq, asv)
+    np.testing.assert_array_equal(host(gu), ref.astype(np.float32))     # integer-exact
+    np.testing.assert_array_equal(host(hq96), host(hq2))                  # fused SwiGLU == standalone
+    np.testing.assert_array_equal(host(sh96), host(sh2))
+    assert torch.equal(hq0, hq96) and torch.equal(sh0, sh96)              # block_n 0 picked 96
+    a, asc, offsets, q, sinv = _w4a_inputs(17, sizes, N, 1024, False)
+    hq96, sh96 = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_SWIGLU_QUANT, 96, scratch=True)
+    hq64, sh64 = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_SWIGLU_QUANT, 64, scratch=True)
+    gu, _ = _run_w4a(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, 128, scratch=True)
+    _gu_within_fp32_bound(host(gu), ffn.grouped_gemm_w4afp8(a, asc, offsets, q, sinv),
+                          _abs_gemm(a, asc, offsets, lambda g: ffn.dequant_int4g128(q[g], sinv[g])))
+    _swiglu_ok(host(hq96), host(sh96), host(gu).astype(np.float64), N // 2)
+    assert (host(hq96) != host(hq64)).mean() < 1e-3
+    no_device_error(lib)
+
+
 @pytest.mark.parametrize("block_n,epi", [(64, 2), (64, 0), (128, 0), (128, 1)])
 def test_w4afp8_e4m3_copy_path(lib, block_n, epi):
     """Wide token tiles with a workspace that holds the E4M3 weight copy:
