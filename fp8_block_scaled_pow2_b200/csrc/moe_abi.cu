@@ -159,13 +159,12 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   if (dual && N % 256) return MOE_ERR_INVALID;
   const bool auto_bn = block_n == 0;
   if (block_n == 0) block_n = std::min(pick_block_n(a_rows, n_groups), dual ? 64 : 128);
-  // INT4 with gate and up: an automatic choice takes 96-row tiles (eight
-  // promotion warps) when the workspace holds their plan and the E4M3 copy
-  if (!W8 && dual && auto_bn && block_n == 64 &&
-      workspace_bytes >= gemm::ws_layout(a_rows, n_groups, K, 96).total + w4a_scratch_bytes(n_groups, N, K))
+  // with gate and up an automatic choice takes 96-row tiles (eight promotion
+  // warps) when the workspace holds their plan (and, for INT4, the E4M3 copy)
+  if (dual && auto_bn && block_n == 64 &&
+      workspace_bytes >= gemm::ws_layout(a_rows, n_groups, K, 96).total + (W8 ? 0 : w4a_scratch_bytes(n_groups, N, K)))
     block_n = 96;
-  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual) &&
-      !(block_n == 96 && dual && !W8))
+  if (block_n != 16 && block_n != 32 && block_n != 64 && !(block_n == 128 && !dual) && !(block_n == 96 && dual))
     return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w || !w_scale_inv || !out || !workspace) return MOE_ERR_INVALID;
@@ -176,7 +175,7 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
   const bool scratch = !W8 && w4a_uses_scratch(block_n) &&
                        workspace_bytes >= L.total + w4a_scratch_bytes(n_groups, N, K);
-  if (block_n == 96 && !scratch) return MOE_ERR_INVALID;     // 96-row tiles stream the E4M3 copy
+  if (!W8 && block_n == 96 && !scratch) return MOE_ERR_INVALID;     // INT4 96-row tiles stream the E4M3 copy
   uint8_t* e4m3_copy = scratch ? reinterpret_cast<uint8_t*>(workspace) + L.total : nullptr;
   CUtensorMap ta, tb;
   // INT4: raw [rows, K/2] tiles of 64 x 128 bytes; FP8 (and the E4M3 copy of
@@ -236,6 +235,9 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
     switch (block_n) {
       case 16: return launch_w4a<16, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
       case 32: return launch_w4a<32, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
+      case 96:
+        if constexpr (W8) return launch_w4a<96, true, MOE_EPI_SWIGLU_QUANT, true>(ta, tb, args, st);
+        return MOE_ERR_UNSUPPORTED;
       default: return launch_w4a<64, true, MOE_EPI_SWIGLU_QUANT, W8>(ta, tb, args, st);
     }
   }

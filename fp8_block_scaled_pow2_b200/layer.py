@@ -187,7 +187,7 @@ class MoeLayer:
             ws_gemm=torch.empty(ws_g, dtype=u8, device=d), block_n=block_n,
             **(dict(shared_off=torch.tensor([0, T], dtype=i32, device=d),
                     ws_shared=torch.empty(max([moe.moe_gemm_workspace_size(max(T, 1), 1, K, bn)
-                                               for bn in (0, 16, block_n) for K in (H, I)] + [256]),
+                                               for bn in (0, 16, 96, block_n) for K in (H, I)] + [256]),
                                           dtype=u8, device=d))
                if self.shared == "fp8" else {}),
             **(dict(sxf=torch.empty(max(T, 1), dtype=f32, device=d),

@@ -312,7 +312,9 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
  *   other arguments, layouts and epilogues as moe_grouped_gemm_mxfp4;
  *   block_n: 16, 32, 64 or 96 (SWIGLU_QUANT; 96 needs the E4M3-copy workspace
  *   below, and with block_n = 0 is chosen instead of 64 when the workspace
- *   holds it) or up to 128 (STORE_F32 / STORE_BF16);
+ *   holds it) or up to 128 (STORE_F32 / STORE_BF16);  the FP8 block-scaled GEMM
+ *   below takes 96 with SWIGLU_QUANT without a copy, chosen with block_n = 0
+ *   when the workspace holds the plan of 96-row tiles;
  *   workspace: at least moe_gemm_workspace_size(a_rows, G, K, block_n) bytes.
  *   Token tiles of 64 rows or more, given the larger workspace that
  *   moe_w4afp8_workspace_size(a_rows, G, N, K, block_n) returns: the call

@@ -665,15 +665,24 @@ def test_fp8_block_gemm_random(lib, block_n):
     assert (np.abs(got - ref) <= 1024 * 2.0 ** -24 * bound + 1e-30).all()
 
 
-def test_fp8_block_gemm_swiglu_matches_standalone(lib):
+@pytest.mark.parametrize("block_n", [32, 96])
+def test_fp8_block_gemm_swiglu_matches_standalone(lib, block_n):
+    """The fused SwiGLU epilogue equals the standalone kernel on the GEMM's
+    float32 output at 32-row tiles (the float32 epilogue's tile), and at
+    96-row tiles (eight promotion warps, each on half of the token columns)
+    agrees with it except at rare rounding boundaries; both against the
+    oracle's SwiGLU of that float32 output within the silu bound."""
     I = 256
-    a, asc, offsets, q, sinv = _fp8w_inputs(16, [5, 0, 33, 70], 2 * I, 512, False)
+    a, asc, offsets, q, sinv = _fp8w_inputs(16, [5, 0, 33, 70, 1, 200, 97], 2 * I, 512, False)
     gu, _ = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_STORE_F32, 32)
-    hq, sh = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_SWIGLU_QUANT, 32)
+    hq, sh = _run_fp8w(lib, a, asc, offsets, q, sinv, lib.MOE_EPI_SWIGLU_QUANT, block_n)
     hq2, sh2 = torch.empty_like(hq), torch.empty_like(sh)
     lib.moe_swiglu_clamp(gu, hq2, sh2, 10.0)
-    np.testing.assert_array_equal(host(hq), host(hq2))
-    np.testing.assert_array_equal(host(sh), host(sh2))
+    if block_n == 32:
+        np.testing.assert_array_equal(host(hq), host(hq2))
+        np.testing.assert_array_equal(host(sh), host(sh2))
+    else:
+        assert (host(hq) != host(hq2)).mean() < 1e-3 and (host(sh) != host(sh2)).mean() < 1e-3
     _gu_within_fp32_bound(host(gu), ffn.grouped_gemm_fp8_block128(a, asc, offsets, q, sinv),
                           _abs_gemm(a, asc, offsets, lambda g: ffn.dequant_fp8_block128(q[g], sinv[g])))
     _swiglu_ok(host(hq), host(sh), host(gu).astype(np.float64), I)
