@@ -24,8 +24,8 @@
 // CTA roles (persistent kernel, one CTA per SM, 11 warps):
 //   warp 0        TMA producer: weight tiles (FP4 unpacked to one nibble per
 //                 byte in shared memory by the 16U4_ALIGN16B tensor-map type),
-//                 token tile, and the pre-interleaved scale blocks (1-D bulk
-//                 copies)
+//                 their pre-interleaved scale blocks, the token tile and the
+//                 token scales
 //   warp 1        TMEM owner and MMA issuer 0: scale factors shared -> TMEM
 //                 (tcgen05.cp), 4 MMAs of K = 32 per 128-wide K step
 //   warp 10       MMA issuer 1 (tile 1 of a pair, or alternate K steps of a
@@ -59,10 +59,24 @@ constexpr int kWBlock = 8192 + 512;
 constexpr int kMaxGroups = 1024;
 constexpr int kPlanSmemBytes = 16 * (kMaxGroups + 4);
 
-// Pipeline: per 128-wide K step a 3-D TMA copy writes each weight tile
-// straight into the unpacked one-nibble-per-byte layout the MMA reads
-// (16U4_ALIGN16B), a 1-D bulk copy brings its 512-byte scale block, a 2-D TMA
-// copy the token tile, and every fourth step a bulk copy the token scales.
+// Pipeline: per 128-wide K step one 4-D TMA copy writes the item's weight
+// tiles (both tiles of a pair: its box holds two prepared blocks) straight
+// into the unpacked one-nibble-per-byte layout the MMA reads (16U4_ALIGN16B),
+// one TMA copy over a view of the prepared blocks' scale parts brings their
+// 512-byte scale blocks, a 2-D TMA copy the token tile, and every fourth step
+// a bulk copy the token scales: 3.25 copy instructions per K step.
+//
+// Shared memory bandwidth is what the pipeline spends: per K step of a full
+// tile pair the tensor core reads 64 KB (8 MMAs x (4 KB of weights + 4 KB of
+// tokens)) and the copies write ~49 KB.  The token tile is therefore copied
+// with the smallest of four boxes (16, 32, 64 or BN rows) that covers the
+// item's rows: a ragged tile of 20 tokens writes 4 KB per step, not 16 KB.
+//
+// Tensor maps of the prepared weights (built by the host):
+//   tmA  [pairs][2][128 rows][128 nibbles] in paired order (box: one pair),
+//        [row blocks][K steps][128 rows][128 nibbles] in plain order (box: the
+//        item's one or two row blocks at one K step);
+//   tmS  the same views of the scale blocks as 128 32-bit words each.
 template <int BN, bool PAIR>
 struct Cfg {
   static constexpr int NA = (BN + 127) / 128;            // 128-row scale blocks of the token tile
@@ -87,7 +101,8 @@ struct Cfg {
   static constexpr int STAGES = STAGES_FIT > 16 ? 16 : STAGES_FIT;
   // transaction bytes of a step (the TMA counts the packed weight bytes);
   // steps that also load token scales add NA * 512
-  static constexpr int TX = NUM_A * (A_PACKED + SF_BYTES) + B_BYTES;
+  // (plus the token tile's box and, every fourth step, the token scales)
+  static constexpr int TX_W = NUM_A * (A_PACKED + SF_BYTES);
   // MMA issue: one warp issuing block-scaled MMAs is bound by its own issue
   // latency (about 60 cycles per instruction, the tensor work of N = 128),
   // so two warps issue.  With a tile pair issuer 0 computes tile 0 and
@@ -126,6 +141,16 @@ struct Cfg {
   // their width: each warp's column slice starts at a multiple of CW
   static_assert(CW == 8 || CW % 16 == 0, "epilogue column slices must be whole 16-column loads");
 };
+
+// Token-tile tensor maps whose boxes hold 16, 32, 64 and BN rows (capped at
+// BN); an item copies with the smallest box that covers its MMA width.
+struct TokenMaps {
+  CUtensorMap m[4];
+};
+__host__ __device__ __forceinline__ int token_box_rows(int i, int BN) { return (16 << i) < BN ? (16 << i) : BN; }
+__device__ __forceinline__ int token_box_index(int n_mma) {
+  return n_mma <= 16 ? 0 : (n_mma <= 32 ? 1 : (n_mma <= 64 ? 2 : 3));
+}
 
 // ----------------------- plan (work decomposition) -------------------------
 // Workspace layout, all offsets 256-byte aligned:
@@ -190,6 +215,11 @@ constexpr int kPrepPerThread = (kMaxGroups + kPrepThreads) / kPrepThreads;   // 
 // operands or the workspace.  (offsets[0] > 0 lets a caller run a subset of
 // groups, e.g. one group of a larger grouping.)
 //
+// split_tile > 0 splits every group between two kernels, each with its own
+// plan: part 0 takes the group's first floor(rows / split_tile) * split_tile
+// rows (whole tiles of the SM-pair kernel), part 1 the remaining rows.  A
+// group's entry in `groups` then holds the (first row, rows) of its part.
+//
 // With a_corr (the INT4 weight GEMM on narrow token tiles), each block also
 // writes, for every row r of its tile and K step kt, a_corr[r * KT + kt] =
 // 8 * 2^(sx - 127) * (sum of the row's 128 E4M3 values in that step): the GEMM
@@ -202,11 +232,13 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
                                                                  int* __restrict__ tstart, int2* __restrict__ groups,
                                                                  uint8_t* __restrict__ a_sf,
                                                                  const uint8_t* __restrict__ aq,
-                                                                 float* __restrict__ a_corr) {
+                                                                 float* __restrict__ a_corr, int split_tile,
+                                                                 int split_part) {
   pdl_trigger();
   pdl_wait();
   __shared__ int s_off[kMaxGroups + 1];
   __shared__ int s_t0[kMaxGroups + 1];      // first tile of each group; s_t0[G] = tiles in all
+  __shared__ int s_skip[kMaxGroups];        // rows of the group before this plan's part
   __shared__ int s_warp[kPrepThreads / 32];
   const int tid = threadIdx.x;
   for (int g = tid; g <= G; g += kPrepThreads) s_off[g] = offsets[g];
@@ -222,7 +254,15 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
 #pragma unroll
   for (int i = 0; i < kPrepPerThread; ++i) {
     const int g = g0 + i;
-    nt[i] = (!bad && g < G) ? ceil_div(s_off[g + 1] - s_off[g], BN) : 0;
+    int rows = (!bad && g < G) ? s_off[g + 1] - s_off[g] : 0;
+    int skip = 0;
+    if (split_tile > 0) {
+      const int whole = rows / split_tile * split_tile;
+      if (split_part == 0) rows = whole;
+      else { skip = whole; rows -= whole; }
+    }
+    if (g < G) s_skip[g] = skip;
+    nt[i] = ceil_div(rows, BN);
     local += nt[i];
   }
   const int lane = tid & 31, wid = tid >> 5;
@@ -249,7 +289,9 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
     for (int g = tid; g < G; g += kPrepThreads) {
       tstart[g] = s_t0[g];
       prefix[g] = s_t0[g] * n_ft;
-      groups[g] = bad ? make_int2(0, 0) : make_int2(s_off[g], s_off[g + 1] - s_off[g]);
+      int rows = s_off[g + 1] - s_off[g];
+      if (split_tile > 0) rows = split_part == 0 ? rows / split_tile * split_tile : rows - s_skip[g];
+      groups[g] = bad ? make_int2(0, 0) : make_int2(s_off[g] + s_skip[g], rows);
     }
     if (tid == 0) {
       prefix[G] = n_tiles * n_ft;
@@ -268,8 +310,10 @@ __global__ void __launch_bounds__(kPrepThreads) gemm_prep_kernel(const int32_t* 
     const int mid = (lo + hi + 1) >> 1;
     if (s_t0[mid] <= t) lo = mid; else hi = mid - 1;
   }
-  const int row0 = s_off[lo] + (t - s_t0[lo]) * BN;
-  const int rows = min(BN, s_off[lo + 1] - row0);
+  const int row0 = s_off[lo] + s_skip[lo] + (t - s_t0[lo]) * BN;
+  const int g_end = (split_tile > 0 && split_part == 0) ? s_off[lo] + (s_off[lo + 1] - s_off[lo]) / split_tile * split_tile
+                                                        : s_off[lo + 1];
+  const int rows = min(BN, g_end - row0);
   const int KG = (KT + 3) / 4, NA = ceil_div(BN, 128);
   for (int kg = 0; kg < KG; ++kg) {
     for (int a = 0; a < NA; ++a) {
@@ -335,8 +379,10 @@ struct SmemPlan {
 };
 
 // Work item -> (group, weight tile, token tile).  Items are group-major, then
-// weight tile, then token tile.
-__device__ __forceinline__ Item decode_item(int item, const SmemPlan& plan, int G, int n_ft, int BN) {
+// weight tile, then token tile.  Plan: SmemPlan, or any struct with the same
+// three arrays (prefix, tstart, groups).
+template <class Plan>
+__device__ __forceinline__ Item decode_item(int item, const Plan& plan, int G, int n_ft, int BN) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -525,8 +571,8 @@ __device__ __forceinline__ void mma_issuer(const int iss, uint8_t* smem, const u
 
 template <int BN, bool PAIR, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_mxfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmArgs args) {
+    gemm_mxfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ TokenMaps tmB,
+                      const __grid_constant__ CUtensorMap tmS, const GemmArgs args) {
   using C = Cfg<BN, PAIR>;
   // SwiGLU reads gate and up from the two tiles of a pair (paired weight order)
   constexpr bool PAIRED_ORDER = EPI == MOE_EPI_SWIGLU_QUANT;
@@ -563,7 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *produced = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmB.m[i]);
+    prefetch_tensormap(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -585,20 +633,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t stage = 0, phase = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
-      // prepared block of weight tile a at K step kt: blk0 + kt * kt_step + a * a_step
-      //   paired order: the gate and up blocks of a K step are adjacent;
-      //   plain order: each 128-row block holds its KT steps contiguously
-      size_t blk0, kt_step, a_step;
-      if (PAIRED_ORDER) {
-        blk0 = (size_t)(it.g * n_ft + it.ft) * KT * 2;
-        kt_step = 2;
-        a_step = 1;
-      } else {
-        blk0 = (size_t)(it.g * rb_per_g + (PAIR ? 2 * it.ft : it.ft)) * KT;
-        kt_step = 1;
-        a_step = KT;
-      }
+      // paired order: the gate and up blocks of K step kt are pair p0 + kt;
+      // plain order: the item's first 128-row block is rb (its K steps are
+      // contiguous), the second one rb + 1
+      const int p0 = (it.g * n_ft + it.ft) * KT;
+      const int rb = it.g * rb_per_g + (PAIR ? 2 * it.ft : it.ft);
       const uint8_t* sfb = args.a_sf + (size_t)it.t * ((KT + 3) / 4) * C::NA * 512;
+      // token rows the MMAs read (the issuers' N) and the box that covers them
+      const int box = token_box_index(max(16, (it.rows + 15) & ~15));
+      const CUtensorMap* tm_tok = &tmB.m[box];
+      const uint32_t tx = C::TX_W + token_box_rows(box, BN) * 128;
       bool ok = true;
       for (int kt = 0; kt < KT; ++kt) {
         if (!mbar_wait_warp(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -607,14 +651,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           // token scales: one block per 4 K steps, read by each issuer at its
           // first step of the group (issuers alternate steps without PAIR)
           const bool new_group = PAIR ? (kt & 3) == 0 : (kt & 3) < 2;
-          mbar_arrive_expect_tx(&full[stage], C::TX + (new_group ? C::NA * 512 : 0));
-#pragma unroll
-          for (int a = 0; a < C::NUM_A; ++a) {
-            const size_t blk = blk0 + (size_t)kt * kt_step + (size_t)a * a_step;
-            tma_load_3d(st + C::A0_OFF + a * C::A_BYTES, &tmA, 0, 0, (int)blk, &full[stage]);
-            bulk_load(st + C::SFA_OFF + a * C::SF_BYTES, args.w + blk * kWBlock + 8192, 512, &full[stage]);
+          mbar_arrive_expect_tx(&full[stage], tx + (new_group ? C::NA * 512 : 0));
+          if (PAIRED_ORDER) {
+            tma_load_4d(st + C::A0_OFF, &tmA, 0, 0, 0, p0 + kt, &full[stage]);
+            tma_load_3d(st + C::SFA_OFF, &tmS, 0, 0, p0 + kt, &full[stage]);
+          } else {
+            tma_load_4d(st + C::A0_OFF, &tmA, 0, 0, kt, rb, &full[stage]);
+            tma_load_3d(st + C::SFA_OFF, &tmS, 0, kt, rb, &full[stage]);
           }
-          tma_load_2d(st + C::B_OFF, &tmB, kt * 128, it.row0, &full[stage]);
+          tma_load_2d(st + C::B_OFF, tm_tok, kt * 128, it.row0, &full[stage]);
           if (new_group) bulk_load(st + C::SFB_OFF, sfb + (size_t)(kt >> 2) * C::NA * 512, C::NA * 512, &full[stage]);
           *produced = *produced + 1;
         }
@@ -658,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int a = 0; a < C::NUM_A; ++a) bulk_prefetch(args.w + (blk + (size_t)a * a_step) * kWBlock, kWBlock);
           }
-          tma_prefetch_2d(&tmB, kt * 128, it.row0);
+          tma_prefetch_2d(&tmB.m[token_box_index(max(16, (it.rows + 15) & ~15))], kt * 128, it.row0);
           ++pf;
         }
       }
@@ -681,7 +726,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ab = 0, acc_bits = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item it = decode_item(item, plan, G, n_ft, BN);
-      if (!mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag)) break;
+      bool ok = mbar_wait(&acc_full[ab], (acc_bits >> ab) & 1u, abort_flag);
+      // the SwiGLU epilogue's four warps of a half meet at a named barrier:
+      // they continue or stop together, never one without the others
+      if (EPI == MOE_EPI_SWIGLU_QUANT) ok = named_bar_and(1 + half, 128, ok);
+      if (!ok) break;
       tc_fence_after();
       epilogue_item<BN, PAIR, EPI, C::CW>(it, lane_addr + ab * C::ACC_COLS + half * C::CW, f, q, half, lane, N,
                                           KT, args, red, &acc_empty[ab]);

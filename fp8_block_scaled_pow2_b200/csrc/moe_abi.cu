@@ -3,12 +3,14 @@
 // they share the device error word.
 #include <cudaTypedefs.h>
 
+#include <climits>
 #include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
 #include "elementwise.cuh"
 #include "gemm_mxfp4.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_w4afp8.cuh"
 #include "gemm_ptpc.cuh"
 #include "repack.cuh"
@@ -61,18 +63,22 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
 }
 
 
-// 3-D tiled map (inner dimension first) over equally spaced 2-D blocks.
-bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                 uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1) {
+// Tiled map of any rank (inner dimension first); strides[i] is the byte
+// stride of dimension i + 1.
+bool make_map_nd(CUtensorMap* map, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {stride1, stride2};
-  cuuint32_t box[3] = {b0, b1, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  return fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 
@@ -103,25 +109,64 @@ int pick_block_n(int a_rows, int G) {
 }
 
 template <int BN, bool PAIR, int EPI>
-int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a, cudaStream_t st) {
+int launch_gemm(const CUtensorMap& ta, const gemm::TokenMaps& tb, const CUtensorMap& ts, const gemm::GemmArgs& a,
+                cudaStream_t st) {
   using C = gemm::Cfg<BN, PAIR>;
   auto k = gemm::gemm_mxfp4_kernel<BN, PAIR, EPI>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) != cudaSuccess)
     return MOE_ERR_LAUNCH;
-  launch(k, dim3(sm_count()), dim3(gemm::kThreads), C::SMEM_ALLOC, st, ta, tb, a);
+  launch(k, dim3(sm_count()), dim3(gemm::kThreads), C::SMEM_ALLOC, st, ta, tb, ts, a);
   return launch_status();
 }
 
 template <bool PAIR, int EPI>
-int launch_gemm_bn(int bn, const CUtensorMap& ta, const CUtensorMap& tb, const gemm::GemmArgs& a,
-                   cudaStream_t st) {
+int launch_gemm_bn(int bn, const CUtensorMap& ta, const gemm::TokenMaps& tb, const CUtensorMap& ts,
+                   const gemm::GemmArgs& a, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_gemm<16, PAIR, EPI>(ta, tb, a, st);
-    case 32: return launch_gemm<32, PAIR, EPI>(ta, tb, a, st);
-    case 64: return launch_gemm<64, PAIR, EPI>(ta, tb, a, st);
-    case 128: return launch_gemm<128, PAIR, EPI>(ta, tb, a, st);
+    case 16: return launch_gemm<16, PAIR, EPI>(ta, tb, ts, a, st);
+    case 32: return launch_gemm<32, PAIR, EPI>(ta, tb, ts, a, st);
+    case 64: return launch_gemm<64, PAIR, EPI>(ta, tb, ts, a, st);
+    case 128: return launch_gemm<128, PAIR, EPI>(ta, tb, ts, a, st);
     default: return MOE_ERR_UNSUPPORTED;
   }
+}
+
+// The pair kernel runs as clusters of two CTAs (one per SM); the grid is the
+// number of clusters that can be resident at once, so every cluster of the
+// persistent kernel starts immediately.
+template <int EPI>
+int launch_pair(const CUtensorMap& tw, const pair::PairMaps& tt, const CUtensorMap& ts, const pair::PairArgs& a,
+                cudaStream_t st) {
+  auto k = pair::gemm_pair_kernel<EPI>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::Cfg::SMEM_ALLOC) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2));
+  cfg.blockDim = dim3(pair::kThreads);
+  cfg.dynamicSmemBytes = pair::Cfg::SMEM_ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  static int cached_dev = -1, cached_clusters = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (dev != cached_dev) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(k), &cfg) != cudaSuccess || n <= 0)
+      return MOE_ERR_LAUNCH;
+    cached_clusters = n;
+    cached_dev = dev;
+  }
+  cfg.gridDim = dim3(2 * cached_clusters);
+  if (cudaLaunchKernelEx(&cfg, k, tw, tt, ts, a) != cudaSuccess) return MOE_ERR_LAUNCH;
+  return launch_status();
 }
 
 template <int BN, bool DUAL, int EPI, bool W8, bool ROWS = false>
@@ -215,7 +260,7 @@ int promoted_gemm(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, 
   launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, a_e4m3, a_corr);
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, a_e4m3, a_corr, 0, 0);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   if (scratch) {
     const int64_t chunks = (int64_t)N * K / 32;     // 16 input bytes (32 INT4) per thread
@@ -431,9 +476,19 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
   return launch_status();
 }
 
+// Workspace of an automatic MXFP4 call that splits its groups between the
+// 128-row swap-AB kernel and the SM-pair kernel: both plans, one after the other.
+size_t split_workspace_size(int a_rows, int n_groups, int K) {
+  return gemm::align256(gemm::ws_layout(a_rows, n_groups, K, 128).total) +
+         gemm::ws_layout(a_rows, n_groups, K, pair::BN).total;
+}
+
 size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n) {
   if (a_rows < 0 || n_groups <= 0 || K <= 0) return 0;
-  if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
+  if (block_n == 0) {
+    block_n = pick_block_n(a_rows, n_groups);
+    if (block_n == 128) return split_workspace_size(a_rows, n_groups, K);
+  }
   return gemm::ws_layout(a_rows, n_groups, K, block_n).total;
 }
 
@@ -460,7 +515,7 @@ size_t moe_workspace_size(const MoeConfig* cfg, int path) {
   if (R > (int64_t)INT32_MAX) return 0;
   const int G = c.E + (c.has_shared ? 1 : 0);
   size_t need = moe_permute_workspace_size(c.T, c.E, c.topk);
-  for (int bn : {16, 32, 64, 128})
+  for (int bn : {0, 16, 32, 64, 128, 256})
     for (int K : {c.H, c.I}) need = std::max(need, moe_gemm_workspace_size((int)R, G, K, bn));
   if (path == MOE_PATH_W4AFP8) {   // the E4M3 copy of the weights for wide token tiles
     need = std::max(need, moe_w4afp8_workspace_size((int)R, G, 2 * c.I, c.H, 0));
@@ -477,66 +532,152 @@ int moe_grouped_gemm_mxfp4(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int
     return MOE_ERR_INVALID;
   if (epilogue < MOE_EPI_STORE_F32 || epilogue > MOE_EPI_SWIGLU_QUANT) return MOE_ERR_INVALID;
   if (epilogue == MOE_EPI_SWIGLU_QUANT && N % 256) return MOE_ERR_INVALID;
-  if (block_n == 0) block_n = pick_block_n(a_rows, n_groups);
-  if (block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128)
+  if (block_n != 0 && block_n != 16 && block_n != 32 && block_n != 64 && block_n != 128 && block_n != 256)
     return MOE_ERR_UNSUPPORTED;
+  if (block_n == pair::BN && N % 256) return MOE_ERR_UNSUPPORTED;
   if (a_rows == 0) return MOE_OK;
   if (!a_e4m3 || !a_e8m0_128 || !offsets || !w_prepared || !out || !workspace) return MOE_ERR_INVALID;
   if (epilogue == MOE_EPI_SWIGLU_QUANT && !out_scale) return MOE_ERR_INVALID;
   if (!aligned(a_e4m3, 16) || !aligned(w_prepared, 32) || !aligned(workspace, 256)) return MOE_ERR_INVALID;
-  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, block_n);
+  if (epilogue != MOE_EPI_SWIGLU_QUANT && !aligned(out, 16)) return MOE_ERR_INVALID;
+
+  // Automatic choice: the tile width from the mean rows per group.  For the
+  // SwiGLU projection with at least 192 rows per group on average (long
+  // prefill) and a workspace that holds both plans, every group's whole
+  // 256-row tiles go to the SM-pair kernel and its remaining rows (fewer than
+  // 256) to the swap-AB kernel's 128-row tiles: long-prefill w1/w3 1.97 ->
+  // 1.87 ms.  At 4096 tokens (111 rows per group) and for the float32 w2
+  // projection the split measured 1-6 % slower, so those keep one kernel.
+  bool split = false;
+  if (block_n == 0) {
+    block_n = pick_block_n(a_rows, n_groups);
+    split = block_n == 128 && epilogue == MOE_EPI_SWIGLU_QUANT && a_rows >= 192 * n_groups &&
+            workspace_bytes >= split_workspace_size(a_rows, n_groups, K);
+  }
+  const bool run_swap = block_n != pair::BN;          // the swap-AB kernel (tiles of block_n rows)
+  const bool run_pair = block_n == pair::BN || split;
+  const gemm::WsLayout L = gemm::ws_layout(a_rows, n_groups, K, run_swap ? block_n : pair::BN);
   if (workspace_bytes < L.total) return MOE_ERR_INVALID;
-
-  CUtensorMap ta, tb;
-  // weight tiles: 3-D view [blocks][128 rows][128 nibbles] of the prepared
-  // blocks (the scale block that ends each prepared block is a bulk copy)
-  const uint64_t n_blocks = (uint64_t)n_groups * (N / 128) * (K / 128);
-  if (!make_map_3d(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_prepared, 128, 128, n_blocks, 64,
-                   (uint64_t)gemm::kWBlock, 128, 128))
-    return MOE_ERR_LAUNCH;
-  if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K, 128,
-                (uint32_t)block_n))
-    return MOE_ERR_LAUNCH;
-
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-  gemm::GemmArgs args;
-  args.w = w_prepared;
-  args.a_sf = ws + L.a_sf;
-  args.header = reinterpret_cast<const int*>(ws + L.header);
-  args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
-  args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
-  args.groups = reinterpret_cast<const int2*>(ws + L.groups);
-  args.G = n_groups;
-  args.N = N;
-  args.K = K;
-  args.out = out;
-  args.out_scale = out_scale;
-  args.limit = swiglu_limit;
-  // decode-sized token tiles stream the weights once: an L2 prefetch 4 K steps
-  // ahead of the producer keeps more of that stream in flight (0.270 ->
-  // 0.260 ms for the 64-token w1/w3 GEMM); wider tiles are bound by the MMA
-  // side and lose 6-12 % to the extra L2 traffic, so they do not prefetch
-  args.pf_steps = block_n <= 32 ? 4 : 0;
+  // the pair kernel's plan: after the swap-AB plan when split
+  const gemm::WsLayout LP = gemm::ws_layout(a_rows, n_groups, K, pair::BN);
+  uint8_t* wsp = split ? ws + gemm::align256(L.total) : ws;
+
+  // work items of the swap-AB kernel hold two 128-row weight tiles whenever N
+  // allows (gate + up for SwiGLU, which requires N % 256 == 0)
+  const bool pair_tiles = epilogue == MOE_EPI_SWIGLU_QUANT || N % 256 == 0;
+  const int n_ft = pair_tiles ? N / 256 : N / 128;
+
+  // Weight tiles and their scale blocks, as views of the prepared blocks
+  // (kWBlock bytes each: 128 rows x 64 bytes of nibbles, then the 512-byte
+  // scale block).  Paired order (SwiGLU): [pairs][2][...]; plain order: [row
+  // blocks][K steps][...].  ta: the swap-AB kernel's box (both tiles of an
+  // item), tw: one tile (each CTA of a pair loads its own), ts: the scale
+  // blocks of both tiles.
+  CUtensorMap ta, tw, ts;
+  {
+    const uint64_t KT = (uint64_t)K / 128, n_rb = (uint64_t)n_groups * (N / 128);
+    const uint64_t wb = (uint64_t)gemm::kWBlock;
+    const bool paired_order = epilogue == MOE_EPI_SWIGLU_QUANT;
+    const uint64_t d2 = paired_order ? 2 : KT, d3 = paired_order ? n_rb * KT / 2 : n_rb;
+    const uint64_t s2 = wb, s3 = paired_order ? 2 * wb : KT * wb;
+    const uint32_t b2 = paired_order ? 2 : 1, b3 = (!paired_order && pair_tiles) ? 2 : 1;
+    const uint64_t wdims[4] = {128, 128, d2, d3}, wstr[3] = {64, s2, s3};
+    const uint32_t wbox[4] = {128, 128, b2, b3}, wbox1[4] = {128, 128, 1, 1};
+    if (!make_map_nd(&ta, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_prepared, 4, wdims, wstr, wbox,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_nd(&tw, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w_prepared, 4, wdims, wstr, wbox1,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return MOE_ERR_LAUNCH;
+    // scale blocks as 128 32-bit words at byte 8192 of each prepared block
+    const uint64_t sdims[3] = {128, d2, d3}, sstr[2] = {s2, s3};
+    const uint32_t sbox[3] = {128, b2, b3};
+    if (!make_map_nd(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT32, w_prepared + 8192, 3, sdims, sstr, sbox,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_LAUNCH;
+  }
 
   cudaStream_t st = S(stream);
-  // work items hold two 128-row weight tiles whenever N allows (gate + up for
-  // SwiGLU, which requires N % 256 == 0)
-  const bool pair = epilogue == MOE_EPI_SWIGLU_QUANT || N % 256 == 0;
-  const int n_ft = pair ? N / 256 : N / 128;
-  launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
-      offsets, n_groups, (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
-      reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr);
-  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  switch (epilogue) {
-    case MOE_EPI_STORE_F32:
-      return pair ? launch_gemm_bn<true, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st)
-                  : launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);
-    case MOE_EPI_STORE_BF16:
-      return pair ? launch_gemm_bn<true, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st)
-                  : launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, args, st);
-    default: return launch_gemm_bn<true, MOE_EPI_SWIGLU_QUANT>(block_n, ta, tb, args, st);
+  if (run_swap) {
+    // token tiles: boxes of 16, 32, 64 and block_n rows (capped at block_n)
+    gemm::TokenMaps tb;
+    for (int i = 0; i < 4; ++i)
+      if (!make_map(&tb.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K,
+                    128, (uint32_t)gemm::token_box_rows(i, block_n)))
+        return MOE_ERR_LAUNCH;
+    gemm::GemmArgs args;
+    args.w = w_prepared;
+    args.a_sf = ws + L.a_sf;
+    args.header = reinterpret_cast<const int*>(ws + L.header);
+    args.prefix = reinterpret_cast<const int*>(ws + L.prefix);
+    args.tstart = reinterpret_cast<const int*>(ws + L.tstart);
+    args.groups = reinterpret_cast<const int2*>(ws + L.groups);
+    args.G = n_groups;
+    args.N = N;
+    args.K = K;
+    args.out = out;
+    args.out_scale = out_scale;
+    args.limit = swiglu_limit;
+    // decode-sized token tiles stream the weights once: an L2 prefetch 4 K
+    // steps ahead of the producer keeps more of that stream in flight (0.270
+    // -> 0.260 ms for the 64-token w1/w3 GEMM); wider tiles are bound by
+    // shared-memory traffic and lose 6-12 % to the extra L2 traffic
+    args.pf_steps = block_n <= 32 ? 4 : 0;
+    launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, offsets, n_groups,
+           (int)a_rows, block_n, n_ft, a_e8m0_128, K / 128, reinterpret_cast<int*>(ws + L.header),
+           reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
+           reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr, split ? pair::BN : 0, 1);
+    if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+    int rc;
+    switch (epilogue) {
+      case MOE_EPI_STORE_F32:
+        rc = pair_tiles ? launch_gemm_bn<true, MOE_EPI_STORE_F32>(block_n, ta, tb, ts, args, st)
+                        : launch_gemm_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, ts, args, st);
+        break;
+      case MOE_EPI_STORE_BF16:
+        rc = pair_tiles ? launch_gemm_bn<true, MOE_EPI_STORE_BF16>(block_n, ta, tb, ts, args, st)
+                        : launch_gemm_bn<false, MOE_EPI_STORE_BF16>(block_n, ta, tb, ts, args, st);
+        break;
+      default: rc = launch_gemm_bn<true, MOE_EPI_SWIGLU_QUANT>(block_n, ta, tb, ts, args, st);
+    }
+    if (rc != MOE_OK) return rc;
   }
+  if (run_pair) {
+    if (LP.total > workspace_bytes - (size_t)(wsp - ws)) return MOE_ERR_INVALID;
+    pair::PairMaps tt;
+    for (int i = 0; i < 4; ++i)
+      if (!make_map(&tt.tok[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, a_e4m3, (uint64_t)K, (uint64_t)a_rows, (uint64_t)K,
+                    128, (uint32_t)gemm::token_box_rows(i, 128)))
+        return MOE_ERR_LAUNCH;
+    // token scales: the plan's interleaved blocks (two 512-byte blocks per
+    // tile and group of four K steps, one per CTA) as rows of 128 words
+    const uint64_t n_sf = (uint64_t)LP.max_tiles * ((K / 128 + 3) / 4) * 2;
+    if (!make_map(&tt.tok_sf, CU_TENSOR_MAP_DATA_TYPE_UINT32, wsp + LP.a_sf, 128, n_sf, 512, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_LAUNCH;
+    pair::PairArgs pa;
+    pa.header = reinterpret_cast<const int*>(wsp + LP.header);
+    pa.prefix = reinterpret_cast<const int*>(wsp + LP.prefix);
+    pa.tstart = reinterpret_cast<const int*>(wsp + LP.tstart);
+    pa.groups = reinterpret_cast<const int2*>(wsp + LP.groups);
+    pa.G = n_groups;
+    pa.N = N;
+    pa.K = K;
+    pa.out = out;
+    pa.out_scale = out_scale;
+    pa.limit = swiglu_limit;
+    launch(gemm::gemm_prep_kernel, dim3(LP.max_tiles), dim3(gemm::kPrepThreads), 0, st, offsets, n_groups,
+           (int)a_rows, pair::BN, N / 256, a_e8m0_128, K / 128, reinterpret_cast<int*>(wsp + LP.header),
+           reinterpret_cast<int*>(wsp + LP.prefix), reinterpret_cast<int*>(wsp + LP.tstart),
+           reinterpret_cast<int2*>(wsp + LP.groups), wsp + LP.a_sf, nullptr, nullptr, split ? pair::BN : 0, 0);
+    if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+    switch (epilogue) {
+      case MOE_EPI_STORE_F32: return launch_pair<MOE_EPI_STORE_F32>(tw, tt, ts, pa, st);
+      case MOE_EPI_STORE_BF16: return launch_pair<MOE_EPI_STORE_BF16>(tw, tt, ts, pa, st);
+      default: return launch_pair<MOE_EPI_SWIGLU_QUANT>(tw, tt, ts, pa, st);
+    }
+  }
+  return MOE_OK;
 }
 
 int moe_grouped_gemm_w4afp8(const uint8_t* a_e4m3, const uint8_t* a_e8m0_128, int a_rows, const int32_t* offsets,
@@ -601,7 +742,7 @@ int moe_grouped_gemm_fp8_ptpc(const uint8_t* a_e4m3, const float* a_scale, int a
   launch(gemm::gemm_prep_kernel, dim3(L.max_tiles), dim3(gemm::kPrepThreads), 0, st, 
       offsets, n_groups, (int)a_rows, block_n, n_ft, nullptr, K / 128, reinterpret_cast<int*>(ws + L.header),
       reinterpret_cast<int*>(ws + L.prefix), reinterpret_cast<int*>(ws + L.tstart),
-      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr);
+      reinterpret_cast<int2*>(ws + L.groups), ws + L.a_sf, nullptr, nullptr, 0, 0);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
   if (dual) return launch_ptpc_bn<true, MOE_EPI_SWIGLU_F32>(block_n, ta, tb, args, st);
   if (epilogue == MOE_EPI_STORE_F32) return launch_ptpc_bn<false, MOE_EPI_STORE_F32>(block_n, ta, tb, args, st);

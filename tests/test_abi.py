@@ -59,6 +59,9 @@ def test_argument_validation_without_gpu():
                                       ctypes.c_float(10), 0, None, None, None, 0, None) == -1
     assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 256, 128, 0,
                                       ctypes.c_float(10), 48, None, None, None, 0, None) == -2
+    # the SM-pair kernel (block_n 256) needs N % 256 == 0
+    assert lib.moe_grouped_gemm_mxfp4(None, None, 4, None, 2, None, 384, 128, 0,
+                                      ctypes.c_float(10), 256, None, None, None, 0, None) == -2
     assert lib.moe_prepared_weights_size(3, 256, 512) == 3 * 2 * 4 * 8704
     assert lib.repack_mxfp4_to_int4g128(None, None, 1, 8, 96, None, None, None) == -1
     assert lib.repack_mxfp4_to_fp8_block128(None, None, 1, 100, 128, None, None, None) == -1   # N % 128
@@ -89,13 +92,24 @@ def test_layer_workspace_size_without_gpu():
     ws = moe.moe_workspace_size(T, H, I, E, k)
     R, G = T * k + T, E + 1
     need = [lib.moe_permute_workspace_size(T, E, k)]
-    need += [lib.moe_gemm_workspace_size(R, G, K, bn) for K in (H, I) for bn in (16, 32, 64, 128)]
+    need += [lib.moe_gemm_workspace_size(R, G, K, bn) for K in (H, I) for bn in (0, 16, 32, 64, 128, 256)]
     assert ws >= max(need) and ws % 256 == 0
     assert moe.moe_workspace_size(T, H, I, E, k, path=moe.MOE_PATH_PTPC) == ws
     assert moe.moe_workspace_size(T, 100, I, E, k) == 0            # H % 128
     assert moe.moe_workspace_size(T, H, I, E, 7, path=3) == 0      # unknown path
     assert moe.moe_workspace_size(T, H, I, 4, 6) == 0              # topk > E
     assert moe.moe_workspace_size(0, H, I, E, k) > 0               # empty batch still valid
+
+
+def test_split_gemm_workspace_without_gpu():
+    """With block_n = 0 a prefill-sized call (128-row tiles) may split its
+    groups between the swap-AB and the SM-pair kernel: its workspace holds
+    both plans; decode-sized calls keep one plan."""
+    from fp8_block_scaled_pow2_b200 import moe
+    R, G, K = 28672, 257, 4096
+    w128, w256 = moe.moe_gemm_workspace_size(R, G, K, 128), moe.moe_gemm_workspace_size(R, G, K, 256)
+    assert w256 > 0 and moe.moe_gemm_workspace_size(R, G, K, 0) == (w128 + 255) // 256 * 256 + w256
+    assert moe.moe_gemm_workspace_size(384, 257, K, 0) == moe.moe_gemm_workspace_size(384, 257, K, 16)
 
 
 def test_w4afp8_workspace_sizes_without_gpu():

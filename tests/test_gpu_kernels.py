@@ -152,15 +152,65 @@ GROUPS = [0, 1, 15, 16, 17, 0, 127, 128, 129, 300, 2]
 
 
 @pytest.mark.parametrize("N", [256, 384, 512])
-@pytest.mark.parametrize("block_n", [16, 32, 64, 128])
+@pytest.mark.parametrize("block_n", [16, 32, 64, 128, 256, 0])
 def test_gemm_integer_exact(lib, block_n, N):
     """All scales 2^0 and small-integer operands: every partial sum is an
     integer below 2^24, so the float32 result is exact in any order.  N = 384
-    runs single 128-row weight tiles per work item, N = 256 / 512 pairs."""
+    runs single 128-row weight tiles per work item, N = 256 / 512 pairs.
+    block_n = 256 is the SM-pair kernel (N % 256 == 0 only); block_n = 0
+    picks 128-row tiles here."""
+    if block_n == 256 and N % 256:
+        pytest.skip("the SM-pair kernel needs N % 256 == 0")
     a, asc, offsets, w, wsc = _gemm_inputs(3, GROUPS, N, 512, True)
     out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
     ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
     np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    no_device_error(lib)
+
+
+def test_gemm_split_swiglu_integer(lib):
+    """block_n = 0 with at least 192 rows per group on average splits the
+    SwiGLU GEMM: each group's whole 256-row tiles run on the SM-pair kernel,
+    the rest (here 0, 1, 44, 255 and 7 rows) on 128-row tiles.  With small
+    integers and unit scales every sum is exact, so the split result equals
+    the 128-row-tile-only and the SM-pair-only results bit for bit, and the
+    float32 gate/up equal the oracle's."""
+    I = 256
+    sizes = [256, 257, 300, 0, 511, 263, 128, 512]
+    a, asc, offsets, w, wsc = _gemm_inputs(23, sizes, 2 * I, 512, True)
+    assert sum(sizes) >= 192 * len(sizes)
+    res = {bn: _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_SWIGLU_QUANT, bn) for bn in (0, 128, 256)}
+    for bn in (128, 256):
+        np.testing.assert_array_equal(host(res[0][0]), host(res[bn][0]))
+        np.testing.assert_array_equal(host(res[0][1]), host(res[bn][1]))
+    gu, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, 256)
+    np.testing.assert_array_equal(host(gu), ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc).astype(np.float32))
+    hq2, sh2 = torch.empty_like(res[0][0]), torch.empty_like(res[0][1])
+    lib.moe_swiglu_clamp(gu, hq2, sh2, 10.0)
+    np.testing.assert_array_equal(host(res[0][0]), host(hq2))
+    np.testing.assert_array_equal(host(res[0][1]), host(sh2))
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("epi", [0, 1])
+def test_gemm_pair_tile_edges(lib, epi):
+    """SM-pair kernel (block_n = 256) on group sizes around its tile edges:
+    each 256-row tile gives rank 0 its first 128 rows and rank 1 the rest, so
+    128 / 129 / 255 / 256 / 257 / 511 rows leave one CTA's half empty, with a
+    single row, or full; random scales over three groups of four K steps
+    (K = 1536).  Float32 within the accumulation bound; bf16 the rounding of
+    the float32 result of the same kernel."""
+    sizes = [128, 129, 0, 255, 256, 257, 511, 7]
+    a, asc, offsets, w, wsc = _gemm_inputs(21, sizes, 512, 1536, False)
+    out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, 256)
+    ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
+    bound = _abs_gemm(a, asc, offsets, lambda g: ffn.dequant_mxfp4(w[g], wsc[g]))
+    got = out.cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= 1536 * 2.0 ** -24 * bound + 1e-30).all()
+    if epi == 1:
+        out16, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_BF16, 256)
+        np.testing.assert_array_equal(out16.view(torch.int16).cpu().numpy(),
+                                      torch.from_numpy(got.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy())
     no_device_error(lib)
 
 
@@ -178,8 +228,12 @@ def test_gemm_max_groups(lib):
 
 
 @pytest.mark.parametrize("N", [384, 512])
-@pytest.mark.parametrize("block_n", [16, 128])
+@pytest.mark.parametrize("block_n", [16, 128, 256])
 def test_gemm_random_scaled(lib, block_n, N):
+    """Random operands and scales (every per-32 weight scale and per-128
+    token scale differs), so a misplaced scale factor fails the bound."""
+    if block_n == 256 and N % 256:
+        pytest.skip("the SM-pair kernel needs N % 256 == 0")
     a, asc, offsets, w, wsc = _gemm_inputs(5, [3, 0, 40, 130, 1], N, 1024, False)
     out, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
     ref = ffn.grouped_gemm_mxfp4(a, asc, offsets, w, wsc)
@@ -241,10 +295,10 @@ def _swiglu_ok(hq, sh, gu_ref, I, limit=10.0):
     assert sbad.mean() < 1e-3
 
 
-@pytest.mark.parametrize("block_n", [32, 128])
+@pytest.mark.parametrize("block_n", [32, 128, 256, 0])
 def test_gemm_swiglu_epilogue_matches_standalone(lib, block_n):
     I = 256
-    a, asc, offsets, w, wsc = _gemm_inputs(9, [5, 0, 33, 140, 97, 200], 2 * I, 512, False)
+    a, asc, offsets, w, wsc = _gemm_inputs(9, [5, 0, 33, 140, 97, 300, 512], 2 * I, 512, False)
     wsc[:] = np.clip(wsc, 0, 124)                          # keep gu mostly inside the clamp
     gu, _ = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_STORE_F32, block_n)
     hq, sh = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_SWIGLU_QUANT, block_n)
