@@ -74,7 +74,7 @@ def read_peaks():
 
 GEMM_ENTRY = {"mxfp4": "moe_grouped_gemm_mxfp4", "w4afp8": "moe_grouped_gemm_w4afp8",
               "ptpc": "moe_grouped_gemm_fp8_ptpc"}
-GEMM_SOURCES = {"mxfp4": ("common.cuh", "gemm_mxfp4.cuh", "sm100.cuh"),
+GEMM_SOURCES = {"mxfp4": ("common.cuh", "gemm_mxfp4.cuh", "gemm_pair.cuh", "sm100.cuh"),
                 "w4afp8": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh"),
                 "ptpc": ("common.cuh", "gemm_mxfp4.cuh", "gemm_w4afp8.cuh", "sm100.cuh")}
 

@@ -251,9 +251,17 @@ int moe_prepare_weights(const uint8_t* fp4, const uint8_t* e8m0, int64_t n_mats,
  *             h = silu(clamp(g, +-limit)) * clamp(u, +-limit) in float32,
  *             then the a1 rule per 128 columns of h: out = E4M3 [a_rows, I],
  *             out_scale = E8M0 [a_rows, I/128]
- *   block_n   token rows per tile: 16, 32, 64 or 128 (0 = choose from
- *             a_rows and G)
- *   workspace scratch of moe_gemm_workspace_size(a_rows, G, K, block_n) bytes
+ *   block_n   token rows per tile: 16, 32, 64 or 128 (one CTA per SM, the
+ *             weight tile as the MMA's M operand), or 256 (SM pairs: clusters
+ *             of two CTAs share one tcgen05.mma.cta_group::2 of 256 tokens x
+ *             256 weight rows; needs N % 256 == 0, else MOE_ERR_UNSUPPORTED).
+ *             0 = choose from a_rows and G; for SWIGLU_QUANT with at least
+ *             192 rows per group on average, when the workspace holds both
+ *             plans, each group's whole 256-row tiles run on SM pairs and its
+ *             remaining rows on 128-row tiles (two kernel launches, disjoint
+ *             output rows).
+ *   workspace scratch of moe_gemm_workspace_size(a_rows, G, K, block_n) bytes;
+ *             with block_n = 0 this covers the two plans of a split call
  */
 size_t moe_gemm_workspace_size(int a_rows, int n_groups, int K, int block_n);
 
