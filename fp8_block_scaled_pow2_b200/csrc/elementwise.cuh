@@ -9,26 +9,55 @@
 namespace moe {
 
 // ------------------------------- a1 ---------------------------------------
-// One warp per (row, 128-column group): each lane owns 4 consecutive columns
-// (8 bytes of bf16 in, 4 bytes of E4M3 out).  "DeepSeek-V4-Flash-SI",
-// 低精度计算: FP8 E4M3 per 128 elements with a power-of-two scale.
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint2* __restrict__ x, int64_t n_groups,
-                                                        int gpr, uint32_t* __restrict__ xq,
-                                                        uint8_t* __restrict__ sx) {
+// Each half-warp quantises one (row, 128-column) group: a lane owns 8
+// consecutive columns (16 bytes of bf16 in, 8 bytes of E4M3 out).  A warp
+// takes kQuantSlots pairs of groups and issues all their loads before using
+// any, so each SM keeps enough bytes in flight to stream at the copy rate.
+// "DeepSeek-V4-Flash-SI", 低精度计算: FP8 E4M3 per 128 elements with a
+// power-of-two scale.
+constexpr int kQuantSlots = 4;
+constexpr int kQuantGroupsPerBlock = 8 * 2 * kQuantSlots;     // 8 warps of 256 threads
+
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint4* __restrict__ x, int64_t n_groups,
+                                                        uint2* __restrict__ xq, uint8_t* __restrict__ sx) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int64_t grp = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (grp >= n_groups) return;
-  const int64_t v = grp * 32 + lane;               // index in units of 4 elements
-  const uint2 w = __ldg(x + v);
-  const float a = bf16_lo(w.x), b = bf16_hi(w.x), c = bf16_lo(w.y), d = bf16_hi(w.y);
-  const float m = warp_max_nonneg(fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d))));
-  const int k = pow2_scale_exponent(m);
-  const float s = exp2_int(-k);
-  xq[v] = e4m3x4(__fmul_rn(a, s), __fmul_rn(b, s), __fmul_rn(c, s), __fmul_rn(d, s));
-  if (lane == 0) sx[grp] = (uint8_t)(k + 127);
-  (void)gpr;
+  const int hl = lane & 15;                          // lane within the half-warp
+  // group of slot s: first + 2 s + (lane >> 4)
+  const int64_t first = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * (2 * kQuantSlots);
+  uint4 wv[kQuantSlots];
+#pragma unroll
+  for (int s = 0; s < kQuantSlots; ++s) {
+    const int64_t grp = first + 2 * s + (lane >> 4);
+    wv[s] = grp < n_groups ? __ldg(x + grp * 16 + hl) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int s = 0; s < kQuantSlots; ++s) {
+    const int64_t grp = first + 2 * s + (lane >> 4);
+    const uint32_t u[4] = {wv[s].x, wv[s].y, wv[s].z, wv[s].w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16_lo(u[i]);
+      f[2 * i + 1] = bf16_hi(u[i]);
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    // maximum over the half-warp (offsets below 16 stay within it)
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int k = pow2_scale_exponent(m);
+    const float sc = exp2_int(-k);
+    if (grp < n_groups) {
+      xq[grp * 16 + hl] = make_uint2(e4m3x4(__fmul_rn(f[0], sc), __fmul_rn(f[1], sc), __fmul_rn(f[2], sc),
+                                            __fmul_rn(f[3], sc)),
+                                     e4m3x4(__fmul_rn(f[4], sc), __fmul_rn(f[5], sc), __fmul_rn(f[6], sc),
+                                            __fmul_rn(f[7], sc)));
+      if (hl == 0) sx[grp] = (uint8_t)(k + 127);
+    }
+  }
 }
 
 // ------------------------------- a5 ---------------------------------------

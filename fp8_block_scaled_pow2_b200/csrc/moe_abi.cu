@@ -380,10 +380,10 @@ int moe_get_device_error(int* code, void* stream) {
 int moe_quantize_act_fp8(const void* x, int rows, int cols, uint8_t* xq, uint8_t* sx, void* stream) {
   if (rows < 0 || cols <= 0 || cols % 128) return MOE_ERR_INVALID;
   if (rows == 0) return MOE_OK;
-  if (!x || !xq || !sx || !aligned(x, 8) || !aligned(xq, 4)) return MOE_ERR_INVALID;
+  if (!x || !xq || !sx || !aligned(x, 16) || !aligned(xq, 8)) return MOE_ERR_INVALID;
   const int64_t n_groups = (int64_t)rows * (cols / 128);
-  launch(quant_act_kernel, dim3((unsigned)((n_groups + 7) / 8)), dim3(256), 0, S(stream), 
-      reinterpret_cast<const uint2*>(x), n_groups, cols / 128, reinterpret_cast<uint32_t*>(xq), sx);
+  launch(quant_act_kernel, dim3((unsigned)((n_groups + kQuantGroupsPerBlock - 1) / kQuantGroupsPerBlock)), dim3(256),
+         0, S(stream), reinterpret_cast<const uint4*>(x), n_groups, reinterpret_cast<uint2*>(xq), sx);
   return launch_status();
 }
 

@@ -110,8 +110,8 @@ int moe_selftest_wait_timeout(int64_t timeout_ns, void* stream);
  * divide and the ceiling taken exactly; k clamped to [-127, 127]; k = 0 for
  * an all-zero group.  xq = E4M3(x * 2^-k) rounded to nearest even and
  * saturated to +-448; sx = k + 127 (E8M0).
- *   x   bfloat16 [rows, cols], 8-byte aligned; cols % 128 == 0
- *   xq  uint8 E4M3 [rows, cols], 4-byte aligned
+ *   x   bfloat16 [rows, cols], 16-byte aligned; cols % 128 == 0
+ *   xq  uint8 E4M3 [rows, cols], 8-byte aligned
  *   sx  uint8 E8M0 [rows, cols / 128]
  * rows == 0 is a no-op.  NaN/Inf inputs are a precondition violation.
  */
