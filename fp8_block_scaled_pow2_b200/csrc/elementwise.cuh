@@ -495,40 +495,78 @@ __global__ void __launch_bounds__(256) permute_gather_kernel(const uint4* __rest
 }
 
 // ------------------------------- a7 ---------------------------------------
-// One thread per (token, 4 columns): slot-order float32 sum, one bf16 rounding.
-__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ inv,
-                                                      const float* __restrict__ w, int T, int k, int H,
-                                                      int has_shared, const int32_t* __restrict__ offsets,
-                                                      int E, uint2* __restrict__ y) {
+// Block (token t, 512-column slice): each thread sums two 4-column chunks 256
+// chunks apart, issuing the row loads of up to 8 slots of both before
+// accumulating them (float32, slot order, then the shared expert's row; one
+// bf16 rounding), so a thread keeps up to 18 16-byte loads in flight.  The
+// token's slot indices and weights are read by every thread (through L1).
+constexpr int kCombineThreads = 256;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const float4* __restrict__ o,
+                                                                  const int32_t* __restrict__ inv,
+                                                                  const float* __restrict__ w, int T, int k, int H,
+                                                                  int has_shared, const int32_t* __restrict__ offsets,
+                                                                  int E, uint2* __restrict__ y) {
   pdl_trigger();
   pdl_wait();
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t t = blockIdx.x;
   const int h4 = H / 4;
-  if (i >= (int64_t)T * h4) return;
-  const int t = (int)(i / h4);
-  const int c = (int)(i % h4);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int r = __ldg(inv + (int64_t)t * k + j);
-    if (r < 0) continue;            // a pair the grouping rejected (invalid expert id)
-    const float wj = __ldg(w + (int64_t)t * k + j);
-    const float4 v = __ldg(o + (int64_t)r * h4 + c);
-    acc.x = fmaf(wj, v.x, acc.x);
-    acc.y = fmaf(wj, v.y, acc.y);
-    acc.z = fmaf(wj, v.z, acc.z);
-    acc.w = fmaf(wj, v.w, acc.w);
+  const int c0 = blockIdx.y * 2 * kCombineThreads + threadIdx.x;
+  const int c1 = c0 + kCombineThreads;
+  const bool has0 = c0 < h4, has1 = c1 < h4;
+  if (!has0) return;
+  const int32_t* it = inv + t * k;
+  const float* wt = w + t * k;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 a0 = zero, a1 = zero;
+  for (int jb = 0; jb < k; jb += 8) {
+    int r[8];
+    float wj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const bool in = jb + j < k;
+      r[j] = in ? __ldg(it + jb + j) : -1;       // -1 also: a pair the grouping rejected
+      wj[j] = in ? __ldg(wt + jb + j) : 0.f;
+    }
+    float4 v0[8], v1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v0[j] = r[j] >= 0 ? __ldg(o + (int64_t)r[j] * h4 + c0) : zero;
+      v1[j] = (r[j] >= 0 && has1) ? __ldg(o + (int64_t)r[j] * h4 + c1) : zero;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (r[j] < 0) continue;
+      a0.x = fmaf(wj[j], v0[j].x, a0.x);
+      a0.y = fmaf(wj[j], v0[j].y, a0.y);
+      a0.z = fmaf(wj[j], v0[j].z, a0.z);
+      a0.w = fmaf(wj[j], v0[j].w, a0.w);
+      a1.x = fmaf(wj[j], v1[j].x, a1.x);
+      a1.y = fmaf(wj[j], v1[j].y, a1.y);
+      a1.z = fmaf(wj[j], v1[j].z, a1.z);
+      a1.w = fmaf(wj[j], v1[j].w, a1.w);
+    }
   }
   if (has_shared) {
-    const int r = __ldg(offsets + E) + t;
-    const float4 v = __ldg(o + (int64_t)r * h4 + c);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
+    const int64_t rs = (int64_t)__ldg(offsets + E) + t;
+    const float4 v = __ldg(o + rs * h4 + c0);
+    const float4 u = has1 ? __ldg(o + rs * h4 + c1) : zero;
+    a0.x += v.x;
+    a0.y += v.y;
+    a0.z += v.z;
+    a0.w += v.w;
+    a1.x += u.x;
+    a1.y += u.y;
+    a1.z += u.z;
+    a1.w += u.w;
   }
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  y[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+  auto pack = [](const float4& a) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(a.z, a.w);
+    return make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+  };
+  y[t * h4 + c0] = pack(a0);
+  if (has1) y[t * h4 + c1] = pack(a1);
 }
 
 }  // namespace moe

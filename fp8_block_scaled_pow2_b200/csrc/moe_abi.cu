@@ -789,10 +789,11 @@ int moe_combine(const float* o, const int32_t* inv, const float* w, int T, int k
   if (T == 0) return MOE_OK;
   if (!o || !y || (k > 0 && (!inv || !w)) || (has_shared && !offsets)) return MOE_ERR_INVALID;
   if (!aligned(o, 16) || !aligned(y, 8)) return MOE_ERR_INVALID;
-  const int64_t n = (int64_t)T * (H / 4);
-  launch(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, S(stream), 
-      reinterpret_cast<const float4*>(o), inv, w, T, k, H, has_shared ? 1 : 0, offsets, E,
-      reinterpret_cast<uint2*>(y));
+  // one block per (token, 512 columns): two 4-column chunks a thread
+  const int slices = (H / 4 + 2 * kCombineThreads - 1) / (2 * kCombineThreads);
+  launch(combine_kernel, dim3((unsigned)T, (unsigned)slices), dim3(kCombineThreads), 0, S(stream),
+         reinterpret_cast<const float4*>(o), inv, w, T, k, H, has_shared ? 1 : 0, offsets, E,
+         reinterpret_cast<uint2*>(y));
   return launch_status();
 }
 
