@@ -359,7 +359,7 @@ const char* moe_status_string(int s) {
   }
 }
 
-int moe_version(void) { return 100; }
+int moe_version(void) { return 200; }
 
 int moe_get_device_error(int* code, void* stream) {
   if (!code) return MOE_ERR_INVALID;
