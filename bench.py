@@ -584,7 +584,7 @@ def bench_layer(args, name: str, weights: str, shared: str, steps: int, warmup: 
         # region; StepRunner overlaps those copies with the neighbouring steps'
         # compute on a second stream
         from fp8_block_scaled_pow2_b200.runner import StepRunner, pinned_inputs
-        runner = StepRunner(layer, T, block_n=args.block_n, graphs=use_graph)
+        runner = StepRunner(layer, T, block_n=args.block_n, graphs=use_graph, input_sets=args.input_sets)
         xh, lh, yh = pinned_inputs(x, logits)
         for _ in range(max(1, warmup)):
             runner.submit(xh, lh, yh)
@@ -679,7 +679,8 @@ def run_ours(args, wl):
         "gemm": main["gemm"],
         "segments": main["segments"],
         "e2e": {"value": round(tokens / (r["e2e"]["ms"] / 1e3), 2), "unit": "tokens/s",
-                "api": "StepRunner.submit (pinned host x, logits in; y out; copies on their own streams)",
+                "api": "StepRunner.submit (pinned host x, logits in; y out; copies on their own streams; "
+                       f"{args.input_sets} device input set(s))",
                 "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"]},
         "gpu_launches": kernels_per_step(r["wl"], args.shared, args.weights) * args.steps,
@@ -859,6 +860,8 @@ def main(argv=None):
                     help="replay the layer step as four CUDA graphs (off: eager library calls)")
     ap.add_argument("--block-n", type=int, default=0,
                     help="token rows per GEMM tile (0: the library's choice)")
+    ap.add_argument("--input-sets", type=int, default=2, choices=[1, 2],
+                    help="device copies of the step inputs in the host-buffer (e2e) runs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extras", choices=["default", "none"], default="default",

@@ -251,15 +251,16 @@ def test_empty_batch(lib, weights):
     assert lib.moe_get_device_error() == 0
 
 
-@pytest.mark.parametrize("graphs", [True, False])
-def test_step_runner_overlapped_copies(lib, graphs):
-    """StepRunner (host copies overlapped with the neighbouring steps on a
-    second stream) gives, step after step with changing inputs, the eager
-    forward's y bit for bit."""
+@pytest.mark.parametrize("graphs,input_sets", [(True, 2), (False, 2), (True, 1)])
+def test_step_runner_overlapped_copies(lib, graphs, input_sets):
+    """StepRunner (host copies overlapped with the neighbouring steps on
+    their own streams, into one or two device copies of the inputs) gives,
+    step after step with changing inputs, the eager forward's y bit for
+    bit."""
     from fp8_block_scaled_pow2_b200.runner import StepRunner, pinned_inputs
     wl = synth.tiny_layer(8)
     layer = MoeLayer(wl.w13, wl.w13_e8m0, wl.w2, wl.w2_e8m0, wl.topk)
-    runner = StepRunner(layer, wl.T, graphs=graphs)
+    runner = StepRunner(layer, wl.T, graphs=graphs, input_sets=input_sets)
     steps = [synth.tiny_layer(20 + i) for i in range(4)]
     hosts = [pinned_inputs(s.x_bf16, s.logits) for s in steps]
     for xh, lh, yh in hosts:
