@@ -21,7 +21,7 @@
 // group-major, then weight tile, then token tile, so CTAs running at the same
 // time stream the same weight tiles from L2.
 //
-// CTA roles (persistent kernel, one CTA per SM, 11 warps):
+// CTA roles (persistent kernel, one CTA per SM, 12 warps):
 //   warp 0        TMA producer: weight tiles (FP4 unpacked to one nibble per
 //                 byte in shared memory by the 16U4_ALIGN16B tensor-map type),
 //                 their pre-interleaved scale blocks, the token tile and the
@@ -32,6 +32,7 @@
 //                 single tile; see Cfg::ISSUERS)
 //   warps 2..9    epilogue: TMEM -> registers -> global (float32 / bf16 /
 //                 SwiGLU + per-128 FP8 requantisation)
+//   warp 11       L2 prefetcher on decode-sized token tiles (see GemmArgs::pf_steps)
 // The producer and issuer loops run converged on their whole warp and one
 // elected lane issues the copies and tensor-core instructions.
 #pragma once
