@@ -192,6 +192,21 @@ def test_gemm_split_swiglu_integer(lib):
     no_device_error(lib)
 
 
+def test_gemm_split_without_whole_tiles(lib):
+    """A split call (at least 192 rows per group on average) in which no
+    group holds a whole 256-row tile: the SM-pair kernel runs with no work
+    item (it allocates and frees its tensor memory and meets its peer at the
+    cluster barriers), every row comes from the 128-row tiles, and the result
+    equals the call that runs only those."""
+    I = 256
+    sizes = [200, 255, 192, 230]
+    a, asc, offsets, w, wsc = _gemm_inputs(24, sizes, 2 * I, 512, False)
+    hq0, sh0 = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_SWIGLU_QUANT, 0)
+    hq1, sh1 = _run_gemm(lib, a, asc, offsets, w, wsc, lib.MOE_EPI_SWIGLU_QUANT, 128)
+    assert torch.equal(hq0, hq1) and torch.equal(sh0, sh1)
+    no_device_error(lib)
+
+
 @pytest.mark.parametrize("epi", [0, 1])
 def test_gemm_pair_tile_edges(lib, epi):
     """SM-pair kernel (block_n = 256) on group sizes around its tile edges:
